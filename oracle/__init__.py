@@ -1,0 +1,287 @@
+"""Float64 CPU oracle for the Voxtral Realtime causal sliding-window encoder.
+
+TEST INFRASTRUCTURE ONLY.  Only ``tests/``, ``__graft_entry__.smoke()`` and the
+``cpu_baseline`` / ``--impl reference`` legs of ``bench.py`` may import this
+package.  The product path (the CUDA library and its Python binding) never
+imports, links or runs it, and this package shares no code with it.
+
+Every function is a plain, slow statement of what the encoder computes,
+written from the transcribe.cpp porting notes "Voxtral", section
+"Architecture -> Voxtral Realtime 2602 (voxtral_realtime)": a causal conv stem
+(left-pad-only CausalConv1d, conv2 stride 2), then 32 causal sliding-window
+(750) transformer layers with RoPE (theta 1e6, head_dim 64), RMSNorm pre-norm,
+a SwiGLU/silu MLP, 32-head MHA, no bias on k_proj and FFN bias only on the down
+projection; plus the streaming schedule of the same section (4 encoder frames
+per step).  Numpy matmuls serve as library steps; nothing is blocked, fused or
+reordered beyond the definitions below.
+
+Readings where the page is silent (each pinned by a test in tests/):
+  * window: query i sees keys j with i - W < j <= i (exactly W keys incl. itself);
+  * RoPE: split-halves pairing (x_m, x_{m+D/2}), inv_freq_m = theta^(-2m/D),
+    angle = position * inv_freq_m, applied to q and k after the bias add;
+    positions are absolute 0-based frame indices (pos0 + t);
+  * softmax scale 1/sqrt(head_dim); RMSNorm x / sqrt(mean(x^2) + eps) * g;
+  * SwiGLU: silu(x W_g^T [+ b_g]) * (x W_u^T [+ b_u]) with silu(z) = z * sigmoid(z);
+  * conv stem: left zero padding of k - 1 = 2 frames before each conv, exact
+    (erf) GELU, output length floor((Tm - 1) / 2) + 1;
+  * streaming: the ring holds frame f in slot f mod W; a step reads every old
+    in-window slot before any new frame is written.
+
+Parity against the real checkpoint is unpinned: the pages print no
+activations and no trained weights are available.
+"""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+from scipy.special import erf as _erf
+
+__all__ = [
+    "rms_norm", "rope_inv_freq", "rope", "swa_attention", "swa_attention_rows",
+    "silu", "gelu", "encoder_layer", "ring_from_sequence", "stream_step_layer",
+    "stream_step", "conv_stem", "conv_out_len", "encoder", "as64",
+]
+
+
+def as64(a):
+    """Upcast (bf16-exact float32 or float32) inputs to float64, exactly."""
+    return None if a is None else np.asarray(a, dtype=np.float64)
+
+
+# ---------------------------------------------------------------- elementwise
+
+def rms_norm(x, g, eps=1e-5):
+    """RMSNorm pre-norm ("RMSNorm pre-norm", Voxtral Realtime 2602 architecture):
+    y = x / sqrt(mean(x^2 over the model dimension) + eps) * g."""
+    x = as64(x)
+    ms = np.mean(x * x, axis=-1, keepdims=True)
+    return x / np.sqrt(ms + eps) * as64(g)
+
+
+def silu(z):
+    """silu(z) = z * sigmoid(z) (the MLP activation of the 2602 encoder)."""
+    return z / (1.0 + np.exp(-z))
+
+
+def gelu(z):
+    """Exact GELU, 0.5 z (1 + erf(z / sqrt(2))) (the conv-stem activation)."""
+    return 0.5 * z * (1.0 + _erf(z / math.sqrt(2.0)))
+
+
+# ----------------------------------------------------------------------- RoPE
+
+def rope_inv_freq(head_dim, theta):
+    """inv_freq_m = theta^(-2m / head_dim), m = 0 .. head_dim/2 - 1."""
+    m = np.arange(head_dim // 2, dtype=np.float64)
+    return theta ** (-2.0 * m / head_dim)
+
+
+def rope(x, pos, theta):
+    """Rotary position embedding (theta 1e6, head_dim 64 for the encoder).
+
+    x: [..., T, H, D]; pos: [T] absolute frame positions.  Each pair
+    (x_m, x_{m+D/2}) is rotated by the angle pos * inv_freq_m.
+    """
+    x = as64(x)
+    D = x.shape[-1]
+    half = D // 2
+    ang = np.asarray(pos, dtype=np.float64)[:, None] * rope_inv_freq(D, theta)[None, :]
+    cos = np.cos(ang)[:, None, :]
+    sin = np.sin(ang)[:, None, :]
+    x1, x2 = x[..., :half], x[..., half:]
+    return np.concatenate([x1 * cos - x2 * sin, x2 * cos + x1 * sin], axis=-1)
+
+
+# ------------------------------------------------------------------ attention
+
+def swa_attention_rows(q, k, v, window, rows, scale=None):
+    """Causal sliding-window attention for selected query rows.
+
+    o_i = sum_{j : i - W < j <= i} softmax_j(<q_i, k_j> * scale) v_j, per head
+    ("causal + sliding-window (750)" attention of the 2602 encoder).
+    q, k, v: [B, T, H, D] (RoPE already applied).  Returns [B, len(rows), H, D].
+    """
+    q, k, v = as64(q), as64(k), as64(v)
+    B, T, H, D = q.shape
+    scale = 1.0 / math.sqrt(D) if scale is None else scale
+    out = np.empty((B, len(rows), H, D))
+    for n, i in enumerate(rows):
+        lo = max(0, i - window + 1)
+        s = np.einsum("bhd,bjhd->bhj", q[:, i], k[:, lo:i + 1]) * scale
+        s = s - np.max(s, axis=-1, keepdims=True)
+        p = np.exp(s)
+        p /= np.sum(p, axis=-1, keepdims=True)
+        out[:, n] = np.einsum("bhj,bjhd->bhd", p, v[:, lo:i + 1])
+    return out
+
+
+def swa_attention(q, k, v, window, scale=None):
+    """swa_attention_rows over every query row: [B, T, H, D] -> [B, T, H, D]."""
+    T = np.shape(q)[1]
+    return swa_attention_rows(q, k, v, window, range(T), scale)
+
+
+# ------------------------------------------------------------- encoder layer
+
+def _qkv(y, p, dims, pos):
+    """Projections q = y Wq^T + bq, k = y Wk^T (no bias), v = y Wv^T + bv,
+    split into heads, RoPE on q and k at `pos` (per row of the T axis)."""
+    H, D = dims.n_heads, dims.head_dim
+    lead = y.shape[:-1]
+    q = y @ as64(p["wq"]).T + as64(p["bq"])
+    k = y @ as64(p["wk"]).T
+    v = y @ as64(p["wv"]).T + as64(p["bv"])
+    q = q.reshape(*lead, H, D)
+    k = k.reshape(*lead, H, D)
+    v = v.reshape(*lead, H, D)
+    return rope(q, pos, dims.rope_theta), rope(k, pos, dims.rope_theta), v
+
+
+def _mlp(h, p, dims):
+    """SwiGLU MLP branch: (silu(y Wg^T [+bg]) * (y Wu^T [+bu])) Wd^T + bd, y = RMSNorm(h)."""
+    y1 = rms_norm(h, p["ffn_norm_g"], dims.eps)
+    g = y1 @ as64(p["wg"]).T
+    u = y1 @ as64(p["wu"]).T
+    if p.get("bg") is not None:
+        g = g + as64(p["bg"])
+    if p.get("bu") is not None:
+        u = u + as64(p["bu"])
+    return (silu(g) * u) @ as64(p["wd"]).T + as64(p["bd"])
+
+
+def encoder_layer(x, p, dims, pos0=0, return_kv=False):
+    """One pre-norm encoder layer over whole clips.
+
+    x: [B, T, d] -> [B, T, d]:
+      h   = x + SWA(RoPE(q), RoPE(k), v) Wo^T + bo
+      out = h + MLP(RMSNorm(h))
+    with y0 = RMSNorm(x) feeding the q/k/v projections, positions pos0 + t.
+    """
+    x = as64(x)
+    B, T, d = x.shape
+    pos = pos0 + np.arange(T)
+    y0 = rms_norm(x, p["attn_norm_g"], dims.eps)
+    q, k, v = _qkv(y0, p, dims, pos)
+    a = swa_attention(q, k, v, dims.window).reshape(B, T, dims.hd)
+    h = x + a @ as64(p["wo"]).T + as64(p["bo"])
+    out = h + _mlp(h, p, dims)
+    return (out, k, v) if return_kv else out
+
+
+# ------------------------------------------------------------------ streaming
+
+def ring_from_sequence(k, v, window):
+    """Ring cache after appending a whole sequence: frame f sits in slot f mod W.
+
+    k, v: [S, T, H, D] -> ring_k, ring_v: [S, H, W, D] (slots never written are 0).
+    """
+    k, v = as64(k), as64(v)
+    S, T, H, D = k.shape
+    rk = np.zeros((S, H, window, D))
+    rv = np.zeros((S, H, window, D))
+    for f in range(max(0, T - window), T):
+        rk[:, :, f % window] = k[:, f]
+        rv[:, :, f % window] = v[:, f]
+    return rk, rv
+
+
+def stream_step_layer(x_new, p, dims, ring_k, ring_v, pos):
+    """One layer of an incremental streaming step over a W-slot ring cache.
+
+    x_new: [S, n, d] (frames pos[s] .. pos[s]+n-1 of each stream);
+    ring_k/ring_v: [S, H, W, D] holding frames max(0, pos-W) .. pos-1 at slot f mod W.
+    Query frame f_q attends frames f with f_q - W < f <= f_q; frames before pos[s]
+    come from the ring, the others from this step.  All ring reads happen before
+    the n new frames are written to slots (pos[s] + t) mod W.
+    Returns (out [S, n, d], new ring_k, new ring_v).
+    """
+    x_new = as64(x_new)
+    S, n, d = x_new.shape
+    H, D, W = dims.n_heads, dims.head_dim, dims.window
+    scale = 1.0 / math.sqrt(D)
+    ring_k, ring_v = as64(ring_k), as64(ring_v)
+    y0 = rms_norm(x_new, p["attn_norm_g"], dims.eps)
+    a = np.empty((S, n, H, D))
+    knew_all, vnew_all = [], []
+    for s in range(S):
+        ps = int(pos[s])
+        q, knew, vnew = _qkv(y0[s], p, dims, ps + np.arange(n))     # [n, H, D]
+        knew_all.append(knew)
+        vnew_all.append(vnew)
+        for i in range(n):
+            fq = ps + i
+            keys, vals = [], []
+            for f in range(max(0, fq - W + 1), fq + 1):
+                if f < ps:
+                    keys.append(ring_k[s, :, f % W])
+                    vals.append(ring_v[s, :, f % W])
+                else:
+                    keys.append(knew[f - ps])
+                    vals.append(vnew[f - ps])
+            K = np.stack(keys, axis=1)                  # [H, J, D]
+            V = np.stack(vals, axis=1)
+            sc = np.einsum("hd,hjd->hj", q[i], K) * scale
+            sc = sc - np.max(sc, axis=-1, keepdims=True)
+            pr = np.exp(sc)
+            pr /= np.sum(pr, axis=-1, keepdims=True)
+            a[s, i] = np.einsum("hj,hjd->hd", pr, V)
+    new_k, new_v = ring_k.copy(), ring_v.copy()
+    for s in range(S):
+        ps = int(pos[s])
+        for t in range(n):
+            new_k[s, :, (ps + t) % W] = knew_all[s][t]
+            new_v[s, :, (ps + t) % W] = vnew_all[s][t]
+    h = x_new + a.reshape(S, n, dims.hd) @ as64(p["wo"]).T + as64(p["bo"])
+    out = h + _mlp(h, p, dims)
+    return out, new_k, new_v
+
+
+def stream_step(x_new, layers, dims, rings, pos, final_g=None):
+    """A streaming step through a stack of layers: each layer's output feeds the
+    next; rings is a list of (ring_k, ring_v) per layer.  Returns
+    (out, new_rings, pos + n); a final RMSNorm is applied when final_g is given."""
+    x = as64(x_new)
+    new_rings = []
+    for p, (rk, rv) in zip(layers, rings):
+        x, nk, nv = stream_step_layer(x, p, dims, rk, rv, pos)
+        new_rings.append((nk, nv))
+    if final_g is not None:
+        x = rms_norm(x, final_g, dims.eps)
+    return x, new_rings, np.asarray(pos) + x.shape[1]
+
+
+# ------------------------------------------------------------------ conv stem
+
+def conv_out_len(Tm):
+    """Frames out of the stride-2 causal conv with left padding 2 and kernel 3."""
+    return (Tm - 1) // 2 + 1
+
+
+def conv_stem(mel, w1, b1, w2, b2):
+    """Causal conv stem (left-pad-only CausalConv1d, conv2 stride 2):
+      h1[t] = GELU(b1 + sum_{k,c} w1[:, c, k] x[c, t + k - 2]),      t < Tm
+      h2[t] = GELU(b2 + sum_{k,c} w2[:, c, k] h1[c, 2t + k - 2]),    t < floor((Tm-1)/2)+1
+    with x[., t<0] = h1[., t<0] = 0.  mel: [B, C, Tm] -> [B, T_out, d] (frame-major)."""
+    x = as64(mel)
+    w1, b1, w2, b2 = as64(w1), as64(b1), as64(w2), as64(b2)
+    B, C, Tm = x.shape
+    xp = np.concatenate([np.zeros((B, C, 2)), x], axis=2)            # [B, C, Tm+2]
+    h1 = np.zeros((B, w1.shape[0], Tm)) + b1[None, :, None]
+    for k in range(3):
+        h1 += np.einsum("oc,bct->bot", w1[:, :, k], xp[:, :, k:k + Tm])
+    h1 = gelu(h1)
+    To = conv_out_len(Tm)
+    hp = np.concatenate([np.zeros((B, h1.shape[1], 2)), h1], axis=2)  # [B, d, Tm+2]
+    h2 = np.zeros((B, w2.shape[0], To)) + b2[None, :, None]
+    for k in range(3):
+        h2 += np.einsum("oc,bct->bot", w2[:, :, k], hp[:, :, k:k + 2 * To - 1:2])
+    return np.transpose(gelu(h2), (0, 2, 1))
+
+
+def encoder(mel, conv, layers, final_g, dims):
+    """Whole-clip encoder: conv stem -> layers (positions from 0) -> final RMSNorm."""
+    x = conv_stem(mel, conv["w1"], conv["b1"], conv["w2"], conv["b2"])
+    for p in layers:
+        x = encoder_layer(x, p, dims, pos0=0)
+    return rms_norm(x, final_g, dims.eps)
