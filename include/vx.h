@@ -1,0 +1,232 @@
+/*
+ * vx.h -- C ABI of libvx, B200 (sm_100a) kernels for the Voxtral Realtime
+ * causal sliding-window audio encoder.
+ *
+ * Source of the operations: transcribe.cpp porting notes "Voxtral", section
+ * "Architecture -> Voxtral Realtime 2602 (voxtral_realtime)" (causal conv stem,
+ * 32 causal sliding-window (750) layers, RoPE theta 1e6 / head_dim 64, RMSNorm
+ * pre-norm, SwiGLU MLP, 32-head MHA, no k_proj bias, FFN bias only on down) and
+ * its "Streaming schedule" paragraph (4 encoder frames per 80 ms step); the
+ * Core AI model card "Voxtral Mini 4B Realtime -- Core AI", section "Usage /
+ * Known limitations" (the pages' streaming encoder keeps an append-only frame
+ * buffer; this library replaces it with a W-slot ring).
+ *
+ * Conventions (all entry points):
+ *  - Every pointer argument is a DEVICE pointer owned by the caller unless the
+ *    comment says "host".  The library never allocates or frees device memory;
+ *    scratch space is the caller's workspace `ws` of `ws_bytes` bytes, sized by
+ *    the matching vx_*_workspace() query.  ws must be 256-byte aligned.
+ *  - Work is enqueued on `stream` and is asynchronous; nothing synchronises the
+ *    host except vx_status_check().
+ *  - Activations are row-major and frame-major: [B, T, C] with C contiguous.
+ *    Attention tensors are [B, T, H, D] with D contiguous.
+ *  - bf16 tensors are passed as `const void*` holding IEEE bfloat16 bit patterns.
+ *  - Return value: VX_OK, or an error code with a message in vx_last_error()
+ *    (thread-local).  Argument errors are detected on the host before any work
+ *    is enqueued.  A kernel whose bounded wait ran out records
+ *    VX_ERR_DEVICE_TIMEOUT in the workspace status word (first 256 bytes of
+ *    ws); read it with vx_status_check() and clear it with vx_status_reset().
+ *  - Calls on distinct streams with distinct workspaces are thread-safe.
+ *    Unsupported shapes return VX_ERR_UNSUPPORTED; there is no fallback path.
+ */
+#ifndef VX_H_
+#define VX_H_
+
+#include <stddef.h>
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#if defined(__GNUC__)
+#define VX_API __attribute__((visibility("default")))
+#else
+#define VX_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum vx_status {
+  VX_OK = 0,
+  VX_ERR_INVALID_ARG = 1,     /* null pointer, bad shape, misalignment, small ws */
+  VX_ERR_UNSUPPORTED = 2,     /* valid but not built (e.g. head_dim != 64)       */
+  VX_ERR_CUDA = 3,            /* a CUDA runtime/driver call or launch failed     */
+  VX_ERR_DEVICE_TIMEOUT = 4   /* a bounded in-kernel wait expired                */
+} vx_status;
+
+typedef enum vx_dtype { VX_F32 = 0, VX_BF16 = 1 } vx_dtype;
+
+/* Shape of one encoder layer.  Supported: head_dim 64, d_model a multiple of
+ * 128 and <= 2048, n_heads*head_dim a multiple of 128, ffn_hidden a multiple
+ * of 64, window >= 1.  Voxtral Realtime 2602: {1280, 32, 64, 5120, 750, 1e6, 1e-5}. */
+typedef struct vx_layer_cfg {
+  int d_model;
+  int n_heads;
+  int head_dim;
+  int ffn_hidden;
+  int window;        /* W: query i sees keys j with i - W < j <= i */
+  float rope_theta;  /* inv_freq_m = theta^(-2m/head_dim), split-halves pairing */
+  float eps;         /* RMSNorm epsilon */
+} vx_layer_cfg;
+
+/* One layer's parameters as the checkpoint holds them (PyTorch [out, in]
+ * order, all bf16).  bg/bu may be NULL (the 2602 encoder has no gate/up bias).
+ * Input of vx_pack_layer only. */
+typedef struct vx_layer_params {
+  const void *attn_norm_g;          /* [d]            */
+  const void *wq, *wk, *wv;         /* [HD, d] each   */
+  const void *bq, *bv;              /* [HD] each (k has no bias) */
+  const void *wo;                   /* [d, HD]        */
+  const void *bo;                   /* [d]            */
+  const void *ffn_norm_g;           /* [d]            */
+  const void *wg, *wu;              /* [F, d] each    */
+  const void *bg, *bu;              /* [F] or NULL    */
+  const void *wd;                   /* [d, F]         */
+  const void *bd;                   /* [d]            */
+} vx_layer_params;
+
+/* A layer in the layout the kernels read (built by vx_pack_layer). */
+typedef struct vx_layer_weights {
+  const void *attn_norm_g;  /* [d] bf16                                        */
+  const void *wqkv;         /* [3*HD, d] bf16: rows q | k | v                   */
+  const void *bqkv;         /* [3*HD] bf16: bq | 0 | bv                         */
+  const void *wo;           /* [d, HD] bf16                                     */
+  const void *bo;           /* [d] bf16                                         */
+  const void *ffn_norm_g;   /* [d] bf16                                         */
+  const void *wgu;          /* [2F, d] bf16: gate/up rows interleaved in blocks
+                               of 64 (gate f0..f0+63, up f0..f0+63, gate ...)   */
+  const void *bgu;          /* [2F] bf16, same interleave (zeros if no bias)    */
+  const void *wd;           /* [d, F] bf16                                      */
+  const void *bd;           /* [d] bf16                                         */
+} vx_layer_weights;
+
+/* Per-layer ring-buffer K/V cache of `window` slots for n_streams streams.
+ * k and v are [n_layers][n_streams][n_heads][window][head_dim] bf16; frame f of
+ * stream s sits in slot f mod window.  pos[s] (device int64) counts the frames
+ * already appended to stream s; the ring holds frames max(0,pos-W) .. pos-1. */
+typedef struct vx_kv_ring {
+  void *k;
+  void *v;
+  int64_t *pos;
+  int n_layers;
+  int n_streams;
+  int window;
+} vx_kv_ring;
+
+/* ---------------------------------------------------------------- utilities */
+
+VX_API const char *vx_last_error(void);       /* thread-local message of the last error */
+VX_API const char *vx_version(void);
+/* Bounded-wait limit for every in-kernel wait (default 1e9 ns).  Host setting,
+ * read at launch time; affects launches enqueued afterwards (all threads). */
+VX_API void vx_set_wait_timeout_ns(uint64_t ns);
+/* Clears the status word at the start of ws (async on stream). */
+VX_API vx_status vx_status_reset(void *ws, cudaStream_t stream);
+/* Synchronises `stream`, then returns VX_ERR_DEVICE_TIMEOUT if a kernel
+ * recorded an expired wait in ws, else VX_OK (or VX_ERR_CUDA). */
+VX_API vx_status vx_status_check(const void *ws, cudaStream_t stream);
+
+/* Fills the packed layout of one layer.  packed_wqkv: [3*HD, d] bf16,
+ * packed_bqkv: [3*HD] bf16, packed_wgu: [2F, d] bf16, packed_bgu: [2F] bf16.
+ * The caller then points vx_layer_weights at these buffers and at the
+ * unchanged norm gains, wo, bo, wd, bd. */
+VX_API vx_status vx_pack_layer(const vx_layer_cfg *cfg, const vx_layer_params *in,
+                        void *packed_wqkv, void *packed_bqkv,
+                        void *packed_wgu, void *packed_bgu, cudaStream_t stream);
+
+/* Reorders a Conv1d weight [out, in, 3] (PyTorch) to [out, 3, in], the
+ * layout vx_conv_stem_fwd reads (bf16 both). */
+VX_API vx_status vx_pack_conv_weight(const void *w, void *w_packed, int out_ch, int in_ch,
+                              cudaStream_t stream);
+
+/* ------------------------------------------------------------- operations */
+
+/* Causal sliding-window multi-head attention with RoPE (the encoder's
+ * attention: each frame attends to itself and the W-1 frames before it).
+ *   o_i = sum_{j: i-W < j <= i} softmax_j(<q'_i, k'_j> * scale) v_j per head,
+ * with q', k' = RoPE(q, k) at positions pos0 + t when apply_rope != 0
+ * (split-halves pairing, inv_freq_m = rope_theta^(-2m/D)).
+ * q, k, v, o: [B, T, H, D] of dtype dt (VX_F32: fp32 CUDA-core path;
+ * VX_BF16: tcgen05 tensor-core path, fp32 softmax).  D must be 64.
+ * scale <= 0 selects 1/sqrt(D).  Workspace: vx_swa_attn_workspace(). */
+VX_API vx_status vx_swa_attn_fwd(const void *q, const void *k, const void *v, void *o,
+                          vx_dtype dt, int B, int T, int H, int D, int window,
+                          int apply_rope, float rope_theta, int64_t pos0, float scale,
+                          void *ws, size_t ws_bytes, cudaStream_t stream);
+VX_API size_t vx_swa_attn_workspace(vx_dtype dt, int B, int T, int H, int D, int apply_rope);
+
+/* RMSNorm with optional residual add:
+ *   h = x + r (r may be NULL), y = h / sqrt(mean(h^2) + eps) * g.
+ * x, r, h_out: [M, d] fp32 (h_out may be NULL); g: [d] bf16;
+ * y: [M, d] of dtype y_dt (bf16 for GEMM operands, fp32 for the final norm). */
+VX_API vx_status vx_rms_norm_fwd(const float *x, const float *r, const void *g, float *h_out,
+                          void *y, vx_dtype y_dt, int M, int d, float eps,
+                          void *ws, size_t ws_bytes, cudaStream_t stream);
+
+/* One encoder layer over B clips of T frames (whole-sequence, causal):
+ *   y0 = RMSNorm(x); q,k,v = y0 W^T + b; RoPE(q,k) at pos0 + t;
+ *   h = x + SWA(q,k,v) Wo^T + bo; out = h + (silu(y1 Wg^T + bg) * (y1 Wu^T + bu)) Wd^T + bd,
+ *   y1 = RMSNorm(h).
+ * x, y: [B, T, d] fp32 (y may alias nothing in ws; x == y is allowed).
+ * Workspace: vx_encoder_layer_workspace(). */
+VX_API vx_status vx_encoder_layer_fwd(const vx_layer_cfg *cfg, const vx_layer_weights *w,
+                               const float *x, float *y, int B, int T, int64_t pos0,
+                               void *ws, size_t ws_bytes, cudaStream_t stream);
+VX_API size_t vx_encoder_layer_workspace(const vx_layer_cfg *cfg, int B, int T);
+
+/* Causal conv stem: left-pad-only Conv1d(n_mels -> d, k3, s1) + GELU, then
+ * Conv1d(d -> d, k3, s2) + GELU (exact erf GELU, left zero padding of 2 frames
+ * before each conv).  mel: [B, n_mels, Tm] fp32; w1p: [d, 3, n_mels] and
+ * w2p: [d, 3, d] bf16 (vx_pack_conv_weight); b1, b2: [d] bf16;
+ * out: [B, T_out, d] fp32 with T_out = (Tm - 1) / 2 + 1.
+ * n_mels must be a multiple of 64.  Workspace: vx_conv_stem_workspace(). */
+VX_API vx_status vx_conv_stem_fwd(const float *mel, const void *w1p, const void *b1,
+                           const void *w2p, const void *b2, float *out,
+                           int B, int n_mels, int Tm, int d,
+                           void *ws, size_t ws_bytes, cudaStream_t stream);
+VX_API size_t vx_conv_stem_workspace(int B, int n_mels, int Tm, int d);
+
+/* Whole-clip encoder: conv stem -> n_layers encoder layers (positions from 0)
+ * -> final RMSNorm with gain final_g ([d] bf16).  layers: HOST array of
+ * n_layers weight structs (device pointers inside).  out: [B, T_out, d] fp32.
+ * Workspace: vx_encoder_workspace(). */
+VX_API vx_status vx_encoder_fwd(const vx_layer_cfg *cfg, const float *mel, int B, int n_mels, int Tm,
+                         const void *w1p, const void *b1, const void *w2p, const void *b2,
+                         const vx_layer_weights *layers, int n_layers, const void *final_g,
+                         float *out, void *ws, size_t ws_bytes, cudaStream_t stream);
+VX_API size_t vx_encoder_workspace(const vx_layer_cfg *cfg, int B, int n_mels, int Tm);
+
+/* Streaming prefill: runs the whole-sequence forward over the first T frames
+ * of each of the ring's streams through the ring's n_layers layers, writes
+ * each layer's K/V of frames max(0,T-W) .. T-1 into the ring (slot f mod W)
+ * and sets pos[s] = T.  x: [S, T, d] fp32 layer-0 input, y: [S, T, d] fp32
+ * output of the last layer (final RMSNorm applied when final_g != NULL).
+ * Workspace: vx_encoder_layer_workspace(cfg, S, T). */
+VX_API vx_status vx_stream_prefill(const vx_layer_cfg *cfg, const vx_layer_weights *layers,
+                            const vx_kv_ring *ring, const float *x, float *y, int T,
+                            const void *final_g, void *ws, size_t ws_bytes,
+                            cudaStream_t stream);
+
+/* Streaming step: n_new (1..8) new frames per stream, for every stream of the
+ * ring, through the ring's n_layers layers.  Per layer, new frame f = pos[s]+t
+ * attends frames f' with f - W < f' <= f: older frames from the ring, the rest
+ * from this step; every in-window ring slot is read before the new K/V are
+ * written to slots (pos[s] + t) mod W.  Advances pos[s] += n_new at the end.
+ * x_new, y: [S, n_new, d] fp32 (final RMSNorm applied when final_g != NULL).
+ * The call enqueues only kernels (no host sync), so it can be captured in a
+ * CUDA graph and replayed.  Workspace: vx_stream_step_workspace(). */
+VX_API vx_status vx_stream_step(const vx_layer_cfg *cfg, const vx_layer_weights *layers,
+                         const vx_kv_ring *ring, const float *x_new, float *y, int n_new,
+                         const void *final_g, void *ws, size_t ws_bytes, cudaStream_t stream);
+VX_API size_t vx_stream_step_workspace(const vx_layer_cfg *cfg, int S, int n_new);
+
+/* Test hook for the bounded-wait machinery: launches one CTA that waits on an
+ * mbarrier nothing arrives on, with a limit of timeout_ns, then records
+ * VX_ERR_DEVICE_TIMEOUT in ws and returns.  Nothing faults or hangs. */
+VX_API vx_status vx_selftest_wait_timeout(void *ws, size_t ws_bytes, uint64_t timeout_ns,
+                                   cudaStream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* VX_H_ */

@@ -52,7 +52,7 @@ def as64(a):
 # ---------------------------------------------------------------- elementwise
 
 def rms_norm(x, g, eps=1e-5):
-    """RMSNorm pre-norm ("RMSNorm pre-norm", Voxtral Realtime 2602 architecture):
+    """RMSNorm (the pre-norm of each 2602 encoder sub-block):
     y = x / sqrt(mean(x^2 over the model dimension) + eps) * g."""
     x = as64(x)
     ms = np.mean(x * x, axis=-1, keepdims=True)
@@ -99,7 +99,7 @@ def swa_attention_rows(q, k, v, window, rows, scale=None):
     """Causal sliding-window attention for selected query rows.
 
     o_i = sum_{j : i - W < j <= i} softmax_j(<q_i, k_j> * scale) v_j, per head
-    ("causal + sliding-window (750)" attention of the 2602 encoder).
+    (the 2602 encoder's causal attention restricted to a window of W frames).
     q, k, v: [B, T, H, D] (RoPE already applied).  Returns [B, len(rows), H, D].
     """
     q, k, v = as64(q), as64(k), as64(v)
@@ -269,13 +269,13 @@ def conv_stem(mel, w1, b1, w2, b2):
     xp = np.concatenate([np.zeros((B, C, 2)), x], axis=2)            # [B, C, Tm+2]
     h1 = np.zeros((B, w1.shape[0], Tm)) + b1[None, :, None]
     for k in range(3):
-        h1 += np.einsum("oc,bct->bot", w1[:, :, k], xp[:, :, k:k + Tm])
+        h1 += np.einsum("oc,bct->bot", w1[:, :, k], xp[:, :, k:k + Tm], optimize=True)
     h1 = gelu(h1)
     To = conv_out_len(Tm)
     hp = np.concatenate([np.zeros((B, h1.shape[1], 2)), h1], axis=2)  # [B, d, Tm+2]
     h2 = np.zeros((B, w2.shape[0], To)) + b2[None, :, None]
     for k in range(3):
-        h2 += np.einsum("oc,bct->bot", w2[:, :, k], hp[:, :, k:k + 2 * To - 1:2])
+        h2 += np.einsum("oc,bct->bot", w2[:, :, k], hp[:, :, k:k + 2 * To - 1:2], optimize=True)
     return np.transpose(gelu(h2), (0, 2, 1))
 
 

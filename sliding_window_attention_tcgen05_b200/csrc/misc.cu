@@ -1,0 +1,219 @@
+// misc.cu -- bandwidth-bound helpers: RMSNorm (+ residual), weight packing,
+// conv-stem input staging, and the bounded-wait self test.
+#include "vx_internal.h"
+
+namespace vx {
+
+namespace {
+
+// ---------------------------------------------------------------- RMSNorm --
+// One warp per row of d (multiple of 128, <= 2048) fp32 values; lane i holds
+// float4 columns i, i+32, ...; h = x (+ r); y = h * rsqrt(mean(h^2) + eps) * g.
+template <bool BF16_OUT>
+__global__ void __launch_bounds__(256)
+rmsnorm_kernel(const float* __restrict__ x, const float* __restrict__ r, const uint16_t* __restrict__ g,
+               float* __restrict__ h_out, void* __restrict__ y, int M, int d, float eps) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int row = blockIdx.x * 8 + warp;
+  if (row >= M) return;
+  const int nv = d >> 7;
+  const float4* xr = reinterpret_cast<const float4*>(x + static_cast<int64_t>(row) * d);
+  const float4* rr = r ? reinterpret_cast<const float4*>(r + static_cast<int64_t>(row) * d) : nullptr;
+  float4 v[16];
+  float ss = 0.f;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    if (i < nv) {
+      float4 a = xr[lane + 32 * i];
+      if (rr) {
+        const float4 b = rr[lane + 32 * i];
+        a.x += b.x; a.y += b.y; a.z += b.z; a.w += b.w;
+      }
+      v[i] = a;
+      ss = fmaf(a.x, a.x, fmaf(a.y, a.y, fmaf(a.z, a.z, fmaf(a.w, a.w, ss))));
+    }
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+  const float inv = rsqrtf(ss / static_cast<float>(d) + eps);
+  if (h_out) {
+    float4* hr = reinterpret_cast<float4*>(h_out + static_cast<int64_t>(row) * d);
+#pragma unroll
+    for (int i = 0; i < 16; ++i)
+      if (i < nv) hr[lane + 32 * i] = v[i];
+  }
+  const uint2* gr = reinterpret_cast<const uint2*>(g);
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    if (i < nv) {
+      const int c4 = lane + 32 * i;
+      const uint2 gw = __ldg(gr + c4);
+      const float o0 = v[i].x * inv * bf16lo(gw.x), o1 = v[i].y * inv * bf16hi(gw.x);
+      const float o2 = v[i].z * inv * bf16lo(gw.y), o3 = v[i].w * inv * bf16hi(gw.y);
+      if constexpr (BF16_OUT) {
+        uint2 w;
+        w.x = pack_bf16x2(o0, o1);
+        w.y = pack_bf16x2(o2, o3);
+        reinterpret_cast<uint2*>(static_cast<uint16_t*>(y) + static_cast<int64_t>(row) * d)[c4] = w;
+      } else {
+        reinterpret_cast<float4*>(static_cast<float*>(y) + static_cast<int64_t>(row) * d)[c4] =
+            make_float4(o0, o1, o2, o3);
+      }
+    }
+  }
+}
+
+// ---------------------------------------------------------------- packing --
+// Row gather: output row rr (of `cols` bf16) comes from src_of(rr) or is zero.
+struct PackSrc {
+  const uint16_t* a;   // first source (q rows / gate rows)
+  const uint16_t* b;   // second source (k rows / up rows)
+  const uint16_t* c;   // third source (v rows)
+  int mode;            // 0: concat a|b|c in blocks of `blk` rows; 1: interleave a,b in blocks of `blk`
+  int blk;
+};
+
+__device__ __forceinline__ const uint16_t* pack_src_row(const PackSrc& p, int64_t rr, int64_t cols) {
+  if (p.mode == 0) {
+    const int64_t part = rr / p.blk, r = rr % p.blk;
+    const uint16_t* s = part == 0 ? p.a : (part == 1 ? p.b : p.c);
+    return s ? s + r * cols : nullptr;
+  }
+  const int64_t blk2 = 2 * p.blk;
+  const int64_t g = rr / blk2, w = rr % blk2;
+  const uint16_t* s = w < p.blk ? p.a : p.b;
+  return s ? s + (g * p.blk + (w % p.blk)) * cols : nullptr;
+}
+
+// cols must be a multiple of 8 when > 1 (vector path) ; cols == 1 packs vectors.
+__global__ void pack_rows_kernel(PackSrc p, uint16_t* __restrict__ out, int64_t rows, int64_t cols) {
+  const int64_t chunks = cols >= 8 ? cols / 8 : 1;
+  const int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (cols >= 8) {
+    if (idx >= rows * chunks) return;
+    const int64_t rr = idx / chunks, ch = idx % chunks;
+    const uint16_t* s = pack_src_row(p, rr, cols);
+    uint4 v = make_uint4(0, 0, 0, 0);
+    if (s) v = *reinterpret_cast<const uint4*>(s + ch * 8);
+    *reinterpret_cast<uint4*>(out + rr * cols + ch * 8) = v;
+  } else {
+    if (idx >= rows) return;
+    const uint16_t* s = pack_src_row(p, idx, 1);
+    out[idx] = s ? *s : static_cast<uint16_t>(0);
+  }
+}
+
+// Conv1d weight [O, C, 3] -> [O, 3, C].
+__global__ void pack_conv_kernel(const uint16_t* __restrict__ w, uint16_t* __restrict__ wp, int O, int C) {
+  const int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const int64_t total = static_cast<int64_t>(O) * C * 3;
+  if (idx >= total) return;
+  const int64_t c = idx % C;
+  const int64_t k = (idx / C) % 3;
+  const int64_t o = idx / (3 * static_cast<int64_t>(C));
+  wp[idx] = w[(o * C + c) * 3 + k];
+}
+
+// --------------------------------------------------------------- conv prep --
+// mel [B, C, Tm] fp32 -> xpad [B, P, C] bf16, xpad[b, tp, c] = mel[b, c, tp - 2]
+// for 2 <= tp < Tm + 2, else 0.  32 x 32 tiles through shared memory.
+__global__ void conv_prep_kernel(const float* __restrict__ mel, uint16_t* __restrict__ xpad,
+                                 int C, int Tm, int P) {
+  __shared__ float tile[32][33];
+  const int tp0 = blockIdx.x * 32, c0 = blockIdx.y * 32, b = blockIdx.z;
+  const int tx = threadIdx.x, ty = threadIdx.y;   // 32 x 8
+  for (int k = ty; k < 32; k += 8) {
+    const int c = c0 + k, tp = tp0 + tx;
+    float v = 0.f;
+    if (c < C && tp >= 2 && tp < Tm + 2) v = mel[(static_cast<int64_t>(b) * C + c) * Tm + (tp - 2)];
+    tile[k][tx] = v;
+  }
+  __syncthreads();
+  for (int k = ty; k < 32; k += 8) {
+    const int tp = tp0 + k, c = c0 + tx;
+    if (tp < P && c < C) {
+      const __nv_bfloat16 h = __float2bfloat16_rn(tile[tx][k]);
+      xpad[(static_cast<int64_t>(b) * P + tp) * C + c] = *reinterpret_cast<const uint16_t*>(&h);
+    }
+  }
+}
+
+// Zeroes rows {0, 1} and [Tm + 2, P) of every clip of h1pad [B, P, d].
+__global__ void conv_pad_zero_kernel(uint16_t* __restrict__ h1pad, int Tm, int P, int d) {
+  const int b = blockIdx.y;
+  const int which = blockIdx.x;     // 0, 1, or 2 + (row - Tm - 2)
+  const int row = which < 2 ? which : Tm + which;
+  if (row >= P) return;
+  uint16_t* r = h1pad + (static_cast<int64_t>(b) * P + row) * d;
+  for (int c = threadIdx.x * 8; c < d; c += blockDim.x * 8)
+    *reinterpret_cast<uint4*>(r + c) = make_uint4(0, 0, 0, 0);
+}
+
+// --------------------------------------------------------------- selftest --
+__global__ void selftest_wait_kernel(DevStatus* st, uint64_t limit_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(smem_addr(&bar), 1);
+    abort_flag = 0;
+    fence_barrier_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    const WaitCtx wc{st, &abort_flag, limit_ns};
+    mbar_wait(smem_addr(&bar), 0, wc, 99);   // nothing ever arrives
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_rmsnorm(const Launch& L, const float* x, const float* r, const uint16_t* g, float* h_out,
+                           void* y, bool y_bf16, int M, int d, float eps) {
+  if (M <= 0) return cudaSuccess;
+  const int blocks = (M + 7) / 8;
+  if (y_bf16)
+    rmsnorm_kernel<true><<<blocks, 256, 0, L.stream>>>(x, r, g, h_out, y, M, d, eps);
+  else
+    rmsnorm_kernel<false><<<blocks, 256, 0, L.stream>>>(x, r, g, h_out, y, M, d, eps);
+  return cudaGetLastError();
+}
+
+static cudaError_t pack_rows(const Launch& L, PackSrc p, uint16_t* out, int64_t rows, int64_t cols) {
+  const int64_t work = cols >= 8 ? rows * (cols / 8) : rows;
+  const int threads = 256;
+  pack_rows_kernel<<<static_cast<unsigned>((work + threads - 1) / threads), threads, 0, L.stream>>>(p, out, rows, cols);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_pack_layer(const Launch& L, int d, int HD, int F, const uint16_t* wq, const uint16_t* wk,
+                              const uint16_t* wv, const uint16_t* bq, const uint16_t* bv, const uint16_t* wg,
+                              const uint16_t* wu, const uint16_t* bg, const uint16_t* bu, uint16_t* wqkv,
+                              uint16_t* bqkv, uint16_t* wgu, uint16_t* bgu) {
+  cudaError_t e;
+  if ((e = pack_rows(L, PackSrc{wq, wk, wv, 0, HD}, wqkv, 3LL * HD, d)) != cudaSuccess) return e;
+  if ((e = pack_rows(L, PackSrc{bq, nullptr, bv, 0, HD}, bqkv, 3LL * HD, 1)) != cudaSuccess) return e;
+  if ((e = pack_rows(L, PackSrc{wg, wu, nullptr, 1, 64}, wgu, 2LL * F, d)) != cudaSuccess) return e;
+  return pack_rows(L, PackSrc{bg, bu, nullptr, 1, 64}, bgu, 2LL * F, 1);
+}
+
+cudaError_t launch_pack_conv(const Launch& L, const uint16_t* w, uint16_t* wp, int O, int C) {
+  const int64_t total = static_cast<int64_t>(O) * C * 3;
+  pack_conv_kernel<<<static_cast<unsigned>((total + 255) / 256), 256, 0, L.stream>>>(w, wp, O, C);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_conv_prep(const Launch& L, const float* mel, uint16_t* xpad, uint16_t* h1pad, int B, int C,
+                             int Tm, int P, int d) {
+  conv_prep_kernel<<<dim3((P + 31) / 32, (C + 31) / 32, B), dim3(32, 8), 0, L.stream>>>(mel, xpad, C, Tm, P);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  conv_pad_zero_kernel<<<dim3(2 + (P - Tm - 2), B), 128, 0, L.stream>>>(h1pad, Tm, P, d);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_selftest_wait(const Launch& L) {
+  selftest_wait_kernel<<<1, 32, 0, L.stream>>>(L.status, L.limit_ns);
+  return cudaGetLastError();
+}
+
+}  // namespace vx

@@ -1,0 +1,128 @@
+// vx_internal.h -- host-side launchers shared between the libvx translation
+// units.  Not part of the public ABI (include/vx.h is).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+#include <string>
+
+#include "vx_common.cuh"
+
+namespace vx {
+
+// Error reporting (thread-local message, see vx_last_error()).
+void set_error(const char* fmt, ...);
+const char* last_error();
+
+// Launch context of one public call.
+struct Launch {
+  cudaStream_t stream;
+  DevStatus* status;   // status word inside the caller's workspace
+  uint64_t limit_ns;   // bounded-wait limit
+  int sm_count;        // SMs of the current device
+};
+
+int current_sm_count();
+uint64_t wait_limit_ns();
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no -lcuda).
+bool encode_tmap(CUtensorMap* map, CUtensorMapDataType dt, int rank, const void* base,
+                 const uint64_t* dims, const uint64_t* strides_bytes, const uint32_t* box,
+                 CUtensorMapSwizzle swizzle);
+
+// 2-D bf16 K-major operand view with a 64-element (128-byte) inner box and a
+// 128-byte swizzle: `rows` rows of `cols` elements, `row_stride` elements apart.
+bool tmap_bf16_2d(CUtensorMap* map, const void* base, uint64_t cols, uint64_t rows,
+                  uint64_t row_stride, uint32_t box_rows);
+
+// ------------------------------------------------------------------ GEMM --
+enum EpiKind : int {
+  EPI_F32 = 0,        // out fp32 = acc + bias + residual
+  EPI_QKV_ROPE = 1,   // out bf16 = RoPE(acc + bias) on the first rope_cols columns
+  EPI_SWIGLU = 2,     // out bf16 [.., N/2] = silu(gate + bg) * (up + bu), 64-blocks interleaved
+  EPI_GELU_BF16 = 3,  // out bf16 = GELU(acc + bias)
+  EPI_GELU_F32 = 4,   // out fp32 = GELU(acc + bias)
+};
+
+struct GemmArgs {
+  int M, N, K;
+  // A addressing of K-block kb (64 wide): tap = kb / kb_per_tap,
+  // c = (kb % kb_per_tap) * 64, x = (tap % a_stride) * a_tap_ch + c, y = m0 + tap / a_stride.
+  int kb_per_tap, a_stride, a_tap_ch;
+  void* out;
+  int64_t ld_out;          // elements
+  const uint16_t* bias;    // [N] bf16 or null
+  const float* res;        // [.., ld_res] fp32 or null (EPI_F32 only)
+  int64_t ld_res;
+  // Row mapping: source row m -> (b, t) = (m / in_rows, m % in_rows); rows with
+  // t >= t_valid (or m >= M) are not stored; destination row b * out_rows + out_off + t.
+  int in_rows, t_valid, out_rows, out_off;
+  // RoPE (EPI_QKV_ROPE): position of (b, t) = (pos_arr ? pos_arr[b] : pos0) + t.
+  const int64_t* pos_arr;
+  int64_t pos0;
+  int rope_cols;           // columns [0, rope_cols) are rotated in 64-wide heads
+  float inv_freq_hi[32];   // inv_freq_m as float, and its residual to the exact value
+  float inv_freq_lo[32];
+  DevStatus* status;
+  uint64_t limit_ns;
+};
+
+// D[M, N] = A[M, K] * B[N, K]^T with the given epilogue.  tmA/tmB must be 2-D
+// bf16 maps with 128-byte swizzle and box {64, 128} (A) / {64, bn} (B).
+// bn in {128, 256}; N % bn == 0; K % 64 == 0.
+cudaError_t launch_gemm(const Launch& L, const CUtensorMap& tmA, const CUtensorMap& tmB,
+                        const GemmArgs& args, int epi, int bn);
+
+void fill_rope_freqs(GemmArgs* a, float theta, int head_dim);
+
+// ------------------------------------------------------------- attention --
+struct AttnArgs {
+  void* out;                   // bf16 [B, T, H, 64] with the strides below
+  int64_t o_row, o_head, o_batch;  // element strides of t, h, b in out
+  int B, T, H, window;
+  float scale_log2;            // softmax scale * log2(e)
+  DevStatus* status;
+  uint64_t limit_ns;
+};
+// tmQ/tmK/tmV: 4-D bf16 maps {64 (d), H, T, B} with box {64, 1, 128, 1}.
+cudaError_t launch_attn_bf16(const Launch& L, const CUtensorMap& tmQ, const CUtensorMap& tmK,
+                             const CUtensorMap& tmV, const AttnArgs& a);
+bool tmap_attn_operand(CUtensorMap* map, const void* base, int B, int T, int H,
+                       int64_t row_stride, int64_t batch_stride);
+
+// fp32 CUDA-core sliding-window attention on pre-rotated q, k: [B, T, H, 64].
+cudaError_t launch_attn_f32(const Launch& L, const float* q, const float* k, const float* v,
+                            float* o, int B, int T, int H, int window, float scale);
+
+// RoPE of x ([B, T, H, 64], fp32 or bf16) into y (same layout and dtype).
+cudaError_t launch_rope(const Launch& L, const void* x, void* y, bool bf16, int B, int T, int H,
+                        int64_t pos0, float theta);
+
+// ---------------------------------------------------------------- others --
+cudaError_t launch_rmsnorm(const Launch& L, const float* x, const float* r, const uint16_t* g,
+                           float* h_out, void* y, bool y_bf16, int M, int d, float eps);
+
+// Ring attention of one layer of a streaming step (see vx_stream_step).
+cudaError_t launch_ring_attn(const Launch& L, const uint16_t* qkv, int64_t ld_qkv, int HD,
+                             uint16_t* ring_k, uint16_t* ring_v, const int64_t* pos, int S,
+                             int H, int W, int n_new, uint16_t* out, float scale_log2);
+// Writes the K/V of frames max(0,T-W)..T-1 of qkv ([S*T, ld]) into one layer's ring.
+cudaError_t launch_ring_fill(const Launch& L, const uint16_t* qkv, int64_t ld_qkv, int HD,
+                             uint16_t* ring_k, uint16_t* ring_v, int S, int T, int H, int W);
+cudaError_t launch_pos_add(const Launch& L, int64_t* pos, int S, int64_t n, bool set);
+
+cudaError_t launch_pack_layer(const Launch& L, int d, int HD, int F, const uint16_t* wq,
+                              const uint16_t* wk, const uint16_t* wv, const uint16_t* bq,
+                              const uint16_t* bv, const uint16_t* wg, const uint16_t* wu,
+                              const uint16_t* bg, const uint16_t* bu, uint16_t* wqkv,
+                              uint16_t* bqkv, uint16_t* wgu, uint16_t* bgu);
+cudaError_t launch_pack_conv(const Launch& L, const uint16_t* w, uint16_t* wp, int O, int C);
+// mel [B, C, Tm] fp32 -> xpad [B, P, C] bf16 (rows 0,1 and >= Tm+2 zero); also
+// zeroes rows 0, 1 and Tm+2 .. P-1 of h1pad [B, P, d].
+cudaError_t launch_conv_prep(const Launch& L, const float* mel, uint16_t* xpad, uint16_t* h1pad,
+                             int B, int C, int Tm, int P, int d);
+
+cudaError_t launch_selftest_wait(const Launch& L);
+
+}  // namespace vx
