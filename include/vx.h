@@ -120,6 +120,16 @@ VX_API const char *vx_version(void);
 /* Bounded-wait limit for every in-kernel wait (default 1e9 ns).  Host setting,
  * read at launch time; affects launches enqueued afterwards (all threads). */
 VX_API void vx_set_wait_timeout_ns(uint64_t ns);
+/* Per-launch timing: while enabled (per calling thread), every kernel this
+ * library enqueues is bracketed by CUDA events recorded on its launch stream.
+ * vx_trace_read() synchronises those events, writes one "name milliseconds"
+ * line per launch (in launch order) into buf (host, NUL-terminated, truncated
+ * to cap), forgets them and returns how many there were.  Do not enable it
+ * while capturing a CUDA graph. */
+VX_API void vx_trace_enable(int on);
+VX_API int vx_trace_read(char *buf, size_t cap);
+/* Number of kernels this library has enqueued since it was loaded (all threads). */
+VX_API uint64_t vx_launch_count(void);
 /* Clears the status word at the start of ws (async on stream). */
 VX_API vx_status vx_status_reset(void *ws, cudaStream_t stream);
 /* Synchronises `stream`, then returns VX_ERR_DEVICE_TIMEOUT if a kernel

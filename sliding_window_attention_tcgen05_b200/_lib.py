@@ -45,6 +45,9 @@ SIGNATURES = {
     "vx_last_error": (C.c_char_p, []),
     "vx_version": (C.c_char_p, []),
     "vx_set_wait_timeout_ns": (None, [_U64]),
+    "vx_trace_enable": (None, [_I]),
+    "vx_trace_read": (_I, [C.c_char_p, _S]),
+    "vx_launch_count": (_U64, []),
     "vx_status_reset": (_I, [_P, _P]),
     "vx_status_check": (_I, [_P, _P]),
     "vx_pack_layer": (_I, [_CFG, C.POINTER(VxLayerParams), _P, _P, _P, _P, _P]),
@@ -69,7 +72,7 @@ def load(path: str = LIB_PATH) -> C.CDLL:
     if not os.path.exists(path):
         raise ImportError(
             f"libvx.so not found at {path}; build it with "
-            "`python -m sliding_window_attention_tcgen05_b200.build` (nvcc, sm_100a)")
+            "`python sliding_window_attention_tcgen05_b200/build.py` (nvcc, sm_100a)")
     lib = C.CDLL(path)
     for name, (res, args) in SIGNATURES.items():
         fn = getattr(lib, name)

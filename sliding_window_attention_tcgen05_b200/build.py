@@ -1,7 +1,9 @@
 """Builds libvx.so in-tree with nvcc for sm_100a.
 
-    python -m sliding_window_attention_tcgen05_b200.build        # incremental
-    python -m sliding_window_attention_tcgen05_b200.build --force
+    python sliding_window_attention_tcgen05_b200/build.py          # incremental
+    python sliding_window_attention_tcgen05_b200/build.py --force
+
+(Run it as a script: importing the package itself needs the built library.)
 
 Each csrc/*.cu is compiled to _build/<name>.o (rebuilt when it or any header
 is newer than its object) and the objects are linked into

@@ -17,6 +17,8 @@
 #include <cmath>
 #include <atomic>
 #include <mutex>
+#include <string>
+#include <vector>
 
 #include <cudaTypedefs.h>
 
@@ -38,6 +40,40 @@ const char* last_error() { return g_err; }
 
 static std::atomic<uint64_t> g_wait_limit_ns{1000000000ull};
 uint64_t wait_limit_ns() { return g_wait_limit_ns.load(); }
+
+// ------------------------------------------------------------- tracing --
+// Kernel launches go through traced(): it counts them and, when tracing is on
+// for the calling thread, brackets them with CUDA events on the launch stream.
+static std::atomic<uint64_t> g_launches{0};
+struct TraceRec {
+  const char* name;
+  cudaEvent_t a, b;
+};
+static thread_local bool t_trace = false;
+static thread_local std::vector<TraceRec> t_recs;
+static thread_local std::vector<cudaEvent_t> t_pool;
+static thread_local size_t t_pool_used = 0;
+
+static cudaEvent_t trace_event() {
+  if (t_pool_used == t_pool.size()) {
+    cudaEvent_t e;
+    if (cudaEventCreate(&e) != cudaSuccess) return nullptr;
+    t_pool.push_back(e);
+  }
+  return t_pool[t_pool_used++];
+}
+
+template <class F>
+cudaError_t traced(const Launch& L, const char* name, int kernels, F&& f) {
+  g_launches.fetch_add(static_cast<uint64_t>(kernels));
+  if (!t_trace) return f();
+  cudaEvent_t a = trace_event(), b = trace_event();
+  if (a) cudaEventRecord(a, L.stream);
+  const cudaError_t e = f();
+  if (b) cudaEventRecord(b, L.stream);
+  if (a && b) t_recs.push_back({name, a, b});
+  return e;
+}
 
 int current_sm_count() {
   static int cache[64] = {0};
@@ -219,12 +255,12 @@ GemmArgs base_args(const Launch& L, int M, int N, int K) {
   return a;
 }
 
-vx_status gemm(const Launch& L, const void* A, int64_t lda, const void* Bw, GemmArgs& a, int epi) {
+vx_status gemm(const Launch& L, const char* name, const void* A, int64_t lda, const void* Bw, GemmArgs& a, int epi) {
   const int bn = pick_bn(a.M, a.N, L.sm_count);
   CUtensorMap tmA, tmB;
   if (!tmap_bf16_2d(&tmA, A, a.K, a.M, lda, 128)) return VX_ERR_CUDA;
   if (!tmap_bf16_2d(&tmB, Bw, a.K, a.N, a.K, bn)) return VX_ERR_CUDA;
-  VX_CUDA(launch_gemm(L, tmA, tmB, a, epi, bn));
+  VX_CUDA(traced(L, name, 1, [&] { return launch_gemm(L, tmA, tmB, a, epi, bn); }));
   return VX_OK;
 }
 
@@ -245,7 +281,7 @@ vx_status run_layer(const Launch& L, const vx_layer_cfg& c, const vx_layer_weigh
   const float sl2 = (1.0f / std::sqrt(static_cast<float>(c.head_dim))) * 1.4426950408889634f;
   vx_status st;
   // 1. RMSNorm
-  VX_CUDA(launch_rmsnorm(L, x, nullptr, static_cast<const uint16_t*>(w.attn_norm_g), nullptr, bf.y0, true, M, d, c.eps));
+  VX_CUDA(traced(L, "rmsnorm", 1, [&] { return launch_rmsnorm(L, x, nullptr, static_cast<const uint16_t*>(w.attn_norm_g), nullptr, bf.y0, true, M, d, c.eps); }));
   // 2. QKV + bias + RoPE
   {
     GemmArgs a = base_args(L, M, 3 * HD, d);
@@ -256,11 +292,11 @@ vx_status run_layer(const Launch& L, const vx_layer_cfg& c, const vx_layer_weigh
     a.pos0 = pos0;
     a.rope_cols = 2 * HD;
     fill_rope_freqs(&a, c.rope_theta, c.head_dim);
-    if ((st = gemm(L, bf.y0, d, w.wqkv, a, EPI_QKV_ROPE)) != VX_OK) return st;
+    if ((st = gemm(L, "gemm_qkv_rope", bf.y0, d, w.wqkv, a, EPI_QKV_ROPE)) != VX_OK) return st;
   }
   // 3. attention
   if (ring && ring->step) {
-    VX_CUDA(launch_ring_attn(L, bf.qkv, 3LL * HD, HD, ring->k, ring->v, ring->pos, nseq, H, ring->W, rows, bf.att, sl2));
+    VX_CUDA(traced(L, "ring_attn", 1, [&] { return launch_ring_attn(L, bf.qkv, 3LL * HD, HD, ring->k, ring->v, ring->pos, nseq, H, ring->W, rows, bf.att, sl2); }));
   } else {
     CUtensorMap tq, tk, tv;
     const int64_t rs = 3LL * HD, bs = static_cast<int64_t>(rows) * 3 * HD;
@@ -271,9 +307,9 @@ vx_status run_layer(const Launch& L, const vx_layer_cfg& c, const vx_layer_weigh
     aa.out = bf.att; aa.o_row = HD; aa.o_head = 64; aa.o_batch = static_cast<int64_t>(rows) * HD;
     aa.B = nseq; aa.T = rows; aa.H = H; aa.window = c.window; aa.scale_log2 = sl2;
     aa.status = L.status; aa.limit_ns = L.limit_ns;
-    VX_CUDA(launch_attn_bf16(L, tq, tk, tv, aa));
+    VX_CUDA(traced(L, "swa_attn_tc", 1, [&] { return launch_attn_bf16(L, tq, tk, tv, aa); }));
     if (ring && ring->fill)
-      VX_CUDA(launch_ring_fill(L, bf.qkv, 3LL * HD, HD, ring->k, ring->v, nseq, rows, H, ring->W));
+      VX_CUDA(traced(L, "ring_fill", 1, [&] { return launch_ring_fill(L, bf.qkv, 3LL * HD, HD, ring->k, ring->v, nseq, rows, H, ring->W); }));
   }
   // 4. O-projection + bias + residual
   {
@@ -281,16 +317,16 @@ vx_status run_layer(const Launch& L, const vx_layer_cfg& c, const vx_layer_weigh
     a.out = bf.h; a.ld_out = d;
     a.bias = static_cast<const uint16_t*>(w.bo);
     a.res = x; a.ld_res = d;
-    if ((st = gemm(L, bf.att, HD, w.wo, a, EPI_F32)) != VX_OK) return st;
+    if ((st = gemm(L, "gemm_o_residual", bf.att, HD, w.wo, a, EPI_F32)) != VX_OK) return st;
   }
   // 5. RMSNorm
-  VX_CUDA(launch_rmsnorm(L, bf.h, nullptr, static_cast<const uint16_t*>(w.ffn_norm_g), nullptr, bf.y0, true, M, d, c.eps));
+  VX_CUDA(traced(L, "rmsnorm", 1, [&] { return launch_rmsnorm(L, bf.h, nullptr, static_cast<const uint16_t*>(w.ffn_norm_g), nullptr, bf.y0, true, M, d, c.eps); }));
   // 6. gate/up + SwiGLU
   {
     GemmArgs a = base_args(L, M, 2 * F, d);
     a.out = bf.act; a.ld_out = F;
     a.bias = static_cast<const uint16_t*>(w.bgu);
-    if ((st = gemm(L, bf.y0, d, w.wgu, a, EPI_SWIGLU)) != VX_OK) return st;
+    if ((st = gemm(L, "gemm_gate_up_swiglu", bf.y0, d, w.wgu, a, EPI_SWIGLU)) != VX_OK) return st;
   }
   // 7. down + bias + residual
   {
@@ -298,7 +334,7 @@ vx_status run_layer(const Launch& L, const vx_layer_cfg& c, const vx_layer_weigh
     a.out = y; a.ld_out = d;
     a.bias = static_cast<const uint16_t*>(w.bd);
     a.res = bf.h; a.ld_res = d;
-    if ((st = gemm(L, bf.act, F, w.wd, a, EPI_F32)) != VX_OK) return st;
+    if ((st = gemm(L, "gemm_down_residual", bf.act, F, w.wd, a, EPI_F32)) != VX_OK) return st;
   }
   return VX_OK;
 }
@@ -323,7 +359,7 @@ vx_status run_conv_stem(const Launch& L, const float* mel, const void* w1p, cons
                         const void* b2, float* out, int B, int C, int Tm, int d, const ConvBufs& cb) {
   const int P = conv_rows_per_clip(Tm);
   const int To = (Tm - 1) / 2 + 1;
-  VX_CUDA(launch_conv_prep(L, mel, cb.xpad, cb.h1pad, B, C, Tm, P, d));
+  VX_CUDA(traced(L, "conv_prep", 2, [&] { return launch_conv_prep(L, mel, cb.xpad, cb.h1pad, B, C, Tm, P, d); }));
   vx_status st;
   // conv1: rows r = b*P + t of xpad; taps read rows r, r+1, r+2 -> h1pad row b*P + 2 + t.
   {
@@ -336,7 +372,7 @@ vx_status run_conv_stem(const Launch& L, const float* mel, const void* w1p, cons
     CUtensorMap tmA, tmB;
     if (!tmap_bf16_2d(&tmA, cb.xpad, C, int64_t(B) * P, C, 128)) return VX_ERR_CUDA;
     if (!tmap_bf16_2d(&tmB, w1p, 3 * C, d, 3 * C, bn)) return VX_ERR_CUDA;
-    VX_CUDA(launch_gemm(L, tmA, tmB, a, EPI_GELU_BF16, bn));
+    VX_CUDA(traced(L, "gemm_conv1_gelu", 1, [&] { return launch_gemm(L, tmA, tmB, a, EPI_GELU_BF16, bn); }));
   }
   // conv2 (stride 2): h1pad viewed as [B*P/2, 2d]; output t of clip b reads
   // padded rows 2t, 2t+1, 2t+2 = (pair t, half 0), (pair t, half 1), (pair t+1, half 0).
@@ -351,7 +387,7 @@ vx_status run_conv_stem(const Launch& L, const float* mel, const void* w1p, cons
     CUtensorMap tmA, tmB;
     if (!tmap_bf16_2d(&tmA, cb.h1pad, 2LL * d, int64_t(B) * pairs, 2LL * d, 128)) return VX_ERR_CUDA;
     if (!tmap_bf16_2d(&tmB, w2p, 3 * d, d, 3 * d, bn)) return VX_ERR_CUDA;
-    VX_CUDA(launch_gemm(L, tmA, tmB, a, EPI_GELU_F32, bn));
+    VX_CUDA(traced(L, "gemm_conv2_gelu", 1, [&] { return launch_gemm(L, tmA, tmB, a, EPI_GELU_F32, bn); }));
   }
   (void)st;
   return VX_OK;
@@ -375,6 +411,31 @@ extern "C" {
 const char* vx_last_error(void) { return vx::last_error(); }
 const char* vx_version(void) { return "vx 0.1 (sm_100a)"; }
 void vx_set_wait_timeout_ns(uint64_t ns) { g_wait_limit_ns.store(ns > 0 ? ns : 1); }
+
+void vx_trace_enable(int on) { t_trace = on != 0; }
+
+int vx_trace_read(char* buf, size_t cap) {
+  std::string out;
+  int n = 0;
+  for (const TraceRec& r : t_recs) {
+    float ms = -1.f;
+    if (cudaEventSynchronize(r.b) == cudaSuccess) cudaEventElapsedTime(&ms, r.a, r.b);
+    char line[160];
+    snprintf(line, sizeof(line), "%s %.6f\n", r.name, ms);
+    out += line;
+    ++n;
+  }
+  t_recs.clear();
+  t_pool_used = 0;
+  if (buf && cap > 0) {
+    const size_t m = out.size() < cap - 1 ? out.size() : cap - 1;
+    std::memcpy(buf, out.data(), m);
+    buf[m] = '\0';
+  }
+  return n;
+}
+
+uint64_t vx_launch_count(void) { return g_launches.load(); }
 
 vx_status vx_status_reset(void* ws, cudaStream_t stream) {
   VX_CHECK_ARG(ws != nullptr, "workspace is null");
@@ -404,6 +465,7 @@ vx_status vx_pack_layer(const vx_layer_cfg* cfg, const vx_layer_params* in, void
   for (const void* p : al) VX_CHECK_ARG(aligned16(p), "weight buffers must be 16-byte aligned");
   Launch L{stream, nullptr, wait_limit_ns(), 1};
   const int HD = cfg->n_heads * cfg->head_dim;
+  g_launches.fetch_add(4);
   VX_CUDA(launch_pack_layer(L, cfg->d_model, HD, cfg->ffn_hidden, static_cast<const uint16_t*>(in->wq),
                             static_cast<const uint16_t*>(in->wk), static_cast<const uint16_t*>(in->wv),
                             static_cast<const uint16_t*>(in->bq), static_cast<const uint16_t*>(in->bv),
@@ -417,6 +479,7 @@ vx_status vx_pack_layer(const vx_layer_cfg* cfg, const vx_layer_params* in, void
 vx_status vx_pack_conv_weight(const void* w, void* w_packed, int out_ch, int in_ch, cudaStream_t stream) {
   VX_CHECK_ARG(w && w_packed && out_ch > 0 && in_ch > 0, "bad conv weight arguments");
   Launch L{stream, nullptr, wait_limit_ns(), 1};
+  g_launches.fetch_add(1);
   VX_CUDA(launch_pack_conv(L, static_cast<const uint16_t*>(w), static_cast<uint16_t*>(w_packed), out_ch, in_ch));
   return VX_OK;
 }
@@ -456,14 +519,16 @@ vx_status vx_swa_attn_fwd(const void* q, const void* k, const void* v, void* o, 
     const size_t es = dt == VX_F32 ? 4 : 2;
     void* qr = cv.take(size_t(B) * T * H * D * es);
     void* kr = cv.take(size_t(B) * T * H * D * es);
-    VX_CUDA(launch_rope(L, q, qr, dt == VX_BF16, B, T, H, pos0, rope_theta));
-    VX_CUDA(launch_rope(L, k, kr, dt == VX_BF16, B, T, H, pos0, rope_theta));
+    VX_CUDA(traced(L, "rope", 1, [&] { return launch_rope(L, q, qr, dt == VX_BF16, B, T, H, pos0, rope_theta); }));
+    VX_CUDA(traced(L, "rope", 1, [&] { return launch_rope(L, k, kr, dt == VX_BF16, B, T, H, pos0, rope_theta); }));
     qq = qr;
     kk = kr;
   }
   if (dt == VX_F32) {
-    VX_CUDA(launch_attn_f32(L, static_cast<const float*>(qq), static_cast<const float*>(kk),
-                            static_cast<const float*>(v), static_cast<float*>(o), B, T, H, window, scale));
+    VX_CUDA(traced(L, "swa_attn_f32", 1, [&] {
+      return launch_attn_f32(L, static_cast<const float*>(qq), static_cast<const float*>(kk),
+                             static_cast<const float*>(v), static_cast<float*>(o), B, T, H, window, scale);
+    }));
     return VX_OK;
   }
   CUtensorMap tq, tk, tv;
@@ -476,7 +541,7 @@ vx_status vx_swa_attn_fwd(const void* q, const void* k, const void* v, void* o, 
   aa.B = B; aa.T = T; aa.H = H; aa.window = window;
   aa.scale_log2 = scale * 1.4426950408889634f;
   aa.status = L.status; aa.limit_ns = L.limit_ns;
-  VX_CUDA(launch_attn_bf16(L, tq, tk, tv, aa));
+  VX_CUDA(traced(L, "swa_attn_tc", 1, [&] { return launch_attn_bf16(L, tq, tk, tv, aa); }));
   return VX_OK;
 }
 
@@ -494,7 +559,9 @@ vx_status vx_rms_norm_fwd(const float* x, const float* r, const void* g, float* 
   Launch L;
   vx_status st = make_launch(&L, ws, ws_bytes, kStatusBytes, stream);
   if (st != VX_OK) return st;
-  VX_CUDA(launch_rmsnorm(L, x, r, static_cast<const uint16_t*>(g), h_out, y, y_dt == VX_BF16, M, d, eps));
+  VX_CUDA(traced(L, "rmsnorm", 1, [&] {
+    return launch_rmsnorm(L, x, r, static_cast<const uint16_t*>(g), h_out, y, y_dt == VX_BF16, M, d, eps);
+  }));
   return VX_OK;
 }
 
@@ -580,8 +647,10 @@ vx_status vx_encoder_fwd(const vx_layer_cfg* cfg, const float* mel, int B, int n
   const LayerBufs bf = carve_layer(cv, *cfg, int64_t(B) * To);
   for (int l = 0; l < n_layers; ++l)
     if ((st = run_layer(L, *cfg, layers[l], out, out, B, To, 0, bf, nullptr)) != VX_OK) return st;
-  VX_CUDA(launch_rmsnorm(L, out, nullptr, static_cast<const uint16_t*>(final_g), nullptr, out, false, B * To,
-                         cfg->d_model, cfg->eps));
+  VX_CUDA(traced(L, "rmsnorm", 1, [&] {
+    return launch_rmsnorm(L, out, nullptr, static_cast<const uint16_t*>(final_g), nullptr, out, false, B * To,
+                          cfg->d_model, cfg->eps);
+  }));
   return VX_OK;
 }
 
@@ -607,9 +676,11 @@ vx_status vx_stream_prefill(const vx_layer_cfg* cfg, const vx_layer_weights* lay
     if ((st = run_layer(L, *cfg, layers[l], l == 0 ? x : y, y, S, T, 0, bf, &rl)) != VX_OK) return st;
   }
   if (final_g)
-    VX_CUDA(launch_rmsnorm(L, y, nullptr, static_cast<const uint16_t*>(final_g), nullptr, y, false, S * T,
-                           cfg->d_model, cfg->eps));
-  VX_CUDA(launch_pos_add(L, ring->pos, S, T, true));
+    VX_CUDA(traced(L, "rmsnorm", 1, [&] {
+      return launch_rmsnorm(L, y, nullptr, static_cast<const uint16_t*>(final_g), nullptr, y, false, S * T,
+                            cfg->d_model, cfg->eps);
+    }));
+  VX_CUDA(traced(L, "pos_add", 1, [&] { return launch_pos_add(L, ring->pos, S, T, true); }));
   return VX_OK;
 }
 
@@ -644,9 +715,11 @@ vx_status vx_stream_step(const vx_layer_cfg* cfg, const vx_layer_weights* layers
     if ((st = run_layer(L, *cfg, layers[l], l == 0 ? x_new : y, y, S, n_new, 0, bf, &rl)) != VX_OK) return st;
   }
   if (final_g)
-    VX_CUDA(launch_rmsnorm(L, y, nullptr, static_cast<const uint16_t*>(final_g), nullptr, y, false, S * n_new,
-                           cfg->d_model, cfg->eps));
-  VX_CUDA(launch_pos_add(L, ring->pos, S, n_new, false));
+    VX_CUDA(traced(L, "rmsnorm", 1, [&] {
+      return launch_rmsnorm(L, y, nullptr, static_cast<const uint16_t*>(final_g), nullptr, y, false, S * n_new,
+                            cfg->d_model, cfg->eps);
+    }));
+  VX_CUDA(traced(L, "pos_add", 1, [&] { return launch_pos_add(L, ring->pos, S, n_new, false); }));
   return VX_OK;
 }
 
@@ -655,7 +728,7 @@ vx_status vx_selftest_wait_timeout(void* ws, size_t ws_bytes, uint64_t timeout_n
   vx_status st = make_launch(&L, ws, ws_bytes, kStatusBytes, stream);
   if (st != VX_OK) return st;
   L.limit_ns = timeout_ns > 0 ? timeout_ns : 1;
-  VX_CUDA(launch_selftest_wait(L));
+  VX_CUDA(traced(L, "selftest_wait", 1, [&] { return launch_selftest_wait(L); }));
   return VX_OK;
 }
 

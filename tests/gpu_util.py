@@ -24,15 +24,27 @@ def host(t) -> np.ndarray:
     return t.detach().float().cpu().numpy().astype(np.float64)
 
 
-def compare_bf16(got, want, what=""):
+def _log(what, **kv):
+    """Appends measured errors to $VX_PARITY_LOG (one JSON line per check)."""
+    import json
+    import os
+    path = os.environ.get("VX_PARITY_LOG")
+    if path:
+        with open(path, "a") as f:
+            f.write(json.dumps({"check": what, **kv}) + "\n")
+
+
+def compare_bf16(got, want, what="", max_abs=BF16_MAX_ABS, rel_l2=BF16_REL_L2):
     got = np.asarray(got, dtype=np.float64)
     want = np.asarray(want, dtype=np.float64)
     assert got.shape == want.shape, (got.shape, want.shape)
     assert np.all(np.isfinite(got)), f"{what}: non-finite output"
+    max_abs_bar = max_abs
     err = np.abs(got - want)
     max_abs = float(err.max()) if err.size else 0.0
     rel = float(np.linalg.norm(got - want) / max(np.linalg.norm(want), 1e-30))
-    assert max_abs <= BF16_MAX_ABS and rel <= BF16_REL_L2, f"{what}: max_abs={max_abs:.3e} rel_l2={rel:.3e}"
+    _log(what, max_abs=max_abs, rel_l2=rel, bar_max_abs=max_abs_bar, bar_rel_l2=rel_l2)
+    assert max_abs <= max_abs_bar and rel <= rel_l2, f"{what}: max_abs={max_abs:.3e} rel_l2={rel:.3e}"
     return max_abs, rel
 
 
@@ -41,6 +53,7 @@ def compare_f32(got, want, what=""):
     want = np.asarray(want, dtype=np.float64)
     assert got.shape == want.shape
     max_abs = float(np.abs(got - want).max())
+    _log(what, max_abs=max_abs, bar_max_abs=F32_MAX_ABS)
     assert max_abs <= F32_MAX_ABS, f"{what}: max_abs={max_abs:.3e}"
     return max_abs
 

@@ -8,6 +8,7 @@ import torch
 
 import oracle
 import synth
+from test_rounding_floor import C4_MAX_ABS
 from gpu_util import cfg_of, compare_bf16, compare_f32, dev, host, layer_params_dev, layer_stack
 
 pytestmark = pytest.mark.gpu
@@ -132,7 +133,9 @@ def test_c4_full_encoder_prefix():
     out = host(vx.encoder_fwd(cfg_of(dims), dev(mel), *_conv_dev(conv), Ls, dev(g, torch.bfloat16)))
     assert out.shape == (4, 3000, 1280) and np.all(np.isfinite(out))
     want = oracle.encoder(mel[:1, :, :512], conv, layers, g, dims)
-    compare_bf16(out[:1, :256], want, "C4 prefix")
+    # 32 layers: rel-L2 keeps the 1e-2 bar; max-abs is bounded by the bf16
+    # operand-rounding floor derived in test_rounding_floor.py.
+    compare_bf16(out[:1, :256], want, "C4 prefix", max_abs=C4_MAX_ABS)
     # final RMSNorm: every frame's RMS of out / g is ~1
     rms = np.sqrt(np.mean((out / g.astype(np.float64)) ** 2, axis=-1))
     assert np.all(np.abs(rms - 1) < 1e-2)

@@ -1,0 +1,84 @@
+"""Derivation of the 32-layer encoder tolerance (CPU only).
+
+The GPU path rounds every tensor-core operand to bf16: the RMSNorm outputs,
+q/k/v, the softmax probabilities P, the attention output, the SwiGLU
+activation, and the conv-stem hidden frames.  This test runs the oracle's
+float64 arithmetic with exactly those roundings added (nothing else changed)
+and measures its distance to the plain oracle on the frames that
+tests/test_gpu_layer.py::test_c4_full_encoder_prefix compares.  That distance
+is a floor for ANY implementation with bf16 activations: it exceeds the 3e-2
+max-abs bar after 32 layers while the relative L2 error stays under 1e-2.
+Hence the 32-layer encoder test keeps rel-L2 <= 1e-2 and bounds max-abs by
+C4_MAX_ABS below (the floor measured here, 3.6e-2, plus headroom); every
+single-layer and attention test keeps the 3e-2 bar.
+"""
+import numpy as np
+import pytest
+
+import oracle
+import synth
+
+C4_MAX_ABS = 5e-2
+C4_FRAMES = 256
+
+
+def _r(x):
+    return synth.bf16_round(np.asarray(x, dtype=np.float32)).astype(np.float64)
+
+
+def _layer_bf16_operands(x, p, dims):
+    B, T, _ = x.shape
+    H, D, W = dims.n_heads, dims.head_dim, dims.window
+    pos = np.arange(T)
+    f = lambda a: np.asarray(a, dtype=np.float64)
+    y0 = _r(oracle.rms_norm(x, p["attn_norm_g"], dims.eps))
+    q = _r(oracle.rope((y0 @ f(p["wq"]).T + f(p["bq"])).reshape(B, T, H, D), pos, dims.rope_theta))
+    k = _r(oracle.rope((y0 @ f(p["wk"]).T).reshape(B, T, H, D), pos, dims.rope_theta))
+    v = _r((y0 @ f(p["wv"]).T + f(p["bv"])).reshape(B, T, H, D))
+    a = np.empty((B, T, H, D))
+    for i in range(T):
+        lo = max(0, i - W + 1)
+        s = np.einsum("bhd,bjhd->bhj", q[:, i], k[:, lo:i + 1]) / np.sqrt(D)
+        e = np.exp(s - s.max(-1, keepdims=True))
+        a[:, i] = np.einsum("bhj,bjhd->bhd", _r(e), v[:, lo:i + 1]) / e.sum(-1, keepdims=True)
+    h = x + _r(a.reshape(B, T, H * D)) @ f(p["wo"]).T + f(p["bo"])
+    y1 = _r(oracle.rms_norm(h, p["ffn_norm_g"], dims.eps))
+    act = _r(oracle.silu(y1 @ f(p["wg"]).T) * (y1 @ f(p["wu"]).T))
+    return h + act @ f(p["wd"]).T + f(p["bd"])
+
+
+def _stem_bf16_operands(mel, conv):
+    f = lambda a: np.asarray(a, dtype=np.float64)
+    w1, b1, w2, b2 = f(conv["w1"]), f(conv["b1"]), f(conv["w2"]), f(conv["b2"])
+    B, C, Tm = mel.shape
+    xp = _r(np.concatenate([np.zeros((B, C, 2)), mel], axis=2))
+    h1 = np.zeros((B, w1.shape[0], Tm)) + b1[None, :, None]
+    for k in range(3):
+        h1 += np.einsum("oc,bct->bot", w1[:, :, k], xp[:, :, k:k + Tm], optimize=True)
+    h1 = _r(oracle.gelu(h1))
+    To = oracle.conv_out_len(Tm)
+    hp = np.concatenate([np.zeros((B, h1.shape[1], 2)), h1], axis=2)
+    h2 = np.zeros((B, w2.shape[0], To)) + b2[None, :, None]
+    for k in range(3):
+        h2 += np.einsum("oc,bct->bot", w2[:, :, k], hp[:, :, k:k + 2 * To - 1:2], optimize=True)
+    return np.transpose(oracle.gelu(h2), (0, 2, 1))
+
+
+@pytest.mark.slow
+def test_bf16_operand_floor_of_the_32_layer_encoder():
+    dims = synth.VOXTRAL_RT
+    layers = [synth.layer_params(dims, seed=synth.layer_seed(1, l)) for l in range(32)]
+    conv = synth.conv_params(seed=3)
+    g = synth.final_norm_gain(dims.d_model, seed=5)
+    mel = synth.mel(4, 128, 6000, seed=4)[:1, :, :2 * C4_FRAMES].astype(np.float64)
+    ref = oracle.encoder(mel, conv, layers, g, dims)
+    x = _stem_bf16_operands(mel, conv)
+    for p in layers:
+        x = _layer_bf16_operands(x, p, dims)
+    out = oracle.rms_norm(x, g, dims.eps)
+    err = out - ref
+    max_abs = np.abs(err).max()
+    rel = np.linalg.norm(err) / np.linalg.norm(ref)
+    # the floor exceeds the single-layer bar but not the derived one
+    assert 3e-2 < max_abs < C4_MAX_ABS, max_abs
+    assert rel < 1e-2, rel
