@@ -37,7 +37,6 @@ ring_attn_kernel(const uint16_t* __restrict__ qkv, int64_t ld_qkv, int HD,
   const int h = blockIdx.x;
   const int s = blockIdx.y;
   const int tid = threadIdx.x;
-  const int grp = tid >> 3;        // 0..31
   const int sub = tid & 7;         // dims sub*8 .. sub*8+7
   const int64_t p = pos[s];
   const int n_old = static_cast<int>(p < W - 1 ? p : W - 1);
@@ -64,25 +63,32 @@ ring_attn_kernel(const uint16_t* __restrict__ qkv, int64_t ld_qkv, int HD,
     for (int d = 0; d < 8; ++d) o[qi][d] = 0.f;
   }
 
-  // The first old frame is p - n_old; frame f of key index kk.
+  // The first old frame is p - n_old; key index kk is frame f0 + kk.  Every
+  // lane of a warp runs the same number of iterations (the shuffles below are
+  // warp-collective); keys past the end are masked.
   const int64_t f0 = p - n_old;
-  int slot = static_cast<int>((f0 + grp) % W);
-  const int slot_step = kGroups % W;
-  for (int kk = grp; kk < total; kk += kGroups) {
-    const uint16_t* krow;
-    const uint16_t* vrow;
-    if (kk < n_old) {
+  const int f0_slot = static_cast<int>(f0 % W);
+  const int warp_id = tid >> 5;
+  const int gw = (tid >> 3) & 3;           // group within the warp
+  for (int kb = warp_id * 4; kb < total; kb += kGroups) {
+    const int kk = kb + gw;
+    const bool live = kk < total;
+    const uint16_t* krow = nullptr;
+    const uint16_t* vrow = nullptr;
+    if (live && kk < n_old) {
+      const int slot = (f0_slot + kk) % W;
       krow = rk + static_cast<int64_t>(slot) * 64;
       vrow = rv + static_cast<int64_t>(slot) * 64;
-    } else {
+    } else if (live) {
       const int t = kk - n_old;
       krow = qkv + (static_cast<int64_t>(s) * NQ + t) * ld_qkv + HD + h * 64;
       vrow = krow + HD;
     }
-    slot += slot_step;
-    if (slot >= W) slot -= W;
-    const uint4 kw = ld_global_cs_v4(krow + sub * 8);
-    const uint4 vw = ld_global_cs_v4(vrow + sub * 8);
+    uint4 kw = make_uint4(0, 0, 0, 0), vw = make_uint4(0, 0, 0, 0);
+    if (live) {
+      kw = ld_global_cs_v4(krow + sub * 8);
+      vw = ld_global_cs_v4(vrow + sub * 8);
+    }
     const float kf[8] = {bf16lo(kw.x), bf16hi(kw.x), bf16lo(kw.y), bf16hi(kw.y),
                          bf16lo(kw.z), bf16hi(kw.z), bf16lo(kw.w), bf16hi(kw.w)};
     const float vf[8] = {bf16lo(vw.x), bf16hi(vw.x), bf16lo(vw.y), bf16hi(vw.y),
@@ -100,6 +106,7 @@ ring_attn_kernel(const uint16_t* __restrict__ qkv, int64_t ld_qkv, int HD,
 #pragma unroll
       for (int qi = 0; qi < NQ; ++qi) sc[qi] += __shfl_xor_sync(0xffffffffu, sc[qi], off);
     }
+    if (!live) continue;
     const int64_t f = f0 + kk;   // absolute frame of this key
 #pragma unroll
     for (int qi = 0; qi < NQ; ++qi) {
