@@ -11,6 +11,7 @@ import torch
 
 import oracle
 import synth
+from test_rounding_floor import C3_MAX_ABS, C3_SAMPLE
 from gpu_util import cfg_of, compare_bf16, dev, host, layer_params_dev, layer_stack
 
 pytestmark = pytest.mark.gpu
@@ -125,7 +126,7 @@ def test_c3_full_size_sampled_streams():
     ring.k.normal_(generator=gen)
     ring.v.normal_(generator=gen)
     ring.pos.fill_(P)
-    sample = [0, 37, 63]
+    sample = list(C3_SAMPLE)
     host_rings = []
     for l in range(L):
         k, v = synth.ring_kv(len(sample), dims.n_heads, dims.window, dims.head_dim, seed=1000 + l)
@@ -136,7 +137,9 @@ def test_c3_full_size_sampled_streams():
     got = host(vx.stream_step(cfg_of(dims), Ls, ring, dev(x)))
     assert np.all(np.isfinite(got))
     want, new_rings, _ = oracle.stream_step(x[sample], layers, dims, host_rings, np.full(len(sample), P))
-    compare_bf16(got[sample], want, "C3 sampled streams")
+    # 32 layers of unnormalised residual stream: rel-L2 keeps the 1e-2 bar;
+    # max-abs is bounded by the bf16 operand floor (test_rounding_floor.py).
+    compare_bf16(got[sample], want, "C3 sampled streams", max_abs=C3_MAX_ABS)
     assert torch.all(ring.pos == P + n)
     # the step wrote the 4 new frames' K/V into slots (1000 + t) mod 750 = 250..253
     for l in (0, 31):
