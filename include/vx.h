@@ -165,6 +165,31 @@ VX_API vx_status vx_swa_attn_fwd(const void *q, const void *k, const void *v, vo
                           void *ws, size_t ws_bytes, cudaStream_t stream);
 VX_API size_t vx_swa_attn_workspace(vx_dtype dt, int B, int T, int H, int D, int apply_rope);
 
+/* vx_swa_attn_fwd_noalloc: the same operation, arguments and results as
+ * vx_swa_attn_fwd, for callers that cannot allocate device memory when they
+ * run attention (real-time audio callbacks that must not wait on the
+ * driver's allocator, plug-in hosts that own every device allocation, code
+ * under a fixed memory budget).  It takes no workspace and allocates nothing:
+ * its scratch (the RoPE-rotated q and k, and the status word of the bounded
+ * waits) is one static device array of 32 MiB + 256 bytes inside this
+ * library, held by every GPU that loads the library until the process exits.
+ * Inputs and outputs are still the caller's.
+ * Limit: with apply_rope, B*T*H*64 elements of q plus as many of k must fit in
+ * 32 MiB (B*T*H <= 131072 for bf16, 65536 for fp32); larger calls return
+ * VX_ERR_INVALID_ARG with a message and enqueue nothing.
+ * The first call on each device looks up the array's device address (with
+ * that device current) and caches it; make that first call before any stream
+ * capture.  Every call clears the status word and overwrites the rotated q/k,
+ * and all calls share the one array: calls whose work overlaps on the GPU
+ * (other streams, other threads) race on it.  A bounded wait that expires is
+ * recorded only in that private status word; use vx_swa_attn_fwd with a
+ * workspace to read it through vx_status_check.  (The pages describe no
+ * counterpart: this entry point exists for those callers only.) */
+VX_API vx_status vx_swa_attn_fwd_noalloc(const void *q, const void *k, const void *v, void *o,
+                                         vx_dtype dt, int B, int T, int H, int D, int window,
+                                         int apply_rope, float rope_theta, int64_t pos0, float scale,
+                                         cudaStream_t stream);
+
 /* RMSNorm with optional residual add:
  *   h = x + r (r may be NULL), y = h / sqrt(mean(h^2) + eps) * g.
  * x, r, h_out: [M, d] fp32 (h_out may be NULL); g: [d] bf16;

@@ -54,6 +54,7 @@ SIGNATURES = {
     "vx_pack_conv_weight": (_I, [_P, _P, _I, _I, _P]),
     "vx_swa_attn_fwd": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _I64, _F, _P, _S, _P]),
     "vx_swa_attn_workspace": (_S, [_I, _I, _I, _I, _I, _I]),
+    "vx_swa_attn_fwd_noalloc": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _I64, _F, _P]),
     "vx_rms_norm_fwd": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _F, _P, _S, _P]),
     "vx_encoder_layer_fwd": (_I, [_CFG, _W, _P, _P, _I, _I, _I64, _P, _S, _P]),
     "vx_encoder_layer_workspace": (_S, [_CFG, _I, _I]),
