@@ -60,6 +60,8 @@ def parse_args(argv=None):
     ap.add_argument("--no-components", action="store_true", help="skip the C2/C3/C4 component timings")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--components-only", default="", help="comma list of c2,c3,c4 (profiling runs)")
+    ap.add_argument("--no-e2e", action="store_true", help="skip the host-copy end-to-end pass (profiling runs)")
+    ap.add_argument("--no-trace", action="store_true", help="skip the traced per-kernel pass (profiling runs)")
     return ap.parse_args(argv)
 
 
@@ -496,20 +498,26 @@ def main(argv=None):
         step()
         yh.copy_(y, non_blocking=True)
 
-    for _ in range(3):
-        e2e_step()
-    torch.cuda.synchronize()
-    barrier(device)
-    ms_e2e_local, _, t1b = timed_steps(torch, e2e_step, max(20, min(args.steps, 200)), flush, stream)
-    ms_e2e = reduce_max(ms_e2e_local, device)
+    ms_e2e = float("nan")
+    if not args.no_e2e:
+        for _ in range(3):
+            e2e_step()
+        torch.cuda.synchronize()
+        barrier(device)
+        ms_e2e_local, _, _ = timed_steps(torch, e2e_step, max(20, min(args.steps, 200)), flush, stream)
+        ms_e2e = reduce_max(ms_e2e_local, device)
     sampler.stop()
     clocks = sampler.summary(t0, t1)
 
     # dominant kernel, timed live per launch (trace mode), and its roofline
-    tr = traced_kernels(vx, torch, step, 50, flush)
+    tr = traced_kernels(vx, torch, step, 0 if args.no_trace else 50, flush)
+    if not tr:
+        tr = {"none": {"ms_per_launch": float("nan"), "launches_per_step": 0, "ms_per_step": 0.0}}
     dom = max(tr, key=lambda k: tr[k]["ms_per_step"])
     work, wunit, bound = kernel_work(dom, B, T)
-    if bound == "tensor":
+    if work is None:
+        roof = {"bound": None, "achieved": None, "peak": None, "unit": None, "frac": None}
+    elif bound == "tensor":
         achieved = work / (tr[dom]["ms_per_launch"] / 1e3) / 1e12
         roof = {"bound": "tensor", "achieved": achieved, "peak": tf_burst, "unit": "TFLOP/s",
                 "frac": achieved / tf_burst, "peak_kind": f"{peak_kind} bf16 dense (burst)"}
