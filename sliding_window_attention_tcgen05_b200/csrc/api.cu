@@ -13,6 +13,7 @@
 //   7. act Wd^T + bd + h          -> y    (fp32)
 #include <cstdarg>
 #include <cstdio>
+#include <cstdlib>
 #include <cstring>
 #include <cmath>
 #include <atomic>
@@ -40,6 +41,14 @@ const char* last_error() { return g_err; }
 
 static std::atomic<uint64_t> g_wait_limit_ns{1000000000ull};
 uint64_t wait_limit_ns() { return g_wait_limit_ns.load(); }
+
+bool pdl_enabled() {
+  static const bool on = [] {
+    const char* e = std::getenv("VX_PDL");
+    return !(e && e[0] == '0');
+  }();
+  return on;
+}
 
 // ------------------------------------------------------------- tracing --
 // Kernel launches go through traced(): it counts them and, when tracing is on
@@ -237,17 +246,32 @@ size_t layer_ws_bytes(const vx_layer_cfg& c, int64_t M) {
   return align_up(cv.off, kAlign);
 }
 
-// Chooses the N tile: 256 when that still fills the GPU, else 128.
-int pick_bn(int M, int N, int sm) {
+// Chooses the N tile: the widest of 256 / 128 that still fills the GPU;
+// for few-row GEMMs (weight streaming) also 64, down to min_bn.
+int pick_bn(int M, int N, int sm, int min_bn = 128) {
   const int mt = (M + 127) / 128;
-  if (N % 256 == 0 && mt * (N / 256) >= sm) return 256;
-  return 128;
+  int bn = 256;
+  for (; bn > min_bn; bn /= 2)
+    if (N % bn == 0 && mt * (N / bn) >= sm) return bn;
+  return bn;
+}
+
+// Split-K factor for a few-row GEMM: the largest of 1, 2, 4, 8 that divides the
+// K blocks and keeps the work units within about one wave.
+int pick_splits(int M, int N, int K, int bn, int sm) {
+  const int units = ((M + 127) / 128) * (N / bn);
+  const int nkb = K / 64;
+  int s = 1;
+  for (int c = 2; c <= 8; c *= 2)
+    if (nkb % c == 0 && nkb / c >= 4 && units * c <= sm + sm / 8) s = c;
+  return s;
 }
 
 GemmArgs base_args(const Launch& L, int M, int N, int K) {
   GemmArgs a;
   std::memset(&a, 0, sizeof(a));
   a.M = M; a.N = N; a.K = K;
+  a.k_splits = 1;
   a.kb_per_tap = K / 64; a.a_stride = 1; a.a_tap_ch = K;
   a.in_rows = M; a.t_valid = M; a.out_rows = M; a.out_off = 0;
   a.status = L.status;
@@ -255,8 +279,9 @@ GemmArgs base_args(const Launch& L, int M, int N, int K) {
   return a;
 }
 
-vx_status gemm(const Launch& L, const char* name, const void* A, int64_t lda, const void* Bw, GemmArgs& a, int epi) {
-  const int bn = pick_bn(a.M, a.N, L.sm_count);
+vx_status gemm(const Launch& L, const char* name, const void* A, int64_t lda, const void* Bw, GemmArgs& a, int epi,
+               int bn = 0) {
+  if (bn == 0) bn = pick_bn(a.M, a.N, L.sm_count);
   CUtensorMap tmA, tmB;
   if (!tmap_bf16_2d(&tmA, A, a.K, a.M, lda, 128)) return VX_ERR_CUDA;
   if (!tmap_bf16_2d(&tmB, Bw, a.K, a.N, a.K, bn)) return VX_ERR_CUDA;
@@ -281,7 +306,7 @@ vx_status run_layer(const Launch& L, const vx_layer_cfg& c, const vx_layer_weigh
   const float sl2 = (1.0f / std::sqrt(static_cast<float>(c.head_dim))) * 1.4426950408889634f;
   vx_status st;
   // 1. RMSNorm
-  VX_CUDA(traced(L, "rmsnorm", 1, [&] { return launch_rmsnorm(L, x, nullptr, static_cast<const uint16_t*>(w.attn_norm_g), nullptr, bf.y0, true, M, d, c.eps); }));
+  VX_CUDA(traced(L, "rmsnorm", 1, [&] { return launch_rmsnorm(L, x, nullptr, 0, 0, nullptr, static_cast<const uint16_t*>(w.attn_norm_g), nullptr, bf.y0, true, M, d, c.eps); }));
   // 2. QKV + bias + RoPE
   {
     GemmArgs a = base_args(L, M, 3 * HD, d);
@@ -320,7 +345,7 @@ vx_status run_layer(const Launch& L, const vx_layer_cfg& c, const vx_layer_weigh
     if ((st = gemm(L, "gemm_o_residual", bf.att, HD, w.wo, a, EPI_F32)) != VX_OK) return st;
   }
   // 5. RMSNorm
-  VX_CUDA(traced(L, "rmsnorm", 1, [&] { return launch_rmsnorm(L, bf.h, nullptr, static_cast<const uint16_t*>(w.ffn_norm_g), nullptr, bf.y0, true, M, d, c.eps); }));
+  VX_CUDA(traced(L, "rmsnorm", 1, [&] { return launch_rmsnorm(L, bf.h, nullptr, 0, 0, nullptr, static_cast<const uint16_t*>(w.ffn_norm_g), nullptr, bf.y0, true, M, d, c.eps); }));
   // 6. gate/up + SwiGLU
   {
     GemmArgs a = base_args(L, M, 2 * F, d);
@@ -335,6 +360,112 @@ vx_status run_layer(const Launch& L, const vx_layer_cfg& c, const vx_layer_weigh
     a.bias = static_cast<const uint16_t*>(w.bd);
     a.res = bf.h; a.ld_res = d;
     if ((st = gemm(L, "gemm_down_residual", bf.act, F, w.wd, a, EPI_F32)) != VX_OK) return st;
+  }
+  return VX_OK;
+}
+
+// ------------------------------------------------------ streaming layers --
+// Few-row layers (a streaming step: M = streams x new frames) stream their
+// weights from HBM; the O-projection and down GEMMs then have too few output
+// tiles to fill the GPU, so they run split-K and write fp32 partial sums.  The
+// partial sums, bias and residual are reduced inside the RMSNorm that follows:
+//   layer input  x_l = H_{l-1} + bd_{l-1} + sum P_down   (RMSNorm 1 also writes x_l)
+//   h            = x_l + bo + sum P_o                    (RMSNorm 2 writes h)
+// so the per-layer kernel count stays seven.
+struct StreamBufs {
+  LayerBufs lb;    // y0 (y1), qkv, att, act; lb.h is H
+  float* xmat;     // [M, d] materialised layer input
+  float* parts;    // [kMaxSplits, M, d] fp32 partial sums
+};
+constexpr int kMaxSplits = 8;
+
+StreamBufs carve_stream(Carve& cv, const vx_layer_cfg& c, int64_t M) {
+  StreamBufs b;
+  b.lb = carve_layer(cv, c, M);
+  b.xmat = static_cast<float*>(cv.take(M * c.d_model * 4));
+  b.parts = static_cast<float*>(cv.take(kMaxSplits * M * c.d_model * 4));
+  return b;
+}
+
+size_t stream_ws_bytes(const vx_layer_cfg& c, int64_t M) {
+  Carve cv{nullptr, kStatusBytes};
+  carve_stream(cv, c, M);
+  return align_up(cv.off, kAlign);
+}
+
+// The pending (unreduced) output of a layer: base + bias + sum of parts.
+struct Pending {
+  const float* base;
+  const float* parts;
+  int nparts;
+  const uint16_t* bias;
+};
+
+vx_status run_layer_stream(const Launch& L, const vx_layer_cfg& c, const vx_layer_weights& w, const Pending& in,
+                           Pending* out, int nseq, int rows, const StreamBufs& sb, const RingLayer& ring) {
+  const int d = c.d_model, H = c.n_heads, HD = H * c.head_dim, F = c.ffn_hidden;
+  const int M = nseq * rows;
+  const int64_t pstride = static_cast<int64_t>(M) * d;
+  const float sl2 = (1.0f / std::sqrt(static_cast<float>(c.head_dim))) * 1.4426950408889634f;
+  const LayerBufs& bf = sb.lb;
+  vx_status st;
+  // 1. x_l = reduce(in); y0 = RMSNorm(x_l)
+  const bool pending_in = in.parts != nullptr || in.bias != nullptr;
+  const float* xl = pending_in ? sb.xmat : in.base;
+  VX_CUDA(traced(L, "rmsnorm", 1, [&] {
+    return launch_rmsnorm(L, in.base, in.parts, in.nparts, pstride, in.bias,
+                          static_cast<const uint16_t*>(w.attn_norm_g), pending_in ? sb.xmat : nullptr, bf.y0, true,
+                          M, d, c.eps);
+  }));
+  // 2. QKV + bias + RoPE at pos[s] + t
+  {
+    GemmArgs a = base_args(L, M, 3 * HD, d);
+    a.out = bf.qkv; a.ld_out = 3 * HD;
+    a.bias = static_cast<const uint16_t*>(w.bqkv);
+    a.in_rows = rows; a.t_valid = rows; a.out_rows = rows;
+    a.pos_arr = ring.pos;
+    a.rope_cols = 2 * HD;
+    fill_rope_freqs(&a, c.rope_theta, c.head_dim);
+    if ((st = gemm(L, "gemm_qkv_rope", bf.y0, d, w.wqkv, a, EPI_QKV_ROPE, pick_bn(M, 3 * HD, L.sm_count, 64))) != VX_OK)
+      return st;
+  }
+  // 3. ring attention (reads every old in-window slot, then appends)
+  VX_CUDA(traced(L, "ring_attn", 1, [&] {
+    return launch_ring_attn(L, bf.qkv, 3LL * HD, HD, ring.k, ring.v, ring.pos, nseq, H, ring.W, rows, bf.att, sl2);
+  }));
+  // 4. O-projection, split-K partial sums
+  int so;
+  {
+    const int bn = pick_bn(M, d, L.sm_count, 64);
+    so = pick_splits(M, d, HD, bn, L.sm_count);
+    GemmArgs a = base_args(L, M, d, HD);
+    a.out = sb.parts; a.ld_out = d;
+    a.k_splits = so; a.split_stride = pstride;
+    if ((st = gemm(L, "gemm_o_splitk", bf.att, HD, w.wo, a, EPI_F32, bn)) != VX_OK) return st;
+  }
+  // 5. h = x_l + bo + sum P_o; y1 = RMSNorm(h)
+  VX_CUDA(traced(L, "rmsnorm", 1, [&] {
+    return launch_rmsnorm(L, xl, sb.parts, so, pstride, static_cast<const uint16_t*>(w.bo),
+                          static_cast<const uint16_t*>(w.ffn_norm_g), bf.h, bf.y0, true, M, d, c.eps);
+  }));
+  // 6. gate/up + SwiGLU
+  {
+    GemmArgs a = base_args(L, M, 2 * F, d);
+    a.out = bf.act; a.ld_out = F;
+    a.bias = static_cast<const uint16_t*>(w.bgu);
+    if ((st = gemm(L, "gemm_gate_up_swiglu", bf.y0, d, w.wgu, a, EPI_SWIGLU, pick_bn(M, 2 * F, L.sm_count, 128))) !=
+        VX_OK)
+      return st;
+  }
+  // 7. down, split-K partial sums; the layer output stays pending
+  {
+    const int bn = pick_bn(M, d, L.sm_count, 64);
+    const int sd = pick_splits(M, d, F, bn, L.sm_count);
+    GemmArgs a = base_args(L, M, d, F);
+    a.out = sb.parts; a.ld_out = d;
+    a.k_splits = sd; a.split_stride = pstride;
+    if ((st = gemm(L, "gemm_down_splitk", bf.act, F, w.wd, a, EPI_F32, bn)) != VX_OK) return st;
+    *out = Pending{bf.h, sb.parts, sd, static_cast<const uint16_t*>(w.bd)};
   }
   return VX_OK;
 }
@@ -560,7 +691,8 @@ vx_status vx_rms_norm_fwd(const float* x, const float* r, const void* g, float* 
   vx_status st = make_launch(&L, ws, ws_bytes, kStatusBytes, stream);
   if (st != VX_OK) return st;
   VX_CUDA(traced(L, "rmsnorm", 1, [&] {
-    return launch_rmsnorm(L, x, r, static_cast<const uint16_t*>(g), h_out, y, y_dt == VX_BF16, M, d, eps);
+    return launch_rmsnorm(L, x, r, r ? 1 : 0, 0, nullptr, static_cast<const uint16_t*>(g), h_out, y, y_dt == VX_BF16,
+                          M, d, eps);
   }));
   return VX_OK;
 }
@@ -648,8 +780,8 @@ vx_status vx_encoder_fwd(const vx_layer_cfg* cfg, const float* mel, int B, int n
   for (int l = 0; l < n_layers; ++l)
     if ((st = run_layer(L, *cfg, layers[l], out, out, B, To, 0, bf, nullptr)) != VX_OK) return st;
   VX_CUDA(traced(L, "rmsnorm", 1, [&] {
-    return launch_rmsnorm(L, out, nullptr, static_cast<const uint16_t*>(final_g), nullptr, out, false, B * To,
-                          cfg->d_model, cfg->eps);
+    return launch_rmsnorm(L, out, nullptr, 0, 0, nullptr, static_cast<const uint16_t*>(final_g), nullptr, out, false,
+                          B * To, cfg->d_model, cfg->eps);
   }));
   return VX_OK;
 }
@@ -677,8 +809,8 @@ vx_status vx_stream_prefill(const vx_layer_cfg* cfg, const vx_layer_weights* lay
   }
   if (final_g)
     VX_CUDA(traced(L, "rmsnorm", 1, [&] {
-      return launch_rmsnorm(L, y, nullptr, static_cast<const uint16_t*>(final_g), nullptr, y, false, S * T,
-                            cfg->d_model, cfg->eps);
+      return launch_rmsnorm(L, y, nullptr, 0, 0, nullptr, static_cast<const uint16_t*>(final_g), nullptr, y, false,
+                            S * T, cfg->d_model, cfg->eps);
     }));
   VX_CUDA(traced(L, "pos_add", 1, [&] { return launch_pos_add(L, ring->pos, S, T, true); }));
   return VX_OK;
@@ -686,7 +818,7 @@ vx_status vx_stream_prefill(const vx_layer_cfg* cfg, const vx_layer_weights* lay
 
 size_t vx_stream_step_workspace(const vx_layer_cfg* cfg, int S, int n_new) {
   if (!cfg || S <= 0 || n_new <= 0) return kStatusBytes;
-  return layer_ws_bytes(*cfg, int64_t(S) * n_new);
+  return stream_ws_bytes(*cfg, int64_t(S) * n_new);
 }
 
 vx_status vx_stream_step(const vx_layer_cfg* cfg, const vx_layer_weights* layers, const vx_kv_ring* ring,
@@ -699,26 +831,33 @@ vx_status vx_stream_step(const vx_layer_cfg* cfg, const vx_layer_weights* layers
   for (int l = 0; l < ring->n_layers; ++l)
     if ((st = check_weights(*cfg, &layers[l])) != VX_OK) return st;
   VX_CHECK_ARG(x_new && y && aligned16(x_new) && aligned16(y), "bad x_new/y");
+  VX_CHECK_ARG(!final_g || (reinterpret_cast<uintptr_t>(final_g) & 7) == 0, "final_g must be 8-byte aligned");
   if (n_new < 1 || n_new > 8 || n_new > cfg->window) {
     set_error("n_new=%d unsupported (1..8 and <= window)", n_new);
     return VX_ERR_UNSUPPORTED;
   }
   const int S = ring->n_streams;
+  const int M = S * n_new;
   Launch L;
   if ((st = make_launch(&L, ws, ws_bytes, vx_stream_step_workspace(cfg, S, n_new), stream)) != VX_OK) return st;
   Carve cv{static_cast<uint8_t*>(ws), kStatusBytes};
-  const LayerBufs bf = carve_layer(cv, *cfg, int64_t(S) * n_new);
+  const StreamBufs sb = carve_stream(cv, *cfg, M);
   const int64_t layer_elems = int64_t(S) * cfg->n_heads * ring->window * cfg->head_dim;
+  Pending cur{x_new, nullptr, 0, nullptr};
   for (int l = 0; l < ring->n_layers; ++l) {
     RingLayer rl{static_cast<uint16_t*>(ring->k) + l * layer_elems, static_cast<uint16_t*>(ring->v) + l * layer_elems,
                  ring->pos, ring->window, false, true};
-    if ((st = run_layer(L, *cfg, layers[l], l == 0 ? x_new : y, y, S, n_new, 0, bf, &rl)) != VX_OK) return st;
+    Pending next;
+    if ((st = run_layer_stream(L, *cfg, layers[l], cur, &next, S, n_new, sb, rl)) != VX_OK) return st;
+    cur = next;
   }
-  if (final_g)
-    VX_CUDA(traced(L, "rmsnorm", 1, [&] {
-      return launch_rmsnorm(L, y, nullptr, static_cast<const uint16_t*>(final_g), nullptr, y, false, S * n_new,
-                            cfg->d_model, cfg->eps);
-    }));
+  // y = reduce(last layer output), then the optional final RMSNorm.
+  const int64_t pstride = static_cast<int64_t>(M) * cfg->d_model;
+  VX_CUDA(traced(L, "rmsnorm", 1, [&] {
+    return launch_rmsnorm(L, cur.base, cur.parts, cur.nparts, pstride, cur.bias,
+                          static_cast<const uint16_t*>(final_g), final_g ? nullptr : y, final_g ? y : nullptr, false,
+                          M, cfg->d_model, cfg->eps);
+  }));
   VX_CUDA(traced(L, "pos_add", 1, [&] { return launch_pos_add(L, ring->pos, S, n_new, false); }));
   return VX_OK;
 }

@@ -80,6 +80,8 @@ swa_attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const WaitCtx wc{a.status, abort_flag, a.limit_ns};
+  pdl_wait();
+  pdl_trigger();
 
   if (warp == 4) {
     if (lane == 0) {
@@ -285,6 +287,8 @@ swa_attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
 __global__ void __launch_bounds__(128)
 swa_attn_f32_kernel(const float* __restrict__ q, const float* __restrict__ k, const float* __restrict__ v,
                     float* __restrict__ o, int T, int H, int W, float scale) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ float qs[4][64];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int i = blockIdx.x * 4 + warp;
@@ -346,6 +350,8 @@ struct RopeArgs {
 template <bool BF16>
 __global__ void rope_kernel(const void* __restrict__ x, void* __restrict__ y, int64_t rows, int T, int H,
                             int64_t pos0, const __grid_constant__ RopeArgs f) {
+  pdl_wait();
+  pdl_trigger();
   const int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   const int64_t total = rows * H * 32;
   if (idx >= total) return;
@@ -393,15 +399,13 @@ cudaError_t launch_attn_bf16(const Launch& L, const CUtensorMap& tmQ, const CUte
     attr_set = true;
   }
   const dim3 grid((a.T + 127) / 128, a.H, a.B);
-  swa_attn_tc_kernel<<<grid, kAttnThreads, kAttnSmem, L.stream>>>(tmQ, tmK, tmV, a);
-  return cudaGetLastError();
+  return launch_kernel(swa_attn_tc_kernel, grid, dim3(kAttnThreads), kAttnSmem, L.stream, tmQ, tmK, tmV, a);
 }
 
 cudaError_t launch_attn_f32(const Launch& L, const float* q, const float* k, const float* v, float* o,
                             int B, int T, int H, int window, float scale) {
   const dim3 grid((T + 3) / 4, H, B);
-  swa_attn_f32_kernel<<<grid, 128, 0, L.stream>>>(q, k, v, o, T, H, window, scale);
-  return cudaGetLastError();
+  return launch_kernel(swa_attn_f32_kernel, grid, dim3(128), 0, L.stream, q, k, v, o, T, H, window, scale);
 }
 
 cudaError_t launch_rope(const Launch& L, const void* x, void* y, bool bf16, int B, int T, int H,
@@ -417,10 +421,10 @@ cudaError_t launch_rope(const Launch& L, const void* x, void* y, bool bf16, int 
   const int threads = 256;
   const int64_t blocks = (total + threads - 1) / threads;
   if (bf16)
-    rope_kernel<true><<<static_cast<unsigned>(blocks), threads, 0, L.stream>>>(x, y, rows, T, H, pos0, f);
-  else
-    rope_kernel<false><<<static_cast<unsigned>(blocks), threads, 0, L.stream>>>(x, y, rows, T, H, pos0, f);
-  return cudaGetLastError();
+    return launch_kernel(rope_kernel<true>, dim3(static_cast<unsigned>(blocks)), dim3(threads), 0, L.stream, x, y,
+                         rows, T, H, pos0, f);
+  return launch_kernel(rope_kernel<false>, dim3(static_cast<unsigned>(blocks)), dim3(threads), 0, L.stream, x, y,
+                       rows, T, H, pos0, f);
 }
 
 }  // namespace vx

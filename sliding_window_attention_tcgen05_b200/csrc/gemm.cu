@@ -25,7 +25,7 @@ constexpr int kABytes = kBM * kBK * 2;
 
 template <int BN>
 struct GemmCfg {
-  static constexpr int kStages = (BN == 256) ? 4 : 6;
+  static constexpr int kStages = (BN == 256) ? 4 : (BN == 128 ? 6 : 8);
   static constexpr int kBBytes = BN * kBK * 2;
   static constexpr int kStageBytes = kABytes + kBBytes;
   static constexpr int kTmemCols = 2 * BN;  // two accumulators
@@ -68,7 +68,7 @@ __device__ __forceinline__ void store_f32x32(float* dst, const float (&v)[32]) {
 }
 
 template <int BN, int EPI>
-__device__ __forceinline__ void epilogue_tile(const GemmArgs& a, uint32_t tacc, int m, int n0) {
+__device__ __forceinline__ void epilogue_tile(const GemmArgs& a, uint32_t tacc, int m, int n0, int ks) {
   const bool in_range = m < a.M;
   const int b = m / a.in_rows;
   const int t = m - b * a.in_rows;
@@ -151,7 +151,7 @@ __device__ __forceinline__ void epilogue_tile(const GemmArgs& a, uint32_t tacc, 
               v[4 * j] += q.x; v[4 * j + 1] += q.y; v[4 * j + 2] += q.z; v[4 * j + 3] += q.w;
             }
           }
-          store_f32x32(static_cast<float*>(a.out) + drow * a.ld_out + n, v);
+          store_f32x32(static_cast<float*>(a.out) + ks * a.split_stride + drow * a.ld_out + n, v);
         } else {
 #pragma unroll
           for (int i = 0; i < 32; ++i) v[i] = gelu_erf(v[i]);
@@ -209,10 +209,24 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
+  // Inputs written by the previous kernel of the stream are read below.
+  pdl_wait();
+  pdl_trigger();
+
   const WaitCtx wc{a.status, abort_flag, a.limit_ns};
+  // Work unit u -> (m tile, K split, n tile), M fastest so that the units
+  // resident at one time share a weight panel through L2.
   const int m_tiles = (a.M + kBM - 1) / kBM;
-  const int num_tiles = m_tiles * (a.N / BN);
-  const int nkb = a.K / kBK;
+  const int splits = a.k_splits;
+  const int num_tiles = m_tiles * (a.N / BN) * splits;
+  const int nkb = a.K / kBK / splits;
+  auto decode = [&](int u, int& m0, int& n0, int& ks) {
+    const int mt = u % m_tiles;
+    const int r = u / m_tiles;
+    ks = r % splits;
+    m0 = mt * kBM;
+    n0 = (r / splits) * BN;
+  };
 
   if (warp == 4) {
     if (lane == 0) {
@@ -221,10 +235,10 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
       uint32_t issued = 0;  // bit s: stage s was filled at least once
       uint32_t last_par = 0;  // bit s: parity of the last fill of stage s
       for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
-        const int m0 = (tile % m_tiles) * kBM;
-        const int n0 = (tile / m_tiles) * BN;
+        int m0, n0, ks;
+        decode(tile, m0, n0, ks);
         bool ok = true;
-        for (int kb = 0; kb < nkb; ++kb) {
+        for (int kb = ks * nkb; kb < (ks + 1) * nkb; ++kb) {
           if (!mbar_wait(empty(stage), phase ^ 1, wc, 1)) { ok = false; break; }
           mbar_arrive_expect_tx(full(stage), C::kStageBytes);
           const int tap = kb / a.kb_per_tap;
@@ -285,8 +299,8 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
   } else {
     int local = 0;
     for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++local) {
-      const int m0 = (tile % m_tiles) * kBM;
-      const int n0 = (tile / m_tiles) * BN;
+      int m0, n0, ks;
+      decode(tile, m0, n0, ks);
       const int ab = local & 1;
       const uint32_t acc_par = (local >> 1) & 1;
       bool ok = mbar_wait(acc_full(ab), acc_par, wc, 4);
@@ -294,7 +308,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
       if (!ok) break;
       tc_fence_after();
       const uint32_t tacc = tmem_base + ab * BN + (static_cast<uint32_t>(warp * 32) << 16);
-      epilogue_tile<BN, EPI>(a, tacc, m0 + warp * 32 + lane, n0);
+      epilogue_tile<BN, EPI>(a, tacc, m0 + warp * 32 + lane, n0, ks);
       tc_fence_before();
       mbar_arrive(acc_empty(ab));
     }
@@ -318,10 +332,9 @@ cudaError_t launch_one(const Launch& L, const CUtensorMap& tmA, const CUtensorMa
     attr_set = true;
   }
   const int m_tiles = (a.M + kBM - 1) / kBM;
-  const int tiles = m_tiles * (a.N / BN);
+  const int tiles = m_tiles * (a.N / BN) * a.k_splits;
   const int grid = tiles < L.sm_count ? tiles : L.sm_count;
-  gemm_tc_kernel<BN, EPI><<<grid, kThreads, C::kSmem, L.stream>>>(tmA, tmB, a);
-  return cudaGetLastError();
+  return launch_kernel(gemm_tc_kernel<BN, EPI>, dim3(grid), dim3(kThreads), C::kSmem, L.stream, tmA, tmB, a);
 }
 
 template <int BN>
@@ -330,7 +343,9 @@ cudaError_t launch_bn(const Launch& L, const CUtensorMap& tmA, const CUtensorMap
   switch (epi) {
     case EPI_F32: return launch_one<BN, EPI_F32>(L, tmA, tmB, a);
     case EPI_QKV_ROPE: return launch_one<BN, EPI_QKV_ROPE>(L, tmA, tmB, a);
-    case EPI_SWIGLU: return launch_one<BN, EPI_SWIGLU>(L, tmA, tmB, a);
+    case EPI_SWIGLU:
+      if constexpr (BN >= 128) return launch_one<BN, EPI_SWIGLU>(L, tmA, tmB, a);
+      else return cudaErrorInvalidValue;
     case EPI_GELU_BF16: return launch_one<BN, EPI_GELU_BF16>(L, tmA, tmB, a);
     case EPI_GELU_F32: return launch_one<BN, EPI_GELU_F32>(L, tmA, tmB, a);
     default: return cudaErrorInvalidValue;
@@ -342,8 +357,10 @@ cudaError_t launch_bn(const Launch& L, const CUtensorMap& tmA, const CUtensorMap
 cudaError_t launch_gemm(const Launch& L, const CUtensorMap& tmA, const CUtensorMap& tmB,
                         const GemmArgs& args, int epi, int bn) {
   if (args.M <= 0) return cudaSuccess;
+  if (args.k_splits < 1 || (args.K / kBK) % args.k_splits != 0) return cudaErrorInvalidValue;
   if (bn == 256) return launch_bn<256>(L, tmA, tmB, args, epi);
   if (bn == 128) return launch_bn<128>(L, tmA, tmB, args, epi);
+  if (bn == 64) return launch_bn<64>(L, tmA, tmB, args, epi);
   return cudaErrorInvalidValue;
 }
 

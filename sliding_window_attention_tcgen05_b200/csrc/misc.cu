@@ -8,40 +8,51 @@ namespace {
 
 // ---------------------------------------------------------------- RMSNorm --
 // One warp per row of d (multiple of 128, <= 2048) fp32 values; lane i holds
-// float4 columns i, i+32, ...; h = x (+ r); y = h * rsqrt(mean(h^2) + eps) * g.
+// float4 columns i, i+32, ...
+//   h = x + bias + sum_k parts[k]   (split-K partial sums of the GEMM before)
+//   y = h * rsqrt(mean(h^2) + eps) * g
 template <bool BF16_OUT>
 __global__ void __launch_bounds__(256)
-rmsnorm_kernel(const float* __restrict__ x, const float* __restrict__ r, const uint16_t* __restrict__ g,
-               float* __restrict__ h_out, void* __restrict__ y, int M, int d, float eps) {
+rmsnorm_kernel(const float* __restrict__ x, const float* __restrict__ parts, int nparts, int64_t part_stride,
+               const uint16_t* __restrict__ bias, const uint16_t* __restrict__ g, float* __restrict__ h_out,
+               void* __restrict__ y, int M, int d, float eps) {
+  pdl_wait();
+  pdl_trigger();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int row = blockIdx.x * 8 + warp;
   if (row >= M) return;
   const int nv = d >> 7;
-  const float4* xr = reinterpret_cast<const float4*>(x + static_cast<int64_t>(row) * d);
-  const float4* rr = r ? reinterpret_cast<const float4*>(r + static_cast<int64_t>(row) * d) : nullptr;
+  const int64_t roff = static_cast<int64_t>(row) * d;
+  const float4* xr = reinterpret_cast<const float4*>(x + roff);
   float4 v[16];
   float ss = 0.f;
 #pragma unroll
   for (int i = 0; i < 16; ++i) {
     if (i < nv) {
-      float4 a = xr[lane + 32 * i];
-      if (rr) {
-        const float4 b = rr[lane + 32 * i];
+      const int c4 = lane + 32 * i;
+      float4 a = xr[c4];
+      for (int k = 0; k < nparts; ++k) {
+        const float4 b = reinterpret_cast<const float4*>(parts + k * part_stride + roff)[c4];
         a.x += b.x; a.y += b.y; a.z += b.z; a.w += b.w;
+      }
+      if (bias) {
+        const uint2 bw = __ldg(reinterpret_cast<const uint2*>(bias) + c4);
+        a.x += bf16lo(bw.x); a.y += bf16hi(bw.x); a.z += bf16lo(bw.y); a.w += bf16hi(bw.y);
       }
       v[i] = a;
       ss = fmaf(a.x, a.x, fmaf(a.y, a.y, fmaf(a.z, a.z, fmaf(a.w, a.w, ss))));
     }
   }
-#pragma unroll
-  for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
-  const float inv = rsqrtf(ss / static_cast<float>(d) + eps);
   if (h_out) {
-    float4* hr = reinterpret_cast<float4*>(h_out + static_cast<int64_t>(row) * d);
+    float4* hr = reinterpret_cast<float4*>(h_out + roff);
 #pragma unroll
     for (int i = 0; i < 16; ++i)
       if (i < nv) hr[lane + 32 * i] = v[i];
   }
+  if (y == nullptr) return;
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+  const float inv = rsqrtf(ss / static_cast<float>(d) + eps);
   const uint2* gr = reinterpret_cast<const uint2*>(g);
 #pragma unroll
   for (int i = 0; i < 16; ++i) {
@@ -54,10 +65,9 @@ rmsnorm_kernel(const float* __restrict__ x, const float* __restrict__ r, const u
         uint2 w;
         w.x = pack_bf16x2(o0, o1);
         w.y = pack_bf16x2(o2, o3);
-        reinterpret_cast<uint2*>(static_cast<uint16_t*>(y) + static_cast<int64_t>(row) * d)[c4] = w;
+        reinterpret_cast<uint2*>(static_cast<uint16_t*>(y) + roff)[c4] = w;
       } else {
-        reinterpret_cast<float4*>(static_cast<float*>(y) + static_cast<int64_t>(row) * d)[c4] =
-            make_float4(o0, o1, o2, o3);
+        reinterpret_cast<float4*>(static_cast<float*>(y) + roff)[c4] = make_float4(o0, o1, o2, o3);
       }
     }
   }
@@ -119,6 +129,8 @@ __global__ void pack_conv_kernel(const uint16_t* __restrict__ w, uint16_t* __res
 // for 2 <= tp < Tm + 2, else 0.  32 x 32 tiles through shared memory.
 __global__ void conv_prep_kernel(const float* __restrict__ mel, uint16_t* __restrict__ xpad,
                                  int C, int Tm, int P) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ float tile[32][33];
   const int tp0 = blockIdx.x * 32, c0 = blockIdx.y * 32, b = blockIdx.z;
   const int tx = threadIdx.x, ty = threadIdx.y;   // 32 x 8
@@ -140,6 +152,8 @@ __global__ void conv_prep_kernel(const float* __restrict__ mel, uint16_t* __rest
 
 // Zeroes rows {0, 1} and [Tm + 2, P) of every clip of h1pad [B, P, d].
 __global__ void conv_pad_zero_kernel(uint16_t* __restrict__ h1pad, int Tm, int P, int d) {
+  pdl_wait();
+  pdl_trigger();
   const int b = blockIdx.y;
   const int which = blockIdx.x;     // 0, 1, or 2 + (row - Tm - 2)
   const int row = which < 2 ? which : Tm + which;
@@ -167,15 +181,16 @@ __global__ void selftest_wait_kernel(DevStatus* st, uint64_t limit_ns) {
 
 }  // namespace
 
-cudaError_t launch_rmsnorm(const Launch& L, const float* x, const float* r, const uint16_t* g, float* h_out,
-                           void* y, bool y_bf16, int M, int d, float eps) {
+cudaError_t launch_rmsnorm(const Launch& L, const float* x, const float* parts, int nparts, int64_t part_stride,
+                           const uint16_t* bias, const uint16_t* g, float* h_out, void* y, bool y_bf16, int M,
+                           int d, float eps) {
   if (M <= 0) return cudaSuccess;
-  const int blocks = (M + 7) / 8;
+  const dim3 blocks((M + 7) / 8);
   if (y_bf16)
-    rmsnorm_kernel<true><<<blocks, 256, 0, L.stream>>>(x, r, g, h_out, y, M, d, eps);
-  else
-    rmsnorm_kernel<false><<<blocks, 256, 0, L.stream>>>(x, r, g, h_out, y, M, d, eps);
-  return cudaGetLastError();
+    return launch_kernel(rmsnorm_kernel<true>, blocks, dim3(256), 0, L.stream, x, parts, nparts, part_stride, bias,
+                         g, h_out, y, M, d, eps);
+  return launch_kernel(rmsnorm_kernel<false>, blocks, dim3(256), 0, L.stream, x, parts, nparts, part_stride, bias,
+                       g, h_out, y, M, d, eps);
 }
 
 static cudaError_t pack_rows(const Launch& L, PackSrc p, uint16_t* out, int64_t rows, int64_t cols) {
@@ -204,11 +219,10 @@ cudaError_t launch_pack_conv(const Launch& L, const uint16_t* w, uint16_t* wp, i
 
 cudaError_t launch_conv_prep(const Launch& L, const float* mel, uint16_t* xpad, uint16_t* h1pad, int B, int C,
                              int Tm, int P, int d) {
-  conv_prep_kernel<<<dim3((P + 31) / 32, (C + 31) / 32, B), dim3(32, 8), 0, L.stream>>>(mel, xpad, C, Tm, P);
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e = launch_kernel(conv_prep_kernel, dim3((P + 31) / 32, (C + 31) / 32, B), dim3(32, 8), 0, L.stream,
+                                mel, xpad, C, Tm, P);
   if (e != cudaSuccess) return e;
-  conv_pad_zero_kernel<<<dim3(2 + (P - Tm - 2), B), 128, 0, L.stream>>>(h1pad, Tm, P, d);
-  return cudaGetLastError();
+  return launch_kernel(conv_pad_zero_kernel, dim3(2 + (P - Tm - 2), B), dim3(128), 0, L.stream, h1pad, Tm, P, d);
 }
 
 cudaError_t launch_selftest_wait(const Launch& L) {

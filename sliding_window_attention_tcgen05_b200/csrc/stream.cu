@@ -24,7 +24,7 @@ constexpr int kRingThreads = 256;
 constexpr int kGroups = kRingThreads / 8;   // 8-lane groups per CTA
 
 template <int NQ>
-__global__ void __launch_bounds__(kRingThreads)
+__global__ void __launch_bounds__(kRingThreads, 2)
 ring_attn_kernel(const uint16_t* __restrict__ qkv, int64_t ld_qkv, int HD,
                  uint16_t* __restrict__ ring_k, uint16_t* __restrict__ ring_v,
                  const int64_t* __restrict__ pos, int H, int W, uint16_t* __restrict__ out,
@@ -34,6 +34,8 @@ ring_attn_kernel(const uint16_t* __restrict__ qkv, int64_t ld_qkv, int HD,
   __shared__ float sm_l[kWarps][NQ];
   __shared__ float sm_o[kWarps][NQ][64];
 
+  pdl_wait();
+  pdl_trigger();
   const int h = blockIdx.x;
   const int s = blockIdx.y;
   const int tid = threadIdx.x;
@@ -63,62 +65,73 @@ ring_attn_kernel(const uint16_t* __restrict__ qkv, int64_t ld_qkv, int HD,
     for (int d = 0; d < 8; ++d) o[qi][d] = 0.f;
   }
 
-  // The first old frame is p - n_old; key index kk is frame f0 + kk.  Every
-  // lane of a warp runs the same number of iterations (the shuffles below are
-  // warp-collective); keys past the end are masked.
+  // The first old frame is p - n_old; key index kk is frame f0 + kk.  Each
+  // 8-lane group takes kU keys per iteration (kk = kb + gw + 32u), issuing all
+  // their K/V loads before any math so that 2 * kU 16-byte loads per lane are
+  // in flight.  Every lane of a warp runs the same number of iterations (the
+  // shuffles are warp-collective); keys past the end are masked.
+  constexpr int kU = 4;
   const int64_t f0 = p - n_old;
   const int f0_slot = static_cast<int>(f0 % W);
   const int warp_id = tid >> 5;
   const int gw = (tid >> 3) & 3;           // group within the warp
-  for (int kb = warp_id * 4; kb < total; kb += kGroups) {
-    const int kk = kb + gw;
-    const bool live = kk < total;
-    const uint16_t* krow = nullptr;
-    const uint16_t* vrow = nullptr;
-    if (live && kk < n_old) {
-      const int slot = (f0_slot + kk) % W;
-      krow = rk + static_cast<int64_t>(slot) * 64;
-      vrow = rv + static_cast<int64_t>(slot) * 64;
-    } else if (live) {
-      const int t = kk - n_old;
-      krow = qkv + (static_cast<int64_t>(s) * NQ + t) * ld_qkv + HD + h * 64;
-      vrow = krow + HD;
-    }
-    uint4 kw = make_uint4(0, 0, 0, 0), vw = make_uint4(0, 0, 0, 0);
-    if (live) {
-      kw = ld_global_cs_v4(krow + sub * 8);
-      vw = ld_global_cs_v4(vrow + sub * 8);
-    }
-    const float kf[8] = {bf16lo(kw.x), bf16hi(kw.x), bf16lo(kw.y), bf16hi(kw.y),
-                         bf16lo(kw.z), bf16hi(kw.z), bf16lo(kw.w), bf16hi(kw.w)};
-    const float vf[8] = {bf16lo(vw.x), bf16hi(vw.x), bf16lo(vw.y), bf16hi(vw.y),
-                         bf16lo(vw.z), bf16hi(vw.z), bf16lo(vw.w), bf16hi(vw.w)};
-    float sc[NQ];
+  for (int kb = warp_id * 4; kb < total; kb += kGroups * kU) {
+    uint4 kw[kU], vw[kU];
 #pragma unroll
-    for (int qi = 0; qi < NQ; ++qi) {
-      float d = 0.f;
-#pragma unroll
-      for (int e = 0; e < 8; ++e) d = fmaf(q[qi][e], kf[e], d);
-      sc[qi] = d;
+    for (int u = 0; u < kU; ++u) {
+      const int kk = kb + gw + kGroups * u;
+      kw[u] = make_uint4(0, 0, 0, 0);
+      vw[u] = make_uint4(0, 0, 0, 0);
+      if (kk < total) {
+        const uint16_t* krow;
+        const uint16_t* vrow;
+        if (kk < n_old) {
+          const int slot = (f0_slot + kk) % W;
+          krow = rk + static_cast<int64_t>(slot) * 64;
+          vrow = rv + static_cast<int64_t>(slot) * 64;
+        } else {
+          const int t = kk - n_old;
+          krow = qkv + (static_cast<int64_t>(s) * NQ + t) * ld_qkv + HD + h * 64;
+          vrow = krow + HD;
+        }
+        kw[u] = ld_global_cs_v4(krow + sub * 8);
+        vw[u] = ld_global_cs_v4(vrow + sub * 8);
+      }
     }
 #pragma unroll
-    for (int off = 1; off < 8; off <<= 1) {
+    for (int u = 0; u < kU; ++u) {
+      const int kk = kb + gw + kGroups * u;
+      const float kf[8] = {bf16lo(kw[u].x), bf16hi(kw[u].x), bf16lo(kw[u].y), bf16hi(kw[u].y),
+                           bf16lo(kw[u].z), bf16hi(kw[u].z), bf16lo(kw[u].w), bf16hi(kw[u].w)};
+      float sc[NQ];
 #pragma unroll
-      for (int qi = 0; qi < NQ; ++qi) sc[qi] += __shfl_xor_sync(0xffffffffu, sc[qi], off);
-    }
-    if (!live) continue;
-    const int64_t f = f0 + kk;   // absolute frame of this key
+      for (int qi = 0; qi < NQ; ++qi) {
+        float d = 0.f;
 #pragma unroll
-    for (int qi = 0; qi < NQ; ++qi) {
-      const int64_t fq = p + qi;
-      if (f > fq || f <= fq - W) continue;   // outside the causal window of query qi
-      const float m_new = fmaxf(m[qi], sc[qi]);
-      const float alpha = ex2_approx(m[qi] - m_new);
-      const float pr = ex2_approx(sc[qi] - m_new);
-      l[qi] = fmaf(l[qi], alpha, pr);
+        for (int e = 0; e < 8; ++e) d = fmaf(q[qi][e], kf[e], d);
+        sc[qi] = d;
+      }
 #pragma unroll
-      for (int e = 0; e < 8; ++e) o[qi][e] = fmaf(o[qi][e], alpha, pr * vf[e]);
-      m[qi] = m_new;
+      for (int off = 1; off < 8; off <<= 1) {
+#pragma unroll
+        for (int qi = 0; qi < NQ; ++qi) sc[qi] += __shfl_xor_sync(0xffffffffu, sc[qi], off);
+      }
+      if (kk >= total) continue;
+      const float vf[8] = {bf16lo(vw[u].x), bf16hi(vw[u].x), bf16lo(vw[u].y), bf16hi(vw[u].y),
+                           bf16lo(vw[u].z), bf16hi(vw[u].z), bf16lo(vw[u].w), bf16hi(vw[u].w)};
+      const int64_t f = f0 + kk;   // absolute frame of this key
+#pragma unroll
+      for (int qi = 0; qi < NQ; ++qi) {
+        const int64_t fq = p + qi;
+        if (f > fq || f <= fq - W) continue;   // outside the causal window of query qi
+        const float m_new = fmaxf(m[qi], sc[qi]);
+        const float alpha = ex2_approx(m[qi] - m_new);
+        const float pr = ex2_approx(sc[qi] - m_new);
+        l[qi] = fmaf(l[qi], alpha, pr);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) o[qi][e] = fmaf(o[qi][e], alpha, pr * vf[e]);
+        m[qi] = m_new;
+      }
     }
   }
 
@@ -183,6 +196,8 @@ ring_attn_kernel(const uint16_t* __restrict__ qkv, int64_t ld_qkv, int HD,
 __global__ void ring_fill_kernel(const uint16_t* __restrict__ qkv, int64_t ld_qkv, int HD,
                                  uint16_t* __restrict__ ring_k, uint16_t* __restrict__ ring_v,
                                  int T, int H, int W, int first) {
+  pdl_wait();
+  pdl_trigger();
   const int f = first + blockIdx.x;
   const int s = blockIdx.y;
   const int slot = f % W;
@@ -198,6 +213,8 @@ __global__ void ring_fill_kernel(const uint16_t* __restrict__ qkv, int64_t ld_qk
 }
 
 __global__ void pos_add_kernel(int64_t* pos, int S, int64_t n, int set) {
+  pdl_wait();
+  pdl_trigger();
   const int s = blockIdx.x * blockDim.x + threadIdx.x;
   if (s < S) pos[s] = set ? n : pos[s] + n;
 }
@@ -205,8 +222,8 @@ __global__ void pos_add_kernel(int64_t* pos, int S, int64_t n, int set) {
 template <int NQ>
 cudaError_t launch_ring_nq(const Launch& L, const uint16_t* qkv, int64_t ld_qkv, int HD, uint16_t* rk,
                            uint16_t* rv, const int64_t* pos, int S, int H, int W, uint16_t* out, float sl2) {
-  ring_attn_kernel<NQ><<<dim3(H, S), kRingThreads, 0, L.stream>>>(qkv, ld_qkv, HD, rk, rv, pos, H, W, out, sl2);
-  return cudaGetLastError();
+  return launch_kernel(ring_attn_kernel<NQ>, dim3(H, S), dim3(kRingThreads), 0, L.stream, qkv, ld_qkv, HD, rk, rv,
+                       pos, H, W, out, sl2);
 }
 
 }  // namespace
@@ -232,13 +249,12 @@ cudaError_t launch_ring_fill(const Launch& L, const uint16_t* qkv, int64_t ld_qk
   const int first = T > W ? T - W : 0;
   const int nf = T - first;
   if (nf <= 0 || S <= 0) return cudaSuccess;
-  ring_fill_kernel<<<dim3(nf, S), 256, 0, L.stream>>>(qkv, ld_qkv, HD, ring_k, ring_v, T, H, W, first);
-  return cudaGetLastError();
+  return launch_kernel(ring_fill_kernel, dim3(nf, S), dim3(256), 0, L.stream, qkv, ld_qkv, HD, ring_k, ring_v, T, H,
+                       W, first);
 }
 
 cudaError_t launch_pos_add(const Launch& L, int64_t* pos, int S, int64_t n, bool set) {
-  pos_add_kernel<<<(S + 127) / 128, 128, 0, L.stream>>>(pos, S, n, set ? 1 : 0);
-  return cudaGetLastError();
+  return launch_kernel(pos_add_kernel, dim3((S + 127) / 128), dim3(128), 0, L.stream, pos, S, n, set ? 1 : 0);
 }
 
 }  // namespace vx

@@ -234,6 +234,14 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr, uint32_t lbo
   return d;
 }
 
+// ------------------------------------------------- programmatic launch --
+// With programmatic dependent launch, a kernel may start while the previous
+// kernel of the stream is still running; pdl_wait() blocks until that kernel
+// has completed and its memory is visible (a no-op without the attribute).
+// pdl_trigger() lets the next kernel of the stream begin its prologue.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // ------------------------------------------------------------------ bf16 --
 __device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }

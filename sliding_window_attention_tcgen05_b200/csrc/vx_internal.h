@@ -6,6 +6,7 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 #include <string>
+#include <utility>
 
 #include "vx_common.cuh"
 
@@ -25,6 +26,24 @@ struct Launch {
 
 int current_sm_count();
 uint64_t wait_limit_ns();
+bool pdl_enabled();   // programmatic dependent launch (default on; VX_PDL=0 disables)
+
+// Launches `k` on `stream`, with programmatic dependent launch when enabled.
+template <class... KArgs, class... Args>
+cudaError_t launch_kernel(void (*k)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                          Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl_enabled() ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, k, std::forward<Args>(args)...);
+}
 
 // cuTensorMapEncodeTiled through the runtime's driver entry point (no -lcuda).
 bool encode_tmap(CUtensorMap* map, CUtensorMapDataType dt, int rank, const void* base,
@@ -47,6 +66,10 @@ enum EpiKind : int {
 
 struct GemmArgs {
   int M, N, K;
+  // Split-K: the K loop is cut into k_splits equal parts; part ks writes its
+  // fp32 partial sums (EPI_F32, no bias / residual) at out + ks * split_stride.
+  int k_splits;
+  int64_t split_stride;
   // A addressing of K-block kb (64 wide): tap = kb / kb_per_tap,
   // c = (kb % kb_per_tap) * 64, x = (tap % a_stride) * a_tap_ch + c, y = m0 + tap / a_stride.
   int kb_per_tap, a_stride, a_tap_ch;
@@ -70,7 +93,8 @@ struct GemmArgs {
 
 // D[M, N] = A[M, K] * B[N, K]^T with the given epilogue.  tmA/tmB must be 2-D
 // bf16 maps with 128-byte swizzle and box {64, 128} (A) / {64, bn} (B).
-// bn in {128, 256}; N % bn == 0; K % 64 == 0.
+// bn in {64, 128, 256} (EPI_SWIGLU: 128 or 256); N % bn == 0; K % 64 == 0;
+// (K / 64) % k_splits == 0.
 cudaError_t launch_gemm(const Launch& L, const CUtensorMap& tmA, const CUtensorMap& tmB,
                         const GemmArgs& args, int epi, int bn);
 
@@ -100,8 +124,11 @@ cudaError_t launch_rope(const Launch& L, const void* x, void* y, bool bf16, int 
                         int64_t pos0, float theta);
 
 // ---------------------------------------------------------------- others --
-cudaError_t launch_rmsnorm(const Launch& L, const float* x, const float* r, const uint16_t* g,
-                           float* h_out, void* y, bool y_bf16, int M, int d, float eps);
+// h = x + bias + sum_{k < nparts} parts[k * part_stride + .]  (parts/bias optional);
+// h_out (optional) = h; y (optional, with g) = h * rsqrt(mean(h^2) + eps) * g.
+cudaError_t launch_rmsnorm(const Launch& L, const float* x, const float* parts, int nparts, int64_t part_stride,
+                           const uint16_t* bias, const uint16_t* g, float* h_out, void* y, bool y_bf16, int M,
+                           int d, float eps);
 
 // Ring attention of one layer of a streaming step (see vx_stream_step).
 cudaError_t launch_ring_attn(const Launch& L, const uint16_t* qkv, int64_t ld_qkv, int HD,
