@@ -263,7 +263,7 @@ int pick_splits(int M, int N, int K, int bn, int sm) {
   const int nkb = K / 64;
   int s = 1;
   for (int c = 2; c <= 8; c *= 2)
-    if (nkb % c == 0 && nkb / c >= 4 && units * c <= sm + sm / 8) s = c;
+    if (nkb % c == 0 && nkb / c >= 4 && units * c <= sm) s = c;
   return s;
 }
 
@@ -280,12 +280,12 @@ GemmArgs base_args(const Launch& L, int M, int N, int K) {
 }
 
 vx_status gemm(const Launch& L, const char* name, const void* A, int64_t lda, const void* Bw, GemmArgs& a, int epi,
-               int bn = 0) {
+               int bn = 0, bool lean = false) {
   if (bn == 0) bn = pick_bn(a.M, a.N, L.sm_count);
   CUtensorMap tmA, tmB;
   if (!tmap_bf16_2d(&tmA, A, a.K, a.M, lda, 128)) return VX_ERR_CUDA;
   if (!tmap_bf16_2d(&tmB, Bw, a.K, a.N, a.K, bn)) return VX_ERR_CUDA;
-  VX_CUDA(traced(L, name, 1, [&] { return launch_gemm(L, tmA, tmB, a, epi, bn); }));
+  VX_CUDA(traced(L, name, 1, [&] { return launch_gemm(L, tmA, tmB, a, epi, bn, lean); }));
   return VX_OK;
 }
 
@@ -408,6 +408,7 @@ vx_status run_layer_stream(const Launch& L, const vx_layer_cfg& c, const vx_laye
   const int64_t pstride = static_cast<int64_t>(M) * d;
   const float sl2 = (1.0f / std::sqrt(static_cast<float>(c.head_dim))) * 1.4426950408889634f;
   const LayerBufs& bf = sb.lb;
+  const int slots = 2 * L.sm_count;   // lean GEMMs: two CTAs per SM
   vx_status st;
   // 1. x_l = reduce(in); y0 = RMSNorm(x_l)
   const bool pending_in = in.parts != nullptr || in.bias != nullptr;
@@ -426,7 +427,8 @@ vx_status run_layer_stream(const Launch& L, const vx_layer_cfg& c, const vx_laye
     a.pos_arr = ring.pos;
     a.rope_cols = 2 * HD;
     fill_rope_freqs(&a, c.rope_theta, c.head_dim);
-    if ((st = gemm(L, "gemm_qkv_rope", bf.y0, d, w.wqkv, a, EPI_QKV_ROPE, pick_bn(M, 3 * HD, L.sm_count, 64))) != VX_OK)
+    if ((st = gemm(L, "gemm_qkv_rope", bf.y0, d, w.wqkv, a, EPI_QKV_ROPE, pick_bn(M, 3 * HD, slots, 64), true)) !=
+        VX_OK)
       return st;
   }
   // 3. ring attention (reads every old in-window slot, then appends)
@@ -436,12 +438,12 @@ vx_status run_layer_stream(const Launch& L, const vx_layer_cfg& c, const vx_laye
   // 4. O-projection, split-K partial sums
   int so;
   {
-    const int bn = pick_bn(M, d, L.sm_count, 64);
-    so = pick_splits(M, d, HD, bn, L.sm_count);
+    const int bn = pick_bn(M, d, slots, 64);
+    so = pick_splits(M, d, HD, bn, slots);
     GemmArgs a = base_args(L, M, d, HD);
     a.out = sb.parts; a.ld_out = d;
     a.k_splits = so; a.split_stride = pstride;
-    if ((st = gemm(L, "gemm_o_splitk", bf.att, HD, w.wo, a, EPI_F32, bn)) != VX_OK) return st;
+    if ((st = gemm(L, "gemm_o_splitk", bf.att, HD, w.wo, a, EPI_F32, bn, true)) != VX_OK) return st;
   }
   // 5. h = x_l + bo + sum P_o; y1 = RMSNorm(h)
   VX_CUDA(traced(L, "rmsnorm", 1, [&] {
@@ -453,18 +455,16 @@ vx_status run_layer_stream(const Launch& L, const vx_layer_cfg& c, const vx_laye
     GemmArgs a = base_args(L, M, 2 * F, d);
     a.out = bf.act; a.ld_out = F;
     a.bias = static_cast<const uint16_t*>(w.bgu);
-    if ((st = gemm(L, "gemm_gate_up_swiglu", bf.y0, d, w.wgu, a, EPI_SWIGLU, pick_bn(M, 2 * F, L.sm_count, 128))) !=
-        VX_OK)
-      return st;
+    if ((st = gemm(L, "gemm_gate_up_swiglu", bf.y0, d, w.wgu, a, EPI_SWIGLU, 128, true)) != VX_OK) return st;
   }
   // 7. down, split-K partial sums; the layer output stays pending
   {
-    const int bn = pick_bn(M, d, L.sm_count, 64);
-    const int sd = pick_splits(M, d, F, bn, L.sm_count);
+    const int bn = pick_bn(M, d, slots, 64);
+    const int sd = pick_splits(M, d, F, bn, slots);
     GemmArgs a = base_args(L, M, d, F);
     a.out = sb.parts; a.ld_out = d;
     a.k_splits = sd; a.split_stride = pstride;
-    if ((st = gemm(L, "gemm_down_splitk", bf.act, F, w.wd, a, EPI_F32, bn)) != VX_OK) return st;
+    if ((st = gemm(L, "gemm_down_splitk", bf.act, F, w.wd, a, EPI_F32, bn, true)) != VX_OK) return st;
     *out = Pending{bf.h, sb.parts, sd, static_cast<const uint16_t*>(w.bd)};
   }
   return VX_OK;

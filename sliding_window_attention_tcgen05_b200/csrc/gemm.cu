@@ -23,11 +23,13 @@ constexpr int kBM = 128;
 constexpr int kBK = 64;
 constexpr int kABytes = kBM * kBK * 2;
 
-template <int BN>
+// LEAN: about 96 KB of pipeline so that two CTAs share an SM (few-row GEMMs,
+// whose work units must all be resident in one round).
+template <int BN, bool LEAN>
 struct GemmCfg {
-  static constexpr int kStages = (BN == 256) ? 4 : (BN == 128 ? 6 : 8);
   static constexpr int kBBytes = BN * kBK * 2;
   static constexpr int kStageBytes = kABytes + kBBytes;
+  static constexpr int kStages = LEAN ? (96 * 1024) / kStageBytes : ((BN == 256) ? 4 : (BN == 128 ? 6 : 8));
   static constexpr int kTmemCols = 2 * BN;  // two accumulators
   static constexpr int kSmem = kStages * kStageBytes + 1024 + 256;
 };
@@ -75,7 +77,33 @@ __device__ __forceinline__ void epilogue_tile(const GemmArgs& a, uint32_t tacc, 
   const bool valid = in_range && t < a.t_valid;
   const int64_t drow = static_cast<int64_t>(b) * a.out_rows + a.out_off + t;
 
-  if constexpr (EPI == EPI_QKV_ROPE) {
+  if constexpr (EPI == EPI_QKV_ROPE && BN == 64) {
+    // one head per tile: rotate while reading (no sin/cos table kept)
+    uint32_t r0[32], r1[32];
+    tmem_ld32(tacc, r0);
+    tmem_ld32(tacc + 32, r1);
+    tmem_ld_wait();
+    if (valid) {
+      float x0[32], x1[32];
+#pragma unroll
+      for (int i = 0; i < 32; ++i) { x0[i] = __uint_as_float(r0[i]); x1[i] = __uint_as_float(r1[i]); }
+      if (a.bias) { add_bias32(x0, a.bias + n0); add_bias32(x1, a.bias + n0 + 32); }
+      if (n0 < a.rope_cols) {
+        const float posf = static_cast<float>((a.pos_arr ? a.pos_arr[b] : a.pos0) + t);
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          float sn, cs;
+          rope_sincos(posf, a.inv_freq_hi[j], a.inv_freq_lo[j], &sn, &cs);
+          const float u = x0[j], w = x1[j];
+          x0[j] = u * cs - w * sn;
+          x1[j] = w * cs + u * sn;
+        }
+      }
+      uint16_t* dst = static_cast<uint16_t*>(a.out) + drow * a.ld_out + n0;
+      store_bf16x32(dst, x0);
+      store_bf16x32(dst + 32, x1);
+    }
+  } else if constexpr (EPI == EPI_QKV_ROPE) {
     float cs[32], sn[32];
     const bool rope_tile = n0 < a.rope_cols;
     if (rope_tile && valid) {
@@ -166,11 +194,11 @@ __device__ __forceinline__ void epilogue_tile(const GemmArgs& a, uint32_t tacc, 
   }
 }
 
-template <int BN, int EPI>
-__global__ void __launch_bounds__(kThreads, 1)
+template <int BN, int EPI, bool LEAN>
+__global__ void __launch_bounds__(kThreads, LEAN ? 2 : 1)
 gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                const __grid_constant__ GemmArgs a) {
-  using C = GemmCfg<BN>;
+  using C = GemmCfg<BN, LEAN>;
   constexpr int S = C::kStages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -321,33 +349,38 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
   }
 }
 
-template <int BN, int EPI>
+template <int BN, int EPI, bool LEAN>
 cudaError_t launch_one(const Launch& L, const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmArgs& a) {
-  using C = GemmCfg<BN>;
+  using C = GemmCfg<BN, LEAN>;
   static bool attr_set = false;  // per instantiation; benign race (idempotent call)
   if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<BN, EPI>,
+    cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<BN, EPI, LEAN>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
   const int m_tiles = (a.M + kBM - 1) / kBM;
   const int tiles = m_tiles * (a.N / BN) * a.k_splits;
-  const int grid = tiles < L.sm_count ? tiles : L.sm_count;
-  return launch_kernel(gemm_tc_kernel<BN, EPI>, dim3(grid), dim3(kThreads), C::kSmem, L.stream, tmA, tmB, a);
+  const int slots = (LEAN ? 2 : 1) * L.sm_count;
+  const int grid = tiles < slots ? tiles : slots;
+  return launch_kernel(gemm_tc_kernel<BN, EPI, LEAN>, dim3(grid), dim3(kThreads), C::kSmem, L.stream, tmA, tmB, a);
 }
 
-template <int BN>
+template <int BN, bool LEAN>
 cudaError_t launch_bn(const Launch& L, const CUtensorMap& tmA, const CUtensorMap& tmB,
                       const GemmArgs& a, int epi) {
   switch (epi) {
-    case EPI_F32: return launch_one<BN, EPI_F32>(L, tmA, tmB, a);
-    case EPI_QKV_ROPE: return launch_one<BN, EPI_QKV_ROPE>(L, tmA, tmB, a);
+    case EPI_F32: return launch_one<BN, EPI_F32, LEAN>(L, tmA, tmB, a);
+    case EPI_QKV_ROPE: return launch_one<BN, EPI_QKV_ROPE, LEAN>(L, tmA, tmB, a);
     case EPI_SWIGLU:
-      if constexpr (BN >= 128) return launch_one<BN, EPI_SWIGLU>(L, tmA, tmB, a);
+      if constexpr (BN >= 128) return launch_one<BN, EPI_SWIGLU, LEAN>(L, tmA, tmB, a);
       else return cudaErrorInvalidValue;
-    case EPI_GELU_BF16: return launch_one<BN, EPI_GELU_BF16>(L, tmA, tmB, a);
-    case EPI_GELU_F32: return launch_one<BN, EPI_GELU_F32>(L, tmA, tmB, a);
+    case EPI_GELU_BF16:
+      if constexpr (!LEAN) return launch_one<BN, EPI_GELU_BF16, LEAN>(L, tmA, tmB, a);
+      else return cudaErrorInvalidValue;
+    case EPI_GELU_F32:
+      if constexpr (!LEAN) return launch_one<BN, EPI_GELU_F32, LEAN>(L, tmA, tmB, a);
+      else return cudaErrorInvalidValue;
     default: return cudaErrorInvalidValue;
   }
 }
@@ -355,12 +388,17 @@ cudaError_t launch_bn(const Launch& L, const CUtensorMap& tmA, const CUtensorMap
 }  // namespace
 
 cudaError_t launch_gemm(const Launch& L, const CUtensorMap& tmA, const CUtensorMap& tmB,
-                        const GemmArgs& args, int epi, int bn) {
+                        const GemmArgs& args, int epi, int bn, bool lean) {
   if (args.M <= 0) return cudaSuccess;
   if (args.k_splits < 1 || (args.K / kBK) % args.k_splits != 0) return cudaErrorInvalidValue;
-  if (bn == 256) return launch_bn<256>(L, tmA, tmB, args, epi);
-  if (bn == 128) return launch_bn<128>(L, tmA, tmB, args, epi);
-  if (bn == 64) return launch_bn<64>(L, tmA, tmB, args, epi);
+  if (lean) {
+    if (bn == 128) return launch_bn<128, true>(L, tmA, tmB, args, epi);
+    if (bn == 64) return launch_bn<64, true>(L, tmA, tmB, args, epi);
+    return cudaErrorInvalidValue;
+  }
+  if (bn == 256) return launch_bn<256, false>(L, tmA, tmB, args, epi);
+  if (bn == 128) return launch_bn<128, false>(L, tmA, tmB, args, epi);
+  if (bn == 64) return launch_bn<64, false>(L, tmA, tmB, args, epi);
   return cudaErrorInvalidValue;
 }
 

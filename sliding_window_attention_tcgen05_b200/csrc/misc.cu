@@ -73,6 +73,51 @@ rmsnorm_kernel(const float* __restrict__ x, const float* __restrict__ parts, int
   }
 }
 
+// Few-row variant: one CTA of d/4 threads per row (one float4 each), so that a
+// handful of rows still spreads over the SMs; same arithmetic as above.
+template <bool BF16_OUT>
+__global__ void __launch_bounds__(512)
+rmsnorm_row_kernel(const float* __restrict__ x, const float* __restrict__ parts, int nparts, int64_t part_stride,
+                   const uint16_t* __restrict__ bias, const uint16_t* __restrict__ g, float* __restrict__ h_out,
+                   void* __restrict__ y, int M, int d, float eps) {
+  __shared__ float red[16];
+  pdl_wait();
+  pdl_trigger();
+  const int row = blockIdx.x;
+  const int c4 = threadIdx.x;
+  const int64_t roff = static_cast<int64_t>(row) * d;
+  float4 a = reinterpret_cast<const float4*>(x + roff)[c4];
+  for (int k = 0; k < nparts; ++k) {
+    const float4 b = reinterpret_cast<const float4*>(parts + k * part_stride + roff)[c4];
+    a.x += b.x; a.y += b.y; a.z += b.z; a.w += b.w;
+  }
+  if (bias) {
+    const uint2 bw = __ldg(reinterpret_cast<const uint2*>(bias) + c4);
+    a.x += bf16lo(bw.x); a.y += bf16hi(bw.x); a.z += bf16lo(bw.y); a.w += bf16hi(bw.y);
+  }
+  if (h_out) reinterpret_cast<float4*>(h_out + roff)[c4] = a;
+  if (y == nullptr) return;   // uniform over the CTA
+  float ss = fmaf(a.x, a.x, fmaf(a.y, a.y, fmaf(a.z, a.z, a.w * a.w)));
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = ss;
+  __syncthreads();
+  float tot = 0.f;
+  for (int w = 0; w < static_cast<int>(blockDim.x >> 5); ++w) tot += red[w];
+  const float inv = rsqrtf(tot / static_cast<float>(d) + eps);
+  const uint2 gw = __ldg(reinterpret_cast<const uint2*>(g) + c4);
+  const float o0 = a.x * inv * bf16lo(gw.x), o1 = a.y * inv * bf16hi(gw.x);
+  const float o2 = a.z * inv * bf16lo(gw.y), o3 = a.w * inv * bf16hi(gw.y);
+  if constexpr (BF16_OUT) {
+    uint2 w;
+    w.x = pack_bf16x2(o0, o1);
+    w.y = pack_bf16x2(o2, o3);
+    reinterpret_cast<uint2*>(static_cast<uint16_t*>(y) + roff)[c4] = w;
+  } else {
+    reinterpret_cast<float4*>(static_cast<float*>(y) + roff)[c4] = make_float4(o0, o1, o2, o3);
+  }
+}
+
 // ---------------------------------------------------------------- packing --
 // Row gather: output row rr (of `cols` bf16) comes from src_of(rr) or is zero.
 struct PackSrc {
@@ -185,6 +230,14 @@ cudaError_t launch_rmsnorm(const Launch& L, const float* x, const float* parts, 
                            const uint16_t* bias, const uint16_t* g, float* h_out, void* y, bool y_bf16, int M,
                            int d, float eps) {
   if (M <= 0) return cudaSuccess;
+  if (M <= 2048) {   // few rows: a CTA per row
+    const dim3 threads(d / 4);
+    if (y_bf16)
+      return launch_kernel(rmsnorm_row_kernel<true>, dim3(M), threads, 0, L.stream, x, parts, nparts, part_stride,
+                           bias, g, h_out, y, M, d, eps);
+    return launch_kernel(rmsnorm_row_kernel<false>, dim3(M), threads, 0, L.stream, x, parts, nparts, part_stride,
+                         bias, g, h_out, y, M, d, eps);
+  }
   const dim3 blocks((M + 7) / 8);
   if (y_bf16)
     return launch_kernel(rmsnorm_kernel<true>, blocks, dim3(256), 0, L.stream, x, parts, nparts, part_stride, bias,

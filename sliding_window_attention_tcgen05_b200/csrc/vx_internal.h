@@ -95,8 +95,9 @@ struct GemmArgs {
 // bf16 maps with 128-byte swizzle and box {64, 128} (A) / {64, bn} (B).
 // bn in {64, 128, 256} (EPI_SWIGLU: 128 or 256); N % bn == 0; K % 64 == 0;
 // (K / 64) % k_splits == 0.
+// lean: a ~96 KB pipeline so two CTAs share an SM (bn 64 or 128; no GELU).
 cudaError_t launch_gemm(const Launch& L, const CUtensorMap& tmA, const CUtensorMap& tmB,
-                        const GemmArgs& args, int epi, int bn);
+                        const GemmArgs& args, int epi, int bn, bool lean = false);
 
 void fill_rope_freqs(GemmArgs* a, float theta, int head_dim);
 
