@@ -170,13 +170,14 @@ VX_API size_t vx_swa_attn_workspace(vx_dtype dt, int B, int T, int H, int D, int
  * run attention (real-time audio callbacks that must not wait on the
  * driver's allocator, plug-in hosts that own every device allocation, code
  * under a fixed memory budget).  It takes no workspace and allocates nothing:
- * its scratch (the RoPE-rotated q and k, and the status word of the bounded
- * waits) is one static device array of 32 MiB + 256 bytes inside this
- * library, held by every GPU that loads the library until the process exits.
- * Inputs and outputs are still the caller's.
- * Limit: with apply_rope, B*T*H*64 elements of q plus as many of k must fit in
- * 32 MiB (B*T*H <= 131072 for bf16, 65536 for fp32); larger calls return
- * VX_ERR_INVALID_ARG with a message and enqueue nothing.
+ * its scratch (the RoPE-rotated q and k, their per-position cos/sin table,
+ * and the status word of the bounded waits) is one static device array of
+ * 32 MiB + 256 bytes inside this library, held by every GPU that loads the
+ * library until the process exits.  Inputs and outputs are still the caller's.
+ * Limit: with apply_rope, the rotated q and k (2 * B*T*H*64 elements) plus
+ * T * 256 bytes of table must fit in 32 MiB (about B*T*H <= 126000 for bf16,
+ * half that for fp32); larger calls return VX_ERR_INVALID_ARG with a message
+ * and enqueue nothing.
  * The first call on each device looks up the array's device address (with
  * that device current) and caches it; make that first call before any stream
  * capture.  Every call clears the status word and overwrites the rotated q/k,

@@ -1,15 +1,15 @@
 // attn.cu -- causal sliding-window attention kernels.
 //
 // swa_attn_tc_kernel: flash-style bf16 attention on tcgen05 tensor cores.
-//   One CTA per (128-query tile, head, clip).  Only the key tiles that meet
-//   the causal window (i - W, i] of some query of the tile are visited; the
-//   masks are evaluated only on the edge tiles.  K/V tiles arrive by TMA into
-//   a 3-stage ring; S = Q K^T and O_j = P_j V_j accumulate in TMEM
-//   (S double-buffered in columns 0..255, O_j in 256..383); the softmax warps
-//   read S from TMEM, keep the running max / sum in registers, write P (bf16)
-//   to shared memory as the A operand of the P V product, and fold each O_j
-//   into a register accumulator with the online-softmax rescale.
-//   Warps 0-3: softmax (TMEM lane = query row), warp 4: TMA, warp 5: MMA.
+//   One CTA per (two adjacent 128-query tiles, head, clip); the two softmax
+//   warpgroups ping-pong against one MMA warp and share every K/V tile.  Only
+//   the key tiles that meet the causal window (i - W, i] of some query are
+//   visited; the masks are evaluated only on the edge tiles.  K/V tiles arrive
+//   by TMA into a 3-stage ring; S = Q K^T and O_j = P_j V_j accumulate in
+//   TMEM; the softmax warps read S from TMEM (two passes: max, then
+//   exponentials), keep the running max / sum in registers, write P (bf16) to
+//   shared memory as the A operand of the P V product, and fold each O_j into
+//   a register accumulator with the online-softmax rescale.
 // swa_attn_f32_kernel: fp32 CUDA-core reference-precision path (one warp per
 //   query row), used for fp32 inputs.
 // rope_kernel: RoPE pre-pass for vx_swa_attn_fwd on raw q, k.
@@ -21,58 +21,84 @@ namespace vx {
 
 namespace {
 
-constexpr int kAttnThreads = 192;
+constexpr int kAttnThreads = 320;           // 2 softmax warpgroups, TMA warp, MMA warp
 constexpr int kNS = 3;                      // K/V pipeline stages
 constexpr int kTile = 128 * 64 * 2;         // one 128 x 64 bf16 tile
 constexpr int kPBytes = 128 * 128 * 2;      // one P tile (128 queries x 128 keys)
-constexpr int kAttnSmem = kTile * (1 + 2 * kNS) + 2 * kPBytes + 1024 + 512;
+constexpr int kAttnSmem = kTile * (2 + 2 * kNS) + 2 * kPBytes + 1024 + 512;
 constexpr uint32_t kTmemCols = 512;
 
+// Max / sum of 32 values as a balanced tree (short dependency chains).
+__device__ __forceinline__ float tree_max32(const float (&v)[32]) {
+  float t[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) t[i] = fmaxf(v[i], v[i + 16]);
+#pragma unroll
+  for (int w = 8; w >= 1; w >>= 1)
+#pragma unroll
+    for (int i = 0; i < w; ++i) t[i] = fmaxf(t[i], t[i + w]);
+  return t[0];
+}
+
+// One CTA per (two adjacent 128-query tiles X = 0, 1; head; clip).  Key tiles
+// of 128 are visited from the first one meeting tile 0's window to the
+// diagonal of tile 1, each loaded once by TMA and used by both query tiles.
+// TMEM columns: S_X at 128 X, O_X double buffer at 256 + 128 X + 64 j.
+// Warps 0-3 / 4-7: softmax of tile 0 / 1 (TMEM lane = query row), warp 8:
+// TMA, warp 9: MMA (S_X = Q_X K^T and O_X,j = P_X V_j).
 __global__ void __launch_bounds__(kAttnThreads, 1)
 swa_attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                    const __grid_constant__ CUtensorMap tmV, const __grid_constant__ AttnArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* sQ = smem;
-  uint8_t* sK = sQ + kTile;
+  uint8_t* sQ = smem;                       // Q_0 | Q_1
+  uint8_t* sK = sQ + 2 * kTile;
   uint8_t* sV = sK + kNS * kTile;
-  uint8_t* sP = sV + kNS * kTile;
+  uint8_t* sP = sV + kNS * kTile;           // P_0 | P_1
   uint64_t* bars = reinterpret_cast<uint64_t*>(sP + 2 * kPBytes);
-  // barrier indices
-  constexpr int QF = 0, KF = 1, VF = KF + kNS, KVE = VF + kNS, SF = KVE + kNS, SE = SF + 2,
-                PF = SE + 2, PE = PF + 2, OF = PE + 2, OE = OF + 2, DR = OE + 2, NBAR = DR + 1;
+  // barrier indices (per query tile X where doubled)
+  constexpr int QF = 0, KF = 1, VF = KF + kNS, KVE = VF + kNS, SF = KVE + kNS, SE = SF + 2, PF = SE + 2,
+                PE = PF + 2, OF = PE + 2, OE = OF + 4, DR = OE + 4, NBAR = DR + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + NBAR);
   int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
   auto bar = [&](int i) { return smem_addr(bars + i); };
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int q0 = blockIdx.x * 128;
+  const int q0 = blockIdx.x * 256;
   const int h = blockIdx.y;
   const int b = blockIdx.z;
   const int W = a.window;
-  const int lo_key = max(0, q0 - W + 1);
-  const int hi_key = min(a.T - 1, q0 + 127);
-  const int kt0 = lo_key / 128;
-  const int n = hi_key / 128 - kt0 + 1;
+  const int T = a.T;
+  const bool has1 = q0 + 128 < T;
+  // key-tile ranges of the two query tiles
+  const int kt0[2] = {max(0, q0 - W + 1) / 128, max(0, q0 + 128 - W + 1) / 128};
+  const int kt1[2] = {min(T - 1, q0 + 127) / 128, min(T - 1, q0 + 255) / 128};
+  const int klo = kt0[0];
+  const int khi = has1 ? kt1[1] : kt1[0];
+  const int nu = khi - klo + 1;
+  auto valid = [&](int X, int u) {
+    const int kt = klo + u;
+    return (X == 0 || has1) && kt >= kt0[X] && kt <= kt1[X];
+  };
 
   if (threadIdx.x == 0) {
     mbar_init(bar(QF), 1);
     for (int s = 0; s < kNS; ++s) { mbar_init(bar(KF + s), 1); mbar_init(bar(VF + s), 1); mbar_init(bar(KVE + s), 1); }
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(bar(SF + i), 1); mbar_init(bar(SE + i), 128);
-      mbar_init(bar(PF + i), 128); mbar_init(bar(PE + i), 1);
-      mbar_init(bar(OF + i), 1); mbar_init(bar(OE + i), 128);
+    for (int X = 0; X < 2; ++X) {
+      mbar_init(bar(SF + X), 1); mbar_init(bar(SE + X), 128);
+      mbar_init(bar(PF + X), 128); mbar_init(bar(PE + X), 1);
+      for (int j = 0; j < 2; ++j) { mbar_init(bar(OF + 2 * X + j), 1); mbar_init(bar(OE + 2 * X + j), 128); }
     }
     mbar_init(bar(DR), 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
-  if (warp == 5) {
+  if (warp == 9) {
     tmem_alloc(smem_addr(tmem_slot), kTmemCols);
     tmem_relinquish();
   }
-  if (warp == 4 && lane == 0) {
+  if (warp == 8 && lane == 0) {
     tma_prefetch_desc(&tmQ); tma_prefetch_desc(&tmK); tma_prefetch_desc(&tmV);
   }
   tc_fence_before();
@@ -83,23 +109,24 @@ swa_attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
   pdl_wait();
   pdl_trigger();
 
-  if (warp == 4) {
+  if (warp == 8) {
     if (lane == 0) {
-      mbar_arrive_expect_tx(bar(QF), kTile);
+      mbar_arrive_expect_tx(bar(QF), has1 ? 2 * kTile : kTile);
       tma_load_4d(smem_addr(sQ), &tmQ, bar(QF), 0, h, q0, b);
+      if (has1) tma_load_4d(smem_addr(sQ + kTile), &tmQ, bar(QF), 0, h, q0 + 128, b);
       uint32_t last_par = 0;
       int filled = 0;
-      for (int j = 0; j < n; ++j) {
-        const int st = j % kNS;
-        const uint32_t ph = (j / kNS) & 1;
+      for (int u = 0; u < nu; ++u) {
+        const int st = u % kNS;
+        const uint32_t ph = (u / kNS) & 1;
         if (!mbar_wait(bar(KVE + st), ph ^ 1, wc, 11)) break;
-        const int key0 = (kt0 + j) * 128;
+        const int key0 = (klo + u) * 128;
         mbar_arrive_expect_tx(bar(KF + st), kTile);
         tma_load_4d(smem_addr(sK + st * kTile), &tmK, bar(KF + st), 0, h, key0, b);
         mbar_arrive_expect_tx(bar(VF + st), kTile);
         tma_load_4d(smem_addr(sV + st * kTile), &tmV, bar(VF + st), 0, h, key0, b);
         last_par = (last_par & ~(1u << st)) | (ph << st);
-        filled = j + 1;
+        filled = u + 1;
       }
       // Bounded wait for every copy still in flight (also after an abort).
       int zero = 0;
@@ -111,48 +138,58 @@ swa_attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
         mbar_wait(bar(VF + s), (last_par >> s) & 1u, dw, 12);
       }
     }
-  } else if (warp == 5) {
+  } else if (warp == 9) {
     if (lane == 0) {
       const uint32_t idesc_s = idesc_bf16_f32(128, 128, 0);
       const uint32_t idesc_o = idesc_bf16_f32(128, 64, 1);
       bool ok = mbar_wait(bar(QF), 0, wc, 13);
-      const uint32_t qa = smem_addr(sQ);
-      auto issue_pv = [&](int jj) -> bool {
-        const int st = jj % kNS;
-        const int pb = jj & 1;
-        const uint32_t pph = (jj >> 1) & 1;
-        if (!mbar_wait(bar(PF + pb), pph, wc, 14)) return false;
-        if (!mbar_wait(bar(VF + st), (jj / kNS) & 1, wc, 15)) return false;
-        if (!mbar_wait(bar(OE + pb), pph ^ 1, wc, 16)) return false;
+      int js[2] = {0, 0};   // S products issued per query tile
+      int jo[2] = {0, 0};   // P V products issued per query tile
+      auto issue_s = [&](int X, int u) -> bool {
+        const int st = u % kNS;
+        if (!mbar_wait(bar(SE + X), (js[X] & 1) ^ 1, wc, 17)) return false;
+        if (!mbar_wait(bar(KF + st), (u / kNS) & 1, wc, 18)) return false;
         tc_fence_after();
-        const uint32_t pa = smem_addr(sP + pb * kPBytes);
+        const uint32_t qa = smem_addr(sQ + X * kTile);
+        const uint32_t ka = smem_addr(sK + st * kTile);
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+          umma_bf16(tmem + X * 128, smem_desc_sw128(qa + 32 * k, 16, 1024), smem_desc_sw128(ka + 32 * k, 16, 1024),
+                    idesc_s, k > 0);
+        umma_commit(bar(SF + X));
+        ++js[X];
+        return true;
+      };
+      auto issue_pv = [&](int X, int u) -> bool {
+        const int st = u % kNS;
+        const int j = jo[X];
+        const int ob = j & 1;
+        if (!mbar_wait(bar(PF + X), j & 1, wc, 14)) return false;
+        if (!mbar_wait(bar(VF + st), (u / kNS) & 1, wc, 15)) return false;
+        if (!mbar_wait(bar(OE + 2 * X + ob), ((j >> 1) & 1) ^ 1, wc, 16)) return false;
+        tc_fence_after();
+        const uint32_t pa = smem_addr(sP + X * kPBytes);
         const uint32_t va = smem_addr(sV + st * kTile);
 #pragma unroll
         for (int k = 0; k < 8; ++k) {
           const uint64_t ad = smem_desc_sw128(pa + (k >> 2) * (kPBytes / 2) + (k & 3) * 32, 16, 1024);
           const uint64_t bd = smem_desc_sw128(va + k * 2048, kTile, 1024);
-          umma_bf16(tmem + 256 + pb * 64, ad, bd, idesc_o, k > 0);
+          umma_bf16(tmem + 256 + X * 128 + ob * 64, ad, bd, idesc_o, k > 0);
         }
-        umma_commit(bar(OF + pb));
-        umma_commit(bar(PE + pb));
-        umma_commit(bar(KVE + st));
+        umma_commit(bar(OF + 2 * X + ob));
+        umma_commit(bar(PE + X));
+        ++jo[X];
         return true;
       };
-      for (int j = 0; ok && j < n; ++j) {
-        const int st = j % kNS;
-        const int sb = j & 1;
-        if (!(ok = mbar_wait(bar(SE + sb), ((j >> 1) & 1) ^ 1, wc, 17))) break;
-        if (!(ok = mbar_wait(bar(KF + st), (j / kNS) & 1, wc, 18))) break;
-        tc_fence_after();
-        const uint32_t ka = smem_addr(sK + st * kTile);
-#pragma unroll
-        for (int k = 0; k < 4; ++k)
-          umma_bf16(tmem + sb * 128, smem_desc_sw128(qa + 32 * k, 16, 1024),
-                    smem_desc_sw128(ka + 32 * k, 16, 1024), idesc_s, k > 0);
-        umma_commit(bar(SF + sb));
-        if (j > 0) ok = issue_pv(j - 1);
+      for (int X = 0; X < 2 && ok; ++X)
+        if (valid(X, 0)) ok = issue_s(X, 0);
+      for (int u = 0; ok && u < nu; ++u) {
+        for (int X = 0; X < 2 && ok; ++X) {
+          if (valid(X, u)) ok = issue_pv(X, u);
+          if (ok && u + 1 < nu && valid(X, u + 1)) ok = issue_s(X, u + 1);
+        }
+        if (ok) umma_commit(bar(KVE + u % kNS));   // K/V stage u is free once these finish
       }
-      if (ok) issue_pv(n - 1);
       umma_commit(bar(DR));
       int zero = 0;
       WaitCtx dw = wc;
@@ -160,28 +197,33 @@ swa_attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
       mbar_wait(bar(DR), 0, dw, 19);
     }
   } else {
-    // ---------------- softmax / output warps: thread r owns query row q0 + r
-    const int r = threadIdx.x;
-    const int i = q0 + r;
-    const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+    // ------------- softmax / output: warpgroup X, thread r owns query row q0 + 128 X + r
+    const int X = warp >> 2;
+    const int r = threadIdx.x & 127;
+    const int i = q0 + 128 * X + r;
+    const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const uint32_t tS = tmem + X * 128 + lane_off;
+    const uint32_t tO = tmem + 256 + X * 128 + lane_off;
     const float sl2 = a.scale_log2;
+    const int q_lo = q0 + 128 * X;          // first query row of this tile
     float o[64];
 #pragma unroll
     for (int d = 0; d < 64; ++d) o[d] = 0.f;
     float m_run = -INFINITY, l_run = 0.f, mu_o = -INFINITY, mu0 = 0.f, mu1 = 0.f;
     bool ok = true;
+    const int nX = (X == 0 || has1) ? kt1[X] - kt0[X] + 1 : 0;
 
     auto consume_o = [&](int jj) -> bool {
       const int ob = jj & 1;
-      bool w = mbar_wait(bar(OF + ob), (jj >> 1) & 1, wc, 20);
+      bool w = mbar_wait(bar(OF + 2 * X + ob), (jj >> 1) & 1, wc, 20);
       if (!__all_sync(0xffffffffu, w)) return false;
       tc_fence_after();
       uint32_t r0[32], r1[32];
-      tmem_ld32(tmem + 256 + ob * 64 + lane_off, r0);
-      tmem_ld32(tmem + 256 + ob * 64 + 32 + lane_off, r1);
+      tmem_ld32(tO + ob * 64, r0);
+      tmem_ld32(tO + ob * 64 + 32, r1);
       tmem_ld_wait();
       tc_fence_before();
-      mbar_arrive(bar(OE + ob));
+      mbar_arrive(bar(OE + 2 * X + ob));
       const float mu_j = ob ? mu1 : mu0;
       const float f = (mu_o == -INFINITY) ? 0.f : ex2_approx(mu_o - mu_j);
 #pragma unroll
@@ -193,76 +235,85 @@ swa_attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
       return true;
     };
 
-    for (int j = 0; j < n; ++j) {
-      const int sb = j & 1;
-      const uint32_t sph = (j >> 1) & 1;
-      bool w = mbar_wait(bar(SF + sb), sph, wc, 21);
+    for (int j = 0; j < nX; ++j) {
+      const int key0 = (kt0[X] + j) * 128;
+      bool w = mbar_wait(bar(SF + X), j & 1, wc, 21);
       if (!__all_sync(0xffffffffu, w)) { ok = false; break; }
       tc_fence_after();
-      float x[128];
-      {
-        uint32_t s0[32], s1[32], s2[32], s3[32];
-        const uint32_t ta = tmem + sb * 128 + lane_off;
-        tmem_ld32(ta, s0);
-        tmem_ld32(ta + 32, s1);
-        tmem_ld32(ta + 64, s2);
-        tmem_ld32(ta + 96, s3);
+      // Edge tile: some (row, key) pair of the tile is outside (i - W, i].
+      const bool edge = key0 + 127 > q_lo || key0 <= q_lo + 127 - W;
+      // pass 1: row max of the raw scores (masked)
+      float smax = -INFINITY;
+#pragma unroll 1
+      for (int c = 0; c < 4; ++c) {
+        uint32_t rr[32];
+        tmem_ld32(tS + c * 32, rr);
         tmem_ld_wait();
+        float v[32];
 #pragma unroll
-        for (int c = 0; c < 32; ++c) {
-          x[c] = __uint_as_float(s0[c]) * sl2;
-          x[c + 32] = __uint_as_float(s1[c]) * sl2;
-          x[c + 64] = __uint_as_float(s2[c]) * sl2;
-          x[c + 96] = __uint_as_float(s3[c]) * sl2;
+        for (int e = 0; e < 32; ++e) {
+          v[e] = __uint_as_float(rr[e]);
+          if (edge) {
+            const int key = key0 + c * 32 + e;
+            if (key > i || key <= i - W) v[e] = -INFINITY;
+          }
+        }
+        smax = fmaxf(smax, tree_max32(v));
+      }
+      const float m_new = fmaxf(m_run, smax * sl2);
+      const float mu = (m_new == -INFINITY) ? 0.f : m_new;
+      const float alpha = ex2_approx(m_run - mu);
+      m_run = m_new;
+      if (j & 1) mu1 = mu; else mu0 = mu;
+
+      w = mbar_wait(bar(PE + X), (j & 1) ^ 1, wc, 22);
+      if (!__all_sync(0xffffffffu, w)) { ok = false; break; }
+      // pass 2: p = 2^(s * scale_log2 - mu), row sum, P (bf16) into shared memory:
+      // row r, 128-byte rows, 16-byte chunk index XOR (r & 7), keys 64.. in the second half.
+      float rs = 0.f;
+      uint8_t* prow = sP + X * kPBytes + r * 128;
+#pragma unroll 1
+      for (int c = 0; c < 4; ++c) {
+        uint32_t rr[32];
+        tmem_ld32(tS + c * 32, rr);
+        tmem_ld_wait();
+        float pv[32];
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          float x = fmaf(__uint_as_float(rr[e]), sl2, -mu);
+          if (edge) {
+            const int key = key0 + c * 32 + e;
+            if (key > i || key <= i - W) x = -INFINITY;
+          }
+          pv[e] = ex2_approx(x);
+        }
+        float t[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) t[e] = pv[e] + pv[e + 16];
+#pragma unroll
+        for (int wdt = 8; wdt >= 1; wdt >>= 1)
+#pragma unroll
+          for (int e = 0; e < wdt; ++e) t[e] += t[e + wdt];
+        rs += t[0];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const int cc = c * 4 + q;     // 16-byte chunk 0..15 of the row
+          const uint32_t off = (cc >> 3) * (kPBytes / 2) + ((((cc & 7) ^ (r & 7))) << 4);
+          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(smem_addr(prow + off)),
+                       "r"(pack_bf16x2(pv[q * 8 + 0], pv[q * 8 + 1])), "r"(pack_bf16x2(pv[q * 8 + 2], pv[q * 8 + 3])),
+                       "r"(pack_bf16x2(pv[q * 8 + 4], pv[q * 8 + 5])), "r"(pack_bf16x2(pv[q * 8 + 6], pv[q * 8 + 7]))
+                       : "memory");
         }
       }
       tc_fence_before();
-      mbar_arrive(bar(SE + sb));
-      const int key0 = (kt0 + j) * 128;
-      // Edge tile: some (row, key) pair of the tile is outside (i - W, i].
-      if (key0 + 127 > q0 || key0 <= q0 + 127 - W) {
-#pragma unroll
-        for (int c = 0; c < 128; ++c) {
-          const int key = key0 + c;
-          if (key > i || key <= i - W) x[c] = -INFINITY;
-        }
-      }
-      float tmax = x[0];
-#pragma unroll
-      for (int c = 1; c < 128; ++c) tmax = fmaxf(tmax, x[c]);
-      const float m_new = fmaxf(m_run, tmax);
-      const float mu = (m_new == -INFINITY) ? 0.f : m_new;
-      const float alpha = ex2_approx(m_run - mu);
-      float rs = 0.f;
-#pragma unroll
-      for (int c = 0; c < 128; ++c) {
-        x[c] = ex2_approx(x[c] - mu);
-        rs += x[c];
-      }
-      l_run = fmaf(l_run, alpha, rs);
-      m_run = m_new;
-      if (sb) mu1 = mu; else mu0 = mu;
-
-      w = mbar_wait(bar(PE + sb), sph ^ 1, wc, 22);
-      if (!__all_sync(0xffffffffu, w)) { ok = false; break; }
-      // P row r: keys 0..63 in the first 16 KB half, 64..127 in the second,
-      // 128-byte rows with the 16-byte chunk index XOR-ed by (r & 7).
-      uint8_t* prow = sP + sb * kPBytes + r * 128;
-#pragma unroll
-      for (int cc = 0; cc < 16; ++cc) {
-        const uint32_t off = (cc >> 3) * (kPBytes / 2) + ((((cc & 7) ^ (r & 7))) << 4);
-        const uint32_t addr = smem_addr(prow + off);
-        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr),
-                     "r"(pack_bf16x2(x[cc * 8 + 0], x[cc * 8 + 1])), "r"(pack_bf16x2(x[cc * 8 + 2], x[cc * 8 + 3])),
-                     "r"(pack_bf16x2(x[cc * 8 + 4], x[cc * 8 + 5])), "r"(pack_bf16x2(x[cc * 8 + 6], x[cc * 8 + 7]))
-                     : "memory");
-      }
+      mbar_arrive(bar(SE + X));
       fence_proxy_async_smem();
-      mbar_arrive(bar(PF + sb));
+      mbar_arrive(bar(PF + X));
+      l_run = fmaf(l_run, alpha, rs);
       if (j > 0 && !(ok = consume_o(j - 1))) break;
     }
-    if (ok) ok = consume_o(n - 1);
-    if (ok && i < a.T) {
+    if (ok && nX > 0) ok = consume_o(nX - 1);
+    if (ok && nX > 0 && i < T) {
       const float inv_l = 1.0f / l_run;
       uint16_t* dst = static_cast<uint16_t*>(a.out) + static_cast<int64_t>(b) * a.o_batch +
                       static_cast<int64_t>(i) * a.o_row + static_cast<int64_t>(h) * a.o_head;
@@ -277,7 +328,7 @@ swa_attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
   }
 
   __syncthreads();
-  if (warp == 5) {
+  if (warp == 9) {
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
   }
@@ -347,35 +398,66 @@ struct RopeArgs {
   float lo[32];
 };
 
+// table[t][m] = (cos, sin) of (pos0 + t) * inv_freq_m, t < T, m < 32.
+__global__ void rope_table_kernel(float2* __restrict__ table, int T, int64_t pos0, const __grid_constant__ RopeArgs f) {
+  pdl_wait();
+  pdl_trigger();
+  const int idx = blockIdx.x * blockDim.x + threadIdx.x;
+  if (idx >= T * 32) return;
+  const int t = idx >> 5, m = idx & 31;
+  float sn, cs;
+  rope_sincos(static_cast<float>(pos0 + t), f.hi[m], f.lo[m], &sn, &cs);
+  table[idx] = make_float2(cs, sn);
+}
+
+// Rotates q and k ([B, T, H, 64]) into qr and kr with the table: thread
+// handles pairs (m, m + 32) for 8 consecutive m of one (tensor, row, head).
 template <bool BF16>
-__global__ void rope_kernel(const void* __restrict__ x, void* __restrict__ y, int64_t rows, int T, int H,
-                            int64_t pos0, const __grid_constant__ RopeArgs f) {
+__global__ void rope_apply_kernel(const void* __restrict__ q, const void* __restrict__ k, void* __restrict__ qr,
+                                  void* __restrict__ kr, const float2* __restrict__ table, int64_t rows, int T, int H) {
   pdl_wait();
   pdl_trigger();
   const int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  const int64_t total = rows * H * 32;
-  if (idx >= total) return;
-  const int m = static_cast<int>(idx & 31);
-  const int64_t rh = idx >> 5;          // (row, head)
-  const int64_t row = rh / H;
-  const int t = static_cast<int>(row % T);
-  float s, c;
-  rope_sincos(static_cast<float>(pos0 + t), f.hi[m], f.lo[m], &s, &c);
-  const int64_t e = rh * 64 + m;
+  const int64_t per = rows * H * 4;          // per tensor: (row, head, 8-pair group)
+  if (idx >= 2 * per) return;
+  const int which = idx >= per;
+  const int64_t j = which ? idx - per : idx;
+  const int g = static_cast<int>(j & 3);      // m = 8 g .. 8 g + 7
+  const int64_t rh = j >> 2;
+  const int t = static_cast<int>((rh / H) % T);
+  const int64_t e = rh * 64 + g * 8;
+  const float2* tb = table + t * 32 + g * 8;
+  float u[8], w[8];
   if constexpr (BF16) {
-    const uint16_t* xs = static_cast<const uint16_t*>(x);
-    uint16_t* ys = static_cast<uint16_t*>(y);
-    const float u = bf16_to_f(xs[e]), w = bf16_to_f(xs[e + 32]);
-    const __nv_bfloat16 r1 = __float2bfloat16_rn(u * c - w * s);
-    const __nv_bfloat16 r2 = __float2bfloat16_rn(w * c + u * s);
-    ys[e] = *reinterpret_cast<const uint16_t*>(&r1);
-    ys[e + 32] = *reinterpret_cast<const uint16_t*>(&r2);
+    const uint16_t* src = static_cast<const uint16_t*>(which ? k : q);
+    const uint4 a = *reinterpret_cast<const uint4*>(src + e);
+    const uint4 c = *reinterpret_cast<const uint4*>(src + e + 32);
+    u[0] = bf16lo(a.x); u[1] = bf16hi(a.x); u[2] = bf16lo(a.y); u[3] = bf16hi(a.y);
+    u[4] = bf16lo(a.z); u[5] = bf16hi(a.z); u[6] = bf16lo(a.w); u[7] = bf16hi(a.w);
+    w[0] = bf16lo(c.x); w[1] = bf16hi(c.x); w[2] = bf16lo(c.y); w[3] = bf16hi(c.y);
+    w[4] = bf16lo(c.z); w[5] = bf16hi(c.z); w[6] = bf16lo(c.w); w[7] = bf16hi(c.w);
   } else {
-    const float* xs = static_cast<const float*>(x);
-    float* ys = static_cast<float*>(y);
-    const float u = xs[e], w = xs[e + 32];
-    ys[e] = u * c - w * s;
-    ys[e + 32] = w * c + u * s;
+    const float* src = static_cast<const float*>(which ? k : q);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) { u[i] = src[e + i]; w[i] = src[e + 32 + i]; }
+  }
+  float y1[8], y2[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const float2 cs = tb[i];
+    y1[i] = u[i] * cs.x - w[i] * cs.y;
+    y2[i] = w[i] * cs.x + u[i] * cs.y;
+  }
+  if constexpr (BF16) {
+    uint16_t* dst = static_cast<uint16_t*>(which ? kr : qr);
+    *reinterpret_cast<uint4*>(dst + e) = make_uint4(pack_bf16x2(y1[0], y1[1]), pack_bf16x2(y1[2], y1[3]),
+                                                    pack_bf16x2(y1[4], y1[5]), pack_bf16x2(y1[6], y1[7]));
+    *reinterpret_cast<uint4*>(dst + e + 32) = make_uint4(pack_bf16x2(y2[0], y2[1]), pack_bf16x2(y2[2], y2[3]),
+                                                         pack_bf16x2(y2[4], y2[5]), pack_bf16x2(y2[6], y2[7]));
+  } else {
+    float* dst = static_cast<float*>(which ? kr : qr);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) { dst[e + i] = y1[i]; dst[e + 32 + i] = y2[i]; }
   }
 }
 
@@ -398,7 +480,7 @@ cudaError_t launch_attn_bf16(const Launch& L, const CUtensorMap& tmQ, const CUte
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  const dim3 grid((a.T + 127) / 128, a.H, a.B);
+  const dim3 grid((a.T + 255) / 256, a.H, a.B);
   return launch_kernel(swa_attn_tc_kernel, grid, dim3(kAttnThreads), kAttnSmem, L.stream, tmQ, tmK, tmV, a);
 }
 
@@ -408,23 +490,25 @@ cudaError_t launch_attn_f32(const Launch& L, const float* q, const float* k, con
   return launch_kernel(swa_attn_f32_kernel, grid, dim3(128), 0, L.stream, q, k, v, o, T, H, window, scale);
 }
 
-cudaError_t launch_rope(const Launch& L, const void* x, void* y, bool bf16, int B, int T, int H,
-                        int64_t pos0, float theta) {
+cudaError_t launch_rope(const Launch& L, const void* q, const void* k, void* qr, void* kr, void* table, bool bf16,
+                        int B, int T, int H, int64_t pos0, float theta) {
   RopeArgs f;
   for (int m = 0; m < 32; ++m) {
     const double inv = std::pow(static_cast<double>(theta), -2.0 * m / 64.0);
     f.hi[m] = static_cast<float>(inv);
     f.lo[m] = static_cast<float>(inv - static_cast<double>(f.hi[m]));
   }
+  float2* tb = static_cast<float2*>(table);
+  cudaError_t e = launch_kernel(rope_table_kernel, dim3((T * 32 + 255) / 256), dim3(256), 0, L.stream, tb, T, pos0, f);
+  if (e != cudaSuccess) return e;
   const int64_t rows = static_cast<int64_t>(B) * T;
-  const int64_t total = rows * H * 32;
-  const int threads = 256;
-  const int64_t blocks = (total + threads - 1) / threads;
+  const int64_t total = 2 * rows * H * 4;
+  const dim3 grid(static_cast<unsigned>((total + 255) / 256));
   if (bf16)
-    return launch_kernel(rope_kernel<true>, dim3(static_cast<unsigned>(blocks)), dim3(threads), 0, L.stream, x, y,
-                         rows, T, H, pos0, f);
-  return launch_kernel(rope_kernel<false>, dim3(static_cast<unsigned>(blocks)), dim3(threads), 0, L.stream, x, y,
-                       rows, T, H, pos0, f);
+    return launch_kernel(rope_apply_kernel<true>, grid, dim3(256), 0, L.stream, q, k, qr, kr,
+                         static_cast<const float2*>(tb), rows, T, H);
+  return launch_kernel(rope_apply_kernel<false>, grid, dim3(256), 0, L.stream, q, k, qr, kr,
+                       static_cast<const float2*>(tb), rows, T, H);
 }
 
 }  // namespace vx

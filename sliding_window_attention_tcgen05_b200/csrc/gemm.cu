@@ -237,10 +237,6 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
-  // Inputs written by the previous kernel of the stream are read below.
-  pdl_wait();
-  pdl_trigger();
-
   const WaitCtx wc{a.status, abort_flag, a.limit_ns};
   // Work unit u -> (m tile, K split, n tile), M fastest so that the units
   // resident at one time share a weight panel through L2.
@@ -256,25 +252,45 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     n0 = (r / splits) * BN;
   };
 
+  // The weights (B) do not depend on the previous kernel of the stream: the
+  // producer starts streaming the first stages' B tiles before waiting for it.
+  int npre = 0;
+  if (warp == 4 && lane == 0 && blockIdx.x < num_tiles) {
+    int m0, n0, ks;
+    decode(blockIdx.x, m0, n0, ks);
+    npre = nkb < S ? nkb : S;
+    for (int i = 0; i < npre; ++i) {
+      mbar_arrive_expect_tx(full(i), C::kStageBytes);
+      tma_load_2d(smem_addr(sB + i * C::kBBytes), &tmB, full(i), (ks * nkb + i) * kBK, n0);
+    }
+  }
+  // Inputs written by the previous kernel of the stream are read below.
+  pdl_wait();
+  pdl_trigger();
+
   if (warp == 4) {
     if (lane == 0) {
       int stage = 0;
       uint32_t phase = 0;
       uint32_t issued = 0;  // bit s: stage s was filled at least once
       uint32_t last_par = 0;  // bit s: parity of the last fill of stage s
+      int it = 0;           // k-block iterations issued so far
       for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
         int m0, n0, ks;
         decode(tile, m0, n0, ks);
         bool ok = true;
-        for (int kb = ks * nkb; kb < (ks + 1) * nkb; ++kb) {
-          if (!mbar_wait(empty(stage), phase ^ 1, wc, 1)) { ok = false; break; }
-          mbar_arrive_expect_tx(full(stage), C::kStageBytes);
+        for (int kb = ks * nkb; kb < (ks + 1) * nkb; ++kb, ++it) {
+          const bool pre = it < npre;   // B already in flight, barrier already armed
+          if (!pre) {
+            if (!mbar_wait(empty(stage), phase ^ 1, wc, 1)) { ok = false; break; }
+            mbar_arrive_expect_tx(full(stage), C::kStageBytes);
+          }
           const int tap = kb / a.kb_per_tap;
           const int c = (kb - tap * a.kb_per_tap) * kBK;
           const int ax = (tap % a.a_stride) * a.a_tap_ch + c;
           const int ay = m0 + tap / a.a_stride;
           tma_load_2d(smem_addr(sA + stage * kABytes), &tmA, full(stage), ax, ay);
-          tma_load_2d(smem_addr(sB + stage * C::kBBytes), &tmB, full(stage), kb * kBK, n0);
+          if (!pre) tma_load_2d(smem_addr(sB + stage * C::kBBytes), &tmB, full(stage), kb * kBK, n0);
           issued |= 1u << stage;
           last_par = (last_par & ~(1u << stage)) | (phase << stage);
           if (++stage == S) { stage = 0; phase ^= 1; }

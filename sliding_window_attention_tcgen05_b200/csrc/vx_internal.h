@@ -120,9 +120,10 @@ bool tmap_attn_operand(CUtensorMap* map, const void* base, int B, int T, int H,
 cudaError_t launch_attn_f32(const Launch& L, const float* q, const float* k, const float* v,
                             float* o, int B, int T, int H, int window, float scale);
 
-// RoPE of x ([B, T, H, 64], fp32 or bf16) into y (same layout and dtype).
-cudaError_t launch_rope(const Launch& L, const void* x, void* y, bool bf16, int B, int T, int H,
-                        int64_t pos0, float theta);
+// RoPE of q and k ([B, T, H, 64], fp32 or bf16) into qr and kr (same layout
+// and dtype); table: T * 32 float2 of scratch for the per-position cos / sin.
+cudaError_t launch_rope(const Launch& L, const void* q, const void* k, void* qr, void* kr, void* table, bool bf16,
+                        int B, int T, int H, int64_t pos0, float theta);
 
 // ---------------------------------------------------------------- others --
 // h = x + bias + sum_{k < nparts} parts[k * part_stride + .]  (parts/bias optional);
