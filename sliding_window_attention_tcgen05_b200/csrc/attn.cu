@@ -1,10 +1,12 @@
 // attn.cu -- causal sliding-window attention kernels.
 //
 // swa_attn_tc_kernel: flash-style bf16 attention on tcgen05 tensor cores.
-//   One CTA per (two adjacent 128-query tiles, head, clip); the two softmax
-//   warpgroups ping-pong against one MMA warp and share every K/V tile.  Only
-//   the key tiles that meet the causal window (i - W, i] of some query are
-//   visited; the masks are evaluated only on the edge tiles.  K/V tiles arrive
+//   One CTA per (128-query tile, head, clip); its key tiles alternate between
+//   two softmax warpgroups (each with its own running max / sum / output,
+//   merged at the end) so that one warpgroup's exponentials overlap the other
+//   warpgroup's tensor-core products.  Only the key tiles that meet the causal
+//   window (i - W, i] of some query are visited; the masks are evaluated only
+//   on the edge tiles.  K/V tiles arrive
 //   by TMA into a 3-stage ring; S = Q K^T and O_j = P_j V_j accumulate in
 //   TMEM; the softmax warps read S from TMEM (two passes: max, then
 //   exponentials), keep the running max / sum in registers, write P (bf16) to
@@ -25,7 +27,7 @@ constexpr int kAttnThreads = 320;           // 2 softmax warpgroups, TMA warp, M
 constexpr int kNS = 3;                      // K/V pipeline stages
 constexpr int kTile = 128 * 64 * 2;         // one 128 x 64 bf16 tile
 constexpr int kPBytes = 128 * 128 * 2;      // one P tile (128 queries x 128 keys)
-constexpr int kAttnSmem = kTile * (2 + 2 * kNS) + 2 * kPBytes + 1024 + 512;
+constexpr int kAttnSmem = kTile * (2 + 2 * kNS) + 2 * kPBytes + 1024 + 512;   // Q slot 2 spare
 constexpr uint32_t kTmemCols = 512;
 
 // Max / sum of 32 values as a balanced tree (short dependency chains).
@@ -40,23 +42,25 @@ __device__ __forceinline__ float tree_max32(const float (&v)[32]) {
   return t[0];
 }
 
-// One CTA per (two adjacent 128-query tiles X = 0, 1; head; clip).  Key tiles
-// of 128 are visited from the first one meeting tile 0's window to the
-// diagonal of tile 1, each loaded once by TMA and used by both query tiles.
+// One CTA per (128-query tile, head, clip).  The key tiles of 128 that meet
+// the tile's causal window are split between two softmax warpgroups: tile u
+// goes to warpgroup X = u % 2, which keeps its own online-softmax state for
+// the same 128 rows; the two states are merged at the end.  The MMA warp
+// issues in key-tile order -- S(0), S(1), PV(0), S(2), PV(1), ... -- so one
+// warpgroup's exponentials overlap the other's products.
 // TMEM columns: S_X at 128 X, O_X double buffer at 256 + 128 X + 64 j.
-// Warps 0-3 / 4-7: softmax of tile 0 / 1 (TMEM lane = query row), warp 8:
-// TMA, warp 9: MMA (S_X = Q_X K^T and O_X,j = P_X V_j).
+// Warps 0-3 / 4-7: warpgroups X = 0 / 1 (TMEM lane = query row), warp 8: TMA,
+// warp 9: MMA.  K/V tiles arrive by TMA into a 3-stage ring.
 __global__ void __launch_bounds__(kAttnThreads, 1)
 swa_attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                    const __grid_constant__ CUtensorMap tmV, const __grid_constant__ AttnArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* sQ = smem;                       // Q_0 | Q_1
-  uint8_t* sK = sQ + 2 * kTile;
+  uint8_t* sQ = smem;
+  uint8_t* sK = sQ + 2 * kTile;             // (second Q slot unused)
   uint8_t* sV = sK + kNS * kTile;
   uint8_t* sP = sV + kNS * kTile;           // P_0 | P_1
   uint64_t* bars = reinterpret_cast<uint64_t*>(sP + 2 * kPBytes);
-  // barrier indices (per query tile X where doubled)
   constexpr int QF = 0, KF = 1, VF = KF + kNS, KVE = VF + kNS, SF = KVE + kNS, SE = SF + 2, PF = SE + 2,
                 PE = PF + 2, OF = PE + 2, OE = OF + 4, DR = OE + 4, NBAR = DR + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + NBAR);
@@ -65,22 +69,13 @@ swa_attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int q0 = blockIdx.x * 256;
+  const int q0 = blockIdx.x * 128;
   const int h = blockIdx.y;
   const int b = blockIdx.z;
   const int W = a.window;
   const int T = a.T;
-  const bool has1 = q0 + 128 < T;
-  // key-tile ranges of the two query tiles
-  const int kt0[2] = {max(0, q0 - W + 1) / 128, max(0, q0 + 128 - W + 1) / 128};
-  const int kt1[2] = {min(T - 1, q0 + 127) / 128, min(T - 1, q0 + 255) / 128};
-  const int klo = kt0[0];
-  const int khi = has1 ? kt1[1] : kt1[0];
-  const int nu = khi - klo + 1;
-  auto valid = [&](int X, int u) {
-    const int kt = klo + u;
-    return (X == 0 || has1) && kt >= kt0[X] && kt <= kt1[X];
-  };
+  const int kt0 = max(0, q0 - W + 1) / 128;
+  const int n = min(T - 1, q0 + 127) / 128 - kt0 + 1;   // key tiles of this query tile
 
   if (threadIdx.x == 0) {
     mbar_init(bar(QF), 1);
@@ -111,16 +106,15 @@ swa_attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
 
   if (warp == 8) {
     if (lane == 0) {
-      mbar_arrive_expect_tx(bar(QF), has1 ? 2 * kTile : kTile);
+      mbar_arrive_expect_tx(bar(QF), kTile);
       tma_load_4d(smem_addr(sQ), &tmQ, bar(QF), 0, h, q0, b);
-      if (has1) tma_load_4d(smem_addr(sQ + kTile), &tmQ, bar(QF), 0, h, q0 + 128, b);
       uint32_t last_par = 0;
       int filled = 0;
-      for (int u = 0; u < nu; ++u) {
+      for (int u = 0; u < n; ++u) {
         const int st = u % kNS;
         const uint32_t ph = (u / kNS) & 1;
         if (!mbar_wait(bar(KVE + st), ph ^ 1, wc, 11)) break;
-        const int key0 = (klo + u) * 128;
+        const int key0 = (kt0 + u) * 128;
         mbar_arrive_expect_tx(bar(KF + st), kTile);
         tma_load_4d(smem_addr(sK + st * kTile), &tmK, bar(KF + st), 0, h, key0, b);
         mbar_arrive_expect_tx(bar(VF + st), kTile);
@@ -143,27 +137,23 @@ swa_attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
       const uint32_t idesc_s = idesc_bf16_f32(128, 128, 0);
       const uint32_t idesc_o = idesc_bf16_f32(128, 64, 1);
       bool ok = mbar_wait(bar(QF), 0, wc, 13);
-      int js[2] = {0, 0};   // S products issued per query tile
-      int jo[2] = {0, 0};   // P V products issued per query tile
-      auto issue_s = [&](int X, int u) -> bool {
-        const int st = u % kNS;
-        if (!mbar_wait(bar(SE + X), (js[X] & 1) ^ 1, wc, 17)) return false;
+      const uint32_t qa = smem_addr(sQ);
+      // S(u) -> S_{u%2}: tile u is the (u/2)-th of its warpgroup.
+      auto issue_s = [&](int u) -> bool {
+        const int X = u & 1, j = u >> 1, st = u % kNS;
+        if (!mbar_wait(bar(SE + X), (j & 1) ^ 1, wc, 17)) return false;
         if (!mbar_wait(bar(KF + st), (u / kNS) & 1, wc, 18)) return false;
         tc_fence_after();
-        const uint32_t qa = smem_addr(sQ + X * kTile);
         const uint32_t ka = smem_addr(sK + st * kTile);
 #pragma unroll
         for (int k = 0; k < 4; ++k)
           umma_bf16(tmem + X * 128, smem_desc_sw128(qa + 32 * k, 16, 1024), smem_desc_sw128(ka + 32 * k, 16, 1024),
                     idesc_s, k > 0);
         umma_commit(bar(SF + X));
-        ++js[X];
         return true;
       };
-      auto issue_pv = [&](int X, int u) -> bool {
-        const int st = u % kNS;
-        const int j = jo[X];
-        const int ob = j & 1;
+      auto issue_pv = [&](int u) -> bool {
+        const int X = u & 1, j = u >> 1, st = u % kNS, ob = j & 1;
         if (!mbar_wait(bar(PF + X), j & 1, wc, 14)) return false;
         if (!mbar_wait(bar(VF + st), (u / kNS) & 1, wc, 15)) return false;
         if (!mbar_wait(bar(OE + 2 * X + ob), ((j >> 1) & 1) ^ 1, wc, 16)) return false;
@@ -178,17 +168,14 @@ swa_attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
         }
         umma_commit(bar(OF + 2 * X + ob));
         umma_commit(bar(PE + X));
-        ++jo[X];
+        umma_commit(bar(KVE + st));   // K/V tile u: its S and PV products are the last users
         return true;
       };
-      for (int X = 0; X < 2 && ok; ++X)
-        if (valid(X, 0)) ok = issue_s(X, 0);
-      for (int u = 0; ok && u < nu; ++u) {
-        for (int X = 0; X < 2 && ok; ++X) {
-          if (valid(X, u)) ok = issue_pv(X, u);
-          if (ok && u + 1 < nu && valid(X, u + 1)) ok = issue_s(X, u + 1);
-        }
-        if (ok) umma_commit(bar(KVE + u % kNS));   // K/V stage u is free once these finish
+      if (ok) ok = issue_s(0);
+      if (ok && n > 1) ok = issue_s(1);
+      for (int u = 0; ok && u < n; ++u) {
+        ok = issue_pv(u);
+        if (ok && u + 2 < n) ok = issue_s(u + 2);
       }
       umma_commit(bar(DR));
       int zero = 0;
@@ -197,21 +184,20 @@ swa_attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
       mbar_wait(bar(DR), 0, dw, 19);
     }
   } else {
-    // ------------- softmax / output: warpgroup X, thread r owns query row q0 + 128 X + r
+    // ------------- softmax: warpgroup X takes key tiles X, X + 2, ...; thread r owns row q0 + r
     const int X = warp >> 2;
     const int r = threadIdx.x & 127;
-    const int i = q0 + 128 * X + r;
+    const int i = q0 + r;
     const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const uint32_t tS = tmem + X * 128 + lane_off;
     const uint32_t tO = tmem + 256 + X * 128 + lane_off;
     const float sl2 = a.scale_log2;
-    const int q_lo = q0 + 128 * X;          // first query row of this tile
     float o[64];
 #pragma unroll
     for (int d = 0; d < 64; ++d) o[d] = 0.f;
     float m_run = -INFINITY, l_run = 0.f, mu_o = -INFINITY, mu0 = 0.f, mu1 = 0.f;
     bool ok = true;
-    const int nX = (X == 0 || has1) ? kt1[X] - kt0[X] + 1 : 0;
+    const int nX = (n + 1 - X) / 2;   // tiles u = X, X + 2, ... < n
 
     auto consume_o = [&](int jj) -> bool {
       const int ob = jj & 1;
@@ -236,12 +222,12 @@ swa_attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
     };
 
     for (int j = 0; j < nX; ++j) {
-      const int key0 = (kt0[X] + j) * 128;
+      const int key0 = (kt0 + X + 2 * j) * 128;
       bool w = mbar_wait(bar(SF + X), j & 1, wc, 21);
       if (!__all_sync(0xffffffffu, w)) { ok = false; break; }
       tc_fence_after();
       // Edge tile: some (row, key) pair of the tile is outside (i - W, i].
-      const bool edge = key0 + 127 > q_lo || key0 <= q_lo + 127 - W;
+      const bool edge = key0 + 127 > q0 || key0 <= q0 + 127 - W;
       // pass 1: row max of the raw scores (masked)
       float smax = -INFINITY;
 #pragma unroll 1
@@ -277,6 +263,10 @@ swa_attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
         uint32_t rr[32];
         tmem_ld32(tS + c * 32, rr);
         tmem_ld_wait();
+        if (c == 3) {   // S_X fully read: the next S of this warpgroup may overwrite it
+          tc_fence_before();
+          mbar_arrive(bar(SE + X));
+        }
         float pv[32];
 #pragma unroll
         for (int e = 0; e < 32; ++e) {
@@ -305,24 +295,47 @@ swa_attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
                        : "memory");
         }
       }
-      tc_fence_before();
-      mbar_arrive(bar(SE + X));
       fence_proxy_async_smem();
       mbar_arrive(bar(PF + X));
       l_run = fmaf(l_run, alpha, rs);
       if (j > 0 && !(ok = consume_o(j - 1))) break;
     }
     if (ok && nX > 0) ok = consume_o(nX - 1);
-    if (ok && nX > 0 && i < T) {
-      const float inv_l = 1.0f / l_run;
-      uint16_t* dst = static_cast<uint16_t*>(a.out) + static_cast<int64_t>(b) * a.o_batch +
-                      static_cast<int64_t>(i) * a.o_row + static_cast<int64_t>(h) * a.o_head;
+
+    // Merge: warpgroup 1 hands (m, l, o) to warpgroup 0 through shared memory
+    // (the P buffers are idle now); warpgroup 0 writes the output.
+    float* xo = reinterpret_cast<float*>(sP + kPBytes);          // [128][64]
+    float* xm = reinterpret_cast<float*>(sP);                    // [128] m, [128] l
+    const bool okall = ok;
+    if (X == 1) {
+      asm volatile("bar.sync 1, 256;" ::: "memory");   // P_1 no longer read by the tensor cores
 #pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        st_global_v4(dst + 8 * c, pack_bf16x2(o[8 * c] * inv_l, o[8 * c + 1] * inv_l),
-                     pack_bf16x2(o[8 * c + 2] * inv_l, o[8 * c + 3] * inv_l),
-                     pack_bf16x2(o[8 * c + 4] * inv_l, o[8 * c + 5] * inv_l),
-                     pack_bf16x2(o[8 * c + 6] * inv_l, o[8 * c + 7] * inv_l));
+      for (int d = 0; d < 64; ++d) xo[r * 64 + ((d + r) & 63)] = o[d];
+      xm[r] = m_run;
+      xm[128 + r] = okall ? l_run : 0.f;
+      asm volatile("bar.sync 2, 256;" ::: "memory");
+    } else {
+      asm volatile("bar.sync 1, 256;" ::: "memory");
+      asm volatile("bar.sync 2, 256;" ::: "memory");
+      const float m1 = xm[r], l1 = xm[128 + r];
+      const float M = fmaxf(m_run, m1);
+      const float f0 = (m_run == -INFINITY) ? 0.f : ex2_approx(m_run - M);
+      const float f1 = (m1 == -INFINITY) ? 0.f : ex2_approx(m1 - M);
+      const float inv_l = 1.0f / (l_run * f0 + l1 * f1);
+      if (ok && i < T) {
+        uint16_t* dst = static_cast<uint16_t*>(a.out) + static_cast<int64_t>(b) * a.o_batch +
+                        static_cast<int64_t>(i) * a.o_row + static_cast<int64_t>(h) * a.o_head;
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          float v[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const int d = 8 * c + e;
+            v[e] = (o[d] * f0 + xo[r * 64 + ((d + r) & 63)] * f1) * inv_l;
+          }
+          st_global_v4(dst + 8 * c, pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]), pack_bf16x2(v[4], v[5]),
+                       pack_bf16x2(v[6], v[7]));
+        }
       }
     }
   }
@@ -480,7 +493,7 @@ cudaError_t launch_attn_bf16(const Launch& L, const CUtensorMap& tmQ, const CUte
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  const dim3 grid((a.T + 255) / 256, a.H, a.B);
+  const dim3 grid((a.T + 127) / 128, a.H, a.B);
   return launch_kernel(swa_attn_tc_kernel, grid, dim3(kAttnThreads), kAttnSmem, L.stream, tmQ, tmK, tmV, a);
 }
 
