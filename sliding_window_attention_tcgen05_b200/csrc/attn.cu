@@ -6,15 +6,13 @@
 //   merged at the end) so that one warpgroup's exponentials overlap the other
 //   warpgroup's tensor-core products.  Only the key tiles that meet the causal
 //   window (i - W, i] of some query are visited; the masks are evaluated only
-//   on the edge tiles.  K/V tiles arrive
-//   by TMA into a 3-stage ring; S = Q K^T and O_j = P_j V_j accumulate in
-//   TMEM; the softmax warps read S from TMEM (two passes: max, then
-//   exponentials), keep the running max / sum in registers, write P (bf16) to
-//   shared memory as the A operand of the P V product, and fold each O_j into
-//   a register accumulator with the online-softmax rescale.
+//   on the edge tiles.  K/V tiles arrive by TMA into a 4-stage ring; S, P and
+//   O all live in TMEM (P is the TMEM A operand of the P V product, O is
+//   accumulated in place and rescaled lazily).
 // swa_attn_f32_kernel: fp32 CUDA-core reference-precision path (one warp per
 //   query row), used for fp32 inputs.
-// rope_kernel: RoPE pre-pass for vx_swa_attn_fwd on raw q, k.
+// rope_table_kernel / rope_apply_kernel: RoPE pre-pass of vx_swa_attn_fwd on raw
+//   q, k (a per-position cos/sin table, then one vectorised rotation pass).
 #include <cmath>
 
 #include "vx_internal.h"
@@ -24,14 +22,21 @@ namespace vx {
 namespace {
 
 constexpr int kAttnThreads = 320;           // 2 softmax warpgroups, TMA warp, MMA warp
-constexpr int kNS = 3;                      // K/V pipeline stages
+constexpr int kNS = 4;                      // K/V pipeline stages
 constexpr int kTile = 128 * 64 * 2;         // one 128 x 64 bf16 tile
-constexpr int kPBytes = 128 * 128 * 2;      // one P tile (128 queries x 128 keys)
-constexpr int kAttnSmem = kTile * (2 + 2 * kNS) + 2 * kPBytes + 1024 + 512;   // Q slot 2 spare
+constexpr int kAttnSmem = kTile * (1 + 2 * kNS) + 1024 + 512;
 constexpr uint32_t kTmemCols = 512;
+constexpr float kRescaleSlack = 8.0f;       // O is rescaled only when a row max grows by more than 2^8
 
-// Max / sum of 32 values as a balanced tree (short dependency chains).
-__device__ __forceinline__ float tree_max32(const float (&v)[32]) {
+__device__ __forceinline__ void store_bf16x32(uint16_t* dst, const float (&v)[32]) {
+#pragma unroll
+  for (int j = 0; j < 4; ++j)
+    st_global_v4(dst + 8 * j, pack_bf16x2(v[8 * j + 0], v[8 * j + 1]), pack_bf16x2(v[8 * j + 2], v[8 * j + 3]),
+                 pack_bf16x2(v[8 * j + 4], v[8 * j + 5]), pack_bf16x2(v[8 * j + 6], v[8 * j + 7]));
+}
+
+// Max of 32 values as a balanced tree (short dependency chains).
+__device__ __forceinline__ float tree_max32(const float* v) {
   float t[16];
 #pragma unroll
   for (int i = 0; i < 16; ++i) t[i] = fmaxf(v[i], v[i + 16]);
@@ -43,28 +48,31 @@ __device__ __forceinline__ float tree_max32(const float (&v)[32]) {
 }
 
 // One CTA per (128-query tile, head, clip).  The key tiles of 128 that meet
-// the tile's causal window are split between two softmax warpgroups: tile u
-// goes to warpgroup X = u % 2, which keeps its own online-softmax state for
-// the same 128 rows; the two states are merged at the end.  The MMA warp
-// issues in key-tile order -- S(0), S(1), PV(0), S(2), PV(1), ... -- so one
-// warpgroup's exponentials overlap the other's products.
-// TMEM columns: S_X at 128 X, O_X double buffer at 256 + 128 X + 64 j.
-// Warps 0-3 / 4-7: warpgroups X = 0 / 1 (TMEM lane = query row), warp 8: TMA,
-// warp 9: MMA.  K/V tiles arrive by TMA into a 3-stage ring.
+// the tile's causal window alternate between two softmax warpgroups (tile u
+// -> warpgroup u % 2), each keeping its own running max / sum / output for the
+// same 128 rows; the two are merged at the end.  Per warpgroup X, TMEM holds
+// S_X (128 columns fp32), P_X (64 columns, bf16 pairs) and O_X (64 columns):
+// the softmax threads copy S_X to registers and release it at once, so the
+// next S of the warpgroup is computed while they exponentiate; P goes back to
+// TMEM and is the A operand of O_X += P_X V; O_X is rescaled in place only when
+// a row's max grows by more than kRescaleSlack (the exponents are taken
+// against a stale max otherwise, which cancels in O / l).
+// Warps 0-3 / 4-7: warpgroups 0 / 1 (TMEM lane = query row), warp 8: TMA,
+// warp 9: MMA, issuing S(0), S(1), then S(u+2), PV(u) for u = 0, 1, ...
 __global__ void __launch_bounds__(kAttnThreads, 1)
 swa_attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                    const __grid_constant__ CUtensorMap tmV, const __grid_constant__ AttnArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sQ = smem;
-  uint8_t* sK = sQ + 2 * kTile;             // (second Q slot unused)
+  uint8_t* sK = sQ + kTile;
   uint8_t* sV = sK + kNS * kTile;
-  uint8_t* sP = sV + kNS * kTile;           // P_0 | P_1
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sP + 2 * kPBytes);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sV + kNS * kTile);
   constexpr int QF = 0, KF = 1, VF = KF + kNS, KVE = VF + kNS, SF = KVE + kNS, SE = SF + 2, PF = SE + 2,
-                PE = PF + 2, OF = PE + 2, OE = OF + 4, DR = OE + 4, NBAR = DR + 1;
+                PE = PF + 2, OD = PE + 2, DR = OD + 2, NBAR = DR + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + NBAR);
   int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
+  float* xml = reinterpret_cast<float*>(abort_flag + 1);   // [128] m, [128] l of warpgroup 1 (padded below)
   auto bar = [&](int i) { return smem_addr(bars + i); };
 
   const int warp = threadIdx.x >> 5;
@@ -83,7 +91,7 @@ swa_attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
     for (int X = 0; X < 2; ++X) {
       mbar_init(bar(SF + X), 1); mbar_init(bar(SE + X), 128);
       mbar_init(bar(PF + X), 128); mbar_init(bar(PE + X), 1);
-      for (int j = 0; j < 2; ++j) { mbar_init(bar(OF + 2 * X + j), 1); mbar_init(bar(OE + 2 * X + j), 128); }
+      mbar_init(bar(OD + X), 1);
     }
     mbar_init(bar(DR), 1);
     *abort_flag = 0;
@@ -138,7 +146,7 @@ swa_attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
       const uint32_t idesc_o = idesc_bf16_f32(128, 64, 1);
       bool ok = mbar_wait(bar(QF), 0, wc, 13);
       const uint32_t qa = smem_addr(sQ);
-      // S(u) -> S_{u%2}: tile u is the (u/2)-th of its warpgroup.
+      // S(u) into S_{u%2}; it is the (u/2)-th tile of warpgroup u%2.
       auto issue_s = [&](int u) -> bool {
         const int X = u & 1, j = u >> 1, st = u % kNS;
         if (!mbar_wait(bar(SE + X), (j & 1) ^ 1, wc, 17)) return false;
@@ -147,36 +155,33 @@ swa_attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
         const uint32_t ka = smem_addr(sK + st * kTile);
 #pragma unroll
         for (int k = 0; k < 4; ++k)
-          umma_bf16(tmem + X * 128, smem_desc_sw128(qa + 32 * k, 16, 1024), smem_desc_sw128(ka + 32 * k, 16, 1024),
+          umma_bf16(tmem + X * 256, smem_desc_sw128(qa + 32 * k, 16, 1024), smem_desc_sw128(ka + 32 * k, 16, 1024),
                     idesc_s, k > 0);
         umma_commit(bar(SF + X));
         return true;
       };
       auto issue_pv = [&](int u) -> bool {
-        const int X = u & 1, j = u >> 1, st = u % kNS, ob = j & 1;
+        const int X = u & 1, j = u >> 1, st = u % kNS;
         if (!mbar_wait(bar(PF + X), j & 1, wc, 14)) return false;
         if (!mbar_wait(bar(VF + st), (u / kNS) & 1, wc, 15)) return false;
-        if (!mbar_wait(bar(OE + 2 * X + ob), ((j >> 1) & 1) ^ 1, wc, 16)) return false;
         tc_fence_after();
-        const uint32_t pa = smem_addr(sP + X * kPBytes);
         const uint32_t va = smem_addr(sV + st * kTile);
 #pragma unroll
-        for (int k = 0; k < 8; ++k) {
-          const uint64_t ad = smem_desc_sw128(pa + (k >> 2) * (kPBytes / 2) + (k & 3) * 32, 16, 1024);
-          const uint64_t bd = smem_desc_sw128(va + k * 2048, kTile, 1024);
-          umma_bf16(tmem + 256 + X * 128 + ob * 64, ad, bd, idesc_o, k > 0);
-        }
-        umma_commit(bar(OF + 2 * X + ob));
+        for (int k = 0; k < 8; ++k)   // 16 keys per step: 8 TMEM columns of P, 2 K-rows groups of V
+          umma_bf16_ts(tmem + X * 256 + 192, tmem + X * 256 + 128 + 8 * k, smem_desc_sw128(va + k * 2048, kTile, 1024),
+                       idesc_o, (j > 0 || k > 0) ? 1u : 0u);
         umma_commit(bar(PE + X));
-        umma_commit(bar(KVE + st));   // K/V tile u: its S and PV products are the last users
+        umma_commit(bar(KVE + st));   // K/V tile u: S(u) and PV(u) were its last users
         return true;
       };
       if (ok) ok = issue_s(0);
       if (ok && n > 1) ok = issue_s(1);
       for (int u = 0; ok && u < n; ++u) {
-        ok = issue_pv(u);
-        if (ok && u + 2 < n) ok = issue_s(u + 2);
+        if (u + 2 < n) ok = issue_s(u + 2);
+        if (ok) ok = issue_pv(u);
       }
+      umma_commit(bar(OD + 0));
+      umma_commit(bar(OD + 1));
       umma_commit(bar(DR));
       int zero = 0;
       WaitCtx dw = wc;
@@ -189,94 +194,81 @@ swa_attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
     const int r = threadIdx.x & 127;
     const int i = q0 + r;
     const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
-    const uint32_t tS = tmem + X * 128 + lane_off;
-    const uint32_t tO = tmem + 256 + X * 128 + lane_off;
+    const uint32_t tS = tmem + X * 256 + lane_off;
+    const uint32_t tP = tS + 128;
+    const uint32_t tO = tS + 192;
     const float sl2 = a.scale_log2;
-    float o[64];
-#pragma unroll
-    for (int d = 0; d < 64; ++d) o[d] = 0.f;
-    float m_run = -INFINITY, l_run = 0.f, mu_o = -INFINITY, mu0 = 0.f, mu1 = 0.f;
+    float m_used = -INFINITY, l_run = 0.f;
     bool ok = true;
     const int nX = (n + 1 - X) / 2;   // tiles u = X, X + 2, ... < n
-
-    auto consume_o = [&](int jj) -> bool {
-      const int ob = jj & 1;
-      bool w = mbar_wait(bar(OF + 2 * X + ob), (jj >> 1) & 1, wc, 20);
-      if (!__all_sync(0xffffffffu, w)) return false;
-      tc_fence_after();
-      uint32_t r0[32], r1[32];
-      tmem_ld32(tO + ob * 64, r0);
-      tmem_ld32(tO + ob * 64 + 32, r1);
-      tmem_ld_wait();
-      tc_fence_before();
-      mbar_arrive(bar(OE + 2 * X + ob));
-      const float mu_j = ob ? mu1 : mu0;
-      const float f = (mu_o == -INFINITY) ? 0.f : ex2_approx(mu_o - mu_j);
-#pragma unroll
-      for (int d = 0; d < 32; ++d) {
-        o[d] = fmaf(o[d], f, __uint_as_float(r0[d]));
-        o[d + 32] = fmaf(o[d + 32], f, __uint_as_float(r1[d]));
-      }
-      mu_o = mu_j;
-      return true;
-    };
 
     for (int j = 0; j < nX; ++j) {
       const int key0 = (kt0 + X + 2 * j) * 128;
       bool w = mbar_wait(bar(SF + X), j & 1, wc, 21);
       if (!__all_sync(0xffffffffu, w)) { ok = false; break; }
       tc_fence_after();
-      // Edge tile: some (row, key) pair of the tile is outside (i - W, i].
-      const bool edge = key0 + 127 > q0 || key0 <= q0 + 127 - W;
-      // pass 1: row max of the raw scores (masked)
-      float smax = -INFINITY;
-#pragma unroll 1
-      for (int c = 0; c < 4; ++c) {
-        uint32_t rr[32];
-        tmem_ld32(tS + c * 32, rr);
+      float sv[128];
+      {
+        uint32_t r0[32], r1[32], r2[32], r3[32];
+        tmem_ld32(tS, r0);
+        tmem_ld32(tS + 32, r1);
+        tmem_ld32(tS + 64, r2);
+        tmem_ld32(tS + 96, r3);
         tmem_ld_wait();
-        float v[32];
 #pragma unroll
         for (int e = 0; e < 32; ++e) {
-          v[e] = __uint_as_float(rr[e]);
-          if (edge) {
-            const int key = key0 + c * 32 + e;
-            if (key > i || key <= i - W) v[e] = -INFINITY;
-          }
+          sv[e] = __uint_as_float(r0[e]);
+          sv[e + 32] = __uint_as_float(r1[e]);
+          sv[e + 64] = __uint_as_float(r2[e]);
+          sv[e + 96] = __uint_as_float(r3[e]);
         }
-        smax = fmaxf(smax, tree_max32(v));
       }
-      const float m_new = fmaxf(m_run, smax * sl2);
-      const float mu = (m_new == -INFINITY) ? 0.f : m_new;
-      const float alpha = ex2_approx(m_run - mu);
-      m_run = m_new;
-      if (j & 1) mu1 = mu; else mu0 = mu;
+      tc_fence_before();
+      mbar_arrive(bar(SE + X));      // S_X may be overwritten by the next product
+      // Edge tile: some (row, key) pair of the tile is outside (i - W, i].
+      if (key0 + 127 > q0 || key0 <= q0 + 127 - W) {
+#pragma unroll
+        for (int e = 0; e < 128; ++e) {
+          const int key = key0 + e;
+          if (key > i || key <= i - W) sv[e] = -INFINITY;
+        }
+      }
+      const float m_tile = fmaxf(fmaxf(tree_max32(sv), tree_max32(sv + 32)),
+                                 fmaxf(tree_max32(sv + 64), tree_max32(sv + 96))) * sl2;
+      // Rescale decision (per row): a first finite max just sets m_used (l and O
+      // are still zero); a max more than the slack above m_used rescales.
+      float corr = 1.f;
+      if (m_tile > m_used + kRescaleSlack) {
+        if (m_used != -INFINITY) corr = ex2_approx(m_used - m_tile);
+        m_used = m_tile;
+      }
+      l_run *= corr;
+      const float mu = (m_used == -INFINITY) ? 0.f : m_used;
 
+      // P_X and O_X are free once the previous P V product of this warpgroup is done.
       w = mbar_wait(bar(PE + X), (j & 1) ^ 1, wc, 22);
       if (!__all_sync(0xffffffffu, w)) { ok = false; break; }
-      // pass 2: p = 2^(s * scale_log2 - mu), row sum, P (bf16) into shared memory:
-      // row r, 128-byte rows, 16-byte chunk index XOR (r & 7), keys 64.. in the second half.
-      float rs = 0.f;
-      uint8_t* prow = sP + X * kPBytes + r * 128;
-#pragma unroll 1
-      for (int c = 0; c < 4; ++c) {
-        uint32_t rr[32];
-        tmem_ld32(tS + c * 32, rr);
+      tc_fence_after();
+      if (j > 0 && __any_sync(0xffffffffu, corr != 1.f)) {
+        uint32_t o0[32], o1[32];
+        tmem_ld32(tO, o0);
+        tmem_ld32(tO + 32, o1);
         tmem_ld_wait();
-        if (c == 3) {   // S_X fully read: the next S of this warpgroup may overwrite it
-          tc_fence_before();
-          mbar_arrive(bar(SE + X));
-        }
-        float pv[32];
 #pragma unroll
         for (int e = 0; e < 32; ++e) {
-          float x = fmaf(__uint_as_float(rr[e]), sl2, -mu);
-          if (edge) {
-            const int key = key0 + c * 32 + e;
-            if (key > i || key <= i - W) x = -INFINITY;
-          }
-          pv[e] = ex2_approx(x);
+          o0[e] = __float_as_uint(__uint_as_float(o0[e]) * corr);
+          o1[e] = __float_as_uint(__uint_as_float(o1[e]) * corr);
         }
+        tmem_st32(tO, o0);
+        tmem_st32(tO + 32, o1);
+      }
+      // p = 2^(s * scale_log2 - mu), row sum, P (bf16 pairs) into TMEM
+      float rs = 0.f;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        float pv[32];
+#pragma unroll
+        for (int e = 0; e < 32; ++e) pv[e] = ex2_approx(fmaf(sv[c * 32 + e], sl2, -mu));
         float t[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e) t[e] = pv[e] + pv[e + 16];
@@ -285,56 +277,51 @@ swa_attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
 #pragma unroll
           for (int e = 0; e < wdt; ++e) t[e] += t[e + wdt];
         rs += t[0];
+        uint32_t pk[16];
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const int cc = c * 4 + q;     // 16-byte chunk 0..15 of the row
-          const uint32_t off = (cc >> 3) * (kPBytes / 2) + ((((cc & 7) ^ (r & 7))) << 4);
-          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(smem_addr(prow + off)),
-                       "r"(pack_bf16x2(pv[q * 8 + 0], pv[q * 8 + 1])), "r"(pack_bf16x2(pv[q * 8 + 2], pv[q * 8 + 3])),
-                       "r"(pack_bf16x2(pv[q * 8 + 4], pv[q * 8 + 5])), "r"(pack_bf16x2(pv[q * 8 + 6], pv[q * 8 + 7]))
-                       : "memory");
-        }
+        for (int e = 0; e < 16; ++e) pk[e] = pack_bf16x2(pv[2 * e], pv[2 * e + 1]);
+        tmem_st16(tP + c * 16, pk);
       }
-      fence_proxy_async_smem();
+      tmem_st_wait();
+      tc_fence_before();
       mbar_arrive(bar(PF + X));
-      l_run = fmaf(l_run, alpha, rs);
-      if (j > 0 && !(ok = consume_o(j - 1))) break;
+      l_run += rs;
     }
-    if (ok && nX > 0) ok = consume_o(nX - 1);
 
-    // Merge: warpgroup 1 hands (m, l, o) to warpgroup 0 through shared memory
-    // (the P buffers are idle now); warpgroup 0 writes the output.
-    float* xo = reinterpret_cast<float*>(sP + kPBytes);          // [128][64]
-    float* xm = reinterpret_cast<float*>(sP);                    // [128] m, [128] l
-    const bool okall = ok;
+    // Merge: warpgroup 1 hands (m, l) over through shared memory; warpgroup 0
+    // reads both O_0 and O_1 from TMEM and writes the output rows.
     if (X == 1) {
-      asm volatile("bar.sync 1, 256;" ::: "memory");   // P_1 no longer read by the tensor cores
-#pragma unroll
-      for (int d = 0; d < 64; ++d) xo[r * 64 + ((d + r) & 63)] = o[d];
-      xm[r] = m_run;
-      xm[128 + r] = okall ? l_run : 0.f;
-      asm volatile("bar.sync 2, 256;" ::: "memory");
+      xml[r] = m_used;
+      xml[128 + r] = ok ? l_run : 0.f;
+      asm volatile("bar.sync 1, 256;" ::: "memory");
     } else {
       asm volatile("bar.sync 1, 256;" ::: "memory");
-      asm volatile("bar.sync 2, 256;" ::: "memory");
-      const float m1 = xm[r], l1 = xm[128 + r];
-      const float M = fmaxf(m_run, m1);
-      const float f0 = (m_run == -INFINITY) ? 0.f : ex2_approx(m_run - M);
+      bool w = mbar_wait(bar(OD + 0), 0, wc, 23) && mbar_wait(bar(OD + 1), 0, wc, 24);
+      if (!__all_sync(0xffffffffu, w)) ok = false;
+      tc_fence_after();
+      const float m1 = xml[r], l1 = xml[128 + r];
+      const float M = fmaxf(m_used, m1);
+      const float f0 = (m_used == -INFINITY) ? 0.f : ex2_approx(m_used - M);
       const float f1 = (m1 == -INFINITY) ? 0.f : ex2_approx(m1 - M);
       const float inv_l = 1.0f / (l_run * f0 + l1 * f1);
-      if (ok && i < T) {
-        uint16_t* dst = static_cast<uint16_t*>(a.out) + static_cast<int64_t>(b) * a.o_batch +
-                        static_cast<int64_t>(i) * a.o_row + static_cast<int64_t>(h) * a.o_head;
+      uint16_t* dst = static_cast<uint16_t*>(a.out) + static_cast<int64_t>(b) * a.o_batch +
+                      static_cast<int64_t>(i) * a.o_row + static_cast<int64_t>(h) * a.o_head;
+#pragma unroll 1
+      for (int half = 0; half < 2; ++half) {
+        uint32_t x0[32], x1[32];
+        tmem_ld32(tmem + 192 + 32 * half + lane_off, x0);
+        tmem_ld32(tmem + 256 + 192 + 32 * half + lane_off, x1);
+        tmem_ld_wait();
+        if (ok && i < T) {
+          float v[32];
 #pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          float v[8];
-#pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            const int d = 8 * c + e;
-            v[e] = (o[d] * f0 + xo[r * 64 + ((d + r) & 63)] * f1) * inv_l;
+          for (int d = 0; d < 32; ++d) {
+            // a warpgroup without keys for this row contributes nothing (its O may be unset)
+            const float y0 = f0 != 0.f ? __uint_as_float(x0[d]) * f0 : 0.f;
+            const float y1 = f1 != 0.f ? __uint_as_float(x1[d]) * f1 : 0.f;
+            v[d] = (y0 + y1) * inv_l;
           }
-          st_global_v4(dst + 8 * c, pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]), pack_bf16x2(v[4], v[5]),
-                       pack_bf16x2(v[6], v[7]));
+          store_bf16x32(dst + 32 * half, v);
         }
       }
     }
