@@ -62,6 +62,7 @@ def parse_args(argv=None):
     ap.add_argument("--components-only", default="", help="comma list of c2,c3,c4 (profiling runs)")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-copy end-to-end pass (profiling runs)")
     ap.add_argument("--no-trace", action="store_true", help="skip the traced per-kernel pass (profiling runs)")
+    ap.add_argument("--c3-layers", type=int, default=32, help="layers of the streaming-step component (profiling runs)")
     return ap.parse_args(argv)
 
 
@@ -309,10 +310,10 @@ def component_c2(vx, torch, flush, hbm, tf):
     return out
 
 
-def component_c3(vx, torch, flush, hbm, tf):
-    cfg, layers = device_layers(vx, torch, 32, 300, "cuda")
+def component_c3(vx, torch, flush, hbm, tf, L=32):
+    cfg, layers = device_layers(vx, torch, L, 300, "cuda")
     S, n, P = 64, 4, 1000
-    ring = vx.KVRing(cfg, 32, S)
+    ring = vx.KVRing(cfg, L, S)
     g = torch.Generator(device="cuda").manual_seed(301)
     ring.k.normal_(generator=g)
     ring.v.normal_(generator=g)
@@ -336,9 +337,9 @@ def component_c3(vx, torch, flush, hbm, tf):
     for _ in range(3):
         gr.replay()
     ms_g, _, _ = timed_steps(torch, gr.replay, 10, lambda: None, torch.cuda.current_stream())
-    kv_read = 749 * 64 * 2 * 2 * 32 * S * 32           # bytes: 749 slots x 64 x bf16 x (K,V) x heads x streams x layers
-    w_read = 32 * 30146560 * 2
-    kv_write = 4 * 64 * 2 * 2 * 32 * S * 32
+    kv_read = 749 * 64 * 2 * 2 * 32 * S * L            # bytes: 749 slots x 64 x bf16 x (K,V) x heads x streams x layers
+    w_read = L * 30146560 * 2
+    kv_write = 4 * 64 * 2 * 2 * 32 * S * L
     io = 2 * S * n * 1280 * 4
     total = kv_read + w_read + kv_write + io
     ring_ms = tr["ring_attn"]["ms_per_launch"]
@@ -457,7 +458,10 @@ def main(argv=None):
     if comps_only:
         out = {}
         for c in comps_only:
-            out[c] = {"c2": component_c2, "c3": component_c3, "c4": component_c4}[c](vx, torch, flush, hbm, tf_burst)
+            if c == "c3":
+                out[c] = component_c3(vx, torch, flush, hbm, tf_burst, L=args.c3_layers)
+            else:
+                out[c] = {"c2": component_c2, "c4": component_c4}[c](vx, torch, flush, hbm, tf_burst)
         if rank == 0:
             print(json.dumps({"components": out}), flush=True)
         return 0
