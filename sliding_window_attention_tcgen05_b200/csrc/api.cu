@@ -285,10 +285,6 @@ vx_status gemm(const Launch& L, const char* name, const void* A, int64_t lda, co
   CUtensorMap tmA, tmB;
   if (!tmap_bf16_2d(&tmA, A, a.K, a.M, lda, 128)) return VX_ERR_CUDA;
   if (!tmap_bf16_2d(&tmB, Bw, a.K, a.N, a.K, bn)) return VX_ERR_CUDA;
-  if (lean) {   // few-row GEMMs stream their weights: prefetch each panel into L2
-    a.b_ptr = Bw;
-    a.ldb = a.K;
-  }
   VX_CUDA(traced(L, name, 1, [&] { return launch_gemm(L, tmA, tmB, a, epi, bn, lean); }));
   return VX_OK;
 }

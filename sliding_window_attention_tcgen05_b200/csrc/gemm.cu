@@ -258,20 +258,6 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
   if (warp == 4 && lane == 0 && blockIdx.x < num_tiles) {
     int m0, n0, ks;
     decode(blockIdx.x, m0, n0, ks);
-    if (a.b_ptr != nullptr) {
-      // Stream this unit's weight panel (BN whole rows, or each row's K slice
-      // under split-K) into L2 as large contiguous reads.
-      const uint8_t* base = static_cast<const uint8_t*>(a.b_ptr) + static_cast<int64_t>(n0) * a.ldb * 2;
-      if (splits == 1 && a.ldb == a.K) {
-        const int64_t bytes = static_cast<int64_t>(BN) * a.K * 2;
-        for (int64_t off = 0; off < bytes; off += 65536)
-          prefetch_l2_bulk(base + off, static_cast<uint32_t>(bytes - off < 65536 ? bytes - off : 65536));
-      } else {
-        const int64_t k0 = static_cast<int64_t>(ks) * nkb * kBK;
-        for (int rr = 0; rr < BN; ++rr)
-          prefetch_l2_bulk(base + (rr * a.ldb + k0) * 2, static_cast<uint32_t>(nkb * kBK * 2));
-      }
-    }
     npre = nkb < S ? nkb : S;
     for (int i = 0; i < npre; ++i) {
       mbar_arrive_expect_tx(full(i), C::kStageBytes);

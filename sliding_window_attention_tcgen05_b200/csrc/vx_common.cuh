@@ -131,12 +131,6 @@ __device__ __forceinline__ void tma_load_4d(uint32_t dst, const CUtensorMap* map
       : "memory");
 }
 
-// Asynchronous prefetch of [p, p + bytes) into L2 (bytes a multiple of 16).
-__device__ __forceinline__ void prefetch_l2_bulk(const void* p, uint32_t bytes) {
-  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(reinterpret_cast<uint64_t>(p)), "r"(bytes)
-               : "memory");
-}
-
 // L2 eviction-priority policies for cache hints.
 __device__ __forceinline__ uint64_t policy_evict_last() {
   uint64_t p;

@@ -73,10 +73,6 @@ struct GemmArgs {
   // A addressing of K-block kb (64 wide): tap = kb / kb_per_tap,
   // c = (kb % kb_per_tap) * 64, x = (tap % a_stride) * a_tap_ch + c, y = m0 + tap / a_stride.
   int kb_per_tap, a_stride, a_tap_ch;
-  // B (weights) as a plain row-major [N, K] matrix, for an L2 prefetch of each
-  // work unit's weight panel (b_ptr may be null: no prefetch).
-  const void* b_ptr;
-  int64_t ldb;
   void* out;
   int64_t ld_out;          // elements
   const uint16_t* bias;    // [N] bf16 or null
