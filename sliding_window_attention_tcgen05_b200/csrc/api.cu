@@ -42,6 +42,14 @@ const char* last_error() { return g_err; }
 static std::atomic<uint64_t> g_wait_limit_ns{1000000000ull};
 uint64_t wait_limit_ns() { return g_wait_limit_ns.load(); }
 
+bool pair_gemm_disabled() {
+  static const bool off = [] {
+    const char* e = std::getenv("VX_PAIR_GEMM");
+    return e && e[0] == '0';
+  }();
+  return off;
+}
+
 bool pdl_enabled() {
   static const bool on = [] {
     const char* e = std::getenv("VX_PDL");
@@ -279,15 +287,35 @@ GemmArgs base_args(const Launch& L, int M, int N, int K) {
   return a;
 }
 
-vx_status gemm(const Launch& L, const char* name, const void* A, int64_t lda, const void* Bw, GemmArgs& a, int epi,
-               int bn = 0, bool lean = false) {
+// Two-CTA tiles (256 x 256 per pair) for many-row GEMMs that still give every
+// pair of SMs a tile.
+bool use_pair(const GemmArgs& a, int sm) {
+  if (pair_gemm_disabled() || a.k_splits != 1 || a.N % 256 != 0) return false;
+  const int tiles = ((a.M + 255) / 256) * (a.N / 256);
+  return tiles >= sm / 2;
+}
+
+vx_status launch_any_gemm(const Launch& L, const char* name, const CUtensorMap* tmA_in, const void* Bw, int64_t ldb,
+                          GemmArgs& a, int epi, int bn, bool lean) {
+  CUtensorMap tmB;
+  if (!lean && bn == 0 && use_pair(a, L.sm_count)) {
+    if (!tmap_bf16_2d(&tmB, Bw, a.K, a.N, ldb, 128)) return VX_ERR_CUDA;
+    VX_CUDA(traced(L, name, 1, [&] { return launch_gemm_pair(L, *tmA_in, tmB, a, epi); }));
+    return VX_OK;
+  }
   if (bn == 0) bn = pick_bn(a.M, a.N, L.sm_count);
-  CUtensorMap tmA, tmB;
-  if (!tmap_bf16_2d(&tmA, A, a.K, a.M, lda, 128)) return VX_ERR_CUDA;
-  if (!tmap_bf16_2d(&tmB, Bw, a.K, a.N, a.K, bn)) return VX_ERR_CUDA;
-  VX_CUDA(traced(L, name, 1, [&] { return launch_gemm(L, tmA, tmB, a, epi, bn, lean); }));
+  if (!tmap_bf16_2d(&tmB, Bw, a.K, a.N, ldb, bn)) return VX_ERR_CUDA;
+  VX_CUDA(traced(L, name, 1, [&] { return launch_gemm(L, *tmA_in, tmB, a, epi, bn, lean); }));
   return VX_OK;
 }
+
+vx_status gemm(const Launch& L, const char* name, const void* A, int64_t lda, const void* Bw, GemmArgs& a, int epi,
+               int bn = 0, bool lean = false) {
+  CUtensorMap tmA;
+  if (!tmap_bf16_2d(&tmA, A, a.K, a.M, lda, 128)) return VX_ERR_CUDA;
+  return launch_any_gemm(L, name, &tmA, Bw, a.K, a, epi, bn, lean);
+}
+
 
 struct RingLayer {
   uint16_t* k;
@@ -499,11 +527,9 @@ vx_status run_conv_stem(const Launch& L, const float* mel, const void* w1p, cons
     a.out = cb.h1pad; a.ld_out = d;
     a.bias = static_cast<const uint16_t*>(b1);
     a.in_rows = P; a.t_valid = Tm; a.out_rows = P; a.out_off = 2;
-    const int bn = pick_bn(a.M, a.N, L.sm_count);
-    CUtensorMap tmA, tmB;
+    CUtensorMap tmA;
     if (!tmap_bf16_2d(&tmA, cb.xpad, C, int64_t(B) * P, C, 128)) return VX_ERR_CUDA;
-    if (!tmap_bf16_2d(&tmB, w1p, 3 * C, d, 3 * C, bn)) return VX_ERR_CUDA;
-    VX_CUDA(traced(L, "gemm_conv1_gelu", 1, [&] { return launch_gemm(L, tmA, tmB, a, EPI_GELU_BF16, bn); }));
+    if ((st = launch_any_gemm(L, "gemm_conv1_gelu", &tmA, w1p, 3 * C, a, EPI_GELU_BF16, 0, false)) != VX_OK) return st;
   }
   // conv2 (stride 2): h1pad viewed as [B*P/2, 2d]; output t of clip b reads
   // padded rows 2t, 2t+1, 2t+2 = (pair t, half 0), (pair t, half 1), (pair t+1, half 0).
@@ -514,13 +540,10 @@ vx_status run_conv_stem(const Launch& L, const float* mel, const void* w1p, cons
     a.out = out; a.ld_out = d;
     a.bias = static_cast<const uint16_t*>(b2);
     a.in_rows = pairs; a.t_valid = To; a.out_rows = To; a.out_off = 0;
-    const int bn = pick_bn(a.M, a.N, L.sm_count);
-    CUtensorMap tmA, tmB;
+    CUtensorMap tmA;
     if (!tmap_bf16_2d(&tmA, cb.h1pad, 2LL * d, int64_t(B) * pairs, 2LL * d, 128)) return VX_ERR_CUDA;
-    if (!tmap_bf16_2d(&tmB, w2p, 3 * d, d, 3 * d, bn)) return VX_ERR_CUDA;
-    VX_CUDA(traced(L, "gemm_conv2_gelu", 1, [&] { return launch_gemm(L, tmA, tmB, a, EPI_GELU_F32, bn); }));
+    if ((st = launch_any_gemm(L, "gemm_conv2_gelu", &tmA, w2p, 3 * d, a, EPI_GELU_F32, 0, false)) != VX_OK) return st;
   }
-  (void)st;
   return VX_OK;
 }
 

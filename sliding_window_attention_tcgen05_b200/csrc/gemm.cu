@@ -365,6 +365,184 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
   }
 }
 
+// ------------------------------------------------------------ CTA pairs --
+// Two-CTA variant for many-row GEMMs: a cluster of two CTAs computes a
+// 256 x 256 tile with tcgen05.mma.cta_group::2 (M = 256).  CTA r loads its own
+// 128 rows of A and rows [128 r, 128 r + 128) of the tile's 256 B rows, so each
+// SM stages 32 KB per 64-wide K block for 128 x 256 x 64 of MMA work (the
+// one-CTA 128 x 256 tile stages 48 KB); the leader (CTA 0) issues the MMAs.
+// TMA completions of both CTAs land on the leader's full barriers; MMA
+// completions are multicast to the empty / accumulator barriers of both CTAs;
+// both CTAs' epilogue warps release an accumulator on the leader's barrier.
+// Each CTA's epilogue handles its 128 rows x 256 columns from its own TMEM.
+constexpr int kPairBN = 256;
+constexpr int kPairStages = 6;
+constexpr int kPairStageBytes = kABytes + 128 * kBK * 2;   // A (128 rows) + half of B (128 rows)
+constexpr int kPairSmem = kPairStages * kPairStageBytes + 1024 + 256;
+
+template <int EPI>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                const __grid_constant__ GemmArgs a) {
+  constexpr int S = kPairStages;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + S * kABytes;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S * kPairStageBytes);
+  // bars: full[S] (used in CTA 0), empty[S], acc_full[2], acc_empty[2] (CTA 0), drain
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * S + 5);
+  int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  auto full = [&](int s) { return smem_addr(bars + s); };
+  auto empty = [&](int s) { return smem_addr(bars + S + s); };
+  auto acc_full = [&](int i) { return smem_addr(bars + 2 * S + i); };
+  auto acc_empty = [&](int i) { return smem_addr(bars + 2 * S + 2 + i); };
+  const uint32_t drain = smem_addr(bars + 2 * S + 4);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) { mbar_init(full(s), 1); mbar_init(empty(s), 1); }
+    for (int i = 0; i < 2; ++i) { mbar_init(acc_full(i), 1); mbar_init(acc_empty(i), 8); }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 5) {
+    tmem_alloc_pair(smem_addr(tmem_slot), 2 * kPairBN);
+    tmem_relinquish_pair();
+  }
+  if (warp == 4 && lane == 0) {
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+  }
+  tc_fence_before();
+  cluster_sync_all();   // both CTAs' barriers initialised and TMEM allocated
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  pdl_wait();
+  pdl_trigger();
+
+  const WaitCtx wc{a.status, abort_flag, a.limit_ns};
+  const int m_tiles = (a.M + 255) / 256;
+  const int num_tiles = m_tiles * (a.N / kPairBN);
+  const int nkb = a.K / kBK;
+  const int cluster = blockIdx.x >> 1;
+  const int nclusters = gridDim.x >> 1;
+
+  if (warp == 4) {
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t issued = 0, last_par = 0;
+      for (int tile = cluster; tile < num_tiles; tile += nclusters) {
+        const int m0 = (tile % m_tiles) * 256 + 128 * rank;
+        const int n0 = (tile / m_tiles) * kPairBN;
+        bool ok = true;
+        for (int kb = 0; kb < nkb; ++kb) {
+          if (!mbar_wait(empty(stage), phase ^ 1, wc, 31)) { ok = false; break; }
+          const uint32_t fb = map_to_cta(full(stage), 0);   // the leader's full barrier
+          if (rank == 0) mbar_arrive_expect_tx(full(stage), 2 * kPairStageBytes);
+          const int tap = kb / a.kb_per_tap;
+          const int c = (kb - tap * a.kb_per_tap) * kBK;
+          const int ax = (tap % a.a_stride) * a.a_tap_ch + c;
+          const int ay = m0 + tap / a.a_stride;
+          tma_load_2d_pair(smem_addr(sA + stage * kABytes), &tmA, fb, ax, ay);
+          tma_load_2d_pair(smem_addr(sB + stage * 128 * kBK * 2), &tmB, fb, kb * kBK, n0 + 128 * rank);
+          issued |= 1u << stage;
+          last_par = (last_par & ~(1u << stage)) | (phase << stage);
+          if (++stage == S) { stage = 0; phase ^= 1; }
+        }
+        if (!ok) break;
+      }
+      if (rank == 0) {   // bounded wait for the pair's copies still in flight
+        int zero = 0;
+        WaitCtx dw = wc;
+        dw.abort_flag = &zero;
+        for (int s = 0; s < S; ++s)
+          if (issued & (1u << s)) mbar_wait(full(s), (last_par >> s) & 1u, dw, 35);
+      }
+    }
+  } else if (warp == 5) {
+    if (lane == 0 && rank == 0) {
+      const uint32_t idesc = idesc_bf16_f32(256, kPairBN, 0);
+      int stage = 0;
+      uint32_t phase = 0;
+      int local = 0;
+      for (int tile = cluster; tile < num_tiles; tile += nclusters, ++local) {
+        const int ab = local & 1;
+        const uint32_t acc_par = (local >> 1) & 1;
+        if (!mbar_wait(acc_empty(ab), acc_par ^ 1, wc, 32)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + ab * kPairBN;
+        bool ok = true;
+        for (int kb = 0; kb < nkb; ++kb) {
+          if (!mbar_wait(full(stage), phase, wc, 33)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t a0 = smem_addr(sA + stage * kABytes);
+          const uint32_t b0 = smem_addr(sB + stage * 128 * kBK * 2);
+#pragma unroll
+          for (int k = 0; k < kBK / 16; ++k)
+            umma_bf16_pair(d_tmem, smem_desc_sw128(a0 + 32 * k, 16, 1024), smem_desc_sw128(b0 + 32 * k, 16, 1024),
+                           idesc, (kb | k) != 0);
+          umma_commit_pair(empty(stage), 0x3);
+          if (++stage == S) { stage = 0; phase ^= 1; }
+        }
+        if (!ok) break;
+        umma_commit_pair(acc_full(ab), 0x3);
+      }
+      umma_commit_pair(drain, 0x1);
+      int zero = 0;
+      WaitCtx dw = wc;
+      dw.abort_flag = &zero;
+      mbar_wait(drain, 0, dw, 36);
+    }
+  } else {
+    int local = 0;
+    const uint32_t acc_empty_leader0 = map_to_cta(acc_empty(0), 0);
+    const uint32_t acc_empty_leader1 = map_to_cta(acc_empty(1), 0);
+    for (int tile = cluster; tile < num_tiles; tile += nclusters, ++local) {
+      const int m0 = (tile % m_tiles) * 256 + 128 * rank;
+      const int n0 = (tile / m_tiles) * kPairBN;
+      const int ab = local & 1;
+      const uint32_t acc_par = (local >> 1) & 1;
+      bool ok = mbar_wait(acc_full(ab), acc_par, wc, 34);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      tc_fence_after();
+      const uint32_t tacc = tmem_base + ab * kPairBN + (static_cast<uint32_t>(warp * 32) << 16);
+      epilogue_tile<kPairBN, EPI>(a, tacc, m0 + warp * 32 + lane, n0, 0);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(ab ? acc_empty_leader1 : acc_empty_leader0);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync_all();   // no CTA of the pair still uses TMEM or the peer's barriers
+  if (warp == 5) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem_base, 2 * kPairBN);
+  }
+}
+
+template <int EPI>
+cudaError_t launch_pair(const Launch& L, const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmArgs& a) {
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(gemm_tc2_kernel<EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize, kPairSmem);
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  const int tiles = ((a.M + 255) / 256) * (a.N / kPairBN);
+  const int pairs = L.sm_count / 2;
+  const int grid = 2 * (tiles < pairs ? tiles : pairs);
+  return launch_kernel(gemm_tc2_kernel<EPI>, dim3(grid), dim3(kThreads), kPairSmem, L.stream, tmA, tmB, a);
+}
+
 template <int BN, int EPI, bool LEAN>
 cudaError_t launch_one(const Launch& L, const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmArgs& a) {
   using C = GemmCfg<BN, LEAN>;
@@ -402,6 +580,20 @@ cudaError_t launch_bn(const Launch& L, const CUtensorMap& tmA, const CUtensorMap
 }
 
 }  // namespace
+
+cudaError_t launch_gemm_pair(const Launch& L, const CUtensorMap& tmA, const CUtensorMap& tmB,
+                             const GemmArgs& args, int epi) {
+  if (args.M <= 0) return cudaSuccess;
+  if (args.k_splits != 1 || args.N % kPairBN != 0 || args.K % kBK != 0) return cudaErrorInvalidValue;
+  switch (epi) {
+    case EPI_F32: return launch_pair<EPI_F32>(L, tmA, tmB, args);
+    case EPI_QKV_ROPE: return launch_pair<EPI_QKV_ROPE>(L, tmA, tmB, args);
+    case EPI_SWIGLU: return launch_pair<EPI_SWIGLU>(L, tmA, tmB, args);
+    case EPI_GELU_BF16: return launch_pair<EPI_GELU_BF16>(L, tmA, tmB, args);
+    case EPI_GELU_F32: return launch_pair<EPI_GELU_F32>(L, tmA, tmB, args);
+    default: return cudaErrorInvalidValue;
+  }
+}
 
 cudaError_t launch_gemm(const Launch& L, const CUtensorMap& tmA, const CUtensorMap& tmB,
                         const GemmArgs& args, int epi, int bn, bool lean) {

@@ -27,6 +27,7 @@ struct Launch {
 int current_sm_count();
 uint64_t wait_limit_ns();
 bool pdl_enabled();   // programmatic dependent launch (default on; VX_PDL=0 disables)
+bool pair_gemm_disabled();   // two-CTA GEMM tiles (default on; VX_PAIR_GEMM=0 disables)
 
 // Launches `k` on `stream`, with programmatic dependent launch when enabled.
 template <class... KArgs, class... Args>
@@ -98,6 +99,11 @@ struct GemmArgs {
 // lean: a ~96 KB pipeline so two CTAs share an SM (bn 64 or 128; no GELU).
 cudaError_t launch_gemm(const Launch& L, const CUtensorMap& tmA, const CUtensorMap& tmB,
                         const GemmArgs& args, int epi, int bn, bool lean = false);
+
+// Two-CTA version (clusters of 2, 256 x 256 tiles, tcgen05.mma.cta_group::2):
+// tmA box {64, 128}, tmB box {64, 128}; N % 256 == 0, no split-K.
+cudaError_t launch_gemm_pair(const Launch& L, const CUtensorMap& tmA, const CUtensorMap& tmB,
+                             const GemmArgs& args, int epi);
 
 void fill_rope_freqs(GemmArgs* a, float theta, int head_dim);
 
