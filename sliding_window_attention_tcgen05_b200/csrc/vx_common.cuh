@@ -82,14 +82,30 @@ struct WaitCtx {
   uint64_t limit_ns;        // per-wait limit
 };
 
+// try_wait with a suspend-time hint: the warp may sleep in hardware for up to
+// hint_ns and is woken as soon as the phase completes.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t bar, uint32_t parity, uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0;
+}
+
 // Waits until the phase with parity `parity` of `bar` has completed.  Returns
 // false (and records a timeout) once limit_ns has passed, or at once when
-// another thread of the CTA already gave up.  Never spins forever.
+// another thread of the CTA already gave up.  Never spins forever.  The wait
+// itself sleeps in hardware (woken on completion); the clock and the abort flag
+// are looked at only between those sleeps.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, const WaitCtx& w, int where) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   while (true) {
-    if (mbar_try_wait(bar, parity)) return true;
+    if (mbar_try_wait_sleep(bar, parity, 20000u)) return true;
     if (*w.abort_flag) return false;
     if (globaltimer_ns() - t0 > w.limit_ns) {
       *w.abort_flag = 1;
