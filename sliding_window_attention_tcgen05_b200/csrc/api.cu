@@ -254,27 +254,6 @@ size_t layer_ws_bytes(const vx_layer_cfg& c, int64_t M) {
   return align_up(cv.off, kAlign);
 }
 
-// Chooses the N tile: the widest of 256 / 128 that still fills the GPU;
-// for few-row GEMMs (weight streaming) also 64, down to min_bn.
-int pick_bn(int M, int N, int sm, int min_bn = 128) {
-  const int mt = (M + 127) / 128;
-  int bn = 256;
-  for (; bn > min_bn; bn /= 2)
-    if (N % bn == 0 && mt * (N / bn) >= sm) return bn;
-  return bn;
-}
-
-// Split-K factor for a few-row GEMM: the largest of 1, 2, 4, 8 that divides the
-// K blocks and keeps the work units within about one wave.
-int pick_splits(int M, int N, int K, int bn, int sm) {
-  const int units = ((M + 127) / 128) * (N / bn);
-  const int nkb = K / 64;
-  int s = 1;
-  for (int c = 2; c <= 8; c *= 2)
-    if (nkb % c == 0 && nkb / c >= 4 && units * c <= sm) s = c;
-  return s;
-}
-
 GemmArgs base_args(const Launch& L, int M, int N, int K) {
   GemmArgs a;
   std::memset(&a, 0, sizeof(a));
@@ -287,33 +266,27 @@ GemmArgs base_args(const Launch& L, int M, int N, int K) {
   return a;
 }
 
-// Two-CTA tiles (256 x 256 per pair) for many-row GEMMs that still give every
-// pair of SMs a tile.
-bool use_pair(const GemmArgs& a, int sm) {
-  if (pair_gemm_disabled() || a.k_splits != 1 || a.N % 256 != 0) return false;
-  const int tiles = ((a.M + 255) / 256) * (a.N / 256);
-  return tiles >= sm / 2;
-}
-
-vx_status launch_any_gemm(const Launch& L, const char* name, const CUtensorMap* tmA_in, const void* Bw, int64_t ldb,
-                          GemmArgs& a, int epi, int bn, bool lean) {
-  CUtensorMap tmB;
-  if (!lean && bn == 0 && use_pair(a, L.sm_count)) {
-    if (!tmap_bf16_2d(&tmB, Bw, a.K, a.N, ldb, 128)) return VX_ERR_CUDA;
-    VX_CUDA(traced(L, name, 1, [&] { return launch_gemm_pair(L, *tmA_in, tmB, a, epi); }));
-    return VX_OK;
+// Plans, encodes B's tensor map for and launches one GEMM; on return
+// a.k_splits holds the number of partial sums written (1 unless max_splits > 1).
+vx_status launch_any_gemm(const Launch& L, const char* name, const CUtensorMap* tmA, const void* Bw, int64_t ldb,
+                          GemmArgs& a, int epi, int max_splits = 1) {
+  const GemmPlan p = plan_gemm(a.M, a.N, a.K, epi, max_splits, L.sm_count);
+  if (p.bn == 0) {
+    set_error("%s: no GEMM tile shape fits N=%d K=%d", name, a.N, a.K);
+    return VX_ERR_UNSUPPORTED;
   }
-  if (bn == 0) bn = pick_bn(a.M, a.N, L.sm_count);
-  if (!tmap_bf16_2d(&tmB, Bw, a.K, a.N, ldb, bn)) return VX_ERR_CUDA;
-  VX_CUDA(traced(L, name, 1, [&] { return launch_gemm(L, *tmA_in, tmB, a, epi, bn, lean); }));
+  a.k_splits = p.splits;
+  CUtensorMap tmB;
+  if (!tmap_bf16_2d(&tmB, Bw, a.K, a.N, ldb, p.pair ? p.bn / 2 : p.bn)) return VX_ERR_CUDA;
+  VX_CUDA(traced(L, name, 1, [&] { return launch_gemm(L, *tmA, tmB, a, epi, p); }));
   return VX_OK;
 }
 
 vx_status gemm(const Launch& L, const char* name, const void* A, int64_t lda, const void* Bw, GemmArgs& a, int epi,
-               int bn = 0, bool lean = false) {
+               int max_splits = 1) {
   CUtensorMap tmA;
   if (!tmap_bf16_2d(&tmA, A, a.K, a.M, lda, 128)) return VX_ERR_CUDA;
-  return launch_any_gemm(L, name, &tmA, Bw, a.K, a, epi, bn, lean);
+  return launch_any_gemm(L, name, &tmA, Bw, a.K, a, epi, max_splits);
 }
 
 
@@ -436,7 +409,6 @@ vx_status run_layer_stream(const Launch& L, const vx_layer_cfg& c, const vx_laye
   const int64_t pstride = static_cast<int64_t>(M) * d;
   const float sl2 = (1.0f / std::sqrt(static_cast<float>(c.head_dim))) * 1.4426950408889634f;
   const LayerBufs& bf = sb.lb;
-  const int slots = 2 * L.sm_count;   // lean GEMMs: two CTAs per SM
   vx_status st;
   // 1. x_l = reduce(in); y0 = RMSNorm(x_l)
   const bool pending_in = in.parts != nullptr || in.bias != nullptr;
@@ -455,9 +427,7 @@ vx_status run_layer_stream(const Launch& L, const vx_layer_cfg& c, const vx_laye
     a.pos_arr = ring.pos;
     a.rope_cols = 2 * HD;
     fill_rope_freqs(&a, c.rope_theta, c.head_dim);
-    if ((st = gemm(L, "gemm_qkv_rope", bf.y0, d, w.wqkv, a, EPI_QKV_ROPE, pick_bn(M, 3 * HD, slots, 64), true)) !=
-        VX_OK)
-      return st;
+    if ((st = gemm(L, "gemm_qkv_rope", bf.y0, d, w.wqkv, a, EPI_QKV_ROPE)) != VX_OK) return st;
   }
   // 3. ring attention (reads every old in-window slot, then appends)
   VX_CUDA(traced(L, "ring_attn", 1, [&] {
@@ -466,12 +436,11 @@ vx_status run_layer_stream(const Launch& L, const vx_layer_cfg& c, const vx_laye
   // 4. O-projection, split-K partial sums
   int so;
   {
-    const int bn = pick_bn(M, d, slots, 64);
-    so = pick_splits(M, d, HD, bn, slots);
     GemmArgs a = base_args(L, M, d, HD);
     a.out = sb.parts; a.ld_out = d;
-    a.k_splits = so; a.split_stride = pstride;
-    if ((st = gemm(L, "gemm_o_splitk", bf.att, HD, w.wo, a, EPI_F32, bn, true)) != VX_OK) return st;
+    a.split_stride = pstride;
+    if ((st = gemm(L, "gemm_o_splitk", bf.att, HD, w.wo, a, EPI_F32, kMaxSplits)) != VX_OK) return st;
+    so = a.k_splits;
   }
   // 5. h = x_l + bo + sum P_o; y1 = RMSNorm(h)
   VX_CUDA(traced(L, "rmsnorm", 1, [&] {
@@ -483,17 +452,15 @@ vx_status run_layer_stream(const Launch& L, const vx_layer_cfg& c, const vx_laye
     GemmArgs a = base_args(L, M, 2 * F, d);
     a.out = bf.act; a.ld_out = F;
     a.bias = static_cast<const uint16_t*>(w.bgu);
-    if ((st = gemm(L, "gemm_gate_up_swiglu", bf.y0, d, w.wgu, a, EPI_SWIGLU, 128, true)) != VX_OK) return st;
+    if ((st = gemm(L, "gemm_gate_up_swiglu", bf.y0, d, w.wgu, a, EPI_SWIGLU)) != VX_OK) return st;
   }
   // 7. down, split-K partial sums; the layer output stays pending
   {
-    const int bn = pick_bn(M, d, slots, 64);
-    const int sd = pick_splits(M, d, F, bn, slots);
     GemmArgs a = base_args(L, M, d, F);
     a.out = sb.parts; a.ld_out = d;
-    a.k_splits = sd; a.split_stride = pstride;
-    if ((st = gemm(L, "gemm_down_splitk", bf.act, F, w.wd, a, EPI_F32, bn, true)) != VX_OK) return st;
-    *out = Pending{bf.h, sb.parts, sd, static_cast<const uint16_t*>(w.bd)};
+    a.split_stride = pstride;
+    if ((st = gemm(L, "gemm_down_splitk", bf.act, F, w.wd, a, EPI_F32, kMaxSplits)) != VX_OK) return st;
+    *out = Pending{bf.h, sb.parts, a.k_splits, static_cast<const uint16_t*>(w.bd)};
   }
   return VX_OK;
 }
@@ -529,7 +496,7 @@ vx_status run_conv_stem(const Launch& L, const float* mel, const void* w1p, cons
     a.in_rows = P; a.t_valid = Tm; a.out_rows = P; a.out_off = 2;
     CUtensorMap tmA;
     if (!tmap_bf16_2d(&tmA, cb.xpad, C, int64_t(B) * P, C, 128)) return VX_ERR_CUDA;
-    if ((st = launch_any_gemm(L, "gemm_conv1_gelu", &tmA, w1p, 3 * C, a, EPI_GELU_BF16, 0, false)) != VX_OK) return st;
+    if ((st = launch_any_gemm(L, "gemm_conv1_gelu", &tmA, w1p, 3 * C, a, EPI_GELU_BF16)) != VX_OK) return st;
   }
   // conv2 (stride 2): h1pad viewed as [B*P/2, 2d]; output t of clip b reads
   // padded rows 2t, 2t+1, 2t+2 = (pair t, half 0), (pair t, half 1), (pair t+1, half 0).
@@ -542,7 +509,7 @@ vx_status run_conv_stem(const Launch& L, const float* mel, const void* w1p, cons
     a.in_rows = pairs; a.t_valid = To; a.out_rows = To; a.out_off = 0;
     CUtensorMap tmA;
     if (!tmap_bf16_2d(&tmA, cb.h1pad, 2LL * d, int64_t(B) * pairs, 2LL * d, 128)) return VX_ERR_CUDA;
-    if ((st = launch_any_gemm(L, "gemm_conv2_gelu", &tmA, w2p, 3 * d, a, EPI_GELU_F32, 0, false)) != VX_OK) return st;
+    if ((st = launch_any_gemm(L, "gemm_conv2_gelu", &tmA, w2p, 3 * d, a, EPI_GELU_F32)) != VX_OK) return st;
   }
   return VX_OK;
 }

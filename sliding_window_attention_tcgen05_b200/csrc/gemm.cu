@@ -1,14 +1,32 @@
-// gemm.cu -- persistent, warp-specialised tcgen05 GEMM for sm_100a with the
+// gemm.cu -- persistent, warp-specialised tcgen05 GEMMs for sm_100a with the
 // fused epilogues of the encoder layer (bias, RoPE, SwiGLU, GELU, residual).
 //
 //   D[M, N] = A[M, K] * B[N, K]^T,  A and B bf16 K-major, fp32 accumulate in TMEM.
 //
-// CTA = 6 warps: warps 0-3 epilogue (TMEM lanes 0-127 = tile rows), warp 4 TMA
-// producer, warp 5 MMA issuer (owns the TMEM allocation).  128 x BN x 64 tiles,
-// a STAGES-deep TMA -> shared memory ring guarded by mbarriers, and two TMEM
-// accumulators so the epilogue of tile i overlaps the main loop of tile i+1.
-// Tiles are visited M-fastest so the CTAs resident at one time share the same
-// weight (B) panel through L2.
+// Two kernels share one structure and one epilogue:
+//   gemm_tc_kernel<BN>   one CTA per 128 x BN tile (BN 128 / 256);
+//   gemm_tc2_kernel<BN>  a cluster of two CTAs per 256 x BN tile, issued as
+//                        tcgen05.mma.cta_group::2 (M = 256) by the leader CTA.
+// CTA = 10 warps: warps 0-7 epilogue (warp w reads TMEM lanes 32 (w % 4) ..,
+// i.e. 32 tile rows, and half of the tile's columns), warp 8 TMA producer,
+// warp 9 MMA issuer (owns the TMEM allocation).  A 192 KB TMA ->
+// shared memory ring guarded by mbarriers feeds the MMAs; two TMEM
+// accumulators let the epilogue of one tile overlap the main loop of the next.
+// Work units (m tile, K split, n tile) are visited M-fastest so the CTAs
+// resident at one time share a weight (B) panel through L2.
+//
+// The main loop is bound by how fast TMA can fill one SM's shared memory, so
+// the tile shape is chosen to move the fewest bytes per MMA: a CTA pair
+// stages 16 KB of A and BN/2 rows of B per 64-wide K block for 128 x BN of
+// MMA work (plan_gemm picks the shape, see below).
+//
+// Epilogue: each warp reads 32 rows x 32 columns at a time from TMEM (one row
+// per lane), applies the row-wise part of the epilogue (bias, RoPE pairs,
+// SwiGLU gate x up, GELU), transposes the chunk through a swizzled 2 KB
+// shared-memory buffer and stores it with four lanes per row, so every store
+// writes whole 32-byte sectors.  The tile's bias is staged in shared memory,
+// and the RoPE angles and the residual of the first chunk are prepared before
+// the accumulator is ready.
 #include <cmath>
 #include <cstdio>
 
@@ -18,33 +36,72 @@ namespace vx {
 
 namespace {
 
-constexpr int kThreads = 192;
+constexpr int kThreads = 320;   // warps 0-7 epilogue, 8 TMA producer, 9 MMA issuer
+constexpr int kProducerWarp = 8;
+constexpr int kMmaWarp = 9;
 constexpr int kBM = 128;
 constexpr int kBK = 64;
 constexpr int kABytes = kBM * kBK * 2;
+constexpr int kRingBytes = 192 * 1024;        // TMA ring per CTA
+constexpr int kStgBytes = 8 * 2048;           // per epilogue warp: 32 rows x 64 bytes
+constexpr int kBiasBytes = 8 * 256 * 2;       // per epilogue warp: the tile's bias, BN <= 256
+constexpr int kBarBytes = 256;
 
-// LEAN: about 96 KB of pipeline so that two CTAs share an SM (few-row GEMMs,
-// whose work units must all be resident in one round).
-template <int BN, bool LEAN>
-struct GemmCfg {
-  static constexpr int kBBytes = BN * kBK * 2;
-  static constexpr int kStageBytes = kABytes + kBBytes;
-  static constexpr int kStages = LEAN ? (96 * 1024) / kStageBytes : ((BN == 256) ? 4 : (BN == 128 ? 6 : 8));
-  static constexpr int kTmemCols = 2 * BN;  // two accumulators
-  static constexpr int kSmem = kStages * kStageBytes + 1024 + 256;
+// Shared memory: [ring][staging][bias][barriers], 1024-aligned base.
+template <int STAGE_BYTES>
+struct SmemCfg {
+  static constexpr int kStages = kRingBytes / STAGE_BYTES;
+  static constexpr int kStg = kStages * STAGE_BYTES;
+  static constexpr int kBias = kStg + kStgBytes;
+  static constexpr int kBars = kBias + kBiasBytes;
+  static constexpr int kTotal = kBars + kBarBytes + 1024;
+  static_assert(kStages >= 4, "ring too shallow");
+  static_assert(kTotal <= 227 * 1024, "shared memory");
 };
 
 __device__ __forceinline__ float gelu_erf(float x) {
   return 0.5f * x * (1.0f + erff(x * 0.70710678118654752f));
 }
 
-__device__ __forceinline__ float silu_f(float x) { return x / (1.0f + expf(-x)); }
+__device__ __forceinline__ float rcp_approx(float x) {
+  float y;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+// silu(x) = x * sigmoid(x) = x / (1 + 2^(-x log2 e)); the hardware 2^x and
+// reciprocal are accurate to ~2^-22 relative, far below the bf16 rounding of
+// the result.  Saturates correctly: x -> -inf gives -0, x -> +inf gives x.
+__device__ __forceinline__ float silu_f(float x) {
+  return x * rcp_approx(1.0f + ex2_approx(-1.4426950408889634f * x));
+}
 
-__device__ __forceinline__ void add_bias32(float (&v)[32], const uint16_t* bias) {
-  const uint4* bp = reinterpret_cast<const uint4*>(bias);
+// Waits for this thread's outstanding tcgen05.ld; the registers are passed
+// through so that no use of them can be scheduled before the wait.
+__device__ __forceinline__ void tmem_ld_wait_regs(uint32_t (&r)[32]) {
+  asm volatile("tcgen05.wait::ld.sync.aligned;"
+               : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]),
+                 "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), "+r"(r[14]),
+                 "+r"(r[15]), "+r"(r[16]), "+r"(r[17]), "+r"(r[18]), "+r"(r[19]), "+r"(r[20]), "+r"(r[21]),
+                 "+r"(r[22]), "+r"(r[23]), "+r"(r[24]), "+r"(r[25]), "+r"(r[26]), "+r"(r[27]), "+r"(r[28]),
+                 "+r"(r[29]), "+r"(r[30]), "+r"(r[31])
+               :
+               : "memory");
+}
+__device__ __forceinline__ void tmem_ld2_wait(uint32_t (&r0)[32], uint32_t (&r1)[32]) {
+  tmem_ld_wait_regs(r0);
+  asm volatile("" : "+r"(r1[0]), "+r"(r1[1]), "+r"(r1[2]), "+r"(r1[3]), "+r"(r1[4]), "+r"(r1[5]), "+r"(r1[6]),
+               "+r"(r1[7]), "+r"(r1[8]), "+r"(r1[9]), "+r"(r1[10]), "+r"(r1[11]), "+r"(r1[12]), "+r"(r1[13]),
+               "+r"(r1[14]), "+r"(r1[15]), "+r"(r1[16]), "+r"(r1[17]), "+r"(r1[18]), "+r"(r1[19]), "+r"(r1[20]),
+               "+r"(r1[21]), "+r"(r1[22]), "+r"(r1[23]), "+r"(r1[24]), "+r"(r1[25]), "+r"(r1[26]), "+r"(r1[27]),
+               "+r"(r1[28]), "+r"(r1[29]), "+r"(r1[30]), "+r"(r1[31]));
+}
+
+// v[i] += bias[i], i < 32, bias in shared memory (every lane reads the same words).
+__device__ __forceinline__ void add_bias32_smem(float (&v)[32], const uint16_t* sb) {
+  const uint4* bp = reinterpret_cast<const uint4*>(sb);
 #pragma unroll
   for (int j = 0; j < 4; ++j) {
-    const uint4 w = __ldg(bp + j);
+    const uint4 w = bp[j];
     v[8 * j + 0] += bf16lo(w.x); v[8 * j + 1] += bf16hi(w.x);
     v[8 * j + 2] += bf16lo(w.y); v[8 * j + 3] += bf16hi(w.y);
     v[8 * j + 4] += bf16lo(w.z); v[8 * j + 5] += bf16hi(w.z);
@@ -52,159 +109,264 @@ __device__ __forceinline__ void add_bias32(float (&v)[32], const uint16_t* bias)
   }
 }
 
-__device__ __forceinline__ void store_bf16x32(uint16_t* dst, const float (&v)[32]) {
+// Staging buffer of one warp: 32 rows x four 16-byte slots (32 bf16 or 16
+// fp32 per row).  Slot j of row r sits at j ^ ((r >> 1) & 3), so that the
+// row-wise writes (one row per lane) and the column-wise reads (four lanes per
+// row) both touch eight distinct 16-byte bank groups per quarter warp.
+__device__ __forceinline__ int stg_slot(int r, int j) { return r * 4 + (j ^ ((r >> 1) & 3)); }
+
+__device__ __forceinline__ void stage_bf16x32(uint4* stg, int lane, const float (&v)[32]) {
 #pragma unroll
-  for (int j = 0; j < 4; ++j) {
-    st_global_v4(dst + 8 * j, pack_bf16x2(v[8 * j + 0], v[8 * j + 1]),
-                 pack_bf16x2(v[8 * j + 2], v[8 * j + 3]), pack_bf16x2(v[8 * j + 4], v[8 * j + 5]),
-                 pack_bf16x2(v[8 * j + 6], v[8 * j + 7]));
+  for (int j = 0; j < 4; ++j)
+    stg[stg_slot(lane, j)] = make_uint4(pack_bf16x2(v[8 * j + 0], v[8 * j + 1]), pack_bf16x2(v[8 * j + 2], v[8 * j + 3]),
+                                        pack_bf16x2(v[8 * j + 4], v[8 * j + 5]), pack_bf16x2(v[8 * j + 6], v[8 * j + 7]));
+}
+__device__ __forceinline__ void stage_f32x16(uint4* stg, int lane, const float* v) {
+#pragma unroll
+  for (int j = 0; j < 4; ++j)
+    stg[stg_slot(lane, j)] = make_uint4(__float_as_uint(v[4 * j]), __float_as_uint(v[4 * j + 1]),
+                                        __float_as_uint(v[4 * j + 2]), __float_as_uint(v[4 * j + 3]));
+}
+
+__device__ __forceinline__ void st_global_u4(void* p, uint4 v) {
+  asm volatile("st.global.v4.b32 [%0], {%1, %2, %3, %4};" ::"l"(p), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
+               : "memory");
+}
+
+// Output row of source row m (see GemmArgs); ok = the row is stored.
+__device__ __forceinline__ int64_t out_row(const GemmArgs& a, int m, bool& ok, int& b, int& t) {
+  b = m / a.in_rows;
+  t = m - b * a.in_rows;
+  ok = m < a.M && t < a.t_valid;
+  return static_cast<int64_t>(b) * a.out_rows + a.out_off + t;
+}
+
+// Rows this lane stores in the column-wise phase: mw + (lane >> 2) + 8 i.
+struct StoreRows {
+  int64_t drow[4];
+  uint32_t ok;
+};
+__device__ __forceinline__ StoreRows store_rows(const GemmArgs& a, int mw, int lane) {
+  StoreRows s;
+  s.ok = 0;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    bool ok;
+    int b, t;
+    s.drow[i] = out_row(a, mw + (lane >> 2) + 8 * i, ok, b, t);
+    s.ok |= static_cast<uint32_t>(ok) << i;
+  }
+  return s;
+}
+
+// Stores the warp's staged bf16 chunk: 8 columns col0 + 8 (lane & 3) .. +7 of
+// rows (lane >> 2) + 8 i.
+__device__ __forceinline__ void store_bf16_chunk(uint16_t* out, int64_t ld_out, const StoreRows& sr, const uint4* stg,
+                                                 int lane, int col0) {
+  const int jj = lane & 3;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int rr = (lane >> 2) + 8 * i;
+    const uint4 v = stg[stg_slot(rr, jj)];
+    if (sr.ok & (1u << i)) st_global_u4(out + sr.drow[i] * ld_out + col0 + 8 * jj, v);
   }
 }
 
-__device__ __forceinline__ void store_f32x32(float* dst, const float (&v)[32]) {
-#pragma unroll
-  for (int j = 0; j < 8; ++j) {
-    st_global_v4(dst + 4 * j, __float_as_uint(v[4 * j + 0]), __float_as_uint(v[4 * j + 1]),
-                 __float_as_uint(v[4 * j + 2]), __float_as_uint(v[4 * j + 3]));
-  }
+// Per warp: TMEM lane quarter q = warp & 3 (tile rows 32 q ..), and one half
+// of the tile's column work (warp >> 2).  Everything of a tile's epilogue
+// that does not need the accumulator is done before waiting for it: the bias
+// into this warp's shared-memory copy, the RoPE angles of this lane's row, the
+// residual of the first chunk.  Warps never wait for one another, so a warp
+// that leaves the tile loop on a timeout cannot stall the others.
+template <int BN, int EPI>
+struct EpiPre {
+  StoreRows sr;
+  float cs[EPI == EPI_QKV_ROPE ? 32 : 1];
+  float sn[EPI == EPI_QKV_ROPE ? 32 : 1];
+  float4 res[EPI == EPI_F32 ? 4 : 1];
+};
+
+// First column of this warp's half of an EPI_F32 / GELU tile.
+template <int BN>
+__device__ __forceinline__ int half_col0(int warp) { return (warp >> 2) * (BN / 2); }
+
+__device__ __forceinline__ float4 ld_res4(const GemmArgs& a, const StoreRows& sr, int i, int col) {
+  return __ldg(reinterpret_cast<const float4*>(a.res + sr.drow[i] * a.ld_res + col));
 }
 
 template <int BN, int EPI>
-__device__ __forceinline__ void epilogue_tile(const GemmArgs& a, uint32_t tacc, int m, int n0, int ks) {
-  const bool in_range = m < a.M;
-  const int b = m / a.in_rows;
-  const int t = m - b * a.in_rows;
-  const bool valid = in_range && t < a.t_valid;
-  const int64_t drow = static_cast<int64_t>(b) * a.out_rows + a.out_off + t;
-
-  if constexpr (EPI == EPI_QKV_ROPE && BN == 64) {
-    // one head per tile: rotate while reading (no sin/cos table kept)
-    uint32_t r0[32], r1[32];
-    tmem_ld32(tacc, r0);
-    tmem_ld32(tacc + 32, r1);
-    tmem_ld_wait();
-    if (valid) {
-      float x0[32], x1[32];
-#pragma unroll
-      for (int i = 0; i < 32; ++i) { x0[i] = __uint_as_float(r0[i]); x1[i] = __uint_as_float(r1[i]); }
-      if (a.bias) { add_bias32(x0, a.bias + n0); add_bias32(x1, a.bias + n0 + 32); }
-      if (n0 < a.rope_cols) {
-        const float posf = static_cast<float>((a.pos_arr ? a.pos_arr[b] : a.pos0) + t);
-#pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          float sn, cs;
-          rope_sincos(posf, a.inv_freq_hi[j], a.inv_freq_lo[j], &sn, &cs);
-          const float u = x0[j], w = x1[j];
-          x0[j] = u * cs - w * sn;
-          x1[j] = w * cs + u * sn;
-        }
-      }
-      uint16_t* dst = static_cast<uint16_t*>(a.out) + drow * a.ld_out + n0;
-      store_bf16x32(dst, x0);
-      store_bf16x32(dst + 32, x1);
-    }
-  } else if constexpr (EPI == EPI_QKV_ROPE) {
-    float cs[32], sn[32];
-    const bool rope_tile = n0 < a.rope_cols;
-    if (rope_tile && valid) {
-      const int64_t pos = (a.pos_arr ? a.pos_arr[b] : a.pos0) + t;
+__device__ __forceinline__ void epilogue_prepare(const GemmArgs& a, EpiPre<BN, EPI>& p, uint16_t* sbias, int m0,
+                                                 int n0, int ks, int warp, int lane) {
+  const bool first_part = ks == 0;
+  if (a.bias && first_part) {   // the previous tile's reads of sbias ended at a __syncwarp
+    const uint4* src = reinterpret_cast<const uint4*>(a.bias + n0);
+    for (int i = lane; i < BN / 8; i += 32) reinterpret_cast<uint4*>(sbias)[i] = __ldg(src + i);
+  }
+  const int mw = m0 + (warp & 3) * 32;
+  p.sr = store_rows(a, mw, lane);
+  if constexpr (EPI == EPI_QKV_ROPE) {
+    if (n0 < a.rope_cols) {
+      bool ok;
+      int b, t;
+      out_row(a, mw + lane, ok, b, t);
+      const int64_t pos = (a.pos_arr ? (ok ? a.pos_arr[b] : 0) : a.pos0) + t;
       const float posf = static_cast<float>(pos);
 #pragma unroll
-      for (int j = 0; j < 32; ++j) rope_sincos(posf, a.inv_freq_hi[j], a.inv_freq_lo[j], &sn[j], &cs[j]);
+      for (int j = 0; j < 32; ++j) rope_sincos(posf, a.inv_freq_hi[j], a.inv_freq_lo[j], &p.sn[j], &p.cs[j]);
     }
+  }
+  if constexpr (EPI == EPI_F32) {
+    const int col = n0 + half_col0<BN>(warp) + 4 * (lane & 3);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      p.res[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (a.res && first_part && (p.sr.ok & (1u << i))) p.res[i] = ld_res4(a, p.sr, i, col);
+    }
+  }
+  __syncwarp();   // the bias is visible to the whole warp
+}
+
+// The accumulator part: tacc = this warp's TMEM lanes at the tile's column 0.
+template <int BN, int EPI>
+__device__ __forceinline__ void epilogue_tile(const GemmArgs& a, EpiPre<BN, EPI>& p, const uint16_t* sbias,
+                                              uint4* stg, uint32_t tacc, int n0, int ks, int warp, int lane) {
+  const bool use_bias = a.bias != nullptr && ks == 0;
+  const int hf = warp >> 2;
+  if constexpr (EPI == EPI_QKV_ROPE) {
+    // heads of 64 columns; this warp takes half of them
+    const bool rope = n0 < a.rope_cols;
+    uint16_t* out = static_cast<uint16_t*>(a.out);
 #pragma unroll 1
-    for (int c = 0; c < BN; c += 64) {
+    for (int c = hf * (BN / 2); c < (hf + 1) * (BN / 2); c += 64) {
       uint32_t r0[32], r1[32];
       tmem_ld32(tacc + c, r0);
       tmem_ld32(tacc + c + 32, r1);
-      tmem_ld_wait();
-      if (valid) {
-        const int n = n0 + c;
-        float x0[32], x1[32];
+      tmem_ld2_wait(r0, r1);
+      float x0[32], x1[32];
 #pragma unroll
-        for (int i = 0; i < 32; ++i) { x0[i] = __uint_as_float(r0[i]); x1[i] = __uint_as_float(r1[i]); }
-        if (a.bias) { add_bias32(x0, a.bias + n); add_bias32(x1, a.bias + n + 32); }
-        if (n < a.rope_cols) {
+      for (int i = 0; i < 32; ++i) { x0[i] = __uint_as_float(r0[i]); x1[i] = __uint_as_float(r1[i]); }
+      if (use_bias) { add_bias32_smem(x0, sbias + c); add_bias32_smem(x1, sbias + c + 32); }
+      if (rope) {
 #pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            const float u = x0[j], w = x1[j];
-            x0[j] = u * cs[j] - w * sn[j];
-            x1[j] = w * cs[j] + u * sn[j];
-          }
+        for (int j = 0; j < 32; ++j) {
+          const float u = x0[j], w = x1[j];
+          x0[j] = u * p.cs[j] - w * p.sn[j];
+          x1[j] = w * p.cs[j] + u * p.sn[j];
         }
-        uint16_t* dst = static_cast<uint16_t*>(a.out) + drow * a.ld_out + n;
-        store_bf16x32(dst, x0);
-        store_bf16x32(dst + 32, x1);
       }
+      stage_bf16x32(stg, lane, x0);
+      __syncwarp();
+      store_bf16_chunk(out, a.ld_out, p.sr, stg, lane, n0 + c);
+      __syncwarp();
+      stage_bf16x32(stg, lane, x1);
+      __syncwarp();
+      store_bf16_chunk(out, a.ld_out, p.sr, stg, lane, n0 + c + 32);
+      __syncwarp();
     }
   } else if constexpr (EPI == EPI_SWIGLU) {
+    // units of 32 outputs: gate columns g + hh .., up columns g + 64 + hh ..
+    constexpr int kUnits = BN / 64;
+    uint16_t* out = static_cast<uint16_t*>(a.out);
 #pragma unroll 1
-    for (int g = 0; g < BN; g += 128) {
-#pragma unroll 1
-      for (int hh = 0; hh < 64; hh += 32) {
-        uint32_t rg[32], ru[32];
-        tmem_ld32(tacc + g + hh, rg);
-        tmem_ld32(tacc + g + 64 + hh, ru);
-        tmem_ld_wait();
-        if (valid) {
-          float gv[32], uv[32];
+    for (int u = hf * (kUnits / 2); u < (hf + 1) * (kUnits / 2); ++u) {
+      const int g = (u >> 1) * 128, hh = (u & 1) * 32;
+      uint32_t rg[32], ru[32];
+      tmem_ld32(tacc + g + hh, rg);
+      tmem_ld32(tacc + g + 64 + hh, ru);
+      tmem_ld2_wait(rg, ru);
+      float gv[32], uv[32];
 #pragma unroll
-          for (int i = 0; i < 32; ++i) { gv[i] = __uint_as_float(rg[i]); uv[i] = __uint_as_float(ru[i]); }
-          if (a.bias) { add_bias32(gv, a.bias + n0 + g + hh); add_bias32(uv, a.bias + n0 + g + 64 + hh); }
+      for (int i = 0; i < 32; ++i) { gv[i] = __uint_as_float(rg[i]); uv[i] = __uint_as_float(ru[i]); }
+      if (use_bias) { add_bias32_smem(gv, sbias + g + hh); add_bias32_smem(uv, sbias + g + 64 + hh); }
 #pragma unroll
-          for (int i = 0; i < 32; ++i) gv[i] = silu_f(gv[i]) * uv[i];
-          const int f = (n0 + g) / 2 + hh;
-          store_bf16x32(static_cast<uint16_t*>(a.out) + drow * a.ld_out + f, gv);
-        }
-      }
+      for (int i = 0; i < 32; ++i) gv[i] = silu_f(gv[i]) * uv[i];
+      stage_bf16x32(stg, lane, gv);
+      __syncwarp();
+      store_bf16_chunk(out, a.ld_out, p.sr, stg, lane, (n0 + g) / 2 + hh);
+      __syncwarp();
     }
   } else {
+    const bool use_res = EPI == EPI_F32 && a.res != nullptr && ks == 0;
+    const int jj = lane & 3;
+    const int c0 = half_col0<BN>(warp);
 #pragma unroll 1
-    for (int c = 0; c < BN; c += 32) {
+    for (int c = c0; c < c0 + BN / 2; c += 32) {
       uint32_t r[32];
       tmem_ld32(tacc + c, r);
-      tmem_ld_wait();
-      if (valid) {
-        const int n = n0 + c;
-        float v[32];
+      tmem_ld_wait_regs(r);
+      float v[32];
 #pragma unroll
-        for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
-        if (a.bias) add_bias32(v, a.bias + n);
-        if constexpr (EPI == EPI_F32) {
-          if (a.res) {
-            const float4* rp = reinterpret_cast<const float4*>(a.res + drow * a.ld_res + n);
+      for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+      if (use_bias) add_bias32_smem(v, sbias + c);
+      if constexpr (EPI == EPI_GELU_BF16) {
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
-              const float4 q = rp[j];
-              v[4 * j] += q.x; v[4 * j + 1] += q.y; v[4 * j + 2] += q.z; v[4 * j + 3] += q.w;
-            }
-          }
-          store_f32x32(static_cast<float*>(a.out) + ks * a.split_stride + drow * a.ld_out + n, v);
-        } else {
+        for (int i = 0; i < 32; ++i) v[i] = gelu_erf(v[i]);
+        stage_bf16x32(stg, lane, v);
+        __syncwarp();
+        store_bf16_chunk(static_cast<uint16_t*>(a.out), a.ld_out, p.sr, stg, lane, n0 + c);
+        __syncwarp();
+      } else {
+        float* out = static_cast<float*>(a.out);
+        if constexpr (EPI == EPI_F32) out += ks * a.split_stride;
+        if constexpr (EPI == EPI_GELU_F32) {
 #pragma unroll
           for (int i = 0; i < 32; ++i) v[i] = gelu_erf(v[i]);
-          if constexpr (EPI == EPI_GELU_BF16) {
-            store_bf16x32(static_cast<uint16_t*>(a.out) + drow * a.ld_out + n, v);
-          } else {
-            store_f32x32(static_cast<float*>(a.out) + drow * a.ld_out + n, v);
+        }
+#pragma unroll
+        for (int h16 = 0; h16 < 32; h16 += 16) {
+          stage_f32x16(stg, lane, v + h16);
+          __syncwarp();
+          float4 o[4];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const uint4 w = stg[stg_slot((lane >> 2) + 8 * i, jj)];
+            o[i] = make_float4(__uint_as_float(w.x), __uint_as_float(w.y), __uint_as_float(w.z), __uint_as_float(w.w));
+            if constexpr (EPI == EPI_F32) {
+              o[i].x += p.res[i].x; o[i].y += p.res[i].y; o[i].z += p.res[i].z; o[i].w += p.res[i].w;
+            }
           }
+          __syncwarp();
+          const int col = n0 + c + h16 + 4 * jj;
+          if constexpr (EPI == EPI_F32) {
+            const int nxt = c + h16 + 16;   // the next 16 columns' residual, in flight during the stores
+            if (use_res && nxt < c0 + BN / 2) {
+#pragma unroll
+              for (int i = 0; i < 4; ++i)
+                if (p.sr.ok & (1u << i)) p.res[i] = ld_res4(a, p.sr, i, n0 + nxt + 4 * jj);
+            }
+          }
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+            if (p.sr.ok & (1u << i)) st_global_u4(out + p.sr.drow[i] * a.ld_out + col,
+                                                  make_uint4(__float_as_uint(o[i].x), __float_as_uint(o[i].y),
+                                                             __float_as_uint(o[i].z), __float_as_uint(o[i].w)));
         }
       }
     }
   }
 }
 
-template <int BN, int EPI, bool LEAN>
-__global__ void __launch_bounds__(kThreads, LEAN ? 2 : 1)
+// ---------------------------------------------------------------- 1 CTA --
+template <int BN>
+struct OneCfg {
+  static constexpr int kBBytes = BN * kBK * 2;
+  using S = SmemCfg<kABytes + kBBytes>;
+  static constexpr int kTmemCols = 2 * BN;   // two accumulators
+};
+
+template <int BN, int EPI>
+__global__ void __launch_bounds__(kThreads, 1)
 gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                const __grid_constant__ GemmArgs a) {
-  using C = GemmCfg<BN, LEAN>;
-  constexpr int S = C::kStages;
+  using C = OneCfg<BN>;
+  constexpr int S = C::S::kStages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
   uint8_t* sB = smem + S * kABytes;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S * C::kStageBytes);
+  uint8_t* stg_all = smem + C::S::kStg;
+  uint16_t* sbias_all = reinterpret_cast<uint16_t*>(smem + C::S::kBias);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::S::kBars);
   // bars: full[S], empty[S], acc_full[2], acc_empty[2], drain
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * S + 5);
   int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
@@ -219,16 +381,16 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) { mbar_init(full(s), 1); mbar_init(empty(s), 1); }
-    for (int i = 0; i < 2; ++i) { mbar_init(acc_full(i), 1); mbar_init(acc_empty(i), 128); }
+    for (int i = 0; i < 2; ++i) { mbar_init(acc_full(i), 1); mbar_init(acc_empty(i), 8); }
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
-  if (warp == 5) {
+  if (warp == kMmaWarp) {
     tmem_alloc(smem_addr(tmem_slot), C::kTmemCols);
     tmem_relinquish();
   }
-  if (warp == 4 && lane == 0) {
+  if (warp == kProducerWarp && lane == 0) {
     tma_prefetch_desc(&tmA);
     tma_prefetch_desc(&tmB);
   }
@@ -238,8 +400,6 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
   const uint32_t tmem_base = *tmem_slot;
 
   const WaitCtx wc{a.status, abort_flag, a.limit_ns};
-  // Work unit u -> (m tile, K split, n tile), M fastest so that the units
-  // resident at one time share a weight panel through L2.
   const int m_tiles = (a.M + kBM - 1) / kBM;
   const int splits = a.k_splits;
   const int num_tiles = m_tiles * (a.N / BN) * splits;
@@ -255,12 +415,12 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
   // The weights (B) do not depend on the previous kernel of the stream: the
   // producer starts streaming the first stages' B tiles before waiting for it.
   int npre = 0;
-  if (warp == 4 && lane == 0 && blockIdx.x < num_tiles) {
+  if (warp == kProducerWarp && lane == 0 && blockIdx.x < num_tiles) {
     int m0, n0, ks;
     decode(blockIdx.x, m0, n0, ks);
     npre = nkb < S ? nkb : S;
     for (int i = 0; i < npre; ++i) {
-      mbar_arrive_expect_tx(full(i), C::kStageBytes);
+      mbar_arrive_expect_tx(full(i), kABytes + C::kBBytes);
       tma_load_2d(smem_addr(sB + i * C::kBBytes), &tmB, full(i), (ks * nkb + i) * kBK, n0);
     }
   }
@@ -268,13 +428,13 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
   pdl_wait();
   pdl_trigger();
 
-  if (warp == 4) {
+  if (warp == kProducerWarp) {
     if (lane == 0) {
       int stage = 0;
       uint32_t phase = 0;
-      uint32_t issued = 0;  // bit s: stage s was filled at least once
+      uint32_t issued = 0;    // bit s: stage s was filled at least once
       uint32_t last_par = 0;  // bit s: parity of the last fill of stage s
-      int it = 0;           // k-block iterations issued so far
+      int it = 0;             // k-block iterations issued so far
       for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
         int m0, n0, ks;
         decode(tile, m0, n0, ks);
@@ -283,7 +443,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
           const bool pre = it < npre;   // B already in flight, barrier already armed
           if (!pre) {
             if (!mbar_wait(empty(stage), phase ^ 1, wc, 1)) { ok = false; break; }
-            mbar_arrive_expect_tx(full(stage), C::kStageBytes);
+            mbar_arrive_expect_tx(full(stage), kABytes + C::kBBytes);
           }
           const int tap = kb / a.kb_per_tap;
           const int c = (kb - tap * a.kb_per_tap) * kBK;
@@ -304,7 +464,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
       for (int s = 0; s < S; ++s)
         if (issued & (1u << s)) mbar_wait(full(s), (last_par >> s) & 1u, dw, 5);
     }
-  } else if (warp == 5) {
+  } else if (warp == kMmaWarp) {
     if (lane == 0) {
       const uint32_t idesc = idesc_bf16_f32(kBM, BN, 0);
       int stage = 0;
@@ -341,55 +501,64 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
       mbar_wait(drain, 0, dw, 6);
     }
   } else {
+    uint4* stg = reinterpret_cast<uint4*>(stg_all) + warp * 128;
     int local = 0;
     for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++local) {
       int m0, n0, ks;
       decode(tile, m0, n0, ks);
       const int ab = local & 1;
       const uint32_t acc_par = (local >> 1) & 1;
+      uint16_t* sbias = sbias_all + warp * 256;
+      EpiPre<BN, EPI> pre;
+      epilogue_prepare<BN, EPI>(a, pre, sbias, m0, n0, ks, warp, lane);
       bool ok = mbar_wait(acc_full(ab), acc_par, wc, 4);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       tc_fence_after();
-      const uint32_t tacc = tmem_base + ab * BN + (static_cast<uint32_t>(warp * 32) << 16);
-      epilogue_tile<BN, EPI>(a, tacc, m0 + warp * 32 + lane, n0, ks);
+      const uint32_t tacc = tmem_base + ab * BN + (static_cast<uint32_t>((warp & 3) * 32) << 16);
+      epilogue_tile<BN, EPI>(a, pre, sbias, stg, tacc, n0, ks, warp, lane);
       tc_fence_before();
-      mbar_arrive(acc_empty(ab));
+      __syncwarp();
+      if (lane == 0) mbar_arrive(acc_empty(ab));
     }
   }
 
   __syncthreads();
-  if (warp == 5) {
+  if (warp == kMmaWarp) {
     tc_fence_after();
     tmem_dealloc(tmem_base, C::kTmemCols);
   }
 }
 
 // ------------------------------------------------------------ CTA pairs --
-// Two-CTA variant for many-row GEMMs: a cluster of two CTAs computes a
-// 256 x 256 tile with tcgen05.mma.cta_group::2 (M = 256).  CTA r loads its own
-// 128 rows of A and rows [128 r, 128 r + 128) of the tile's 256 B rows, so each
-// SM stages 32 KB per 64-wide K block for 128 x 256 x 64 of MMA work (the
-// one-CTA 128 x 256 tile stages 48 KB); the leader (CTA 0) issues the MMAs.
-// TMA completions of both CTAs land on the leader's full barriers; MMA
-// completions are multicast to the empty / accumulator barriers of both CTAs;
-// both CTAs' epilogue warps release an accumulator on the leader's barrier.
-// Each CTA's epilogue handles its 128 rows x 256 columns from its own TMEM.
-constexpr int kPairBN = 256;
-constexpr int kPairStages = 6;
-constexpr int kPairStageBytes = kABytes + 128 * kBK * 2;   // A (128 rows) + half of B (128 rows)
-constexpr int kPairSmem = kPairStages * kPairStageBytes + 1024 + 256;
+// A cluster of two CTAs computes a 256 x BN tile with tcgen05.mma.cta_group::2
+// (M = 256).  CTA r loads its own 128 rows of A and rows [r BN/2, (r+1) BN/2)
+// of the tile's B rows; the leader (CTA 0) issues the MMAs.  TMA completions of
+// both CTAs land on the leader's full barriers; MMA completions are multicast
+// to the empty / accumulator barriers of both CTAs; both CTAs' epilogue warps
+// release an accumulator on the leader's barrier.  Each CTA's epilogue handles
+// its 128 rows x BN columns from its own TMEM.
+template <int BN>
+struct PairCfg {
+  static constexpr int kBHalfBytes = (BN / 2) * kBK * 2;
+  static constexpr int kStageBytes = kABytes + kBHalfBytes;
+  using S = SmemCfg<kStageBytes>;
+  static constexpr int kTmemCols = 2 * BN;
+};
 
-template <int EPI>
+template <int BN, int EPI>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                 const __grid_constant__ GemmArgs a) {
-  constexpr int S = kPairStages;
+  using C = PairCfg<BN>;
+  constexpr int S = C::S::kStages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
   uint8_t* sB = smem + S * kABytes;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S * kPairStageBytes);
+  uint8_t* stg_all = smem + C::S::kStg;
+  uint16_t* sbias_all = reinterpret_cast<uint16_t*>(smem + C::S::kBias);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::S::kBars);
   // bars: full[S] (used in CTA 0), empty[S], acc_full[2], acc_empty[2] (CTA 0), drain
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * S + 5);
   int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
@@ -405,16 +574,16 @@ gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) { mbar_init(full(s), 1); mbar_init(empty(s), 1); }
-    for (int i = 0; i < 2; ++i) { mbar_init(acc_full(i), 1); mbar_init(acc_empty(i), 8); }
+    for (int i = 0; i < 2; ++i) { mbar_init(acc_full(i), 1); mbar_init(acc_empty(i), 16); }
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
-  if (warp == 5) {
-    tmem_alloc_pair(smem_addr(tmem_slot), 2 * kPairBN);
+  if (warp == kMmaWarp) {
+    tmem_alloc_pair(smem_addr(tmem_slot), C::kTmemCols);
     tmem_relinquish_pair();
   }
-  if (warp == 4 && lane == 0) {
+  if (warp == kProducerWarp && lane == 0) {
     tma_prefetch_desc(&tmA);
     tma_prefetch_desc(&tmB);
   }
@@ -427,30 +596,38 @@ gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
 
   const WaitCtx wc{a.status, abort_flag, a.limit_ns};
   const int m_tiles = (a.M + 255) / 256;
-  const int num_tiles = m_tiles * (a.N / kPairBN);
-  const int nkb = a.K / kBK;
+  const int splits = a.k_splits;
+  const int num_tiles = m_tiles * (a.N / BN) * splits;
+  const int nkb = a.K / kBK / splits;
   const int cluster = blockIdx.x >> 1;
   const int nclusters = gridDim.x >> 1;
+  auto decode = [&](int u, int& m0, int& n0, int& ks) {
+    const int mt = u % m_tiles;
+    const int r = u / m_tiles;
+    ks = r % splits;
+    m0 = mt * 256 + 128 * rank;
+    n0 = (r / splits) * BN;
+  };
 
-  if (warp == 4) {
+  if (warp == kProducerWarp) {
     if (lane == 0) {
       int stage = 0;
       uint32_t phase = 0;
       uint32_t issued = 0, last_par = 0;
       for (int tile = cluster; tile < num_tiles; tile += nclusters) {
-        const int m0 = (tile % m_tiles) * 256 + 128 * rank;
-        const int n0 = (tile / m_tiles) * kPairBN;
+        int m0, n0, ks;
+        decode(tile, m0, n0, ks);
         bool ok = true;
-        for (int kb = 0; kb < nkb; ++kb) {
+        for (int kb = ks * nkb; kb < (ks + 1) * nkb; ++kb) {
           if (!mbar_wait(empty(stage), phase ^ 1, wc, 31)) { ok = false; break; }
           const uint32_t fb = map_to_cta(full(stage), 0);   // the leader's full barrier
-          if (rank == 0) mbar_arrive_expect_tx(full(stage), 2 * kPairStageBytes);
+          if (rank == 0) mbar_arrive_expect_tx(full(stage), 2 * C::kStageBytes);
           const int tap = kb / a.kb_per_tap;
           const int c = (kb - tap * a.kb_per_tap) * kBK;
           const int ax = (tap % a.a_stride) * a.a_tap_ch + c;
           const int ay = m0 + tap / a.a_stride;
           tma_load_2d_pair(smem_addr(sA + stage * kABytes), &tmA, fb, ax, ay);
-          tma_load_2d_pair(smem_addr(sB + stage * 128 * kBK * 2), &tmB, fb, kb * kBK, n0 + 128 * rank);
+          tma_load_2d_pair(smem_addr(sB + stage * C::kBHalfBytes), &tmB, fb, kb * kBK, n0 + (BN / 2) * rank);
           issued |= 1u << stage;
           last_par = (last_par & ~(1u << stage)) | (phase << stage);
           if (++stage == S) { stage = 0; phase ^= 1; }
@@ -465,9 +642,9 @@ gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
           if (issued & (1u << s)) mbar_wait(full(s), (last_par >> s) & 1u, dw, 35);
       }
     }
-  } else if (warp == 5) {
+  } else if (warp == kMmaWarp) {
     if (lane == 0 && rank == 0) {
-      const uint32_t idesc = idesc_bf16_f32(256, kPairBN, 0);
+      const uint32_t idesc = idesc_bf16_f32(256, BN, 0);
       int stage = 0;
       uint32_t phase = 0;
       int local = 0;
@@ -476,13 +653,13 @@ gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
         const uint32_t acc_par = (local >> 1) & 1;
         if (!mbar_wait(acc_empty(ab), acc_par ^ 1, wc, 32)) break;
         tc_fence_after();
-        const uint32_t d_tmem = tmem_base + ab * kPairBN;
+        const uint32_t d_tmem = tmem_base + ab * BN;
         bool ok = true;
         for (int kb = 0; kb < nkb; ++kb) {
           if (!mbar_wait(full(stage), phase, wc, 33)) { ok = false; break; }
           tc_fence_after();
           const uint32_t a0 = smem_addr(sA + stage * kABytes);
-          const uint32_t b0 = smem_addr(sB + stage * 128 * kBK * 2);
+          const uint32_t b0 = smem_addr(sB + stage * C::kBHalfBytes);
 #pragma unroll
           for (int k = 0; k < kBK / 16; ++k)
             umma_bf16_pair(d_tmem, smem_desc_sw128(a0 + 32 * k, 16, 1024), smem_desc_sw128(b0 + 32 * k, 16, 1024),
@@ -500,20 +677,24 @@ gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
       mbar_wait(drain, 0, dw, 36);
     }
   } else {
+    uint4* stg = reinterpret_cast<uint4*>(stg_all) + warp * 128;
     int local = 0;
     const uint32_t acc_empty_leader0 = map_to_cta(acc_empty(0), 0);
     const uint32_t acc_empty_leader1 = map_to_cta(acc_empty(1), 0);
     for (int tile = cluster; tile < num_tiles; tile += nclusters, ++local) {
-      const int m0 = (tile % m_tiles) * 256 + 128 * rank;
-      const int n0 = (tile / m_tiles) * kPairBN;
+      int m0, n0, ks;
+      decode(tile, m0, n0, ks);
       const int ab = local & 1;
       const uint32_t acc_par = (local >> 1) & 1;
+      uint16_t* sbias = sbias_all + warp * 256;
+      EpiPre<BN, EPI> pre;
+      epilogue_prepare<BN, EPI>(a, pre, sbias, m0, n0, ks, warp, lane);
       bool ok = mbar_wait(acc_full(ab), acc_par, wc, 34);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       tc_fence_after();
-      const uint32_t tacc = tmem_base + ab * kPairBN + (static_cast<uint32_t>(warp * 32) << 16);
-      epilogue_tile<kPairBN, EPI>(a, tacc, m0 + warp * 32 + lane, n0, 0);
+      const uint32_t tacc = tmem_base + ab * BN + (static_cast<uint32_t>((warp & 3) * 32) << 16);
+      epilogue_tile<BN, EPI>(a, pre, sbias, stg, tacc, n0, ks, warp, lane);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(ab ? acc_empty_leader1 : acc_empty_leader0);
@@ -523,91 +704,115 @@ gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
   tc_fence_before();
   __syncthreads();
   cluster_sync_all();   // no CTA of the pair still uses TMEM or the peer's barriers
-  if (warp == 5) {
+  if (warp == kMmaWarp) {
     tc_fence_after();
-    tmem_dealloc_pair(tmem_base, 2 * kPairBN);
+    tmem_dealloc_pair(tmem_base, C::kTmemCols);
   }
+}
+
+// ------------------------------------------------------------- launchers --
+template <class K>
+cudaError_t set_smem(K kernel, int bytes, bool& done) {
+  if (done) return cudaSuccess;
+  cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess) done = true;   // per instantiation; a racing second call is harmless
+  return e;
+}
+
+template <int BN, int EPI>
+cudaError_t launch_one(const Launch& L, const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmArgs& a) {
+  using C = OneCfg<BN>;
+  static bool attr_set = false;
+  if (cudaError_t e = set_smem(gemm_tc_kernel<BN, EPI>, C::S::kTotal, attr_set)) return e;
+  const int tiles = ((a.M + kBM - 1) / kBM) * (a.N / BN) * a.k_splits;
+  const int grid = tiles < L.sm_count ? tiles : L.sm_count;
+  return launch_kernel(gemm_tc_kernel<BN, EPI>, dim3(grid), dim3(kThreads), C::S::kTotal, L.stream, tmA, tmB, a);
+}
+
+template <int BN, int EPI>
+cudaError_t launch_pair(const Launch& L, const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmArgs& a) {
+  using C = PairCfg<BN>;
+  static bool attr_set = false;
+  if (cudaError_t e = set_smem(gemm_tc2_kernel<BN, EPI>, C::S::kTotal, attr_set)) return e;
+  const int tiles = ((a.M + 255) / 256) * (a.N / BN) * a.k_splits;
+  const int pairs = L.sm_count / 2;
+  const int grid = 2 * (tiles < pairs ? tiles : pairs);
+  return launch_kernel(gemm_tc2_kernel<BN, EPI>, dim3(grid), dim3(kThreads), C::S::kTotal, L.stream, tmA, tmB, a);
 }
 
 template <int EPI>
-cudaError_t launch_pair(const Launch& L, const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmArgs& a) {
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(gemm_tc2_kernel<EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize, kPairSmem);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
+cudaError_t launch_epi(const Launch& L, const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmArgs& a,
+                       const GemmPlan& p) {
+  if (p.pair) {
+    if (p.bn == 256) return launch_pair<256, EPI>(L, tmA, tmB, a);
+    if (p.bn == 128) return launch_pair<128, EPI>(L, tmA, tmB, a);
+    return cudaErrorInvalidValue;
   }
-  const int tiles = ((a.M + 255) / 256) * (a.N / kPairBN);
-  const int pairs = L.sm_count / 2;
-  const int grid = 2 * (tiles < pairs ? tiles : pairs);
-  return launch_kernel(gemm_tc2_kernel<EPI>, dim3(grid), dim3(kThreads), kPairSmem, L.stream, tmA, tmB, a);
-}
-
-template <int BN, int EPI, bool LEAN>
-cudaError_t launch_one(const Launch& L, const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmArgs& a) {
-  using C = GemmCfg<BN, LEAN>;
-  static bool attr_set = false;  // per instantiation; benign race (idempotent call)
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<BN, EPI, LEAN>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
-  const int m_tiles = (a.M + kBM - 1) / kBM;
-  const int tiles = m_tiles * (a.N / BN) * a.k_splits;
-  const int slots = (LEAN ? 2 : 1) * L.sm_count;
-  const int grid = tiles < slots ? tiles : slots;
-  return launch_kernel(gemm_tc_kernel<BN, EPI, LEAN>, dim3(grid), dim3(kThreads), C::kSmem, L.stream, tmA, tmB, a);
-}
-
-template <int BN, bool LEAN>
-cudaError_t launch_bn(const Launch& L, const CUtensorMap& tmA, const CUtensorMap& tmB,
-                      const GemmArgs& a, int epi) {
-  switch (epi) {
-    case EPI_F32: return launch_one<BN, EPI_F32, LEAN>(L, tmA, tmB, a);
-    case EPI_QKV_ROPE: return launch_one<BN, EPI_QKV_ROPE, LEAN>(L, tmA, tmB, a);
-    case EPI_SWIGLU:
-      if constexpr (BN >= 128) return launch_one<BN, EPI_SWIGLU, LEAN>(L, tmA, tmB, a);
-      else return cudaErrorInvalidValue;
-    case EPI_GELU_BF16:
-      if constexpr (!LEAN) return launch_one<BN, EPI_GELU_BF16, LEAN>(L, tmA, tmB, a);
-      else return cudaErrorInvalidValue;
-    case EPI_GELU_F32:
-      if constexpr (!LEAN) return launch_one<BN, EPI_GELU_F32, LEAN>(L, tmA, tmB, a);
-      else return cudaErrorInvalidValue;
-    default: return cudaErrorInvalidValue;
-  }
+  if (p.bn == 256) return launch_one<256, EPI>(L, tmA, tmB, a);
+  if (p.bn == 128) return launch_one<128, EPI>(L, tmA, tmB, a);
+  return cudaErrorInvalidValue;
 }
 
 }  // namespace
 
-cudaError_t launch_gemm_pair(const Launch& L, const CUtensorMap& tmA, const CUtensorMap& tmB,
-                             const GemmArgs& args, int epi) {
-  if (args.M <= 0) return cudaSuccess;
-  if (args.k_splits != 1 || args.N % kPairBN != 0 || args.K % kBK != 0) return cudaErrorInvalidValue;
-  switch (epi) {
-    case EPI_F32: return launch_pair<EPI_F32>(L, tmA, tmB, args);
-    case EPI_QKV_ROPE: return launch_pair<EPI_QKV_ROPE>(L, tmA, tmB, args);
-    case EPI_SWIGLU: return launch_pair<EPI_SWIGLU>(L, tmA, tmB, args);
-    case EPI_GELU_BF16: return launch_pair<EPI_GELU_BF16>(L, tmA, tmB, args);
-    case EPI_GELU_F32: return launch_pair<EPI_GELU_F32>(L, tmA, tmB, args);
-    default: return cudaErrorInvalidValue;
-  }
+// Time model of one GEMM launch, used to choose among the shapes below.
+// Measured on B200 (one CTA per SM, 64-wide K blocks):
+//  * a tcgen05.mma with M = 128 rows per CTA and K = 16 takes ~73 ns for any
+//    N <= 256, so a K block costs ~0.29 us whatever the tile width: only
+//    N = 256 runs the tensor core at its peak;
+//  * a TMA tile load costs ~0.13 us of the SM's copy engine (L2 source) to
+//    ~0.17 us (HBM source), nearly independent of its size up to 48 KB, so a
+//    K block (two loads) costs 0.27 - 0.34 us of copy time;
+//  * HBM bounds the weight streaming of few-row GEMMs.
+// A K-split adds the fp32 round trip of its partial sums through L2 and the
+// last tile's epilogue is exposed.
+static double plan_time_us(const GemmPlan& p, int M, int N, int K, int sm) {
+  const int nkb = K / kBK / p.splits;
+  const int rows = p.pair ? 256 : 128;
+  const long units = static_cast<long>((M + rows - 1) / rows) * (N / p.bn) * p.splits;
+  const long slots = p.pair ? sm / 2 : sm;
+  const long waves = (units + slots - 1) / slots;
+  const double kb_us = 0.30;
+  const double hbm_us = (static_cast<double>(N) * K * 2 + static_cast<double>(M) * K * 2) / 6.5e6;
+  const double split_us = p.splits > 1 ? static_cast<double>(p.splits) * M * N * 4 * 2 / 20e6 : 0.0;
+  const double epi_us = 0.5 + 0.004 * p.bn;
+  const double body = waves * nkb * kb_us;
+  return (body > hbm_us ? body : hbm_us) + split_us + epi_us;
 }
 
-cudaError_t launch_gemm(const Launch& L, const CUtensorMap& tmA, const CUtensorMap& tmB,
-                        const GemmArgs& args, int epi, int bn, bool lean) {
-  if (args.M <= 0) return cudaSuccess;
-  if (args.k_splits < 1 || (args.K / kBK) % args.k_splits != 0) return cudaErrorInvalidValue;
-  if (lean) {
-    if (bn == 128) return launch_bn<128, true>(L, tmA, tmB, args, epi);
-    if (bn == 64) return launch_bn<64, true>(L, tmA, tmB, args, epi);
-    return cudaErrorInvalidValue;
+GemmPlan plan_gemm(int M, int N, int K, int epi, int max_splits, int sm) {
+  GemmPlan best{false, 0, 1};
+  double best_t = 1e30;
+  const int nkb = K / kBK;
+  const bool can_split = epi == EPI_F32;
+  for (int pair = pair_gemm_disabled() ? 0 : 1; pair >= 0; --pair) {
+    for (int bn = 256; bn >= 128; bn /= 2) {
+      if (N % bn != 0) continue;
+      for (int s = 1; s <= (can_split ? max_splits : 1); s *= 2) {
+        if (nkb % s != 0 || nkb / s < 2) break;
+        const GemmPlan p{pair != 0, bn, s};
+        const double t = plan_time_us(p, M, N, K, sm);
+        if (t < best_t * 0.98) { best_t = t; best = p; }
+      }
+    }
   }
-  if (bn == 256) return launch_bn<256, false>(L, tmA, tmB, args, epi);
-  if (bn == 128) return launch_bn<128, false>(L, tmA, tmB, args, epi);
-  if (bn == 64) return launch_bn<64, false>(L, tmA, tmB, args, epi);
-  return cudaErrorInvalidValue;
+  return best;
+}
+
+cudaError_t launch_gemm(const Launch& L, const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmArgs& args,
+                        int epi, const GemmPlan& p) {
+  if (args.M <= 0) return cudaSuccess;
+  if (args.k_splits != p.splits || p.splits < 1 || (args.K / kBK) % p.splits != 0 || args.K % kBK != 0 ||
+      p.bn <= 0 || args.N % p.bn != 0 || (p.splits > 1 && epi != EPI_F32))
+    return cudaErrorInvalidValue;
+  switch (epi) {
+    case EPI_F32: return launch_epi<EPI_F32>(L, tmA, tmB, args, p);
+    case EPI_QKV_ROPE: return launch_epi<EPI_QKV_ROPE>(L, tmA, tmB, args, p);
+    case EPI_SWIGLU: return launch_epi<EPI_SWIGLU>(L, tmA, tmB, args, p);
+    case EPI_GELU_BF16: return launch_epi<EPI_GELU_BF16>(L, tmA, tmB, args, p);
+    case EPI_GELU_F32: return launch_epi<EPI_GELU_F32>(L, tmA, tmB, args, p);
+    default: return cudaErrorInvalidValue;
+  }
 }
 
 void fill_rope_freqs(GemmArgs* a, float theta, int head_dim) {

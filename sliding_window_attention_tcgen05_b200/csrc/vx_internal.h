@@ -92,18 +92,24 @@ struct GemmArgs {
   uint64_t limit_ns;
 };
 
-// D[M, N] = A[M, K] * B[N, K]^T with the given epilogue.  tmA/tmB must be 2-D
-// bf16 maps with 128-byte swizzle and box {64, 128} (A) / {64, bn} (B).
-// bn in {64, 128, 256} (EPI_SWIGLU: 128 or 256); N % bn == 0; K % 64 == 0;
-// (K / 64) % k_splits == 0.
-// lean: a ~96 KB pipeline so two CTAs share an SM (bn 64 or 128; no GELU).
-cudaError_t launch_gemm(const Launch& L, const CUtensorMap& tmA, const CUtensorMap& tmB,
-                        const GemmArgs& args, int epi, int bn, bool lean = false);
+// Tile shape of one GEMM launch: one CTA per 128 x bn tile, or a cluster of
+// two CTAs per 256 x bn tile (pair); `splits` K-splits writing fp32 partials.
+struct GemmPlan {
+  bool pair;
+  int bn;       // 64, 128 or 256 (pair: 128 or 256); 0 = no shape fits
+  int splits;
+};
 
-// Two-CTA version (clusters of 2, 256 x 256 tiles, tcgen05.mma.cta_group::2):
-// tmA box {64, 128}, tmB box {64, 128}; N % 256 == 0, no split-K.
-cudaError_t launch_gemm_pair(const Launch& L, const CUtensorMap& tmA, const CUtensorMap& tmB,
-                             const GemmArgs& args, int epi);
+// The fastest shape for an M x N x K GEMM with epilogue `epi` on `sm` SMs by
+// the launch-time model in gemm.cu (split-K only for EPI_F32, up to max_splits).
+GemmPlan plan_gemm(int M, int N, int K, int epi, int max_splits, int sm);
+
+// D[M, N] = A[M, K] * B[N, K]^T with the given epilogue, in the shape `plan`.
+// tmA: 2-D bf16 map with 128-byte swizzle and box {64, 128}; tmB: the same
+// with box {64, plan.pair ? plan.bn / 2 : plan.bn}.  args.k_splits must equal
+// plan.splits; N % bn == 0; K % 64 == 0; (K / 64) % splits == 0.
+cudaError_t launch_gemm(const Launch& L, const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmArgs& args,
+                        int epi, const GemmPlan& plan);
 
 void fill_rope_freqs(GemmArgs* a, float theta, int head_dim);
 
