@@ -7,10 +7,12 @@
 //   2. y0 Wqkv^T + bqkv, RoPE     -> qkv  (bf16, [M, 3*HD], tcgen05 GEMM)
 //   3. sliding-window attention   -> att  (bf16, tcgen05 flash kernel, or the
 //                                          ring kernel in a streaming step)
-//   4. att Wo^T + bo + x          -> h    (fp32, residual fused in the epilogue)
+//   4. att Wo^T + bo + x          -> h    (fp32, residual fused in the epilogue,
+//                                          or split-K partials reduced in 5.)
 //   5. RMSNorm(h)                 -> y1   (bf16)
 //   6. silu(y1 Wg^T) * (y1 Wu^T)  -> act  (bf16, gate/up packed, SwiGLU epilogue)
-//   7. act Wd^T + bd + h          -> y    (fp32)
+//   7. act Wd^T + bd + h          -> y    (fp32; fused, or partials reduced by
+//                                          the next layer's RMSNorm 1.)
 #include <cstdarg>
 #include <cstdio>
 #include <cstdlib>
@@ -230,12 +232,19 @@ vx_status check_weights(const vx_layer_cfg& c, const vx_layer_weights* w) {
 }
 
 struct LayerBufs {
-  uint16_t* y0;    // [M, d] bf16 (reused for y1)
-  uint16_t* qkv;   // [M, 3HD] bf16
-  uint16_t* att;   // [M, HD] bf16
-  float* h;        // [M, d] fp32
-  uint16_t* act;   // [M, F] bf16
+  uint16_t* y0;    // [M, d]     bf16 normed input (reused for the second norm)
+  uint16_t* qkv;   // [M, 3*HD]  bf16
+  uint16_t* att;   // [M, HD]    bf16
+  float* h;        // [M, d]     fp32 post-attention residual stream
+  uint16_t* act;   // [M, F]     bf16 SwiGLU output
+  float* xmat;     // [M, d]     fp32 materialised layer input (when it arrives as partial sums)
+  float* parts;    // [split_cap(M), M, d] fp32 split-K partial sums (null when split_cap(M) == 1)
 };
+
+// Most K-splits a GEMM with M rows may use: few-row GEMMs have too few output
+// tiles to fill the GPU; from a few thousand rows on they never need one.
+constexpr int kMaxSplits = 8;
+int split_cap(int64_t M) { return M <= 512 ? kMaxSplits : (M <= 4096 ? 2 : 1); }
 
 LayerBufs carve_layer(Carve& cv, const vx_layer_cfg& c, int64_t M) {
   const int64_t d = c.d_model, HD = int64_t(c.n_heads) * c.head_dim, F = c.ffn_hidden;
@@ -245,6 +254,9 @@ LayerBufs carve_layer(Carve& cv, const vx_layer_cfg& c, int64_t M) {
   b.att = static_cast<uint16_t*>(cv.take(M * HD * 2));
   b.h = static_cast<float*>(cv.take(M * d * 4));
   b.act = static_cast<uint16_t*>(cv.take(M * F * 2));
+  const int cap = split_cap(M);
+  b.xmat = cap > 1 ? static_cast<float*>(cv.take(M * d * 4)) : nullptr;
+  b.parts = cap > 1 ? static_cast<float*>(cv.take(cap * M * d * 4)) : nullptr;
   return b;
 }
 
@@ -266,27 +278,64 @@ GemmArgs base_args(const Launch& L, int M, int N, int K) {
   return a;
 }
 
-// Plans, encodes B's tensor map for and launches one GEMM; on return
-// a.k_splits holds the number of partial sums written (1 unless max_splits > 1).
-vx_status launch_any_gemm(const Launch& L, const char* name, const CUtensorMap* tmA, const void* Bw, int64_t ldb,
-                          GemmArgs& a, int epi, int max_splits = 1) {
-  const GemmPlan p = plan_gemm(a.M, a.N, a.K, epi, max_splits, L.sm_count);
+// Encodes B's tensor map for and launches one GEMM in the shape `p`
+// (a.k_splits must already equal p.splits).
+vx_status launch_planned(const Launch& L, const char* name, const CUtensorMap* tmA, const void* Bw, int64_t ldb,
+                         const GemmArgs& a, int epi, const GemmPlan& p) {
   if (p.bn == 0) {
     set_error("%s: no GEMM tile shape fits N=%d K=%d", name, a.N, a.K);
     return VX_ERR_UNSUPPORTED;
   }
-  a.k_splits = p.splits;
   CUtensorMap tmB;
   if (!tmap_bf16_2d(&tmB, Bw, a.K, a.N, ldb, p.pair ? p.bn / 2 : p.bn)) return VX_ERR_CUDA;
   VX_CUDA(traced(L, name, 1, [&] { return launch_gemm(L, *tmA, tmB, a, epi, p); }));
   return VX_OK;
 }
 
-vx_status gemm(const Launch& L, const char* name, const void* A, int64_t lda, const void* Bw, GemmArgs& a, int epi,
-               int max_splits = 1) {
+// One GEMM without K-splits: plan, then launch.
+vx_status launch_any_gemm(const Launch& L, const char* name, const CUtensorMap* tmA, const void* Bw, int64_t ldb,
+                          const GemmArgs& a, int epi) {
+  return launch_planned(L, name, tmA, Bw, ldb, a, epi, plan_gemm(a.M, a.N, a.K, epi, 1, L.sm_count));
+}
+
+vx_status gemm(const Launch& L, const char* name, const void* A, int64_t lda, const void* Bw, const GemmArgs& a,
+               int epi, const GemmPlan* p = nullptr) {
   CUtensorMap tmA;
   if (!tmap_bf16_2d(&tmA, A, a.K, a.M, lda, 128)) return VX_ERR_CUDA;
-  return launch_any_gemm(L, name, &tmA, Bw, a.K, a, epi, max_splits);
+  if (p) return launch_planned(L, name, &tmA, Bw, a.K, a, epi, *p);
+  return launch_any_gemm(L, name, &tmA, Bw, a.K, a, epi);
+}
+
+// The pending (unreduced) value of an fp32 [M, d] activation:
+// base + bias + sum_{k < nparts} parts[k].
+struct Pending {
+  const float* base;
+  const float* parts;
+  int nparts;
+  const uint16_t* bias;
+};
+
+// A residual GEMM  out = A W^T + bias + res  in the planned shape: fused into
+// the epilogue when the plan has one K-split, else as fp32 partial sums whose
+// reduction (with bias and residual) is left pending for the next RMSNorm.
+vx_status residual_gemm(const Launch& L, const char* name, const void* A, int64_t lda, const void* W, int M, int N,
+                        int K, const uint16_t* bias, const float* res, float* out, float* parts, int max_splits,
+                        Pending* result) {
+  GemmArgs a = base_args(L, M, N, K);
+  const GemmPlan p = plan_gemm(M, N, K, EPI_F32, parts ? max_splits : 1, L.sm_count);
+  a.ld_out = N;
+  if (p.splits > 1) {
+    a.out = parts;
+    a.k_splits = p.splits;
+    a.split_stride = static_cast<int64_t>(M) * N;
+    *result = Pending{res, parts, p.splits, bias};
+  } else {
+    a.out = out;
+    a.bias = bias;
+    a.res = res; a.ld_res = N;
+    *result = Pending{out, nullptr, 0, nullptr};
+  }
+  return gemm(L, name, A, lda, W, a, EPI_F32, &p);
 }
 
 
@@ -299,30 +348,52 @@ struct RingLayer {
   bool step;   // streaming step: attend through the ring
 };
 
-// One layer over nseq sequences of `rows` frames (x, y: [nseq*rows, d] fp32).
-vx_status run_layer(const Launch& L, const vx_layer_cfg& c, const vx_layer_weights& w, const float* x, float* y,
-                    int nseq, int rows, int64_t pos0, const LayerBufs& bf, const RingLayer* ring) {
+// One layer over nseq sequences of `rows` frames.  The input arrives pending
+// (the previous layer's output may still be split-K partial sums); so may the
+// output: `out` is either y itself or the pending sum that the next RMSNorm
+// (the next layer's, the final norm, or a plain reduction) completes.  With
+// split-K the layer still runs seven kernels: each RMSNorm also reduces.
+//   x_l = reduce(in);  y0 = RMSNorm(x_l)
+//   qkv = RoPE(y0 Wqkv^T + bqkv);  att = attention(qkv)
+//   h   = x_l + bo + att Wo^T         (fused, or pending into RMSNorm 2)
+//   y1  = RMSNorm(h);  act = SwiGLU(y1 Wgu^T + bgu)
+//   out = h + bd + act Wd^T           (fused into y, or pending)
+vx_status run_layer(const Launch& L, const vx_layer_cfg& c, const vx_layer_weights& w, const Pending& in,
+                    Pending* out, float* y, int nseq, int rows, int64_t pos0, const LayerBufs& bf,
+                    const RingLayer* ring) {
   const int d = c.d_model, H = c.n_heads, HD = H * c.head_dim, F = c.ffn_hidden;
   const int M = nseq * rows;
+  const int64_t pstride = static_cast<int64_t>(M) * d;
+  const int cap = bf.parts ? split_cap(M) : 1;
   const float sl2 = (1.0f / std::sqrt(static_cast<float>(c.head_dim))) * 1.4426950408889634f;
+  const bool step = ring && ring->step;
   vx_status st;
-  // 1. RMSNorm
-  VX_CUDA(traced(L, "rmsnorm", 1, [&] { return launch_rmsnorm(L, x, nullptr, 0, 0, nullptr, static_cast<const uint16_t*>(w.attn_norm_g), nullptr, bf.y0, true, M, d, c.eps); }));
-  // 2. QKV + bias + RoPE
+  // 1. x_l = reduce(in); y0 = RMSNorm(x_l)
+  const bool pending_in = in.parts != nullptr || in.bias != nullptr;
+  const float* xl = pending_in ? bf.xmat : in.base;
+  VX_CUDA(traced(L, "rmsnorm", 1, [&] {
+    return launch_rmsnorm(L, in.base, in.parts, in.nparts, pstride, in.bias,
+                          static_cast<const uint16_t*>(w.attn_norm_g), pending_in ? bf.xmat : nullptr, bf.y0, true, M,
+                          d, c.eps);
+  }));
+  // 2. QKV + bias + RoPE at (pos[s] or pos0) + t
   {
     GemmArgs a = base_args(L, M, 3 * HD, d);
     a.out = bf.qkv; a.ld_out = 3 * HD;
     a.bias = static_cast<const uint16_t*>(w.bqkv);
     a.in_rows = rows; a.t_valid = rows; a.out_rows = rows;
-    a.pos_arr = (ring && ring->step) ? ring->pos : nullptr;
+    a.pos_arr = step ? ring->pos : nullptr;
     a.pos0 = pos0;
     a.rope_cols = 2 * HD;
     fill_rope_freqs(&a, c.rope_theta, c.head_dim);
     if ((st = gemm(L, "gemm_qkv_rope", bf.y0, d, w.wqkv, a, EPI_QKV_ROPE)) != VX_OK) return st;
   }
-  // 3. attention
-  if (ring && ring->step) {
-    VX_CUDA(traced(L, "ring_attn", 1, [&] { return launch_ring_attn(L, bf.qkv, 3LL * HD, HD, ring->k, ring->v, ring->pos, nseq, H, ring->W, rows, bf.att, sl2); }));
+  // 3. attention: through the ring (streaming step), or windowed over the sequence
+  if (step) {
+    VX_CUDA(traced(L, "ring_attn", 1, [&] {
+      return launch_ring_attn(L, bf.qkv, 3LL * HD, HD, ring->k, ring->v, ring->pos, nseq, H, ring->W, rows, bf.att,
+                              sl2);
+    }));
   } else {
     CUtensorMap tq, tk, tv;
     const int64_t rs = 3LL * HD, bs = static_cast<int64_t>(rows) * 3 * HD;
@@ -335,117 +406,21 @@ vx_status run_layer(const Launch& L, const vx_layer_cfg& c, const vx_layer_weigh
     aa.status = L.status; aa.limit_ns = L.limit_ns;
     VX_CUDA(traced(L, "swa_attn_tc", 1, [&] { return launch_attn_bf16(L, tq, tk, tv, aa); }));
     if (ring && ring->fill)
-      VX_CUDA(traced(L, "ring_fill", 1, [&] { return launch_ring_fill(L, bf.qkv, 3LL * HD, HD, ring->k, ring->v, nseq, rows, H, ring->W); }));
+      VX_CUDA(traced(L, "ring_fill", 1, [&] {
+        return launch_ring_fill(L, bf.qkv, 3LL * HD, HD, ring->k, ring->v, nseq, rows, H, ring->W);
+      }));
   }
-  // 4. O-projection + bias + residual
-  {
-    GemmArgs a = base_args(L, M, d, HD);
-    a.out = bf.h; a.ld_out = d;
-    a.bias = static_cast<const uint16_t*>(w.bo);
-    a.res = x; a.ld_res = d;
-    if ((st = gemm(L, "gemm_o_residual", bf.att, HD, w.wo, a, EPI_F32)) != VX_OK) return st;
-  }
-  // 5. RMSNorm
-  VX_CUDA(traced(L, "rmsnorm", 1, [&] { return launch_rmsnorm(L, bf.h, nullptr, 0, 0, nullptr, static_cast<const uint16_t*>(w.ffn_norm_g), nullptr, bf.y0, true, M, d, c.eps); }));
-  // 6. gate/up + SwiGLU
-  {
-    GemmArgs a = base_args(L, M, 2 * F, d);
-    a.out = bf.act; a.ld_out = F;
-    a.bias = static_cast<const uint16_t*>(w.bgu);
-    if ((st = gemm(L, "gemm_gate_up_swiglu", bf.y0, d, w.wgu, a, EPI_SWIGLU)) != VX_OK) return st;
-  }
-  // 7. down + bias + residual
-  {
-    GemmArgs a = base_args(L, M, d, F);
-    a.out = y; a.ld_out = d;
-    a.bias = static_cast<const uint16_t*>(w.bd);
-    a.res = bf.h; a.ld_res = d;
-    if ((st = gemm(L, "gemm_down_residual", bf.act, F, w.wd, a, EPI_F32)) != VX_OK) return st;
-  }
-  return VX_OK;
-}
-
-// ------------------------------------------------------ streaming layers --
-// Few-row layers (a streaming step: M = streams x new frames) stream their
-// weights from HBM; the O-projection and down GEMMs then have too few output
-// tiles to fill the GPU, so they run split-K and write fp32 partial sums.  The
-// partial sums, bias and residual are reduced inside the RMSNorm that follows:
-//   layer input  x_l = H_{l-1} + bd_{l-1} + sum P_down   (RMSNorm 1 also writes x_l)
-//   h            = x_l + bo + sum P_o                    (RMSNorm 2 writes h)
-// so the per-layer kernel count stays seven.
-struct StreamBufs {
-  LayerBufs lb;    // y0 (y1), qkv, att, act; lb.h is H
-  float* xmat;     // [M, d] materialised layer input
-  float* parts;    // [kMaxSplits, M, d] fp32 partial sums
-};
-constexpr int kMaxSplits = 8;
-
-StreamBufs carve_stream(Carve& cv, const vx_layer_cfg& c, int64_t M) {
-  StreamBufs b;
-  b.lb = carve_layer(cv, c, M);
-  b.xmat = static_cast<float*>(cv.take(M * c.d_model * 4));
-  b.parts = static_cast<float*>(cv.take(kMaxSplits * M * c.d_model * 4));
-  return b;
-}
-
-size_t stream_ws_bytes(const vx_layer_cfg& c, int64_t M) {
-  Carve cv{nullptr, kStatusBytes};
-  carve_stream(cv, c, M);
-  return align_up(cv.off, kAlign);
-}
-
-// The pending (unreduced) output of a layer: base + bias + sum of parts.
-struct Pending {
-  const float* base;
-  const float* parts;
-  int nparts;
-  const uint16_t* bias;
-};
-
-vx_status run_layer_stream(const Launch& L, const vx_layer_cfg& c, const vx_layer_weights& w, const Pending& in,
-                           Pending* out, int nseq, int rows, const StreamBufs& sb, const RingLayer& ring) {
-  const int d = c.d_model, H = c.n_heads, HD = H * c.head_dim, F = c.ffn_hidden;
-  const int M = nseq * rows;
-  const int64_t pstride = static_cast<int64_t>(M) * d;
-  const float sl2 = (1.0f / std::sqrt(static_cast<float>(c.head_dim))) * 1.4426950408889634f;
-  const LayerBufs& bf = sb.lb;
-  vx_status st;
-  // 1. x_l = reduce(in); y0 = RMSNorm(x_l)
-  const bool pending_in = in.parts != nullptr || in.bias != nullptr;
-  const float* xl = pending_in ? sb.xmat : in.base;
+  // 4. h = x_l + bo + att Wo^T
+  Pending hp;
+  if ((st = residual_gemm(L, "gemm_o_residual", bf.att, HD, w.wo, M, d, HD, static_cast<const uint16_t*>(w.bo), xl,
+                          bf.h, bf.parts, cap, &hp)) != VX_OK)
+    return st;
+  // 5. y1 = RMSNorm(h), materialising h when it is pending
+  const bool pending_h = hp.parts != nullptr;
   VX_CUDA(traced(L, "rmsnorm", 1, [&] {
-    return launch_rmsnorm(L, in.base, in.parts, in.nparts, pstride, in.bias,
-                          static_cast<const uint16_t*>(w.attn_norm_g), pending_in ? sb.xmat : nullptr, bf.y0, true,
-                          M, d, c.eps);
-  }));
-  // 2. QKV + bias + RoPE at pos[s] + t
-  {
-    GemmArgs a = base_args(L, M, 3 * HD, d);
-    a.out = bf.qkv; a.ld_out = 3 * HD;
-    a.bias = static_cast<const uint16_t*>(w.bqkv);
-    a.in_rows = rows; a.t_valid = rows; a.out_rows = rows;
-    a.pos_arr = ring.pos;
-    a.rope_cols = 2 * HD;
-    fill_rope_freqs(&a, c.rope_theta, c.head_dim);
-    if ((st = gemm(L, "gemm_qkv_rope", bf.y0, d, w.wqkv, a, EPI_QKV_ROPE)) != VX_OK) return st;
-  }
-  // 3. ring attention (reads every old in-window slot, then appends)
-  VX_CUDA(traced(L, "ring_attn", 1, [&] {
-    return launch_ring_attn(L, bf.qkv, 3LL * HD, HD, ring.k, ring.v, ring.pos, nseq, H, ring.W, rows, bf.att, sl2);
-  }));
-  // 4. O-projection, split-K partial sums
-  int so;
-  {
-    GemmArgs a = base_args(L, M, d, HD);
-    a.out = sb.parts; a.ld_out = d;
-    a.split_stride = pstride;
-    if ((st = gemm(L, "gemm_o_splitk", bf.att, HD, w.wo, a, EPI_F32, kMaxSplits)) != VX_OK) return st;
-    so = a.k_splits;
-  }
-  // 5. h = x_l + bo + sum P_o; y1 = RMSNorm(h)
-  VX_CUDA(traced(L, "rmsnorm", 1, [&] {
-    return launch_rmsnorm(L, xl, sb.parts, so, pstride, static_cast<const uint16_t*>(w.bo),
-                          static_cast<const uint16_t*>(w.ffn_norm_g), bf.h, bf.y0, true, M, d, c.eps);
+    return launch_rmsnorm(L, hp.base, hp.parts, hp.nparts, pstride, hp.bias,
+                          static_cast<const uint16_t*>(w.ffn_norm_g), pending_h ? bf.h : nullptr, bf.y0, true, M, d,
+                          c.eps);
   }));
   // 6. gate/up + SwiGLU
   {
@@ -454,15 +429,16 @@ vx_status run_layer_stream(const Launch& L, const vx_layer_cfg& c, const vx_laye
     a.bias = static_cast<const uint16_t*>(w.bgu);
     if ((st = gemm(L, "gemm_gate_up_swiglu", bf.y0, d, w.wgu, a, EPI_SWIGLU)) != VX_OK) return st;
   }
-  // 7. down, split-K partial sums; the layer output stays pending
-  {
-    GemmArgs a = base_args(L, M, d, F);
-    a.out = sb.parts; a.ld_out = d;
-    a.split_stride = pstride;
-    if ((st = gemm(L, "gemm_down_splitk", bf.act, F, w.wd, a, EPI_F32, kMaxSplits)) != VX_OK) return st;
-    *out = Pending{bf.h, sb.parts, a.k_splits, static_cast<const uint16_t*>(w.bd)};
-  }
-  return VX_OK;
+  // 7. out = h + bd + act Wd^T
+  return residual_gemm(L, "gemm_down_residual", bf.act, F, w.wd, M, d, F, static_cast<const uint16_t*>(w.bd), bf.h, y,
+                       bf.parts, cap, out);
+}
+
+// y = reduce(p) unless p already is y.
+cudaError_t reduce_into(const Launch& L, const Pending& p, float* y, int M, int d) {
+  if (p.base == y && p.parts == nullptr && p.bias == nullptr) return cudaSuccess;
+  return launch_rmsnorm(L, p.base, p.parts, p.nparts, static_cast<int64_t>(M) * d, p.bias, nullptr, y, nullptr, false,
+                        M, d, 1.0f);
 }
 
 // ------------------------------------------------------------- conv stem --
@@ -706,7 +682,12 @@ vx_status vx_encoder_layer_fwd(const vx_layer_cfg* cfg, const vx_layer_weights* 
   if ((st = make_launch(&L, ws, ws_bytes, vx_encoder_layer_workspace(cfg, B, T), stream)) != VX_OK) return st;
   Carve cv{static_cast<uint8_t*>(ws), kStatusBytes};
   const LayerBufs bf = carve_layer(cv, *cfg, int64_t(B) * T);
-  return run_layer(L, *cfg, *w, x, y, B, T, pos0, bf, nullptr);
+  Pending out;
+  if ((st = run_layer(L, *cfg, *w, Pending{x, nullptr, 0, nullptr}, &out, y, B, T, pos0, bf, nullptr)) != VX_OK)
+    return st;
+  if (out.base != y || out.parts || out.bias)
+    VX_CUDA(traced(L, "reduce_out", 1, [&] { return reduce_into(L, out, y, B * T, cfg->d_model); }));
+  return VX_OK;
 }
 
 size_t vx_conv_stem_workspace(int B, int n_mels, int Tm, int d) {
@@ -770,11 +751,16 @@ vx_status vx_encoder_fwd(const vx_layer_cfg* cfg, const float* mel, int B, int n
   }
   Carve cv{static_cast<uint8_t*>(ws), kStatusBytes};
   const LayerBufs bf = carve_layer(cv, *cfg, int64_t(B) * To);
-  for (int l = 0; l < n_layers; ++l)
-    if ((st = run_layer(L, *cfg, layers[l], out, out, B, To, 0, bf, nullptr)) != VX_OK) return st;
+  Pending cur{out, nullptr, 0, nullptr};
+  for (int l = 0; l < n_layers; ++l) {
+    Pending next;
+    if ((st = run_layer(L, *cfg, layers[l], cur, &next, out, B, To, 0, bf, nullptr)) != VX_OK) return st;
+    cur = next;
+  }
+  const int64_t pstride = static_cast<int64_t>(B) * To * cfg->d_model;
   VX_CUDA(traced(L, "rmsnorm", 1, [&] {
-    return launch_rmsnorm(L, out, nullptr, 0, 0, nullptr, static_cast<const uint16_t*>(final_g), nullptr, out, false,
-                          B * To, cfg->d_model, cfg->eps);
+    return launch_rmsnorm(L, cur.base, cur.parts, cur.nparts, pstride, cur.bias,
+                          static_cast<const uint16_t*>(final_g), nullptr, out, false, B * To, cfg->d_model, cfg->eps);
   }));
   return VX_OK;
 }
@@ -795,23 +781,30 @@ vx_status vx_stream_prefill(const vx_layer_cfg* cfg, const vx_layer_weights* lay
   Carve cv{static_cast<uint8_t*>(ws), kStatusBytes};
   const LayerBufs bf = carve_layer(cv, *cfg, int64_t(S) * T);
   const int64_t layer_elems = int64_t(S) * cfg->n_heads * ring->window * cfg->head_dim;
+  Pending cur{x, nullptr, 0, nullptr};
   for (int l = 0; l < ring->n_layers; ++l) {
     RingLayer rl{static_cast<uint16_t*>(ring->k) + l * layer_elems, static_cast<uint16_t*>(ring->v) + l * layer_elems,
                  ring->pos, ring->window, true, false};
-    if ((st = run_layer(L, *cfg, layers[l], l == 0 ? x : y, y, S, T, 0, bf, &rl)) != VX_OK) return st;
+    Pending next;
+    if ((st = run_layer(L, *cfg, layers[l], cur, &next, y, S, T, 0, bf, &rl)) != VX_OK) return st;
+    cur = next;
   }
-  if (final_g)
+  const int64_t pstride = static_cast<int64_t>(S) * T * cfg->d_model;
+  if (final_g) {
     VX_CUDA(traced(L, "rmsnorm", 1, [&] {
-      return launch_rmsnorm(L, y, nullptr, 0, 0, nullptr, static_cast<const uint16_t*>(final_g), nullptr, y, false,
-                            S * T, cfg->d_model, cfg->eps);
+      return launch_rmsnorm(L, cur.base, cur.parts, cur.nparts, pstride, cur.bias,
+                            static_cast<const uint16_t*>(final_g), nullptr, y, false, S * T, cfg->d_model, cfg->eps);
     }));
+  } else if (cur.base != y || cur.parts || cur.bias) {
+    VX_CUDA(traced(L, "reduce_out", 1, [&] { return reduce_into(L, cur, y, S * T, cfg->d_model); }));
+  }
   VX_CUDA(traced(L, "pos_add", 1, [&] { return launch_pos_add(L, ring->pos, S, T, true); }));
   return VX_OK;
 }
 
 size_t vx_stream_step_workspace(const vx_layer_cfg* cfg, int S, int n_new) {
   if (!cfg || S <= 0 || n_new <= 0) return kStatusBytes;
-  return stream_ws_bytes(*cfg, int64_t(S) * n_new);
+  return layer_ws_bytes(*cfg, int64_t(S) * n_new);
 }
 
 vx_status vx_stream_step(const vx_layer_cfg* cfg, const vx_layer_weights* layers, const vx_kv_ring* ring,
@@ -834,14 +827,14 @@ vx_status vx_stream_step(const vx_layer_cfg* cfg, const vx_layer_weights* layers
   Launch L;
   if ((st = make_launch(&L, ws, ws_bytes, vx_stream_step_workspace(cfg, S, n_new), stream)) != VX_OK) return st;
   Carve cv{static_cast<uint8_t*>(ws), kStatusBytes};
-  const StreamBufs sb = carve_stream(cv, *cfg, M);
+  const LayerBufs bf = carve_layer(cv, *cfg, M);
   const int64_t layer_elems = int64_t(S) * cfg->n_heads * ring->window * cfg->head_dim;
   Pending cur{x_new, nullptr, 0, nullptr};
   for (int l = 0; l < ring->n_layers; ++l) {
     RingLayer rl{static_cast<uint16_t*>(ring->k) + l * layer_elems, static_cast<uint16_t*>(ring->v) + l * layer_elems,
                  ring->pos, ring->window, false, true};
     Pending next;
-    if ((st = run_layer_stream(L, *cfg, layers[l], cur, &next, S, n_new, sb, rl)) != VX_OK) return st;
+    if ((st = run_layer(L, *cfg, layers[l], cur, &next, y, S, n_new, 0, bf, &rl)) != VX_OK) return st;
     cur = next;
   }
   // y = reduce(last layer output), then the optional final RMSNorm.
