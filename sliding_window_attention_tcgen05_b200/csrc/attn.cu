@@ -21,10 +21,10 @@ namespace vx {
 
 namespace {
 
-constexpr int kAttnThreads = 320;           // 2 softmax warpgroups, TMA warp, MMA warp
+constexpr int kAttnThreads = 384;           // 2 softmax warpgroups; TMA, 2 MMA and 1 idle warp
 constexpr int kNS = 4;                      // K/V pipeline stages
 constexpr int kTile = 128 * 64 * 2;         // one 128 x 64 bf16 tile
-constexpr int kAttnSmem = kTile * (1 + 2 * kNS) + 1024 + 512;
+constexpr int kAttnSmem = kTile * (1 + 2 * kNS) + 1024 + 2560;   // + barriers, TMEM slot, merge (m, l)
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleSlack = 8.0f;       // O is rescaled only when a row max grows by more than 2^8
 
@@ -57,8 +57,14 @@ __device__ __forceinline__ float tree_max32(const float* v) {
 // TMEM and is the A operand of O_X += P_X V; O_X is rescaled in place only when
 // a row's max grows by more than kRescaleSlack (the exponents are taken
 // against a stale max otherwise, which cancels in O / l).
-// Warps 0-3 / 4-7: warpgroups 0 / 1 (TMEM lane = query row), warp 8: TMA,
-// warp 9: MMA, issuing S(0), S(1), then S(u+2), PV(u) for u = 0, 1, ...
+// Warps 0-3 / 4-7: softmax warpgroups 0 / 1 (TMEM lane = query row); warp 8:
+// TMA; warps 9 / 10: the tensor-core products of warpgroup 0 / 1 (S(j+1) as
+// soon as S(j) is released, P V(j) when P(j) is ready), so one warpgroup's
+// products never queue behind the other's softmax; warp 11 idles.  The
+// softmax warpgroups take most of the register file (setmaxnreg).
+constexpr int kSoftmaxRegs = 224;   // 8 softmax warps x 224 + 4 other warps x 56 = 384 x 168 launched
+constexpr int kOtherRegs = 56;
+
 __global__ void __launch_bounds__(kAttnThreads, 1)
 swa_attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                    const __grid_constant__ CUtensorMap tmV, const __grid_constant__ AttnArgs a) {
@@ -69,10 +75,10 @@ swa_attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
   uint8_t* sV = sK + kNS * kTile;
   uint64_t* bars = reinterpret_cast<uint64_t*>(sV + kNS * kTile);
   constexpr int QF = 0, KF = 1, VF = KF + kNS, KVE = VF + kNS, SF = KVE + kNS, SE = SF + 2, PF = SE + 2,
-                PE = PF + 2, OD = PE + 2, DR = OD + 2, NBAR = DR + 1;
+                PE = PF + 2, OD = PE + 2, DR = OD + 2, NBAR = DR + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + NBAR);
   int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
-  float* xml = reinterpret_cast<float*>(abort_flag + 1);   // [128] m, [128] l of warpgroup 1 (padded below)
+  float* xml = reinterpret_cast<float*>(abort_flag + 1);   // [2][128] m, [2][128] l of each warpgroup
   auto bar = [&](int i) { return smem_addr(bars + i); };
 
   const int warp = threadIdx.x >> 5;
@@ -92,8 +98,8 @@ swa_attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
       mbar_init(bar(SF + X), 1); mbar_init(bar(SE + X), 128);
       mbar_init(bar(PF + X), 128); mbar_init(bar(PE + X), 1);
       mbar_init(bar(OD + X), 1);
+      mbar_init(bar(DR + X), 1);
     }
-    mbar_init(bar(DR), 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -112,8 +118,9 @@ swa_attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
   pdl_wait();
   pdl_trigger();
 
-  if (warp == 8) {
-    if (lane == 0) {
+  if (warp >= 8) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kOtherRegs));
+    if (warp == 8 && lane == 0) {
       mbar_arrive_expect_tx(bar(QF), kTile);
       tma_load_4d(smem_addr(sQ), &tmQ, bar(QF), 0, h, q0, b);
       uint32_t last_par = 0;
@@ -139,16 +146,16 @@ swa_attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
         mbar_wait(bar(KF + s), (last_par >> s) & 1u, dw, 12);
         mbar_wait(bar(VF + s), (last_par >> s) & 1u, dw, 12);
       }
-    }
-  } else if (warp == 9) {
-    if (lane == 0) {
+    } else if ((warp == 9 || warp == 10) && lane == 0) {
+      // Products of warpgroup X = warp - 9: its tiles u = X, X + 2, ...
+      const int X = warp - 9;
       const uint32_t idesc_s = idesc_bf16_f32(128, 128, 0);
       const uint32_t idesc_o = idesc_bf16_f32(128, 64, 1);
+      const int nX = (n + 1 - X) / 2;
       bool ok = mbar_wait(bar(QF), 0, wc, 13);
       const uint32_t qa = smem_addr(sQ);
-      // S(u) into S_{u%2}; it is the (u/2)-th tile of warpgroup u%2.
-      auto issue_s = [&](int u) -> bool {
-        const int X = u & 1, j = u >> 1, st = u % kNS;
+      auto issue_s = [&](int j) -> bool {   // S(u) into S_X, u = X + 2 j
+        const int u = X + 2 * j, st = u % kNS;
         if (!mbar_wait(bar(SE + X), (j & 1) ^ 1, wc, 17)) return false;
         if (!mbar_wait(bar(KF + st), (u / kNS) & 1, wc, 18)) return false;
         tc_fence_after();
@@ -160,8 +167,8 @@ swa_attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
         umma_commit(bar(SF + X));
         return true;
       };
-      auto issue_pv = [&](int u) -> bool {
-        const int X = u & 1, j = u >> 1, st = u % kNS;
+      auto issue_pv = [&](int j) -> bool {
+        const int u = X + 2 * j, st = u % kNS;
         if (!mbar_wait(bar(PF + X), j & 1, wc, 14)) return false;
         if (!mbar_wait(bar(VF + st), (u / kNS) & 1, wc, 15)) return false;
         tc_fence_after();
@@ -174,21 +181,20 @@ swa_attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
         umma_commit(bar(KVE + st));   // K/V tile u: S(u) and PV(u) were its last users
         return true;
       };
-      if (ok) ok = issue_s(0);
-      if (ok && n > 1) ok = issue_s(1);
-      for (int u = 0; ok && u < n; ++u) {
-        if (u + 2 < n) ok = issue_s(u + 2);
-        if (ok) ok = issue_pv(u);
+      if (ok && nX > 0) ok = issue_s(0);
+      for (int j = 0; ok && j < nX; ++j) {
+        if (j + 1 < nX) ok = issue_s(j + 1);
+        if (ok) ok = issue_pv(j);
       }
-      umma_commit(bar(OD + 0));
-      umma_commit(bar(OD + 1));
-      umma_commit(bar(DR));
+      umma_commit(bar(OD + X));
+      umma_commit(bar(DR + X));
       int zero = 0;
       WaitCtx dw = wc;
       dw.abort_flag = &zero;
-      mbar_wait(bar(DR), 0, dw, 19);
+      mbar_wait(bar(DR + X), 0, dw, 19);
     }
   } else {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kSoftmaxRegs));
     // ------------- softmax: warpgroup X takes key tiles X, X + 2, ...; thread r owns row q0 + r
     const int X = warp >> 2;
     const int r = threadIdx.x & 127;
@@ -225,13 +231,12 @@ swa_attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
       }
       tc_fence_before();
       mbar_arrive(bar(SE + X));      // S_X may be overwritten by the next product
-      // Edge tile: some (row, key) pair of the tile is outside (i - W, i].
+      // Edge tile: keys outside (i - W, i] of this row, i.e. outside columns
+      // [lo, hi] of the tile, are masked.
       if (key0 + 127 > q0 || key0 <= q0 + 127 - W) {
+        const int lo = i - W + 1 - key0, hi = i - key0;
 #pragma unroll
-        for (int e = 0; e < 128; ++e) {
-          const int key = key0 + e;
-          if (key > i || key <= i - W) sv[e] = -INFINITY;
-        }
+        for (int e = 0; e < 128; ++e) sv[e] = (e >= lo && e <= hi) ? sv[e] : -INFINITY;
       }
       const float m_tile = fmaxf(fmaxf(tree_max32(sv), tree_max32(sv + 32)),
                                  fmaxf(tree_max32(sv + 64), tree_max32(sv + 96))) * sl2;
@@ -288,42 +293,35 @@ swa_attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
       l_run += rs;
     }
 
-    // Merge: warpgroup 1 hands (m, l) over through shared memory; warpgroup 0
-    // reads both O_0 and O_1 from TMEM and writes the output rows.
-    if (X == 1) {
-      xml[r] = m_used;
-      xml[128 + r] = ok ? l_run : 0.f;
-      asm volatile("bar.sync 1, 256;" ::: "memory");
-    } else {
-      asm volatile("bar.sync 1, 256;" ::: "memory");
-      bool w = mbar_wait(bar(OD + 0), 0, wc, 23) && mbar_wait(bar(OD + 1), 0, wc, 24);
-      if (!__all_sync(0xffffffffu, w)) ok = false;
-      tc_fence_after();
-      const float m1 = xml[r], l1 = xml[128 + r];
-      const float M = fmaxf(m_used, m1);
-      const float f0 = (m_used == -INFINITY) ? 0.f : ex2_approx(m_used - M);
-      const float f1 = (m1 == -INFINITY) ? 0.f : ex2_approx(m1 - M);
-      const float inv_l = 1.0f / (l_run * f0 + l1 * f1);
-      uint16_t* dst = static_cast<uint16_t*>(a.out) + static_cast<int64_t>(b) * a.o_batch +
-                      static_cast<int64_t>(i) * a.o_row + static_cast<int64_t>(h) * a.o_head;
-#pragma unroll 1
-      for (int half = 0; half < 2; ++half) {
-        uint32_t x0[32], x1[32];
-        tmem_ld32(tmem + 192 + 32 * half + lane_off, x0);
-        tmem_ld32(tmem + 256 + 192 + 32 * half + lane_off, x1);
-        tmem_ld_wait();
-        if (ok && i < T) {
-          float v[32];
+    // Merge: the warpgroups swap (m, l) through shared memory; then each reads
+    // both O_0 and O_1 from TMEM for its half of the 64 output columns.
+    xml[X * 128 + r] = m_used;
+    xml[256 + X * 128 + r] = ok ? l_run : 0.f;
+    asm volatile("bar.sync 1, 256;" ::: "memory");
+    bool w = mbar_wait(bar(OD + 0), 0, wc, 23) && mbar_wait(bar(OD + 1), 0, wc, 24);
+    if (!__all_sync(0xffffffffu, w)) ok = false;
+    tc_fence_after();
+    const float m0v = xml[r], l0v = xml[256 + r], m1v = xml[128 + r], l1v = xml[384 + r];
+    const float M = fmaxf(m0v, m1v);
+    const float f0 = (m0v == -INFINITY) ? 0.f : ex2_approx(m0v - M);
+    const float f1 = (m1v == -INFINITY) ? 0.f : ex2_approx(m1v - M);
+    const float inv_l = 1.0f / (l0v * f0 + l1v * f1);
+    uint16_t* dst = static_cast<uint16_t*>(a.out) + static_cast<int64_t>(b) * a.o_batch +
+                    static_cast<int64_t>(i) * a.o_row + static_cast<int64_t>(h) * a.o_head + 32 * X;
+    uint32_t x0[32], x1[32];
+    tmem_ld32(tmem + 192 + 32 * X + lane_off, x0);
+    tmem_ld32(tmem + 256 + 192 + 32 * X + lane_off, x1);
+    tmem_ld_wait();
+    if (ok && i < T) {
+      float v[32];
 #pragma unroll
-          for (int d = 0; d < 32; ++d) {
-            // a warpgroup without keys for this row contributes nothing (its O may be unset)
-            const float y0 = f0 != 0.f ? __uint_as_float(x0[d]) * f0 : 0.f;
-            const float y1 = f1 != 0.f ? __uint_as_float(x1[d]) * f1 : 0.f;
-            v[d] = (y0 + y1) * inv_l;
-          }
-          store_bf16x32(dst + 32 * half, v);
-        }
+      for (int d = 0; d < 32; ++d) {
+        // a warpgroup without keys for this row contributes nothing (its O may be unset)
+        const float y0 = f0 != 0.f ? __uint_as_float(x0[d]) * f0 : 0.f;
+        const float y1 = f1 != 0.f ? __uint_as_float(x1[d]) * f1 : 0.f;
+        v[d] = (y0 + y1) * inv_l;
       }
+      store_bf16x32(dst, v);
     }
   }
 

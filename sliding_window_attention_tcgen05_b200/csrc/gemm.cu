@@ -591,8 +591,6 @@ gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
   cluster_sync_all();   // both CTAs' barriers initialised and TMEM allocated
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
-  pdl_wait();
-  pdl_trigger();
 
   const WaitCtx wc{a.status, abort_flag, a.limit_ns};
   const int m_tiles = (a.M + 255) / 256;
@@ -609,25 +607,48 @@ gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
     n0 = (r / splits) * BN;
   };
 
+  // The weights (B) do not depend on the previous kernel of the stream: both
+  // CTAs start streaming their halves of the first stages' B tiles before
+  // waiting for it; the leader arms the full barriers for whole stages.
+  int npre = 0;
+  if (warp == kProducerWarp && lane == 0 && cluster < num_tiles) {
+    int m0, n0, ks;
+    decode(cluster, m0, n0, ks);
+    npre = nkb < S ? nkb : S;
+    for (int i = 0; i < npre; ++i) {
+      if (rank == 0) mbar_arrive_expect_tx(full(i), 2 * C::kStageBytes);
+      tma_load_2d_pair(smem_addr(sB + i * C::kBHalfBytes), &tmB, map_to_cta(full(i), 0), (ks * nkb + i) * kBK,
+                       n0 + (BN / 2) * rank);
+    }
+  }
+  // Inputs written by the previous kernel of the stream are read below.
+  pdl_wait();
+  pdl_trigger();
+
   if (warp == kProducerWarp) {
     if (lane == 0) {
       int stage = 0;
       uint32_t phase = 0;
       uint32_t issued = 0, last_par = 0;
+      int it = 0;   // k-block iterations issued so far
       for (int tile = cluster; tile < num_tiles; tile += nclusters) {
         int m0, n0, ks;
         decode(tile, m0, n0, ks);
         bool ok = true;
-        for (int kb = ks * nkb; kb < (ks + 1) * nkb; ++kb) {
-          if (!mbar_wait(empty(stage), phase ^ 1, wc, 31)) { ok = false; break; }
+        for (int kb = ks * nkb; kb < (ks + 1) * nkb; ++kb, ++it) {
+          const bool pre = it < npre;   // B already in flight, barrier already armed
+          if (!pre) {
+            if (!mbar_wait(empty(stage), phase ^ 1, wc, 31)) { ok = false; break; }
+            if (rank == 0) mbar_arrive_expect_tx(full(stage), 2 * C::kStageBytes);
+          }
           const uint32_t fb = map_to_cta(full(stage), 0);   // the leader's full barrier
-          if (rank == 0) mbar_arrive_expect_tx(full(stage), 2 * C::kStageBytes);
           const int tap = kb / a.kb_per_tap;
           const int c = (kb - tap * a.kb_per_tap) * kBK;
           const int ax = (tap % a.a_stride) * a.a_tap_ch + c;
           const int ay = m0 + tap / a.a_stride;
           tma_load_2d_pair(smem_addr(sA + stage * kABytes), &tmA, fb, ax, ay);
-          tma_load_2d_pair(smem_addr(sB + stage * C::kBHalfBytes), &tmB, fb, kb * kBK, n0 + (BN / 2) * rank);
+          if (!pre)
+            tma_load_2d_pair(smem_addr(sB + stage * C::kBHalfBytes), &tmB, fb, kb * kBK, n0 + (BN / 2) * rank);
           issued |= 1u << stage;
           last_par = (last_par & ~(1u << stage)) | (phase << stage);
           if (++stage == S) { stage = 0; phase ^= 1; }
