@@ -52,6 +52,14 @@ bool pair_gemm_disabled() {
   return off;
 }
 
+bool tma_store_disabled() {
+  static const bool off = [] {
+    const char* e = std::getenv("VX_TMA_STORE");
+    return e && e[0] == '0';
+  }();
+  return off;
+}
+
 bool pdl_enabled() {
   static const bool on = [] {
     const char* e = std::getenv("VX_PDL");
@@ -280,15 +288,44 @@ GemmArgs base_args(const Launch& L, int M, int N, int K) {
 
 // Encodes B's tensor map for and launches one GEMM in the shape `p`
 // (a.k_splits must already equal p.splits).
+// Tensor map for TMA stores of a GEMM's output ({columns, M, splits}, a
+// 64-byte x 32-row box with the 64-byte swizzle of the epilogue's staging
+// buffer), or false when the output does not map rows 1:1 or is misaligned.
+bool tmap_gemm_out(CUtensorMap* m, const GemmArgs& a, int epi) {
+  const bool identity = a.out_rows == a.in_rows && a.out_off == 0 && a.t_valid == a.in_rows;
+  if (!identity || !aligned16(a.out)) return false;
+  if (epi == EPI_F32) {
+    const int64_t zs = a.k_splits > 1 ? a.split_stride : a.ld_out * a.M;
+    if ((a.ld_out * 4) % 16 != 0 || (zs * 4) % 16 != 0) return false;
+    const uint64_t dims[3] = {static_cast<uint64_t>(a.N), static_cast<uint64_t>(a.M),
+                              static_cast<uint64_t>(a.k_splits)};
+    const uint64_t strides[2] = {static_cast<uint64_t>(a.ld_out) * 4, static_cast<uint64_t>(zs) * 4};
+    const uint32_t box[3] = {16, 32, 1};
+    return encode_tmap(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, a.out, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_64B);
+  }
+  if (epi == EPI_QKV_ROPE || epi == EPI_SWIGLU) {
+    if ((a.ld_out * 2) % 16 != 0) return false;
+    const uint64_t cols = epi == EPI_SWIGLU ? a.N / 2 : a.N;
+    const uint64_t dims[3] = {cols, static_cast<uint64_t>(a.M), 1};
+    const uint64_t strides[2] = {static_cast<uint64_t>(a.ld_out) * 2, static_cast<uint64_t>(a.ld_out) * 2 * a.M};
+    const uint32_t box[3] = {32, 32, 1};
+    return encode_tmap(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, a.out, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_64B);
+  }
+  return false;
+}
+
 vx_status launch_planned(const Launch& L, const char* name, const CUtensorMap* tmA, const void* Bw, int64_t ldb,
-                         const GemmArgs& a, int epi, const GemmPlan& p) {
+                         const GemmArgs& a_in, int epi, const GemmPlan& p) {
   if (p.bn == 0) {
-    set_error("%s: no GEMM tile shape fits N=%d K=%d", name, a.N, a.K);
+    set_error("%s: no GEMM tile shape fits N=%d K=%d", name, a_in.N, a_in.K);
     return VX_ERR_UNSUPPORTED;
   }
-  CUtensorMap tmB;
-  if (!tmap_bf16_2d(&tmB, Bw, a.K, a.N, ldb, p.pair ? p.bn / 2 : p.bn)) return VX_ERR_CUDA;
-  VX_CUDA(traced(L, name, 1, [&] { return launch_gemm(L, *tmA, tmB, a, epi, p); }));
+  CUtensorMap tmB, tmD;
+  if (!tmap_bf16_2d(&tmB, Bw, a_in.K, a_in.N, ldb, p.pair ? p.bn / 2 : p.bn)) return VX_ERR_CUDA;
+  GemmArgs a = a_in;
+  std::memset(&tmD, 0, sizeof(tmD));
+  a.tma_store = (!tma_store_disabled() && tmap_gemm_out(&tmD, a, epi)) ? 1 : 0;
+  VX_CUDA(traced(L, name, 1, [&] { return launch_gemm(L, *tmA, tmB, tmD, a, epi, p); }));
   return VX_OK;
 }
 

@@ -172,6 +172,30 @@ __device__ __forceinline__ void store_bf16_chunk(uint16_t* out, int64_t ld_out, 
   }
 }
 
+// Output path of one staged chunk.  With TMA stores the chunk leaves shared
+// memory as one 64-byte x 32-row box (the staging swizzle is the tensor map's
+// 64-byte swizzle), written by lane 0; before the staging buffer is refilled,
+// lane 0 waits for the copy engine to have read it.
+struct ChunkOut {
+  const CUtensorMap* tmD;   // null: stores from registers
+  int row0;                 // first tile row of this warp
+  int z;                    // K-split index (third map coordinate)
+};
+__device__ __forceinline__ void stage_reuse(const ChunkOut& co, int lane) {
+  if (co.tmD) {
+    if (lane == 0) bulk_wait_read_all();
+    __syncwarp();
+  }
+}
+__device__ __forceinline__ void tma_flush(const ChunkOut& co, const uint4* stg, int lane, int col0) {
+  fence_proxy_async_smem();   // this lane's staging writes, visible to the copy engine
+  __syncwarp();
+  if (lane == 0) {
+    tma_store_3d(co.tmD, smem_addr(stg), col0, co.row0, co.z);
+    bulk_commit_group();
+  }
+}
+
 // Per warp: TMEM lane quarter q = warp & 3 (tile rows 32 q ..), and one half
 // of the tile's column work (warp >> 2).  Everything of a tile's epilogue
 // that does not need the accumulator is done before waiting for it: the bias
@@ -229,7 +253,8 @@ __device__ __forceinline__ void epilogue_prepare(const GemmArgs& a, EpiPre<BN, E
 // The accumulator part: tacc = this warp's TMEM lanes at the tile's column 0.
 template <int BN, int EPI>
 __device__ __forceinline__ void epilogue_tile(const GemmArgs& a, EpiPre<BN, EPI>& p, const uint16_t* sbias,
-                                              uint4* stg, uint32_t tacc, int n0, int ks, int warp, int lane) {
+                                              uint4* stg, uint32_t tacc, int n0, int ks, int warp, int lane,
+                                              const ChunkOut& co) {
   const bool use_bias = a.bias != nullptr && ks == 0;
   const int hf = warp >> 2;
   if constexpr (EPI == EPI_QKV_ROPE) {
@@ -254,14 +279,18 @@ __device__ __forceinline__ void epilogue_tile(const GemmArgs& a, EpiPre<BN, EPI>
           x1[j] = w * p.cs[j] + u * p.sn[j];
         }
       }
-      stage_bf16x32(stg, lane, x0);
-      __syncwarp();
-      store_bf16_chunk(out, a.ld_out, p.sr, stg, lane, n0 + c);
-      __syncwarp();
-      stage_bf16x32(stg, lane, x1);
-      __syncwarp();
-      store_bf16_chunk(out, a.ld_out, p.sr, stg, lane, n0 + c + 32);
-      __syncwarp();
+#pragma unroll
+      for (int part = 0; part < 2; ++part) {
+        stage_reuse(co, lane);
+        stage_bf16x32(stg, lane, part ? x1 : x0);
+        if (co.tmD) {
+          tma_flush(co, stg, lane, n0 + c + 32 * part);
+        } else {
+          __syncwarp();
+          store_bf16_chunk(out, a.ld_out, p.sr, stg, lane, n0 + c + 32 * part);
+          __syncwarp();
+        }
+      }
     }
   } else if constexpr (EPI == EPI_SWIGLU) {
     // units of 32 outputs: gate columns g + hh .., up columns g + 64 + hh ..
@@ -280,10 +309,15 @@ __device__ __forceinline__ void epilogue_tile(const GemmArgs& a, EpiPre<BN, EPI>
       if (use_bias) { add_bias32_smem(gv, sbias + g + hh); add_bias32_smem(uv, sbias + g + 64 + hh); }
 #pragma unroll
       for (int i = 0; i < 32; ++i) gv[i] = silu_f(gv[i]) * uv[i];
+      stage_reuse(co, lane);
       stage_bf16x32(stg, lane, gv);
-      __syncwarp();
-      store_bf16_chunk(out, a.ld_out, p.sr, stg, lane, (n0 + g) / 2 + hh);
-      __syncwarp();
+      if (co.tmD) {
+        tma_flush(co, stg, lane, (n0 + g) / 2 + hh);
+      } else {
+        __syncwarp();
+        store_bf16_chunk(out, a.ld_out, p.sr, stg, lane, (n0 + g) / 2 + hh);
+        __syncwarp();
+      }
     }
   } else {
     const bool use_res = EPI == EPI_F32 && a.res != nullptr && ks == 0;
@@ -314,6 +348,7 @@ __device__ __forceinline__ void epilogue_tile(const GemmArgs& a, EpiPre<BN, EPI>
         }
 #pragma unroll
         for (int h16 = 0; h16 < 32; h16 += 16) {
+          stage_reuse(co, lane);
           stage_f32x16(stg, lane, v + h16);
           __syncwarp();
           float4 o[4];
@@ -324,6 +359,25 @@ __device__ __forceinline__ void epilogue_tile(const GemmArgs& a, EpiPre<BN, EPI>
             if constexpr (EPI == EPI_F32) {
               o[i].x += p.res[i].x; o[i].y += p.res[i].y; o[i].z += p.res[i].z; o[i].w += p.res[i].w;
             }
+          }
+          if (co.tmD) {
+            if (use_res) {   // the residual went in column-wise: back into the same slots
+#pragma unroll
+              for (int i = 0; i < 4; ++i)
+                stg[stg_slot((lane >> 2) + 8 * i, jj)] =
+                    make_uint4(__float_as_uint(o[i].x), __float_as_uint(o[i].y), __float_as_uint(o[i].z),
+                               __float_as_uint(o[i].w));
+            }
+            if constexpr (EPI == EPI_F32) {
+              const int nxt = c + h16 + 16;
+              if (use_res && nxt < c0 + BN / 2) {
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+                  if (p.sr.ok & (1u << i)) p.res[i] = ld_res4(a, p.sr, i, n0 + nxt + 4 * jj);
+              }
+            }
+            tma_flush(co, stg, lane, n0 + c + h16);
+            continue;
           }
           __syncwarp();
           const int col = n0 + c + h16 + 4 * jj;
@@ -357,7 +411,7 @@ struct OneCfg {
 template <int BN, int EPI>
 __global__ void __launch_bounds__(kThreads, 1)
 gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-               const __grid_constant__ GemmArgs a) {
+               const __grid_constant__ CUtensorMap tmD, const __grid_constant__ GemmArgs a) {
   using C = OneCfg<BN>;
   constexpr int S = C::S::kStages;
   extern __shared__ uint8_t smem_raw[];
@@ -393,6 +447,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
   if (warp == kProducerWarp && lane == 0) {
     tma_prefetch_desc(&tmA);
     tma_prefetch_desc(&tmB);
+    if (a.tma_store) tma_prefetch_desc(&tmD);
   }
   tc_fence_before();
   __syncthreads();
@@ -516,11 +571,13 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
       if (!ok) break;
       tc_fence_after();
       const uint32_t tacc = tmem_base + ab * BN + (static_cast<uint32_t>((warp & 3) * 32) << 16);
-      epilogue_tile<BN, EPI>(a, pre, sbias, stg, tacc, n0, ks, warp, lane);
+      const ChunkOut co{a.tma_store ? &tmD : nullptr, m0 + (warp & 3) * 32, ks};
+      epilogue_tile<BN, EPI>(a, pre, sbias, stg, tacc, n0, ks, warp, lane, co);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(acc_empty(ab));
     }
+    if (a.tma_store && lane == 0) bulk_wait_all();   // this warp's output stores are complete
   }
 
   __syncthreads();
@@ -549,7 +606,7 @@ struct PairCfg {
 template <int BN, int EPI>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                const __grid_constant__ GemmArgs a) {
+                const __grid_constant__ CUtensorMap tmD, const __grid_constant__ GemmArgs a) {
   using C = PairCfg<BN>;
   constexpr int S = C::S::kStages;
   extern __shared__ uint8_t smem_raw[];
@@ -586,6 +643,7 @@ gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
   if (warp == kProducerWarp && lane == 0) {
     tma_prefetch_desc(&tmA);
     tma_prefetch_desc(&tmB);
+    if (a.tma_store) tma_prefetch_desc(&tmD);
   }
   tc_fence_before();
   cluster_sync_all();   // both CTAs' barriers initialised and TMEM allocated
@@ -715,11 +773,13 @@ gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
       if (!ok) break;
       tc_fence_after();
       const uint32_t tacc = tmem_base + ab * BN + (static_cast<uint32_t>((warp & 3) * 32) << 16);
-      epilogue_tile<BN, EPI>(a, pre, sbias, stg, tacc, n0, ks, warp, lane);
+      const ChunkOut co{a.tma_store ? &tmD : nullptr, m0 + (warp & 3) * 32, ks};
+      epilogue_tile<BN, EPI>(a, pre, sbias, stg, tacc, n0, ks, warp, lane, co);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(ab ? acc_empty_leader1 : acc_empty_leader0);
     }
+    if (a.tma_store && lane == 0) bulk_wait_all();   // this warp's output stores are complete
   }
 
   tc_fence_before();
@@ -741,36 +801,40 @@ cudaError_t set_smem(K kernel, int bytes, bool& done) {
 }
 
 template <int BN, int EPI>
-cudaError_t launch_one(const Launch& L, const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmArgs& a) {
+cudaError_t launch_one(const Launch& L, const CUtensorMap& tmA, const CUtensorMap& tmB, const CUtensorMap& tmD,
+                       const GemmArgs& a) {
   using C = OneCfg<BN>;
   static bool attr_set = false;
   if (cudaError_t e = set_smem(gemm_tc_kernel<BN, EPI>, C::S::kTotal, attr_set)) return e;
   const int tiles = ((a.M + kBM - 1) / kBM) * (a.N / BN) * a.k_splits;
   const int grid = tiles < L.sm_count ? tiles : L.sm_count;
-  return launch_kernel(gemm_tc_kernel<BN, EPI>, dim3(grid), dim3(kThreads), C::S::kTotal, L.stream, tmA, tmB, a);
+  return launch_kernel(gemm_tc_kernel<BN, EPI>, dim3(grid), dim3(kThreads), C::S::kTotal, L.stream, tmA, tmB, tmD,
+                       a);
 }
 
 template <int BN, int EPI>
-cudaError_t launch_pair(const Launch& L, const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmArgs& a) {
+cudaError_t launch_pair(const Launch& L, const CUtensorMap& tmA, const CUtensorMap& tmB, const CUtensorMap& tmD,
+                        const GemmArgs& a) {
   using C = PairCfg<BN>;
   static bool attr_set = false;
   if (cudaError_t e = set_smem(gemm_tc2_kernel<BN, EPI>, C::S::kTotal, attr_set)) return e;
   const int tiles = ((a.M + 255) / 256) * (a.N / BN) * a.k_splits;
   const int pairs = L.sm_count / 2;
   const int grid = 2 * (tiles < pairs ? tiles : pairs);
-  return launch_kernel(gemm_tc2_kernel<BN, EPI>, dim3(grid), dim3(kThreads), C::S::kTotal, L.stream, tmA, tmB, a);
+  return launch_kernel(gemm_tc2_kernel<BN, EPI>, dim3(grid), dim3(kThreads), C::S::kTotal, L.stream, tmA, tmB, tmD,
+                       a);
 }
 
 template <int EPI>
-cudaError_t launch_epi(const Launch& L, const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmArgs& a,
-                       const GemmPlan& p) {
+cudaError_t launch_epi(const Launch& L, const CUtensorMap& tmA, const CUtensorMap& tmB, const CUtensorMap& tmD,
+                       const GemmArgs& a, const GemmPlan& p) {
   if (p.pair) {
-    if (p.bn == 256) return launch_pair<256, EPI>(L, tmA, tmB, a);
-    if (p.bn == 128) return launch_pair<128, EPI>(L, tmA, tmB, a);
+    if (p.bn == 256) return launch_pair<256, EPI>(L, tmA, tmB, tmD, a);
+    if (p.bn == 128) return launch_pair<128, EPI>(L, tmA, tmB, tmD, a);
     return cudaErrorInvalidValue;
   }
-  if (p.bn == 256) return launch_one<256, EPI>(L, tmA, tmB, a);
-  if (p.bn == 128) return launch_one<128, EPI>(L, tmA, tmB, a);
+  if (p.bn == 256) return launch_one<256, EPI>(L, tmA, tmB, tmD, a);
+  if (p.bn == 128) return launch_one<128, EPI>(L, tmA, tmB, tmD, a);
   return cudaErrorInvalidValue;
 }
 
@@ -820,18 +884,19 @@ GemmPlan plan_gemm(int M, int N, int K, int epi, int max_splits, int sm) {
   return best;
 }
 
-cudaError_t launch_gemm(const Launch& L, const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmArgs& args,
-                        int epi, const GemmPlan& p) {
+cudaError_t launch_gemm(const Launch& L, const CUtensorMap& tmA, const CUtensorMap& tmB, const CUtensorMap& tmD,
+                        const GemmArgs& args, int epi, const GemmPlan& p) {
   if (args.M <= 0) return cudaSuccess;
   if (args.k_splits != p.splits || p.splits < 1 || (args.K / kBK) % p.splits != 0 || args.K % kBK != 0 ||
-      p.bn <= 0 || args.N % p.bn != 0 || (p.splits > 1 && epi != EPI_F32))
+      p.bn <= 0 || args.N % p.bn != 0 || (p.splits > 1 && epi != EPI_F32) ||
+      (args.tma_store && epi != EPI_F32 && epi != EPI_QKV_ROPE && epi != EPI_SWIGLU))
     return cudaErrorInvalidValue;
   switch (epi) {
-    case EPI_F32: return launch_epi<EPI_F32>(L, tmA, tmB, args, p);
-    case EPI_QKV_ROPE: return launch_epi<EPI_QKV_ROPE>(L, tmA, tmB, args, p);
-    case EPI_SWIGLU: return launch_epi<EPI_SWIGLU>(L, tmA, tmB, args, p);
-    case EPI_GELU_BF16: return launch_epi<EPI_GELU_BF16>(L, tmA, tmB, args, p);
-    case EPI_GELU_F32: return launch_epi<EPI_GELU_F32>(L, tmA, tmB, args, p);
+    case EPI_F32: return launch_epi<EPI_F32>(L, tmA, tmB, tmD, args, p);
+    case EPI_QKV_ROPE: return launch_epi<EPI_QKV_ROPE>(L, tmA, tmB, tmD, args, p);
+    case EPI_SWIGLU: return launch_epi<EPI_SWIGLU>(L, tmA, tmB, tmD, args, p);
+    case EPI_GELU_BF16: return launch_epi<EPI_GELU_BF16>(L, tmA, tmB, tmD, args, p);
+    case EPI_GELU_F32: return launch_epi<EPI_GELU_F32>(L, tmA, tmB, tmD, args, p);
     default: return cudaErrorInvalidValue;
   }
 }

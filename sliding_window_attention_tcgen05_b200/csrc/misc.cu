@@ -7,75 +7,93 @@ namespace vx {
 namespace {
 
 // ---------------------------------------------------------------- RMSNorm --
-// One warp per row of d (multiple of 128, <= 2048) fp32 values; lane i holds
-// float4 columns i, i+32, ...
-//   h = x + bias + sum_k parts[k]   (split-K partial sums of the GEMM before)
-//   y = h * rsqrt(mean(h^2) + eps) * g
+// RMSNorm with the pending residual sum folded in:
+//   h = x + bias + sum_{k < nparts} parts[k]   (split-K partial sums of the GEMM before)
+//   y = h * rsqrt(mean(h^2) + eps) * g          (skipped when y is null)
+// Every load of a row (x, each partial sum, bias, gain) is issued before any
+// arithmetic, so a row costs one memory round trip whatever nparts is.
+
+__device__ __forceinline__ float4 add4f(float4 a, float4 b) {
+  return make_float4(a.x + b.x, a.y + b.y, a.z + b.z, a.w + b.w);
+}
+__device__ __forceinline__ float4 add_bf16x4(float4 a, uint2 w) {
+  return make_float4(a.x + bf16lo(w.x), a.y + bf16hi(w.x), a.z + bf16lo(w.y), a.w + bf16hi(w.y));
+}
+__device__ __forceinline__ float sumsq4(float4 a, float s) {
+  return fmaf(a.x, a.x, fmaf(a.y, a.y, fmaf(a.z, a.z, fmaf(a.w, a.w, s))));
+}
 template <bool BF16_OUT>
-__global__ void __launch_bounds__(256)
+__device__ __forceinline__ void store_norm4(void* y, int64_t idx4, float4 a, float inv, uint2 gw) {
+  const float o0 = a.x * inv * bf16lo(gw.x), o1 = a.y * inv * bf16hi(gw.x);
+  const float o2 = a.z * inv * bf16lo(gw.y), o3 = a.w * inv * bf16hi(gw.y);
+  if constexpr (BF16_OUT) {
+    uint2 w;
+    w.x = pack_bf16x2(o0, o1);
+    w.y = pack_bf16x2(o2, o3);
+    reinterpret_cast<uint2*>(y)[idx4] = w;
+  } else {
+    reinterpret_cast<float4*>(y)[idx4] = make_float4(o0, o1, o2, o3);
+  }
+}
+
+// One warp per row of d = 128 NV fp32 values (lane i holds float4 columns
+// i, i + 32, ...), at most MAXP partial sums; four rows per CTA (a row holds
+// up to 3 NV float4 in flight per lane, so CTAs stay small enough for every
+// row of a one-layer batch to be resident at once).
+template <bool BF16_OUT, int NV, int MAXP>
+__global__ void __launch_bounds__(128)
 rmsnorm_kernel(const float* __restrict__ x, const float* __restrict__ parts, int nparts, int64_t part_stride,
                const uint16_t* __restrict__ bias, const uint16_t* __restrict__ g, float* __restrict__ h_out,
                void* __restrict__ y, int M, int d, float eps) {
   pdl_wait();
   pdl_trigger();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int row = blockIdx.x * 8 + warp;
+  const int row = blockIdx.x * 4 + warp;
   if (row >= M) return;
-  const int nv = d >> 7;
   const int64_t roff = static_cast<int64_t>(row) * d;
-  const float4* xr = reinterpret_cast<const float4*>(x + roff);
-  float4 v[16];
+  float4 v[NV];
+  float4 pp[MAXP][NV];
+  uint2 bw[NV], gw[NV];
+#pragma unroll
+  for (int i = 0; i < NV; ++i) v[i] = reinterpret_cast<const float4*>(x + roff)[lane + 32 * i];
+#pragma unroll
+  for (int k = 0; k < MAXP; ++k)
+    if (k < nparts) {
+#pragma unroll
+      for (int i = 0; i < NV; ++i) pp[k][i] = reinterpret_cast<const float4*>(parts + k * part_stride + roff)[lane + 32 * i];
+    }
+  if (bias) {
+#pragma unroll
+    for (int i = 0; i < NV; ++i) bw[i] = __ldg(reinterpret_cast<const uint2*>(bias) + lane + 32 * i);
+  }
+  if (y) {
+#pragma unroll
+    for (int i = 0; i < NV; ++i) gw[i] = __ldg(reinterpret_cast<const uint2*>(g) + lane + 32 * i);
+  }
   float ss = 0.f;
 #pragma unroll
-  for (int i = 0; i < 16; ++i) {
-    if (i < nv) {
-      const int c4 = lane + 32 * i;
-      float4 a = xr[c4];
-      for (int k = 0; k < nparts; ++k) {
-        const float4 b = reinterpret_cast<const float4*>(parts + k * part_stride + roff)[c4];
-        a.x += b.x; a.y += b.y; a.z += b.z; a.w += b.w;
-      }
-      if (bias) {
-        const uint2 bw = __ldg(reinterpret_cast<const uint2*>(bias) + c4);
-        a.x += bf16lo(bw.x); a.y += bf16hi(bw.x); a.z += bf16lo(bw.y); a.w += bf16hi(bw.y);
-      }
-      v[i] = a;
-      ss = fmaf(a.x, a.x, fmaf(a.y, a.y, fmaf(a.z, a.z, fmaf(a.w, a.w, ss))));
-    }
+  for (int i = 0; i < NV; ++i) {
+#pragma unroll
+    for (int k = 0; k < MAXP; ++k)
+      if (k < nparts) v[i] = add4f(v[i], pp[k][i]);
+    if (bias) v[i] = add_bf16x4(v[i], bw[i]);
+    ss = sumsq4(v[i], ss);
   }
   if (h_out) {
-    float4* hr = reinterpret_cast<float4*>(h_out + roff);
 #pragma unroll
-    for (int i = 0; i < 16; ++i)
-      if (i < nv) hr[lane + 32 * i] = v[i];
+    for (int i = 0; i < NV; ++i) reinterpret_cast<float4*>(h_out + roff)[lane + 32 * i] = v[i];
   }
   if (y == nullptr) return;
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
   const float inv = rsqrtf(ss / static_cast<float>(d) + eps);
-  const uint2* gr = reinterpret_cast<const uint2*>(g);
 #pragma unroll
-  for (int i = 0; i < 16; ++i) {
-    if (i < nv) {
-      const int c4 = lane + 32 * i;
-      const uint2 gw = __ldg(gr + c4);
-      const float o0 = v[i].x * inv * bf16lo(gw.x), o1 = v[i].y * inv * bf16hi(gw.x);
-      const float o2 = v[i].z * inv * bf16lo(gw.y), o3 = v[i].w * inv * bf16hi(gw.y);
-      if constexpr (BF16_OUT) {
-        uint2 w;
-        w.x = pack_bf16x2(o0, o1);
-        w.y = pack_bf16x2(o2, o3);
-        reinterpret_cast<uint2*>(static_cast<uint16_t*>(y) + roff)[c4] = w;
-      } else {
-        reinterpret_cast<float4*>(static_cast<float*>(y) + roff)[c4] = make_float4(o0, o1, o2, o3);
-      }
-    }
-  }
+  for (int i = 0; i < NV; ++i) store_norm4<BF16_OUT>(y, roff / 4 + lane + 32 * i, v[i], inv, gw[i]);
 }
 
 // Few-row variant: one CTA of d/4 threads per row (one float4 each), so that a
-// handful of rows still spreads over the SMs; same arithmetic as above.
-template <bool BF16_OUT>
+// handful of rows still spreads over the SMs; up to MAXP partial sums.
+template <bool BF16_OUT, int MAXP>
 __global__ void __launch_bounds__(512)
 rmsnorm_row_kernel(const float* __restrict__ x, const float* __restrict__ parts, int nparts, int64_t part_stride,
                    const uint16_t* __restrict__ bias, const uint16_t* __restrict__ g, float* __restrict__ h_out,
@@ -87,17 +105,20 @@ rmsnorm_row_kernel(const float* __restrict__ x, const float* __restrict__ parts,
   const int c4 = threadIdx.x;
   const int64_t roff = static_cast<int64_t>(row) * d;
   float4 a = reinterpret_cast<const float4*>(x + roff)[c4];
-  for (int k = 0; k < nparts; ++k) {
-    const float4 b = reinterpret_cast<const float4*>(parts + k * part_stride + roff)[c4];
-    a.x += b.x; a.y += b.y; a.z += b.z; a.w += b.w;
-  }
-  if (bias) {
-    const uint2 bw = __ldg(reinterpret_cast<const uint2*>(bias) + c4);
-    a.x += bf16lo(bw.x); a.y += bf16hi(bw.x); a.z += bf16lo(bw.y); a.w += bf16hi(bw.y);
-  }
+  float4 pp[MAXP];
+#pragma unroll
+  for (int k = 0; k < MAXP; ++k)
+    if (k < nparts) pp[k] = reinterpret_cast<const float4*>(parts + k * part_stride + roff)[c4];
+  uint2 bw = make_uint2(0u, 0u), gw = make_uint2(0u, 0u);
+  if (bias) bw = __ldg(reinterpret_cast<const uint2*>(bias) + c4);
+  if (y) gw = __ldg(reinterpret_cast<const uint2*>(g) + c4);
+#pragma unroll
+  for (int k = 0; k < MAXP; ++k)
+    if (k < nparts) a = add4f(a, pp[k]);
+  if (bias) a = add_bf16x4(a, bw);
   if (h_out) reinterpret_cast<float4*>(h_out + roff)[c4] = a;
   if (y == nullptr) return;   // uniform over the CTA
-  float ss = fmaf(a.x, a.x, fmaf(a.y, a.y, fmaf(a.z, a.z, a.w * a.w)));
+  float ss = sumsq4(a, 0.f);
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
   if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = ss;
@@ -105,17 +126,7 @@ rmsnorm_row_kernel(const float* __restrict__ x, const float* __restrict__ parts,
   float tot = 0.f;
   for (int w = 0; w < static_cast<int>(blockDim.x >> 5); ++w) tot += red[w];
   const float inv = rsqrtf(tot / static_cast<float>(d) + eps);
-  const uint2 gw = __ldg(reinterpret_cast<const uint2*>(g) + c4);
-  const float o0 = a.x * inv * bf16lo(gw.x), o1 = a.y * inv * bf16hi(gw.x);
-  const float o2 = a.z * inv * bf16lo(gw.y), o3 = a.w * inv * bf16hi(gw.y);
-  if constexpr (BF16_OUT) {
-    uint2 w;
-    w.x = pack_bf16x2(o0, o1);
-    w.y = pack_bf16x2(o2, o3);
-    reinterpret_cast<uint2*>(static_cast<uint16_t*>(y) + roff)[c4] = w;
-  } else {
-    reinterpret_cast<float4*>(static_cast<float*>(y) + roff)[c4] = make_float4(o0, o1, o2, o3);
-  }
+  store_norm4<BF16_OUT>(y, roff / 4 + c4, a, inv, gw);
 }
 
 // ---------------------------------------------------------------- packing --
@@ -226,24 +237,37 @@ __global__ void selftest_wait_kernel(DevStatus* st, uint64_t limit_ns) {
 
 }  // namespace
 
+template <bool BF16, int NV>
+static cudaError_t launch_rms_warp(const Launch& L, const float* x, const float* parts, int nparts, int64_t ps,
+                                   const uint16_t* bias, const uint16_t* g, float* h_out, void* y, int M, int d,
+                                   float eps) {
+  return launch_kernel(rmsnorm_kernel<BF16, NV, 2>, dim3((M + 3) / 4), dim3(128), 0, L.stream, x, parts, nparts, ps,
+                       bias, g, h_out, y, M, d, eps);
+}
+
+template <bool BF16>
+static cudaError_t launch_rms(const Launch& L, const float* x, const float* parts, int nparts, int64_t ps,
+                              const uint16_t* bias, const uint16_t* g, float* h_out, void* y, int M, int d, float eps) {
+  if (M <= 512 || nparts > 2)   // few rows, or many partial sums: a CTA per row
+    return launch_kernel(rmsnorm_row_kernel<BF16, 8>, dim3(M), dim3(d / 4), 0, L.stream, x, parts, nparts, ps, bias,
+                         g, h_out, y, M, d, eps);
+  switch (d / 128) {
+#define VX_RMS_NV(n) \
+  case n: return launch_rms_warp<BF16, n>(L, x, parts, nparts, ps, bias, g, h_out, y, M, d, eps);
+    VX_RMS_NV(1) VX_RMS_NV(2) VX_RMS_NV(3) VX_RMS_NV(4) VX_RMS_NV(5) VX_RMS_NV(6) VX_RMS_NV(7) VX_RMS_NV(8)
+    VX_RMS_NV(9) VX_RMS_NV(10) VX_RMS_NV(11) VX_RMS_NV(12) VX_RMS_NV(13) VX_RMS_NV(14) VX_RMS_NV(15) VX_RMS_NV(16)
+#undef VX_RMS_NV
+    default: return cudaErrorInvalidValue;
+  }
+}
+
 cudaError_t launch_rmsnorm(const Launch& L, const float* x, const float* parts, int nparts, int64_t part_stride,
                            const uint16_t* bias, const uint16_t* g, float* h_out, void* y, bool y_bf16, int M,
                            int d, float eps) {
   if (M <= 0) return cudaSuccess;
-  if (M <= 2048) {   // few rows: a CTA per row
-    const dim3 threads(d / 4);
-    if (y_bf16)
-      return launch_kernel(rmsnorm_row_kernel<true>, dim3(M), threads, 0, L.stream, x, parts, nparts, part_stride,
-                           bias, g, h_out, y, M, d, eps);
-    return launch_kernel(rmsnorm_row_kernel<false>, dim3(M), threads, 0, L.stream, x, parts, nparts, part_stride,
-                         bias, g, h_out, y, M, d, eps);
-  }
-  const dim3 blocks((M + 7) / 8);
-  if (y_bf16)
-    return launch_kernel(rmsnorm_kernel<true>, blocks, dim3(256), 0, L.stream, x, parts, nparts, part_stride, bias,
-                         g, h_out, y, M, d, eps);
-  return launch_kernel(rmsnorm_kernel<false>, blocks, dim3(256), 0, L.stream, x, parts, nparts, part_stride, bias,
-                       g, h_out, y, M, d, eps);
+  if (nparts < 0 || nparts > 8 || d % 128 != 0 || d > 2048) return cudaErrorInvalidValue;
+  if (y_bf16) return launch_rms<true>(L, x, parts, nparts, part_stride, bias, g, h_out, y, M, d, eps);
+  return launch_rms<false>(L, x, parts, nparts, part_stride, bias, g, h_out, y, M, d, eps);
 }
 
 static cudaError_t pack_rows(const Launch& L, PackSrc p, uint16_t* out, int64_t rows, int64_t cols) {

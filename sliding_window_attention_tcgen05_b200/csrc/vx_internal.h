@@ -28,6 +28,7 @@ int current_sm_count();
 uint64_t wait_limit_ns();
 bool pdl_enabled();   // programmatic dependent launch (default on; VX_PDL=0 disables)
 bool pair_gemm_disabled();   // two-CTA GEMM tiles (default on; VX_PAIR_GEMM=0 disables)
+bool tma_store_disabled();   // TMA stores of GEMM outputs (default on; VX_TMA_STORE=0 disables)
 
 // Launches `k` on `stream`, with programmatic dependent launch when enabled.
 template <class... KArgs, class... Args>
@@ -88,6 +89,10 @@ struct GemmArgs {
   int rope_cols;           // columns [0, rope_cols) are rotated in 64-wide heads
   float inv_freq_hi[32];   // inv_freq_m as float, and its residual to the exact value
   float inv_freq_lo[32];
+  // Output through TMA tile stores (identity row mapping, EPI_F32 / QKV / SwiGLU):
+  // tmD is then a 3-D map {columns, M, splits} with a 64-byte swizzled box of
+  // 64 bytes x 32 rows.
+  int tma_store;
   DevStatus* status;
   uint64_t limit_ns;
 };
@@ -107,9 +112,10 @@ GemmPlan plan_gemm(int M, int N, int K, int epi, int max_splits, int sm);
 // D[M, N] = A[M, K] * B[N, K]^T with the given epilogue, in the shape `plan`.
 // tmA: 2-D bf16 map with 128-byte swizzle and box {64, 128}; tmB: the same
 // with box {64, plan.pair ? plan.bn / 2 : plan.bn}.  args.k_splits must equal
-// plan.splits; N % bn == 0; K % 64 == 0; (K / 64) % splits == 0.
-cudaError_t launch_gemm(const Launch& L, const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmArgs& args,
-                        int epi, const GemmPlan& plan);
+// plan.splits; N % bn == 0; K % 64 == 0; (K / 64) % splits == 0.  tmD: the
+// output map when args.tma_store (see GemmArgs), else unused.
+cudaError_t launch_gemm(const Launch& L, const CUtensorMap& tmA, const CUtensorMap& tmB, const CUtensorMap& tmD,
+                        const GemmArgs& args, int epi, const GemmPlan& plan);
 
 void fill_rope_freqs(GemmArgs* a, float theta, int head_dim);
 
