@@ -25,7 +25,13 @@ Readings where the page is silent (each pinned by a test in tests/):
   * conv stem: left zero padding of k - 1 = 2 frames before each conv, exact
     (erf) GELU, output length floor((Tm - 1) / 2) + 1;
   * streaming: the ring holds frame f in slot f mod W; a step reads every old
-    in-window slot before any new frame is written.
+    in-window slot before any new frame is written;
+  * streaming conv stem (the "conv padding cache" of the Frontend section):
+    a chunk of an even number of mel frames continues the left context of
+    the previous chunk: the last 2 mel frames (conv1 taps) and the last 2
+    conv1 outputs (conv2 taps) are carried; the first chunk starts from zeros;
+  * projector: frames 4j .. 4j+3 are concatenated in time order into token j
+    (frame-major reshape of [B, T, d] to [B, T/4, 4d]), exact (erf) GELU.
 
 Parity against the real checkpoint is unpinned: the pages print no
 activations and no trained weights are available.
@@ -40,7 +46,8 @@ from scipy.special import erf as _erf
 __all__ = [
     "rms_norm", "rope_inv_freq", "rope", "swa_attention", "swa_attention_rows",
     "silu", "gelu", "encoder_layer", "ring_from_sequence", "stream_step_layer",
-    "stream_step", "conv_stem", "conv_out_len", "encoder", "as64",
+    "stream_step", "conv_stem", "conv_out_len", "encoder", "as64", "conv_stem_step",
+    "projector",
 ]
 
 
@@ -285,3 +292,42 @@ def encoder(mel, conv, layers, final_g, dims):
     for p in layers:
         x = encoder_layer(x, p, dims, pos0=0)
     return rms_norm(x, final_g, dims.eps)
+
+
+def conv_stem_step(mel_new, w1, b1, w2, b2, cache_x, cache_h1):
+    """One streaming chunk of the causal conv stem with a conv padding cache.
+
+    mel_new: [B, C, n] (n even) new mel frames; cache_x: [B, C, 2] the last two
+    mel frames of the previous chunk; cache_h1: [B, d, 2] its last two conv1
+    outputs (GELU applied); zeros before the first chunk (the left padding).
+    Returns (out [B, n/2, d], new cache_x, new cache_h1), where out continues
+    conv_stem of the concatenated stream: conv1 reads mel t-2 .. t, conv2
+    output u reads conv1 outputs 2u-2 .. 2u."""
+    x = as64(mel_new)
+    w1, b1, w2, b2 = as64(w1), as64(b1), as64(w2), as64(b2)
+    B, C, n = x.shape
+    assert n % 2 == 0, "chunks must keep the stride-2 phase"
+    xp = np.concatenate([as64(cache_x), x], axis=2)                      # [B, C, n+2]
+    h1 = np.zeros((B, w1.shape[0], n)) + b1[None, :, None]
+    for k in range(3):
+        h1 += np.einsum("oc,bct->bot", w1[:, :, k], xp[:, :, k:k + n], optimize=True)
+    h1 = gelu(h1)
+    hp = np.concatenate([as64(cache_h1), h1], axis=2)                    # [B, d, n+2]
+    To = n // 2
+    h2 = np.zeros((B, w2.shape[0], To)) + b2[None, :, None]
+    for k in range(3):
+        h2 += np.einsum("oc,bct->bot", w2[:, :, k], hp[:, :, k:k + 2 * To - 1:2], optimize=True)
+    return np.transpose(gelu(h2), (0, 2, 1)), xp[:, :, -2:], hp[:, :, -2:]
+
+
+def projector(x, w1, w2, factor=4):
+    """Audio projector of the 2602 model (transcribe.cpp notes "Voxtral",
+    section "Architecture -> Voxtral Realtime 2602"): reshape [B, T, d] to
+    [B, T // factor, factor * d] (the last T % factor frames dropped, frames
+    4j .. 4j+3 concatenated in time order), then Linear(4d -> H) without bias,
+    GELU, Linear(H -> H) without bias.  w1: [H, 4d], w2: [H, H]."""
+    x = as64(x)
+    B, T, d = x.shape
+    T4 = T // factor
+    tok = x[:, :T4 * factor, :].reshape(B, T4, factor * d)
+    return gelu(tok @ as64(w1).T) @ as64(w2).T

@@ -137,6 +137,15 @@ def mel(B, n_mels, Tm, seed=4):
     return _normal(rng, (B, n_mels, Tm))
 
 
+def projector_params(d=1280, hidden=3072, factor=4, seed=8):
+    """Audio projector weights (no biases): w1 [hidden, factor*d], w2 [hidden, hidden],
+    drawn in that order ~ N(0, 0.02), bf16-exact."""
+    rng = np.random.default_rng(seed)
+    w1 = bf16_round(_normal(rng, (hidden, factor * d), 0.02))
+    w2 = bf16_round(_normal(rng, (hidden, hidden), 0.02))
+    return {"w1": w1, "w2": w2}
+
+
 def final_norm_gain(d=1280, seed=5):
     """Final encoder RMSNorm gain, 1 + N(0, 0.02), bf16-exact."""
     rng = np.random.default_rng(seed)
