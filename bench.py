@@ -59,7 +59,7 @@ def parse_args(argv=None):
     ap.add_argument("--impl", choices=("vx", "reference"), default="vx")
     ap.add_argument("--no-components", action="store_true", help="skip the C2/C3/C4 component timings")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--components-only", default="", help="comma list of c2,c3,c4 (profiling runs)")
+    ap.add_argument("--components-only", default="", help="comma list of c2,c3,c4,next (profiling runs)")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-copy end-to-end pass (profiling runs)")
     ap.add_argument("--no-trace", action="store_true", help="skip the traced per-kernel pass (profiling runs)")
     ap.add_argument("--c3-layers", type=int, default=32, help="layers of the streaming-step component (profiling runs)")
@@ -377,6 +377,45 @@ def component_c4(vx, torch, flush, hbm, tf):
             "kernel_ms_per_forward": {k: v["ms_per_step"] for k, v in tr.items()}}
 
 
+def component_next(vx, torch, flush, hbm, tf):
+    """The widened rows: the streaming conv-stem step (64 streams x 8 mel frames
+    -> 4 frames, warm padding cache) and the audio projector on the encoder
+    output of the 4 x 6000-mel workload ([4, 3000, 1280] -> [4, 750, 3072])."""
+    g = torch.Generator(device="cuda").manual_seed(501)
+
+    def nrm(shape, std):
+        return (torch.randn(shape, generator=g, device="cuda") * std).to(torch.bfloat16)
+
+    w1p = vx.pack_conv_weight(nrm((1280, 128, 3), 0.02))
+    w2p = vx.pack_conv_weight(nrm((1280, 1280, 3), 0.02))
+    b1, b2 = nrm((1280,), 0.01), nrm((1280,), 0.01)
+    S = 64
+    cache = vx.ConvCache(S, 128, 1280)
+    mel = torch.randn(S, 128, 8, generator=g, device="cuda")
+    y = torch.empty(S, 4, 1280, device="cuda")
+    ws = vx.Workspace(vx.lib.vx_conv_stem_step_workspace(S, 128, 8, 1280))
+    step = lambda: vx.conv_stem_step(mel, w1p, b1, w2p, b2, cache, out=y, ws=ws)
+    for _ in range(3):
+        step()
+    ms_c, _, _ = timed_steps(torch, step, 50, lambda: None, torch.cuda.current_stream())
+    conv_flop = 2 * S * 8 * 1280 * 128 * 3 + 2 * S * 4 * 1280 * 1280 * 3
+    conv_bytes = (1280 * 128 * 3 + 1280 * 1280 * 3) * 2 + S * 128 * 8 * 4 + S * 4 * 1280 * 4
+    w1 = nrm((3072, 5120), 0.02)
+    w2 = nrm((3072, 3072), 0.02)
+    x = torch.randn(4, 3000, 1280, generator=g, device="cuda")
+    out = torch.empty(4, 750, 3072, device="cuda")
+    wsp = vx.Workspace(vx.lib.vx_projector_workspace(4, 3000, 1280, 3072))
+    proj = lambda: vx.projector_fwd(x, w1, w2, out=out, ws=wsp)
+    for _ in range(3):
+        proj()
+    ms_p, _, _ = timed_steps(torch, proj, 20, flush, torch.cuda.current_stream())
+    proj_flop = 2 * 3000 * 5120 * 3072 + 2 * 3000 * 3072 * 3072
+    return {"conv_step_64x8": {"ms_per_step": ms_c, "frames_per_s": S * 4 / ms_c * 1e3,
+                               "gbs": conv_bytes / ms_c / 1e6, "tflops": conv_flop / ms_c / 1e9},
+            "projector_4x3000": {"ms_per_call": ms_p, "tokens_per_s": 3000 / ms_p * 1e3,
+                                 "tflops": proj_flop / ms_p / 1e9, "frac_of_measured_peak": proj_flop / ms_p / 1e9 / tf}}
+
+
 # ------------------------------------------------------------- cpu legs
 
 def oracle_sample(frames: int):
@@ -461,7 +500,8 @@ def main(argv=None):
             if c == "c3":
                 out[c] = component_c3(vx, torch, flush, hbm, tf_burst, L=args.c3_layers)
             else:
-                out[c] = {"c2": component_c2, "c4": component_c4}[c](vx, torch, flush, hbm, tf_burst)
+                out[c] = {"c2": component_c2, "c4": component_c4, "next": component_next}[c](vx, torch, flush, hbm,
+                                                                                              tf_burst)
         if rank == 0:
             print(json.dumps({"components": out}), flush=True)
         return 0
@@ -541,7 +581,8 @@ def main(argv=None):
     comps = None
     if world == 1 and not args.no_components:
         comps = {}
-        for name, fn in (("swa_c2", component_c2), ("stream_step_c3", component_c3), ("encoder_c4", component_c4)):
+        for name, fn in (("swa_c2", component_c2), ("stream_step_c3", component_c3), ("encoder_c4", component_c4),
+                         ("next_rows", component_next)):
             try:
                 comps[name] = fn(vx, torch, flush, hbm, tf_burst)
             except Exception as e:   # report, never hide

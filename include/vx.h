@@ -222,6 +222,44 @@ VX_API vx_status vx_conv_stem_fwd(const float *mel, const void *w1p, const void 
                            void *ws, size_t ws_bytes, cudaStream_t stream);
 VX_API size_t vx_conv_stem_workspace(int B, int n_mels, int Tm, int d);
 
+/* Streaming conv stem step with a conv padding cache (transcribe.cpp notes
+ * "Voxtral", section "Frontend": the Realtime model's conv padding cache
+ * carries continuity across streaming chunks; section "Architecture ->
+ * Voxtral Realtime 2602": 8 mel frames = 4 encoder frames per step).
+ * One chunk of n_new mel frames per stream continues the causal conv stem of
+ * everything the stream has seen: conv1 reads mel frames t-2 .. t, conv2
+ * output u reads conv1 outputs 2u-2 .. 2u, and the two frames before the
+ * chunk come from the cache instead of the zero padding of vx_conv_stem_fwd.
+ *   mel_new:  [S, n_mels, n_new] fp32, n_new even (8 for the 80 ms schedule)
+ *   cache_x:  [S, 2, n_mels] bf16, the last two mel frames seen (rounded to bf16)
+ *   cache_h1: [S, 2, d] bf16, the last two conv1 outputs (after GELU)
+ *   out:      [S, n_new / 2, d] fp32
+ * Both caches are read, then overwritten with this chunk's last two rows;
+ * zero them before a stream's first chunk.  Weights as vx_conv_stem_fwd.
+ * Returns VX_ERR_UNSUPPORTED for odd n_new.  Workspace:
+ * vx_conv_stem_step_workspace().  The caches are owned by the caller and must
+ * not be shared by concurrent calls. */
+VX_API vx_status vx_conv_stem_step(const float *mel_new, const void *w1p, const void *b1,
+                            const void *w2p, const void *b2, void *cache_x, void *cache_h1,
+                            float *out, int S, int n_mels, int n_new, int d,
+                            void *ws, size_t ws_bytes, cudaStream_t stream);
+VX_API size_t vx_conv_stem_step_workspace(int S, int n_mels, int n_new, int d);
+
+/* Audio projector (transcribe.cpp notes "Voxtral", section "Architecture ->
+ * Voxtral Realtime 2602", Projector): the encoder output x [B, T, d] fp32 is
+ * reshaped to [B, T/4, 4d] (frames 4j .. 4j+3 concatenated in time order, the
+ * last T % 4 frames dropped), then out = GELU(tok w1^T) w2^T without biases.
+ *   w1: [hidden, 4d] bf16;  w2: [hidden, hidden] bf16;  out: [B, T/4, hidden] fp32
+ * Tokens and the hidden activation are bf16 tensor-core operands (fp32
+ * accumulate); GELU is the exact erf form.  d % 16 == 0, hidden % 128 == 0
+ * (else VX_ERR_UNSUPPORTED).  With T < 4 there is no token: the call returns
+ * VX_OK without reading or writing anything (the pointers may then be null).
+ * Workspace: vx_projector_workspace(). */
+VX_API vx_status vx_projector_fwd(const float *x, const void *w1, const void *w2, float *out,
+                           int B, int T, int d, int hidden,
+                           void *ws, size_t ws_bytes, cudaStream_t stream);
+VX_API size_t vx_projector_workspace(int B, int T, int d, int hidden);
+
 /* Whole-clip encoder: conv stem -> n_layers encoder layers (positions from 0)
  * -> final RMSNorm with gain final_g ([d] bf16).  layers: HOST array of
  * n_layers weight structs (device pointers inside).  out: [B, T_out, d] fp32.

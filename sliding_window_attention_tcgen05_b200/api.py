@@ -208,6 +208,46 @@ def conv_stem_fwd(mel, w1p, b1, w2p, b2, out=None, ws: Workspace | None = None):
     return out
 
 
+class ConvCache:
+    """Conv padding cache of one set of streams for conv_stem_step: the last
+    two mel frames ([S, 2, n_mels] bf16) and conv1 outputs ([S, 2, d] bf16)."""
+
+    def __init__(self, S: int, n_mels: int, d: int, device="cuda"):
+        self.x = torch.zeros(S, 2, n_mels, dtype=torch.bfloat16, device=device)
+        self.h1 = torch.zeros(S, 2, d, dtype=torch.bfloat16, device=device)
+
+    def reset(self):
+        self.x.zero_()
+        self.h1.zero_()
+
+
+def conv_stem_step(mel_new, w1p, b1, w2p, b2, cache: ConvCache, out=None, ws: Workspace | None = None):
+    """One streaming chunk: mel_new [S, n_mels, n_new] fp32 -> [S, n_new // 2, d] fp32; updates cache."""
+    S, nm, n = mel_new.shape
+    d = w1p.shape[0]
+    if out is None:
+        out = torch.empty(S, n // 2, d, dtype=torch.float32, device=mel_new.device)
+    need = lib.vx_conv_stem_step_workspace(S, nm, n, d)
+    ws = _ws(ws, need, mel_new.device)
+    p, nb = ws.get(need)
+    check(lib.vx_conv_stem_step(_p(mel_new), _p(w1p), _p(b1), _p(w2p), _p(b2), _p(cache.x), _p(cache.h1), _p(out),
+                                S, nm, n, d, p, nb, _stream()), "vx_conv_stem_step")
+    return out
+
+
+def projector_fwd(x, w1, w2, out=None, ws: Workspace | None = None):
+    """Audio projector: x [B, T, d] fp32 -> [B, T // 4, hidden] fp32 (w1 [hidden, 4d], w2 [hidden, hidden] bf16)."""
+    B, T, d = x.shape
+    hidden = w1.shape[0]
+    if out is None:
+        out = torch.empty(B, T // 4, hidden, dtype=torch.float32, device=x.device)
+    need = lib.vx_projector_workspace(B, T, d, hidden)
+    ws = _ws(ws, need, x.device)
+    p, n = ws.get(need)
+    check(lib.vx_projector_fwd(_p(x), _p(w1), _p(w2), _p(out), B, T, d, hidden, p, n, _stream()), "vx_projector_fwd")
+    return out
+
+
 def encoder_fwd(cfg: LayerCfg, mel, w1p, b1, w2p, b2, layers, final_g, out=None, ws: Workspace | None = None):
     B, nm, Tm = mel.shape
     To = (Tm - 1) // 2 + 1

@@ -494,11 +494,17 @@ ConvBufs carve_conv(Carve& cv, int B, int C, int Tm, int d) {
   return b;
 }
 
+// cache_x / cache_h1 (both or neither): the conv padding cache of a streaming
+// chunk (see vx_conv_stem_step); rows 0, 1 of xpad / h1pad come from it and
+// are replaced by the chunk's last two rows afterwards.
 vx_status run_conv_stem(const Launch& L, const float* mel, const void* w1p, const void* b1, const void* w2p,
-                        const void* b2, float* out, int B, int C, int Tm, int d, const ConvBufs& cb) {
+                        const void* b2, float* out, int B, int C, int Tm, int d, const ConvBufs& cb,
+                        uint16_t* cache_x = nullptr, uint16_t* cache_h1 = nullptr) {
   const int P = conv_rows_per_clip(Tm);
   const int To = (Tm - 1) / 2 + 1;
-  VX_CUDA(traced(L, "conv_prep", 2, [&] { return launch_conv_prep(L, mel, cb.xpad, cb.h1pad, B, C, Tm, P, d); }));
+  VX_CUDA(traced(L, "conv_prep", 2, [&] {
+    return launch_conv_prep(L, mel, cb.xpad, cb.h1pad, B, C, Tm, P, d, cache_x, cache_h1);
+  }));
   vx_status st;
   // conv1: rows r = b*P + t of xpad; taps read rows r, r+1, r+2 -> h1pad row b*P + 2 + t.
   {
@@ -524,6 +530,10 @@ vx_status run_conv_stem(const Launch& L, const float* mel, const void* w1p, cons
     if (!tmap_bf16_2d(&tmA, cb.h1pad, 2LL * d, int64_t(B) * pairs, 2LL * d, 128)) return VX_ERR_CUDA;
     if ((st = launch_any_gemm(L, "gemm_conv2_gelu", &tmA, w2p, 3 * d, a, EPI_GELU_F32)) != VX_OK) return st;
   }
+  if (cache_x)
+    VX_CUDA(traced(L, "conv_cache_save", 1, [&] {
+      return launch_conv_cache_save(L, cb.xpad, cb.h1pad, cache_x, cache_h1, B, P, C, d);
+    }));
   return VX_OK;
 }
 
@@ -757,6 +767,71 @@ vx_status vx_conv_stem_fwd(const float* mel, const void* w1p, const void* b1, co
   Carve cv{static_cast<uint8_t*>(ws), kStatusBytes};
   const ConvBufs cb = carve_conv(cv, B, n_mels, Tm, d);
   return run_conv_stem(L, mel, w1p, b1, w2p, b2, out, B, n_mels, Tm, d, cb);
+}
+
+size_t vx_conv_stem_step_workspace(int S, int n_mels, int n_new, int d) {
+  return vx_conv_stem_workspace(S, n_mels, n_new, d);
+}
+
+vx_status vx_conv_stem_step(const float* mel_new, const void* w1p, const void* b1, const void* w2p, const void* b2,
+                            void* cache_x, void* cache_h1, float* out, int S, int n_mels, int n_new, int d, void* ws,
+                            size_t ws_bytes, cudaStream_t stream) {
+  vx_status st = check_conv_args(mel_new, w1p, b1, w2p, b2, out, S, n_mels, n_new, d);
+  if (st != VX_OK) return st;
+  VX_CHECK_ARG(cache_x && cache_h1 && aligned16(cache_x) && aligned16(cache_h1),
+               "cache_x / cache_h1 must be non-null and 16-byte aligned");
+  if (n_new % 2 != 0) {
+    set_error("vx_conv_stem_step: n_new=%d must be even (the stride-2 conv keeps its phase across chunks)", n_new);
+    return VX_ERR_UNSUPPORTED;
+  }
+  Launch L;
+  if ((st = make_launch(&L, ws, ws_bytes, vx_conv_stem_step_workspace(S, n_mels, n_new, d), stream)) != VX_OK)
+    return st;
+  Carve cv{static_cast<uint8_t*>(ws), kStatusBytes};
+  const ConvBufs cb = carve_conv(cv, S, n_mels, n_new, d);
+  return run_conv_stem(L, mel_new, w1p, b1, w2p, b2, out, S, n_mels, n_new, d, cb, static_cast<uint16_t*>(cache_x),
+                       static_cast<uint16_t*>(cache_h1));
+}
+
+size_t vx_projector_workspace(int B, int T, int d, int hidden) {
+  if (B <= 0 || T < 4 || d <= 0 || hidden <= 0) return kStatusBytes;
+  const int64_t rows = static_cast<int64_t>(B) * (T / 4);
+  Carve cv{nullptr, kStatusBytes};
+  cv.take(rows * 4 * d * 2);
+  cv.take(rows * hidden * 2);
+  return align_up(cv.off, kAlign);
+}
+
+vx_status vx_projector_fwd(const float* x, const void* w1, const void* w2, float* out, int B, int T, int d, int hidden,
+                           void* ws, size_t ws_bytes, cudaStream_t stream) {
+  VX_CHECK_ARG(B > 0 && T > 0 && d > 0 && hidden > 0, "bad projector shape B=%d T=%d d=%d hidden=%d", B, T, d, hidden);
+  if (d % 16 != 0 || hidden % 128 != 0) {
+    set_error("projector needs d %% 16 == 0 and hidden %% 128 == 0 (got %d, %d)", d, hidden);
+    return VX_ERR_UNSUPPORTED;
+  }
+  const int T4 = T / 4;
+  if (T4 == 0) return VX_OK;   // fewer than 4 frames: no token, nothing is read or written
+  VX_CHECK_ARG(x && w1 && w2 && out, "x / w1 / w2 / out must not be null");
+  VX_CHECK_ARG(aligned16(x) && aligned16(w1) && aligned16(w2) && aligned16(out), "pointers must be 16-byte aligned");
+  Launch L;
+  vx_status st;
+  if ((st = make_launch(&L, ws, ws_bytes, vx_projector_workspace(B, T, d, hidden), stream)) != VX_OK) return st;
+  Carve cv{static_cast<uint8_t*>(ws), kStatusBytes};
+  const int M = B * T4;
+  uint16_t* tok = static_cast<uint16_t*>(cv.take(static_cast<int64_t>(M) * 4 * d * 2));
+  uint16_t* hid = static_cast<uint16_t*>(cv.take(static_cast<int64_t>(M) * hidden * 2));
+  VX_CUDA(traced(L, "frames_to_tokens", 1, [&] { return launch_frames_to_tokens(L, x, tok, B, T, d); }));
+  {
+    GemmArgs a = base_args(L, M, hidden, 4 * d);
+    a.out = hid; a.ld_out = hidden;
+    if ((st = gemm(L, "gemm_proj1_gelu", tok, 4 * d, w1, a, EPI_GELU_BF16)) != VX_OK) return st;
+  }
+  {
+    GemmArgs a = base_args(L, M, hidden, hidden);
+    a.out = out; a.ld_out = hidden;
+    if ((st = gemm(L, "gemm_proj2", hid, hidden, w2, a, EPI_F32)) != VX_OK) return st;
+  }
+  return VX_OK;
 }
 
 size_t vx_encoder_workspace(const vx_layer_cfg* cfg, int B, int n_mels, int Tm) {

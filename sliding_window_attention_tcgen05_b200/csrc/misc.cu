@@ -184,7 +184,7 @@ __global__ void pack_conv_kernel(const uint16_t* __restrict__ w, uint16_t* __res
 // mel [B, C, Tm] fp32 -> xpad [B, P, C] bf16, xpad[b, tp, c] = mel[b, c, tp - 2]
 // for 2 <= tp < Tm + 2, else 0.  32 x 32 tiles through shared memory.
 __global__ void conv_prep_kernel(const float* __restrict__ mel, uint16_t* __restrict__ xpad,
-                                 int C, int Tm, int P) {
+                                 int C, int Tm, int P, const uint16_t* __restrict__ cache_x) {
   pdl_wait();
   pdl_trigger();
   __shared__ float tile[32][33];
@@ -194,6 +194,7 @@ __global__ void conv_prep_kernel(const float* __restrict__ mel, uint16_t* __rest
     const int c = c0 + k, tp = tp0 + tx;
     float v = 0.f;
     if (c < C && tp >= 2 && tp < Tm + 2) v = mel[(static_cast<int64_t>(b) * C + c) * Tm + (tp - 2)];
+    if (c < C && tp < 2 && cache_x) v = bf16_to_f(cache_x[(static_cast<int64_t>(b) * 2 + tp) * C + c]);
     tile[k][tx] = v;
   }
   __syncthreads();
@@ -206,8 +207,10 @@ __global__ void conv_prep_kernel(const float* __restrict__ mel, uint16_t* __rest
   }
 }
 
-// Zeroes rows {0, 1} and [Tm + 2, P) of every clip of h1pad [B, P, d].
-__global__ void conv_pad_zero_kernel(uint16_t* __restrict__ h1pad, int Tm, int P, int d) {
+// Rows {0, 1} of every clip of h1pad [B, P, d]: the two cached conv1 outputs
+// (cache_h1 [B, 2, d]) or zeros; rows [Tm + 2, P): zeros.
+__global__ void conv_pad_zero_kernel(uint16_t* __restrict__ h1pad, int Tm, int P, int d,
+                                     const uint16_t* __restrict__ cache_h1) {
   pdl_wait();
   pdl_trigger();
   const int b = blockIdx.y;
@@ -215,8 +218,46 @@ __global__ void conv_pad_zero_kernel(uint16_t* __restrict__ h1pad, int Tm, int P
   const int row = which < 2 ? which : Tm + which;
   if (row >= P) return;
   uint16_t* r = h1pad + (static_cast<int64_t>(b) * P + row) * d;
+  const uint16_t* src = (which < 2 && cache_h1) ? cache_h1 + (static_cast<int64_t>(b) * 2 + which) * d : nullptr;
   for (int c = threadIdx.x * 8; c < d; c += blockDim.x * 8)
-    *reinterpret_cast<uint4*>(r + c) = make_uint4(0, 0, 0, 0);
+    *reinterpret_cast<uint4*>(r + c) = src ? *reinterpret_cast<const uint4*>(src + c) : make_uint4(0, 0, 0, 0);
+}
+
+// Conv padding cache after a chunk: the last two rows of each clip's xpad
+// [B, P, C] and h1pad [B, P, d] (the chunk's last two mel frames and conv1
+// outputs) into cache_x [B, 2, C] and cache_h1 [B, 2, d].
+__global__ void conv_cache_save_kernel(const uint16_t* __restrict__ xpad, const uint16_t* __restrict__ h1pad,
+                                       uint16_t* __restrict__ cache_x, uint16_t* __restrict__ cache_h1, int P, int C,
+                                       int d) {
+  pdl_wait();
+  pdl_trigger();
+  const int b = blockIdx.y, j = blockIdx.x;   // j: 0, 1 -> xpad rows; 2, 3 -> h1pad rows
+  const bool is_x = j < 2;
+  const int width = is_x ? C : d;
+  const int row = P - 2 + (j & 1);
+  const uint16_t* src = (is_x ? xpad : h1pad) + (static_cast<int64_t>(b) * P + row) * width;
+  uint16_t* dst = (is_x ? cache_x : cache_h1) + (static_cast<int64_t>(b) * 2 + (j & 1)) * width;
+  for (int c = threadIdx.x * 8; c < width; c += blockDim.x * 8)
+    *reinterpret_cast<uint4*>(dst + c) = *reinterpret_cast<const uint4*>(src + c);
+}
+
+// Projector tokens: frames 4j .. 4j+3 of clip b ([B, T, d] fp32) as the bf16
+// row b * T4 + j of tok [B * T4, 4 d]; the last T % 4 frames are not read.
+__global__ void frames_to_tokens_kernel(const float* __restrict__ x, uint16_t* __restrict__ tok, int T, int T4,
+                                        int d, int64_t n8) {
+  pdl_wait();
+  pdl_trigger();
+  const int64_t row_len8 = static_cast<int64_t>(d) / 2;   // 8-element groups per token row (4 d / 8)
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n8;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t row = i / row_len8, e = (i - row * row_len8) * 8;   // element of the token row
+    const int64_t b = row / T4, j = row - b * T4;
+    const float* src = x + (b * T + 4 * j) * d + e;   // 4 consecutive frames are contiguous
+    const float4 lo = *reinterpret_cast<const float4*>(src);
+    const float4 hi = *reinterpret_cast<const float4*>(src + 4);
+    *reinterpret_cast<uint4*>(tok + row * 4 * d + e) =
+        make_uint4(pack_bf16x2(lo.x, lo.y), pack_bf16x2(lo.z, lo.w), pack_bf16x2(hi.x, hi.y), pack_bf16x2(hi.z, hi.w));
+  }
 }
 
 // --------------------------------------------------------------- selftest --
@@ -295,11 +336,27 @@ cudaError_t launch_pack_conv(const Launch& L, const uint16_t* w, uint16_t* wp, i
 }
 
 cudaError_t launch_conv_prep(const Launch& L, const float* mel, uint16_t* xpad, uint16_t* h1pad, int B, int C,
-                             int Tm, int P, int d) {
+                             int Tm, int P, int d, const uint16_t* cache_x, const uint16_t* cache_h1) {
   cudaError_t e = launch_kernel(conv_prep_kernel, dim3((P + 31) / 32, (C + 31) / 32, B), dim3(32, 8), 0, L.stream,
-                                mel, xpad, C, Tm, P);
+                                mel, xpad, C, Tm, P, cache_x);
   if (e != cudaSuccess) return e;
-  return launch_kernel(conv_pad_zero_kernel, dim3(2 + (P - Tm - 2), B), dim3(128), 0, L.stream, h1pad, Tm, P, d);
+  return launch_kernel(conv_pad_zero_kernel, dim3(2 + (P - Tm - 2), B), dim3(128), 0, L.stream, h1pad, Tm, P, d,
+                       cache_h1);
+}
+
+cudaError_t launch_conv_cache_save(const Launch& L, const uint16_t* xpad, const uint16_t* h1pad, uint16_t* cache_x,
+                                   uint16_t* cache_h1, int B, int P, int C, int d) {
+  return launch_kernel(conv_cache_save_kernel, dim3(4, B), dim3(128), 0, L.stream, xpad, h1pad, cache_x, cache_h1, P,
+                       C, d);
+}
+
+cudaError_t launch_frames_to_tokens(const Launch& L, const float* x, uint16_t* tok, int B, int T, int d) {
+  const int T4 = T / 4;
+  const int64_t n8 = static_cast<int64_t>(B) * T4 * d / 2;
+  if (n8 == 0) return cudaSuccess;
+  const int64_t blocks = (n8 + 255) / 256;
+  return launch_kernel(frames_to_tokens_kernel, dim3(static_cast<unsigned>(blocks < 4096 ? blocks : 4096)), dim3(256),
+                       0, L.stream, x, tok, T, T4, d, n8);
 }
 
 cudaError_t launch_selftest_wait(const Launch& L) {

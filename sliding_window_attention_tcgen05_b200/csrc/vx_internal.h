@@ -168,7 +168,14 @@ cudaError_t launch_pack_conv(const Launch& L, const uint16_t* w, uint16_t* wp, i
 // mel [B, C, Tm] fp32 -> xpad [B, P, C] bf16 (rows 0,1 and >= Tm+2 zero); also
 // zeroes rows 0, 1 and Tm+2 .. P-1 of h1pad [B, P, d].
 cudaError_t launch_conv_prep(const Launch& L, const float* mel, uint16_t* xpad, uint16_t* h1pad,
-                             int B, int C, int Tm, int P, int d);
+                             int B, int C, int Tm, int P, int d, const uint16_t* cache_x = nullptr,
+                             const uint16_t* cache_h1 = nullptr);
+// (with cache_x [B, 2, C] / cache_h1 [B, 2, d]: rows 0, 1 come from the caches instead of zeros)
+// Saves the last two rows of each clip of xpad / h1pad into the caches.
+cudaError_t launch_conv_cache_save(const Launch& L, const uint16_t* xpad, const uint16_t* h1pad, uint16_t* cache_x,
+                                   uint16_t* cache_h1, int B, int P, int C, int d);
+// x [B, T, d] fp32 -> tok [B * (T/4), 4 d] bf16 (frames 4j..4j+3 of a clip form token j).
+cudaError_t launch_frames_to_tokens(const Launch& L, const float* x, uint16_t* tok, int B, int T, int d);
 
 cudaError_t launch_selftest_wait(const Launch& L);
 
