@@ -24,7 +24,7 @@ namespace {
 constexpr int kAttnThreads = 384;           // 2 softmax warpgroups; TMA, 2 MMA and 1 idle warp
 constexpr int kNS = 4;                      // K/V pipeline stages
 constexpr int kTile = 128 * 64 * 2;         // one 128 x 64 bf16 tile
-constexpr int kAttnSmem = kTile * (1 + 2 * kNS) + 1024 + 2560;   // + barriers, TMEM slot, merge (m, l)
+constexpr int kAttnSmem = kTile * (2 + 2 * kNS) + 1024 + 4608;   // + barriers, TMEM slot, merge (m, l) x 2
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleSlack = 8.0f;       // O is rescaled only when a row max grows by more than 2^8
 
@@ -47,57 +47,71 @@ __device__ __forceinline__ float tree_max32(const float* v) {
   return t[0];
 }
 
-// One CTA per (128-query tile, head, clip).  The key tiles of 128 that meet
-// the tile's causal window alternate between two softmax warpgroups (tile u
-// -> warpgroup u % 2), each keeping its own running max / sum / output for the
-// same 128 rows; the two are merged at the end.  Per warpgroup X, TMEM holds
-// S_X (128 columns fp32), P_X (64 columns, bf16 pairs) and O_X (64 columns):
-// the softmax threads copy S_X to registers and release it at once, so the
-// next S of the warpgroup is computed while they exponentiate; P goes back to
-// TMEM and is the A operand of O_X += P_X V; O_X is rescaled in place only when
-// a row's max grows by more than kRescaleSlack (the exponents are taken
-// against a stale max otherwise, which cancels in O / l).
+// Persistent: one CTA per SM walks work items (128-query tile, head, clip),
+// item = blockIdx.x + k * gridDim.x, query tiles fastest so that CTAs running
+// at the same time share K/V tiles through L2.  Within an item the key tiles
+// of 128 that meet the tile's causal window alternate between two softmax
+// warpgroups (tile u -> warpgroup u % 2), each keeping its own running max /
+// sum / output for the same 128 rows; the two are merged at the end of the
+// item.  Per warpgroup X, TMEM holds S_X (128 columns fp32), P_X (64 columns,
+// bf16 pairs) and O_X (64 columns): the softmax threads copy S_X to registers
+// and release it at once, so the next S of the warpgroup (possibly of the
+// next item) is computed while they exponentiate or merge; P goes back to TMEM
+// and is the A operand of O_X += P_X V; O_X is rescaled in place only when a
+// row's max grows by more than kRescaleSlack (the exponents are taken against
+// a stale max otherwise, which cancels in O / l).  Q is double-buffered and
+// the K/V ring runs on across items, so the next item's loads and first
+// product overlap the current item's merge.
 // Warps 0-3 / 4-7: softmax warpgroups 0 / 1 (TMEM lane = query row); warp 8:
-// TMA; warps 9 / 10: the tensor-core products of warpgroup 0 / 1 (S(j+1) as
-// soon as S(j) is released, P V(j) when P(j) is ready), so one warpgroup's
-// products never queue behind the other's softmax; warp 11 idles.  The
-// softmax warpgroups take most of the register file (setmaxnreg).
+// TMA; warps 9 / 10: the tensor-core products of warpgroup 0 / 1; warp 11
+// idles.  The softmax warpgroups take most of the register file (setmaxnreg).
 constexpr int kSoftmaxRegs = 224;   // 8 softmax warps x 224 + 4 other warps x 56 = 384 x 168 launched
 constexpr int kOtherRegs = 56;
+
+struct AttnItem {
+  int q0, h, b, kt0, n;   // first query, head, clip, first key tile, key tiles
+};
+__device__ __forceinline__ AttnItem attn_item(const AttnArgs& a, int item) {
+  const int nqt = (a.T + 127) / 128;
+  AttnItem it;
+  const int qt = item % nqt;
+  const int r = item / nqt;
+  it.h = r % a.H;
+  it.b = r / a.H;
+  it.q0 = qt * 128;
+  it.kt0 = max(0, it.q0 - a.window + 1) / 128;
+  it.n = min(a.T - 1, it.q0 + 127) / 128 - it.kt0 + 1;
+  return it;
+}
 
 __global__ void __launch_bounds__(kAttnThreads, 1)
 swa_attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                    const __grid_constant__ CUtensorMap tmV, const __grid_constant__ AttnArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* sQ = smem;
-  uint8_t* sK = sQ + kTile;
+  uint8_t* sQ = smem;                     // two Q buffers
+  uint8_t* sK = sQ + 2 * kTile;
   uint8_t* sV = sK + kNS * kTile;
   uint64_t* bars = reinterpret_cast<uint64_t*>(sV + kNS * kTile);
-  constexpr int QF = 0, KF = 1, VF = KF + kNS, KVE = VF + kNS, SF = KVE + kNS, SE = SF + 2, PF = SE + 2,
-                PE = PF + 2, OD = PE + 2, DR = OD + 2, NBAR = DR + 2;
+  constexpr int QF = 0, QE = 2, KF = 4, VF = KF + kNS, KVE = VF + kNS, SF = KVE + kNS, SE = SF + 2, PF = SE + 2,
+                PE = PF + 2, OD = PE + 2, OFREE = OD + 2, DR = OFREE + 2, NBAR = DR + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + NBAR);
   int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
-  float* xml = reinterpret_cast<float*>(abort_flag + 1);   // [2][128] m, [2][128] l of each warpgroup
+  float* xml = reinterpret_cast<float*>(abort_flag + 3);   // [2 items][2 WG][m 128, l 128]
   auto bar = [&](int i) { return smem_addr(bars + i); };
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int q0 = blockIdx.x * 128;
-  const int h = blockIdx.y;
-  const int b = blockIdx.z;
-  const int W = a.window;
-  const int T = a.T;
-  const int kt0 = max(0, q0 - W + 1) / 128;
-  const int n = min(T - 1, q0 + 127) / 128 - kt0 + 1;   // key tiles of this query tile
+  const int n_items = ((a.T + 127) / 128) * a.H * a.B;
 
   if (threadIdx.x == 0) {
-    mbar_init(bar(QF), 1);
+    for (int i = 0; i < 2; ++i) { mbar_init(bar(QF + i), 1); mbar_init(bar(QE + i), 2); }
     for (int s = 0; s < kNS; ++s) { mbar_init(bar(KF + s), 1); mbar_init(bar(VF + s), 1); mbar_init(bar(KVE + s), 1); }
     for (int X = 0; X < 2; ++X) {
       mbar_init(bar(SF + X), 1); mbar_init(bar(SE + X), 128);
       mbar_init(bar(PF + X), 128); mbar_init(bar(PE + X), 1);
       mbar_init(bar(OD + X), 1);
+      mbar_init(bar(OFREE + X), 8);
       mbar_init(bar(DR + X), 1);
     }
     *abort_flag = 0;
@@ -121,72 +135,97 @@ swa_attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
   if (warp >= 8) {
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kOtherRegs));
     if (warp == 8 && lane == 0) {
-      mbar_arrive_expect_tx(bar(QF), kTile);
-      tma_load_4d(smem_addr(sQ), &tmQ, bar(QF), 0, h, q0, b);
-      uint32_t last_par = 0;
+      uint32_t last_par = 0, q_issued = 0, q_par = 0;
       int filled = 0;
-      for (int u = 0; u < n; ++u) {
-        const int st = u % kNS;
-        const uint32_t ph = (u / kNS) & 1;
-        if (!mbar_wait(bar(KVE + st), ph ^ 1, wc, 11)) break;
-        const int key0 = (kt0 + u) * 128;
-        mbar_arrive_expect_tx(bar(KF + st), kTile);
-        tma_load_4d(smem_addr(sK + st * kTile), &tmK, bar(KF + st), 0, h, key0, b);
-        mbar_arrive_expect_tx(bar(VF + st), kTile);
-        tma_load_4d(smem_addr(sV + st * kTile), &tmV, bar(VF + st), 0, h, key0, b);
-        last_par = (last_par & ~(1u << st)) | (ph << st);
-        filled = u + 1;
+      int U = 0;   // K/V tiles loaded so far (ring position)
+      bool ok = true;
+      for (int item = blockIdx.x, k = 0; ok && item < n_items; item += gridDim.x, ++k) {
+        const AttnItem it = attn_item(a, item);
+        const int qb = k & 1;
+        if (!mbar_wait(bar(QE + qb), ((k >> 1) & 1) ^ 1, wc, 10)) break;   // both issuers are done with it
+        mbar_arrive_expect_tx(bar(QF + qb), kTile);
+        tma_load_4d(smem_addr(sQ + qb * kTile), &tmQ, bar(QF + qb), 0, it.h, it.q0, it.b);
+        q_issued |= 1u << qb;
+        q_par = (q_par & ~(1u << qb)) | (((k >> 1) & 1u) << qb);
+        for (int u = 0; u < it.n; ++u, ++U) {
+          const int st = U % kNS;
+          const uint32_t ph = (U / kNS) & 1;
+          if (!mbar_wait(bar(KVE + st), ph ^ 1, wc, 11)) { ok = false; break; }
+          const int key0 = (it.kt0 + u) * 128;
+          mbar_arrive_expect_tx(bar(KF + st), kTile);
+          tma_load_4d(smem_addr(sK + st * kTile), &tmK, bar(KF + st), 0, it.h, key0, it.b);
+          mbar_arrive_expect_tx(bar(VF + st), kTile);
+          tma_load_4d(smem_addr(sV + st * kTile), &tmV, bar(VF + st), 0, it.h, key0, it.b);
+          last_par = (last_par & ~(1u << st)) | (ph << st);
+          filled = U + 1;
+        }
       }
       // Bounded wait for every copy still in flight (also after an abort).
       int zero = 0;
       WaitCtx dw = wc;
       dw.abort_flag = &zero;
-      mbar_wait(bar(QF), 0, dw, 12);
+      for (int qb = 0; qb < 2; ++qb)
+        if (q_issued & (1u << qb)) mbar_wait(bar(QF + qb), (q_par >> qb) & 1u, dw, 12);
       for (int s = 0; s < kNS && s < filled; ++s) {
         mbar_wait(bar(KF + s), (last_par >> s) & 1u, dw, 12);
         mbar_wait(bar(VF + s), (last_par >> s) & 1u, dw, 12);
       }
     } else if ((warp == 9 || warp == 10) && lane == 0) {
-      // Products of warpgroup X = warp - 9: its tiles u = X, X + 2, ...
+      // Products of warpgroup X = warp - 9: its tiles u = X, X + 2, ... of every item.
       const int X = warp - 9;
       const uint32_t idesc_s = idesc_bf16_f32(128, 128, 0);
       const uint32_t idesc_o = idesc_bf16_f32(128, 64, 1);
-      const int nX = (n + 1 - X) / 2;
-      bool ok = mbar_wait(bar(QF), 0, wc, 13);
-      const uint32_t qa = smem_addr(sQ);
-      auto issue_s = [&](int j) -> bool {   // S(u) into S_X, u = X + 2 j
-        const int u = X + 2 * j, st = u % kNS;
-        if (!mbar_wait(bar(SE + X), (j & 1) ^ 1, wc, 17)) return false;
-        if (!mbar_wait(bar(KF + st), (u / kNS) & 1, wc, 18)) return false;
-        tc_fence_after();
-        const uint32_t ka = smem_addr(sK + st * kTile);
+      int jg = 0;      // this warpgroup's tiles so far (all items)
+      int ubase = 0;   // ring position of the current item's tile 0
+      bool ok = true;
+      for (int item = blockIdx.x, k = 0; ok && item < n_items; item += gridDim.x, ++k) {
+        const AttnItem it = attn_item(a, item);
+        const int nX = (it.n + 1 - X) / 2;
+        const int qb = k & 1;
+        ok = mbar_wait(bar(QF + qb), (k >> 1) & 1, wc, 13);
+        const uint32_t qa = smem_addr(sQ + qb * kTile);
+        auto issue_s = [&](int j) -> bool {   // S(u) into S_X, u = X + 2 j of this item
+          const int U = ubase + X + 2 * j, st = U % kNS, g = jg + j;
+          if (!mbar_wait(bar(SE + X), (g & 1) ^ 1, wc, 17)) return false;
+          if (!mbar_wait(bar(KF + st), (U / kNS) & 1, wc, 18)) return false;
+          tc_fence_after();
+          const uint32_t ka = smem_addr(sK + st * kTile);
 #pragma unroll
-        for (int k = 0; k < 4; ++k)
-          umma_bf16(tmem + X * 256, smem_desc_sw128(qa + 32 * k, 16, 1024), smem_desc_sw128(ka + 32 * k, 16, 1024),
-                    idesc_s, k > 0);
-        umma_commit(bar(SF + X));
-        return true;
-      };
-      auto issue_pv = [&](int j) -> bool {
-        const int u = X + 2 * j, st = u % kNS;
-        if (!mbar_wait(bar(PF + X), j & 1, wc, 14)) return false;
-        if (!mbar_wait(bar(VF + st), (u / kNS) & 1, wc, 15)) return false;
-        tc_fence_after();
-        const uint32_t va = smem_addr(sV + st * kTile);
+          for (int kk = 0; kk < 4; ++kk)
+            umma_bf16(tmem + X * 256, smem_desc_sw128(qa + 32 * kk, 16, 1024), smem_desc_sw128(ka + 32 * kk, 16, 1024),
+                      idesc_s, kk > 0);
+          umma_commit(bar(SF + X));
+          return true;
+        };
+        auto issue_pv = [&](int j) -> bool {
+          const int U = ubase + X + 2 * j, st = U % kNS, g = jg + j;
+          if (!mbar_wait(bar(PF + X), g & 1, wc, 14)) return false;
+          if (!mbar_wait(bar(VF + st), (U / kNS) & 1, wc, 15)) return false;
+          if (j == 0 && !mbar_wait(bar(OFREE + X), (k & 1) ^ 1, wc, 16)) return false;   // previous item merged
+          tc_fence_after();
+          const uint32_t va = smem_addr(sV + st * kTile);
 #pragma unroll
-        for (int k = 0; k < 8; ++k)   // 16 keys per step: 8 TMEM columns of P, 2 K-rows groups of V
-          umma_bf16_ts(tmem + X * 256 + 192, tmem + X * 256 + 128 + 8 * k, smem_desc_sw128(va + k * 2048, kTile, 1024),
-                       idesc_o, (j > 0 || k > 0) ? 1u : 0u);
-        umma_commit(bar(PE + X));
-        umma_commit(bar(KVE + st));   // K/V tile u: S(u) and PV(u) were its last users
-        return true;
-      };
-      if (ok && nX > 0) ok = issue_s(0);
-      for (int j = 0; ok && j < nX; ++j) {
-        if (j + 1 < nX) ok = issue_s(j + 1);
-        if (ok) ok = issue_pv(j);
+          for (int kk = 0; kk < 8; ++kk)   // 16 keys per step: 8 TMEM columns of P, 2 K-rows groups of V
+            umma_bf16_ts(tmem + X * 256 + 192, tmem + X * 256 + 128 + 8 * kk,
+                         smem_desc_sw128(va + kk * 2048, kTile, 1024), idesc_o, (j > 0 || kk > 0) ? 1u : 0u);
+          umma_commit(bar(PE + X));
+          umma_commit(bar(KVE + st));   // K/V tile U: S(U) and PV(U) were its last users
+          return true;
+        };
+        if (ok && nX > 0) ok = issue_s(0);
+        for (int j = 0; ok && j < nX; ++j) {
+          if (j + 1 < nX) ok = issue_s(j + 1);
+          if (ok) ok = issue_pv(j);
+        }
+        // Without a tile in this item, still wait for the previous item's merge
+        // before signalling this one: no per-item barrier may complete twice
+        // before its waiters have seen the first completion (parity waits).
+        if (ok && nX == 0) ok = mbar_wait(bar(OFREE + X), (k & 1) ^ 1, wc, 16);
+        umma_commit(bar(OD + X));   // O_X of this item is final once its products are done
+        umma_commit(bar(QE + qb));  // and so is this issuer's use of the Q buffer
+        jg += nX;
+        ubase += it.n;
       }
-      umma_commit(bar(OD + X));
       umma_commit(bar(DR + X));
       int zero = 0;
       WaitCtx dw = wc;
@@ -198,130 +237,155 @@ swa_attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
     // ------------- softmax: warpgroup X takes key tiles X, X + 2, ...; thread r owns row q0 + r
     const int X = warp >> 2;
     const int r = threadIdx.x & 127;
-    const int i = q0 + r;
     const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const uint32_t tS = tmem + X * 256 + lane_off;
     const uint32_t tP = tS + 128;
     const uint32_t tO = tS + 192;
     const float sl2 = a.scale_log2;
-    float m_used = -INFINITY, l_run = 0.f;
-    bool ok = true;
-    const int nX = (n + 1 - X) / 2;   // tiles u = X, X + 2, ... < n
+    const int W = a.window;
+    int jg = 0;   // this warpgroup's tiles so far (all items)
 
-    for (int j = 0; j < nX; ++j) {
-      const int key0 = (kt0 + X + 2 * j) * 128;
-      bool w = mbar_wait(bar(SF + X), j & 1, wc, 21);
-      if (!__all_sync(0xffffffffu, w)) { ok = false; break; }
-      tc_fence_after();
-      float sv[128];
-      {
-        uint32_t r0[32], r1[32], r2[32], r3[32];
-        tmem_ld32(tS, r0);
-        tmem_ld32(tS + 32, r1);
-        tmem_ld32(tS + 64, r2);
-        tmem_ld32(tS + 96, r3);
-        tmem_ld_wait();
+    for (int item = blockIdx.x, k = 0; item < n_items; item += gridDim.x, ++k) {
+      const AttnItem it = attn_item(a, item);
+      const int q0 = it.q0;
+      const int i = q0 + r;
+      const int nX = (it.n + 1 - X) / 2;   // tiles u = X, X + 2, ... < n
+      float m_used = -INFINITY, l_run = 0.f;
+      bool ok = true;
+
+      for (int j = 0; j < nX; ++j, ++jg) {
+        const int key0 = (it.kt0 + X + 2 * j) * 128;
+        bool w = mbar_wait(bar(SF + X), jg & 1, wc, 21);
+        if (!__all_sync(0xffffffffu, w)) { ok = false; break; }
+        tc_fence_after();
+        float sv[128];
+        {
+          uint32_t r0[32], r1[32], r2[32], r3[32];
+          tmem_ld32(tS, r0);
+          tmem_ld32(tS + 32, r1);
+          tmem_ld32(tS + 64, r2);
+          tmem_ld32(tS + 96, r3);
+          tmem_ld_wait();
 #pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          sv[e] = __uint_as_float(r0[e]);
-          sv[e + 32] = __uint_as_float(r1[e]);
-          sv[e + 64] = __uint_as_float(r2[e]);
-          sv[e + 96] = __uint_as_float(r3[e]);
+          for (int e = 0; e < 32; ++e) {
+            sv[e] = __uint_as_float(r0[e]);
+            sv[e + 32] = __uint_as_float(r1[e]);
+            sv[e + 64] = __uint_as_float(r2[e]);
+            sv[e + 96] = __uint_as_float(r3[e]);
+          }
         }
-      }
-      tc_fence_before();
-      mbar_arrive(bar(SE + X));      // S_X may be overwritten by the next product
-      // Edge tile: keys outside (i - W, i] of this row, i.e. outside columns
-      // [lo, hi] of the tile, are masked.
-      if (key0 + 127 > q0 || key0 <= q0 + 127 - W) {
-        const int lo = i - W + 1 - key0, hi = i - key0;
+        tc_fence_before();
+        mbar_arrive(bar(SE + X));      // S_X may be overwritten by the next product
+        // Edge tile: keys outside (i - W, i] of this row, i.e. outside columns
+        // [lo, hi] of the tile, are masked.
+        if (key0 + 127 > q0 || key0 <= q0 + 127 - W) {
+          const int lo = i - W + 1 - key0, hi = i - key0;
 #pragma unroll
-        for (int e = 0; e < 128; ++e) sv[e] = (e >= lo && e <= hi) ? sv[e] : -INFINITY;
-      }
-      const float m_tile = fmaxf(fmaxf(tree_max32(sv), tree_max32(sv + 32)),
-                                 fmaxf(tree_max32(sv + 64), tree_max32(sv + 96))) * sl2;
-      // Rescale decision (per row): a first finite max just sets m_used (l and O
-      // are still zero); a max more than the slack above m_used rescales.
-      float corr = 1.f;
-      if (m_tile > m_used + kRescaleSlack) {
-        if (m_used != -INFINITY) corr = ex2_approx(m_used - m_tile);
-        m_used = m_tile;
-      }
-      l_run *= corr;
-      const float mu = (m_used == -INFINITY) ? 0.f : m_used;
-
-      // P_X and O_X are free once the previous P V product of this warpgroup is done.
-      w = mbar_wait(bar(PE + X), (j & 1) ^ 1, wc, 22);
-      if (!__all_sync(0xffffffffu, w)) { ok = false; break; }
-      tc_fence_after();
-      if (j > 0 && __any_sync(0xffffffffu, corr != 1.f)) {
-        uint32_t o0[32], o1[32];
-        tmem_ld32(tO, o0);
-        tmem_ld32(tO + 32, o1);
-        tmem_ld_wait();
-#pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          o0[e] = __float_as_uint(__uint_as_float(o0[e]) * corr);
-          o1[e] = __float_as_uint(__uint_as_float(o1[e]) * corr);
+          for (int e = 0; e < 128; ++e) sv[e] = (e >= lo && e <= hi) ? sv[e] : -INFINITY;
         }
-        tmem_st32(tO, o0);
-        tmem_st32(tO + 32, o1);
-      }
-      // p = 2^(s * scale_log2 - mu), row sum, P (bf16 pairs) into TMEM
-      float rs = 0.f;
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        float pv[32];
-#pragma unroll
-        for (int e = 0; e < 32; ++e) pv[e] = ex2_approx(fmaf(sv[c * 32 + e], sl2, -mu));
-        float t[16];
-#pragma unroll
-        for (int e = 0; e < 16; ++e) t[e] = pv[e] + pv[e + 16];
-#pragma unroll
-        for (int wdt = 8; wdt >= 1; wdt >>= 1)
-#pragma unroll
-          for (int e = 0; e < wdt; ++e) t[e] += t[e + wdt];
-        rs += t[0];
-        uint32_t pk[16];
-#pragma unroll
-        for (int e = 0; e < 16; ++e) pk[e] = pack_bf16x2(pv[2 * e], pv[2 * e + 1]);
-        tmem_st16(tP + c * 16, pk);
-      }
-      tmem_st_wait();
-      tc_fence_before();
-      mbar_arrive(bar(PF + X));
-      l_run += rs;
-    }
+        const float m_tile = fmaxf(fmaxf(tree_max32(sv), tree_max32(sv + 32)),
+                                   fmaxf(tree_max32(sv + 64), tree_max32(sv + 96))) * sl2;
+        // Rescale decision (per row): a first finite max just sets m_used (l and O
+        // are still zero); a max more than the slack above m_used rescales.
+        float corr = 1.f;
+        if (m_tile > m_used + kRescaleSlack) {
+          if (m_used != -INFINITY) corr = ex2_approx(m_used - m_tile);
+          m_used = m_tile;
+        }
+        l_run *= corr;
+        const float mu = (m_used == -INFINITY) ? 0.f : m_used;
 
-    // Merge: the warpgroups swap (m, l) through shared memory; then each reads
-    // both O_0 and O_1 from TMEM for its half of the 64 output columns.
-    xml[X * 128 + r] = m_used;
-    xml[256 + X * 128 + r] = ok ? l_run : 0.f;
-    asm volatile("bar.sync 1, 256;" ::: "memory");
-    bool w = mbar_wait(bar(OD + 0), 0, wc, 23) && mbar_wait(bar(OD + 1), 0, wc, 24);
-    if (!__all_sync(0xffffffffu, w)) ok = false;
-    tc_fence_after();
-    const float m0v = xml[r], l0v = xml[256 + r], m1v = xml[128 + r], l1v = xml[384 + r];
-    const float M = fmaxf(m0v, m1v);
-    const float f0 = (m0v == -INFINITY) ? 0.f : ex2_approx(m0v - M);
-    const float f1 = (m1v == -INFINITY) ? 0.f : ex2_approx(m1v - M);
-    const float inv_l = 1.0f / (l0v * f0 + l1v * f1);
-    uint16_t* dst = static_cast<uint16_t*>(a.out) + static_cast<int64_t>(b) * a.o_batch +
-                    static_cast<int64_t>(i) * a.o_row + static_cast<int64_t>(h) * a.o_head + 32 * X;
-    uint32_t x0[32], x1[32];
-    tmem_ld32(tmem + 192 + 32 * X + lane_off, x0);
-    tmem_ld32(tmem + 256 + 192 + 32 * X + lane_off, x1);
-    tmem_ld_wait();
-    if (ok && i < T) {
-      float v[32];
+        // P_X and O_X are free once the previous P V product of this warpgroup is done.
+        w = mbar_wait(bar(PE + X), (jg & 1) ^ 1, wc, 22);
+        if (!__all_sync(0xffffffffu, w)) { ok = false; break; }
+        tc_fence_after();
+        if (j > 0 && __any_sync(0xffffffffu, corr != 1.f)) {
+          uint32_t o0[32], o1[32];
+          tmem_ld32(tO, o0);
+          tmem_ld32(tO + 32, o1);
+          tmem_ld_wait();
 #pragma unroll
-      for (int d = 0; d < 32; ++d) {
-        // a warpgroup without keys for this row contributes nothing (its O may be unset)
-        const float y0 = f0 != 0.f ? __uint_as_float(x0[d]) * f0 : 0.f;
-        const float y1 = f1 != 0.f ? __uint_as_float(x1[d]) * f1 : 0.f;
-        v[d] = (y0 + y1) * inv_l;
+          for (int e = 0; e < 32; ++e) {
+            o0[e] = __float_as_uint(__uint_as_float(o0[e]) * corr);
+            o1[e] = __float_as_uint(__uint_as_float(o1[e]) * corr);
+          }
+          tmem_st32(tO, o0);
+          tmem_st32(tO + 32, o1);
+        }
+        // p = 2^(s * scale_log2 - mu), row sum, P (bf16 pairs) into TMEM
+        float rs = 0.f;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          float pv[32];
+#pragma unroll
+          for (int e = 0; e < 32; ++e) pv[e] = ex2_approx(fmaf(sv[c * 32 + e], sl2, -mu));
+          float t[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) t[e] = pv[e] + pv[e + 16];
+#pragma unroll
+          for (int wdt = 8; wdt >= 1; wdt >>= 1)
+#pragma unroll
+            for (int e = 0; e < wdt; ++e) t[e] += t[e + wdt];
+          rs += t[0];
+          uint32_t pk[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) pk[e] = pack_bf16x2(pv[2 * e], pv[2 * e + 1]);
+          tmem_st16(tP + c * 16, pk);
+        }
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(bar(PF + X));
+        l_run += rs;
       }
-      store_bf16x32(dst, v);
+
+      // Merge: the warpgroups swap (m, l) through shared memory (one buffer per
+      // item parity); then each reads both O_0 and O_1 from TMEM for its half
+      // of the 64 output columns and releases them for the next item.
+      float* xk = xml + (k & 1) * 512;
+      xk[X * 128 + r] = m_used;
+      xk[256 + X * 128 + r] = ok ? l_run : 0.f;
+      asm volatile("bar.sync 1, 256;" ::: "memory");
+      bool w = mbar_wait(bar(OD + 0), k & 1, wc, 23) && mbar_wait(bar(OD + 1), k & 1, wc, 24);
+      if (!__all_sync(0xffffffffu, w)) ok = false;
+      tc_fence_after();
+      const float m0v = xk[r], l0v = xk[256 + r], m1v = xk[128 + r], l1v = xk[384 + r];
+      const float M = fmaxf(m0v, m1v);
+      const float f0 = (m0v == -INFINITY) ? 0.f : ex2_approx(m0v - M);
+      const float f1 = (m1v == -INFINITY) ? 0.f : ex2_approx(m1v - M);
+      const float inv_l = 1.0f / (l0v * f0 + l1v * f1);
+      uint32_t x0[32], x1[32];
+      tmem_ld32(tmem + 192 + 32 * X + lane_off, x0);
+      tmem_ld32(tmem + 256 + 192 + 32 * X + lane_off, x1);
+      tmem_ld_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) { mbar_arrive(bar(OFREE + 0)); mbar_arrive(bar(OFREE + 1)); }
+      if (ok && i < a.T) {
+        uint16_t* dst = static_cast<uint16_t*>(a.out) + static_cast<int64_t>(it.b) * a.o_batch +
+                        static_cast<int64_t>(i) * a.o_row + static_cast<int64_t>(it.h) * a.o_head + 32 * X;
+        float v[32];
+#pragma unroll
+        for (int d = 0; d < 32; ++d) {
+          // a warpgroup without keys for this row contributes nothing (its O may be stale)
+          const float y0 = f0 != 0.f ? __uint_as_float(x0[d]) * f0 : 0.f;
+          const float y1 = f1 != 0.f ? __uint_as_float(x1[d]) * f1 : 0.f;
+          v[d] = (y0 + y1) * inv_l;
+        }
+        store_bf16x32(dst, v);
+      }
+      // Both warpgroups take the same decision on the CTA's abort flag (an OR
+      // over all 256 threads at this barrier), so a timeout ends the item loop
+      // of both and no one is left waiting at the barrier.
+      uint32_t stop;
+      asm volatile(
+          "{\n\t.reg .pred p, q;\n\t"
+          "setp.ne.s32 p, %1, 0;\n\t"
+          "bar.red.or.pred q, 1, 256, p;\n\t"
+          "selp.u32 %0, 1, 0, q;\n\t}"
+          : "=r"(stop)
+          : "r"(*reinterpret_cast<volatile int*>(abort_flag))
+          : "memory");
+      if (stop) break;
     }
   }
 
@@ -478,8 +542,9 @@ cudaError_t launch_attn_bf16(const Launch& L, const CUtensorMap& tmQ, const CUte
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  const dim3 grid((a.T + 127) / 128, a.H, a.B);
-  return launch_kernel(swa_attn_tc_kernel, grid, dim3(kAttnThreads), kAttnSmem, L.stream, tmQ, tmK, tmV, a);
+  const int64_t items = static_cast<int64_t>((a.T + 127) / 128) * a.H * a.B;   // persistent: one CTA per SM
+  const int grid = static_cast<int>(items < L.sm_count ? items : L.sm_count);
+  return launch_kernel(swa_attn_tc_kernel, dim3(grid), dim3(kAttnThreads), kAttnSmem, L.stream, tmQ, tmK, tmV, a);
 }
 
 cudaError_t launch_attn_f32(const Launch& L, const float* q, const float* k, const float* v, float* o,

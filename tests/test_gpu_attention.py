@@ -64,7 +64,10 @@ def test_c2_full_size_sampled_rows(T):
     # Attention-only sweep: B=8, 32 heads, head_dim 64, window 750, RoPE 1e6.
     B, H, W = 8, 32, 750
     q, k, v = synth.attention_qkv(B, T, H, 64, seed=20 + T // 1500, bf16=True)
-    o = _vx().swa_attn_fwd(dev(q, torch.bfloat16), dev(k, torch.bfloat16), dev(v, torch.bfloat16), window=W)
+    vx = _vx()
+    ws = vx.Workspace()
+    o = vx.swa_attn_fwd(dev(q, torch.bfloat16), dev(k, torch.bfloat16), dev(v, torch.bfloat16), window=W, ws=ws)
+    assert vx.status_check(ws) == 0   # no bounded wait ran out
     rng = np.random.default_rng(T)
     rows = sorted(set([0, 1, 127, 128, 749, 750, 751, 1023, T - 129, T - 1] +
                       list(rng.integers(0, T, 6))))
@@ -79,3 +82,18 @@ def test_bf16_deterministic():
     a = _vx().swa_attn_fwd(*args, window=300)
     b = _vx().swa_attn_fwd(*args, window=300)
     assert torch.equal(a, b)
+
+
+def test_bf16_many_items_per_cta_with_single_tile_query_tiles():
+    # More (query tile, head, clip) items than SMs, with many one-key-tile
+    # items (first query tile of each head): every CTA of the persistent kernel
+    # walks several items, including ones where a softmax warpgroup has no tile.
+    B, T, H, W = 4, 256, 48, 100
+    q, k, v = synth.attention_qkv(B, T, H, 64, seed=11, bf16=True)
+    args = [dev(x, torch.bfloat16) for x in (q, k, v)]
+    vx = _vx()
+    ws = vx.Workspace()
+    o = host(vx.swa_attn_fwd(*args, window=W, ws=ws))
+    assert vx.status_check(ws) == 0   # no bounded wait ran out
+    rows = [0, 1, 127, 128, 129, 200, 255]
+    compare_bf16(o[:, rows], _oracle_rows(q, k, v, W, rows), "bf16 many items")
