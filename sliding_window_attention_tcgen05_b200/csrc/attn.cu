@@ -24,7 +24,8 @@ namespace {
 constexpr int kAttnThreads = 384;           // 2 softmax warpgroups; TMA, 2 MMA and 1 idle warp
 constexpr int kNS = 4;                      // K/V pipeline stages
 constexpr int kTile = 128 * 64 * 2;         // one 128 x 64 bf16 tile
-constexpr int kAttnSmem = kTile * (2 + 2 * kNS) + 1024 + 4608;   // + barriers, TMEM slot, merge (m, l) x 2
+constexpr int kAttnSmemPair = kTile * (4 + 2 * kNS) + 1024 + 512;    // + barriers, TMEM slot
+constexpr int kAttnSmemSplit = kTile * (2 + 2 * kNS) + 1024 + 4608;  // + barriers, TMEM slot, merge (m, l) x 2
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleSlack = 8.0f;       // O is rescaled only when a row max grows by more than 2^8
 
@@ -47,21 +48,23 @@ __device__ __forceinline__ float tree_max32(const float* v) {
   return t[0];
 }
 
-// Persistent: one CTA per SM walks work items (128-query tile, head, clip),
-// item = blockIdx.x + k * gridDim.x, query tiles fastest so that CTAs running
-// at the same time share K/V tiles through L2.  Within an item the key tiles
-// of 128 that meet the tile's causal window alternate between two softmax
-// warpgroups (tile u -> warpgroup u % 2), each keeping its own running max /
-// sum / output for the same 128 rows; the two are merged at the end of the
-// item.  Per warpgroup X, TMEM holds S_X (128 columns fp32), P_X (64 columns,
-// bf16 pairs) and O_X (64 columns): the softmax threads copy S_X to registers
-// and release it at once, so the next S of the warpgroup (possibly of the
-// next item) is computed while they exponentiate or merge; P goes back to TMEM
-// and is the A operand of O_X += P_X V; O_X is rescaled in place only when a
-// row's max grows by more than kRescaleSlack (the exponents are taken against
-// a stale max otherwise, which cancels in O / l).  Q is double-buffered and
-// the K/V ring runs on across items, so the next item's loads and first
-// product overlap the current item's merge.
+// swa_attn_pair_kernel (many work items): one CTA per SM walks pairs of work
+// items (128-query tile, head,
+// clip); pair p = blockIdx.x + k * gridDim.x holds items 2p and 2p + 1 (query
+// tiles fastest: usually two neighbouring query tiles of one head, which share
+// most of their key tiles through L2).  Softmax warpgroup X owns item 2p + X
+// entirely: it runs the online softmax over all the key tiles of 128 that meet
+// its tile's causal window and normalises its own output, so there is no
+// merge and the two warpgroups never wait for each other.  Per warpgroup X,
+// TMEM holds S_X (128 columns fp32), P_X (64 columns, bf16 pairs) and O_X (64
+// columns): the softmax threads copy S_X to registers and release it at once,
+// so the next S of the warpgroup (possibly of its next item) is computed while
+// they exponentiate; P goes back to TMEM and is the A operand of
+// O_X += P_X V; O_X is rescaled in place only when a row's max grows by more
+// than kRescaleSlack (the exponents are taken against a stale max otherwise,
+// which cancels in O / l).  Each warpgroup has a double-buffered Q; the K/V
+// ring carries both items' tiles interleaved (A0, B0, A1, B1, ...) and runs on
+// across pairs.
 // Warps 0-3 / 4-7: softmax warpgroups 0 / 1 (TMEM lane = query row); warp 8:
 // TMA; warps 9 / 10: the tensor-core products of warpgroup 0 / 1; warp 11
 // idles.  The softmax warpgroups take most of the register file (setmaxnreg).
@@ -83,9 +86,346 @@ __device__ __forceinline__ AttnItem attn_item(const AttnArgs& a, int item) {
   it.n = min(a.T - 1, it.q0 + 127) / 128 - it.kt0 + 1;
   return it;
 }
+// Ring position of tile t of item X in a pair whose items have nA, nB tiles,
+// loaded interleaved (A0, B0, A1, B1, ...), then the longer item's rest.
+__device__ __forceinline__ int pair_pos(int X, int t, int nA, int nB) {
+  const int m = nA < nB ? nA : nB;
+  return t < m ? 2 * t + X : m + t;
+}
 
 __global__ void __launch_bounds__(kAttnThreads, 1)
-swa_attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+swa_attn_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                   const __grid_constant__ CUtensorMap tmV, const __grid_constant__ AttnArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sQ = smem;                     // Q[X][buffer]: 4 tiles
+  uint8_t* sK = sQ + 4 * kTile;
+  uint8_t* sV = sK + kNS * kTile;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sV + kNS * kTile);
+  // QF/QE: [X * 2 + buffer]
+  constexpr int QF = 0, QE = 4, KF = 8, VF = KF + kNS, KVE = VF + kNS, SF = KVE + kNS, SE = SF + 2, PF = SE + 2,
+                PE = PF + 2, OD = PE + 2, OFREE = OD + 2, DR = OFREE + 2, NBAR = DR + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + NBAR);
+  int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
+  auto bar = [&](int i) { return smem_addr(bars + i); };
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int n_items = ((a.T + 127) / 128) * a.H * a.B;
+  const int n_pairs = (n_items + 1) / 2;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < 4; ++i) { mbar_init(bar(QF + i), 1); mbar_init(bar(QE + i), 1); }
+    for (int s = 0; s < kNS; ++s) { mbar_init(bar(KF + s), 1); mbar_init(bar(VF + s), 1); mbar_init(bar(KVE + s), 1); }
+    for (int X = 0; X < 2; ++X) {
+      mbar_init(bar(SF + X), 1); mbar_init(bar(SE + X), 128);
+      mbar_init(bar(PF + X), 128); mbar_init(bar(PE + X), 1);
+      mbar_init(bar(OD + X), 1);
+      mbar_init(bar(OFREE + X), 4);
+      mbar_init(bar(DR + X), 1);
+    }
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 9) {
+    tmem_alloc(smem_addr(tmem_slot), kTmemCols);
+    tmem_relinquish();
+  }
+  if (warp == 8 && lane == 0) {
+    tma_prefetch_desc(&tmQ); tma_prefetch_desc(&tmK); tma_prefetch_desc(&tmV);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const WaitCtx wc{a.status, abort_flag, a.limit_ns};
+  pdl_wait();
+  pdl_trigger();
+
+  if (warp >= 8) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kOtherRegs));
+    if (warp == 8 && lane == 0) {
+      uint32_t last_par = 0, q_issued = 0, q_par = 0;
+      int filled = 0;
+      int U = 0;   // K/V tiles loaded so far (ring position)
+      bool ok = true;
+      for (int p = blockIdx.x, k = 0; ok && p < n_pairs; p += gridDim.x, ++k) {
+        const int iA = 2 * p;
+        const bool hasB = iA + 1 < n_items;
+        const AttnItem A = attn_item(a, iA);
+        const AttnItem Bi = hasB ? attn_item(a, iA + 1) : A;
+        const int nA = A.n, nB = hasB ? Bi.n : 0;
+        const int qb = k & 1;
+        for (int X = 0; X < (hasB ? 2 : 1); ++X) {
+          const AttnItem& it = X ? Bi : A;
+          const int qi = X * 2 + qb;
+          if (!mbar_wait(bar(QE + qi), ((k >> 1) & 1) ^ 1, wc, 10)) { ok = false; break; }
+          mbar_arrive_expect_tx(bar(QF + qi), kTile);
+          tma_load_4d(smem_addr(sQ + qi * kTile), &tmQ, bar(QF + qi), 0, it.h, it.q0, it.b);
+          q_issued |= 1u << qi;
+          q_par = (q_par & ~(1u << qi)) | (((k >> 1) & 1u) << qi);
+        }
+        const int m = nA < nB ? nA : nB;
+        const int total = nA + nB;
+        for (int pos = 0; ok && pos < total; ++pos, ++U) {
+          // pos -> (item, tile): interleaved while both have tiles, then the longer one
+          int X, t;
+          if (pos < 2 * m) { X = pos & 1; t = pos >> 1; } else { X = nA > nB ? 0 : 1; t = pos - m; }
+          const AttnItem& it = X ? Bi : A;
+          const int st = U % kNS;
+          const uint32_t ph = (U / kNS) & 1;
+          if (!mbar_wait(bar(KVE + st), ph ^ 1, wc, 11)) { ok = false; break; }
+          const int key0 = (it.kt0 + t) * 128;
+          mbar_arrive_expect_tx(bar(KF + st), kTile);
+          tma_load_4d(smem_addr(sK + st * kTile), &tmK, bar(KF + st), 0, it.h, key0, it.b);
+          mbar_arrive_expect_tx(bar(VF + st), kTile);
+          tma_load_4d(smem_addr(sV + st * kTile), &tmV, bar(VF + st), 0, it.h, key0, it.b);
+          last_par = (last_par & ~(1u << st)) | (ph << st);
+          filled = U + 1;
+        }
+      }
+      // Bounded wait for every copy still in flight (also after an abort).
+      int zero = 0;
+      WaitCtx dw = wc;
+      dw.abort_flag = &zero;
+      for (int qi = 0; qi < 4; ++qi)
+        if (q_issued & (1u << qi)) mbar_wait(bar(QF + qi), (q_par >> qi) & 1u, dw, 12);
+      for (int s = 0; s < kNS && s < filled; ++s) {
+        mbar_wait(bar(KF + s), (last_par >> s) & 1u, dw, 12);
+        mbar_wait(bar(VF + s), (last_par >> s) & 1u, dw, 12);
+      }
+    } else if ((warp == 9 || warp == 10) && lane == 0) {
+      // Products of warpgroup X = warp - 9: every key tile of its item of each pair.
+      const int X = warp - 9;
+      const uint32_t idesc_s = idesc_bf16_f32(128, 128, 0);
+      const uint32_t idesc_o = idesc_bf16_f32(128, 64, 1);
+      int jg = 0;      // this warpgroup's tiles so far (all items)
+      int ubase = 0;   // ring position of the current pair's first tile
+      int kc = 0;      // this warpgroup's items so far
+      bool ok = true;
+      for (int p = blockIdx.x, k = 0; ok && p < n_pairs; p += gridDim.x, ++k) {
+        const int iA = 2 * p;
+        const bool hasB = iA + 1 < n_items;
+        const int nA = attn_item(a, iA).n, nB = hasB ? attn_item(a, iA + 1).n : 0;
+        const int nX = X ? nB : nA;
+        if (nX > 0) {
+          const int qi = X * 2 + (k & 1);
+          ok = mbar_wait(bar(QF + qi), (k >> 1) & 1, wc, 13);
+          const uint32_t qa = smem_addr(sQ + qi * kTile);
+          auto issue_s = [&](int j) -> bool {   // S(j) into S_X
+            const int U = ubase + pair_pos(X, j, nA, nB), st = U % kNS, g = jg + j;
+            if (!mbar_wait(bar(SE + X), (g & 1) ^ 1, wc, 17)) return false;
+            if (!mbar_wait(bar(KF + st), (U / kNS) & 1, wc, 18)) return false;
+            tc_fence_after();
+            const uint32_t ka = smem_addr(sK + st * kTile);
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+              umma_bf16(tmem + X * 256, smem_desc_sw128(qa + 32 * kk, 16, 1024),
+                        smem_desc_sw128(ka + 32 * kk, 16, 1024), idesc_s, kk > 0);
+            umma_commit(bar(SF + X));
+            return true;
+          };
+          auto issue_pv = [&](int j) -> bool {
+            const int U = ubase + pair_pos(X, j, nA, nB), st = U % kNS, g = jg + j;
+            if (!mbar_wait(bar(PF + X), g & 1, wc, 14)) return false;
+            if (!mbar_wait(bar(VF + st), (U / kNS) & 1, wc, 15)) return false;
+            // O_X is overwritten by the item's first product: the warpgroup's
+            // previous item must have been read out.
+            if (j == 0 && !mbar_wait(bar(OFREE + X), (kc & 1) ^ 1, wc, 16)) return false;
+            tc_fence_after();
+            const uint32_t va = smem_addr(sV + st * kTile);
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk)   // 16 keys per step: 8 TMEM columns of P, 2 K-rows groups of V
+              umma_bf16_ts(tmem + X * 256 + 192, tmem + X * 256 + 128 + 8 * kk,
+                           smem_desc_sw128(va + kk * 2048, kTile, 1024), idesc_o, (j > 0 || kk > 0) ? 1u : 0u);
+            umma_commit(bar(PE + X));
+            umma_commit(bar(KVE + st));   // K/V tile U: S(U) and PV(U) were its last users
+            return true;
+          };
+          if (ok) ok = issue_s(0);
+          for (int j = 0; ok && j < nX; ++j) {
+            if (j + 1 < nX) ok = issue_s(j + 1);
+            if (ok) ok = issue_pv(j);
+          }
+          umma_commit(bar(OD + X));    // O_X of this item is final once its products are done
+          umma_commit(bar(QE + qi));   // and so is the use of its Q buffer
+          jg += nX;
+          ++kc;
+        }
+        ubase += nA + nB;
+      }
+      umma_commit(bar(DR + X));
+      int zero = 0;
+      WaitCtx dw = wc;
+      dw.abort_flag = &zero;
+      mbar_wait(bar(DR + X), 0, dw, 19);
+    }
+  } else {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kSoftmaxRegs));
+    // ------------- softmax: warpgroup X owns item 2p + X; thread r owns row q0 + r
+    const int X = warp >> 2;
+    const int r = threadIdx.x & 127;
+    const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const uint32_t tS = tmem + X * 256 + lane_off;
+    const uint32_t tP = tS + 128;
+    const uint32_t tO = tS + 192;
+    const float sl2 = a.scale_log2;
+    const int W = a.window;
+    int jg = 0;   // this warpgroup's tiles so far (all items)
+    int kc = 0;   // this warpgroup's items so far
+    bool ok = true;
+
+    for (int p = blockIdx.x; ok && p < n_pairs; p += gridDim.x) {
+      const int item = 2 * p + X;
+      if (item >= n_items) continue;
+      const AttnItem it = attn_item(a, item);
+      const int q0 = it.q0;
+      const int i = q0 + r;
+      float m_used = -INFINITY, l_run = 0.f;
+
+      for (int j = 0; j < it.n; ++j, ++jg) {
+        const int key0 = (it.kt0 + j) * 128;
+        bool w = mbar_wait(bar(SF + X), jg & 1, wc, 21);
+        if (!__all_sync(0xffffffffu, w)) { ok = false; break; }
+        tc_fence_after();
+        float sv[128];
+        {
+          uint32_t r0[32], r1[32], r2[32], r3[32];
+          tmem_ld32(tS, r0);
+          tmem_ld32(tS + 32, r1);
+          tmem_ld32(tS + 64, r2);
+          tmem_ld32(tS + 96, r3);
+          tmem_ld_wait();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            sv[e] = __uint_as_float(r0[e]);
+            sv[e + 32] = __uint_as_float(r1[e]);
+            sv[e + 64] = __uint_as_float(r2[e]);
+            sv[e + 96] = __uint_as_float(r3[e]);
+          }
+        }
+        tc_fence_before();
+        mbar_arrive(bar(SE + X));      // S_X may be overwritten by the next product
+        // Edge tile: keys outside (i - W, i] of this row, i.e. outside columns
+        // [lo, hi] of the tile, are masked.
+        if (key0 + 127 > q0 || key0 <= q0 + 127 - W) {
+          const int lo = i - W + 1 - key0, hi = i - key0;
+#pragma unroll
+          for (int e = 0; e < 128; ++e) sv[e] = (e >= lo && e <= hi) ? sv[e] : -INFINITY;
+        }
+        const float m_tile = fmaxf(fmaxf(tree_max32(sv), tree_max32(sv + 32)),
+                                   fmaxf(tree_max32(sv + 64), tree_max32(sv + 96))) * sl2;
+        // Rescale decision (per row): a first finite max just sets m_used (l and O
+        // are still zero); a max more than the slack above m_used rescales.
+        float corr = 1.f;
+        if (m_tile > m_used + kRescaleSlack) {
+          if (m_used != -INFINITY) corr = ex2_approx(m_used - m_tile);
+          m_used = m_tile;
+        }
+        l_run *= corr;
+        const float mu = (m_used == -INFINITY) ? 0.f : m_used;
+
+        // P_X and O_X are free once the previous P V product of this warpgroup is done.
+        w = mbar_wait(bar(PE + X), (jg & 1) ^ 1, wc, 22);
+        if (!__all_sync(0xffffffffu, w)) { ok = false; break; }
+        tc_fence_after();
+        if (j > 0 && __any_sync(0xffffffffu, corr != 1.f)) {
+          uint32_t o0[32], o1[32];
+          tmem_ld32(tO, o0);
+          tmem_ld32(tO + 32, o1);
+          tmem_ld_wait();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            o0[e] = __float_as_uint(__uint_as_float(o0[e]) * corr);
+            o1[e] = __float_as_uint(__uint_as_float(o1[e]) * corr);
+          }
+          tmem_st32(tO, o0);
+          tmem_st32(tO + 32, o1);
+        }
+        // p = 2^(s * scale_log2 - mu), row sum, P (bf16 pairs) into TMEM
+        float rs = 0.f;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          float pv[32];
+#pragma unroll
+          for (int e = 0; e < 32; ++e) pv[e] = ex2_approx(fmaf(sv[c * 32 + e], sl2, -mu));
+          float t[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) t[e] = pv[e] + pv[e + 16];
+#pragma unroll
+          for (int wdt = 8; wdt >= 1; wdt >>= 1)
+#pragma unroll
+            for (int e = 0; e < wdt; ++e) t[e] += t[e + wdt];
+          rs += t[0];
+          uint32_t pk[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) pk[e] = pack_bf16x2(pv[2 * e], pv[2 * e + 1]);
+          tmem_st16(tP + c * 16, pk);
+        }
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(bar(PF + X));
+        l_run += rs;
+      }
+      if (!ok) break;
+
+      // Output: O_X / l once the item's last product is done; O_X is then
+      // released for the warpgroup's next item.
+      bool w = mbar_wait(bar(OD + X), kc & 1, wc, 23);
+      if (!__all_sync(0xffffffffu, w)) { ok = false; break; }
+      tc_fence_after();
+      uint32_t x0[32], x1[32];
+      tmem_ld32(tO, x0);
+      tmem_ld32(tO + 32, x1);
+      tmem_ld_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(OFREE + X));
+      ++kc;
+      if (i < a.T) {
+        const float inv_l = 1.0f / l_run;
+        uint16_t* dst = static_cast<uint16_t*>(a.out) + static_cast<int64_t>(it.b) * a.o_batch +
+                        static_cast<int64_t>(i) * a.o_row + static_cast<int64_t>(it.h) * a.o_head;
+        float v0[32], v1[32];
+#pragma unroll
+        for (int d = 0; d < 32; ++d) {
+          v0[d] = __uint_as_float(x0[d]) * inv_l;
+          v1[d] = __uint_as_float(x1[d]) * inv_l;
+        }
+        store_bf16x32(dst, v0);
+        store_bf16x32(dst + 32, v1);
+      }
+    }
+  }
+
+  __syncthreads();
+  if (warp == 9) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+// swa_attn_split_kernel (few work items): one CTA per SM walks work items
+// (128-query tile, head, clip),
+// item = blockIdx.x + k * gridDim.x, query tiles fastest so that CTAs running
+// at the same time share K/V tiles through L2.  Within an item the key tiles
+// of 128 that meet the tile's causal window alternate between two softmax
+// warpgroups (tile u -> warpgroup u % 2), each keeping its own running max /
+// sum / output for the same 128 rows; the two are merged at the end of the
+// item.  Per warpgroup X, TMEM holds S_X (128 columns fp32), P_X (64 columns,
+// bf16 pairs) and O_X (64 columns): the softmax threads copy S_X to registers
+// and release it at once, so the next S of the warpgroup (possibly of the
+// next item) is computed while they exponentiate or merge; P goes back to TMEM
+// and is the A operand of O_X += P_X V; O_X is rescaled in place only when a
+// row's max grows by more than kRescaleSlack (the exponents are taken against
+// a stale max otherwise, which cancels in O / l).  Q is double-buffered and
+// the K/V ring runs on across items, so the next item's loads and first
+// product overlap the current item's merge.
+// Warps 0-3 / 4-7: softmax warpgroups 0 / 1 (TMEM lane = query row); warp 8:
+// TMA; warps 9 / 10: the tensor-core products of warpgroup 0 / 1; warp 11
+// idles.  The softmax warpgroups take most of the register file (setmaxnreg).
+__global__ void __launch_bounds__(kAttnThreads, 1)
+swa_attn_split_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                    const __grid_constant__ CUtensorMap tmV, const __grid_constant__ AttnArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -538,13 +878,30 @@ cudaError_t launch_attn_bf16(const Launch& L, const CUtensorMap& tmQ, const CUte
                              const CUtensorMap& tmV, const AttnArgs& a) {
   static bool attr_set = false;
   if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(swa_attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kAttnSmem);
+    cudaError_t e = cudaFuncSetAttribute(swa_attn_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         kAttnSmemPair);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(swa_attn_split_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kAttnSmemSplit);
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  const int64_t items = static_cast<int64_t>((a.T + 127) / 128) * a.H * a.B;   // persistent: one CTA per SM
-  const int grid = static_cast<int>(items < L.sm_count ? items : L.sm_count);
-  return launch_kernel(swa_attn_tc_kernel, dim3(grid), dim3(kAttnThreads), kAttnSmem, L.stream, tmQ, tmK, tmV, a);
+  // Persistent grids of one CTA per SM.  Measured per key tile of an item:
+  // ~1.6 us per round of items when the two warpgroups split an item's tiles
+  // (a merge per item), ~2.6 us per round of item pairs when each warpgroup
+  // owns an item; the rounds count decides which is shorter.
+  const int64_t items = static_cast<int64_t>((a.T + 127) / 128) * a.H * a.B;
+  const int64_t pairs = (items + 1) / 2;
+  const int64_t sm = L.sm_count > 0 ? L.sm_count : 1;
+  const double t_split = 1.6 * static_cast<double>((items + sm - 1) / sm);
+  const double t_pair = 2.6 * static_cast<double>((pairs + sm - 1) / sm);
+  if (t_pair < t_split) {
+    const int grid = static_cast<int>(pairs < sm ? pairs : sm);
+    return launch_kernel(swa_attn_pair_kernel, dim3(grid), dim3(kAttnThreads), kAttnSmemPair, L.stream, tmQ, tmK,
+                         tmV, a);
+  }
+  const int grid = static_cast<int>(items < sm ? items : sm);
+  return launch_kernel(swa_attn_split_kernel, dim3(grid), dim3(kAttnThreads), kAttnSmemSplit, L.stream, tmQ, tmK,
+                       tmV, a);
 }
 
 cudaError_t launch_attn_f32(const Launch& L, const float* q, const float* k, const float* v, float* o,

@@ -97,3 +97,18 @@ def test_bf16_many_items_per_cta_with_single_tile_query_tiles():
     assert vx.status_check(ws) == 0   # no bounded wait ran out
     rows = [0, 1, 127, 128, 129, 200, 255]
     compare_bf16(o[:, rows], _oracle_rows(q, k, v, W, rows), "bf16 many items")
+
+
+def test_bf16_item_pairs_with_odd_item_count():
+    # 5 query tiles x 255 heads = 1275 items: the many-items kernel (two items
+    # per CTA at a time) with pairs that straddle heads and a last pair that
+    # has a single item.
+    B, T, H, W = 1, 640, 255, 300
+    q, k, v = synth.attention_qkv(B, T, H, 64, seed=12, bf16=True)
+    args = [dev(x, torch.bfloat16) for x in (q, k, v)]
+    vx = _vx()
+    ws = vx.Workspace()
+    o = host(vx.swa_attn_fwd(*args, window=W, ws=ws))
+    assert vx.status_check(ws) == 0
+    rows = [0, 127, 128, 383, 384, 639]
+    compare_bf16(o[:, rows], _oracle_rows(q, k, v, W, rows), "bf16 odd item pairs")
