@@ -532,24 +532,53 @@ def main(argv=None):
     frames_all = reduce_sum(B * T, device)
     value = frames_all / (ms / 1e3)
 
-    # end to end: pinned host input -> device -> layer -> host, per step
+    # End to end through the public call from pinned host buffers: every step
+    # copies its input in (H2D), runs the layer and reads its output back (D2H).
+    # Like a server fed a stream of clips, the copies of neighbouring steps run
+    # on their own streams (two device buffers each way), overlapping the
+    # layer; the L2 flush before each step's layer is inside the timed region.
     xh = torch.empty(B, T, d, dtype=torch.float32, pin_memory=True)
     xh.copy_(x.cpu())
     yh = torch.empty_like(xh, pin_memory=True)
+    xs = [x, torch.empty_like(x)]
+    ys = [y, torch.empty_like(y)]
+    s_in, s_out = torch.cuda.Stream(device=device), torch.cuda.Stream(device=device)
 
-    def e2e_step():
-        x.copy_(xh, non_blocking=True)
-        step()
-        yh.copy_(y, non_blocking=True)
+    def e2e_run(K):
+        ev_in = [torch.cuda.Event() for _ in range(K)]
+        ev_comp = [torch.cuda.Event() for _ in range(K)]
+        ev_out = [torch.cuda.Event() for _ in range(K)]
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        s_in.wait_stream(stream)
+        s_out.wait_stream(stream)
+        for i in range(K):
+            bb = i % 2
+            with torch.cuda.stream(s_in):
+                if i >= 2:
+                    s_in.wait_event(ev_comp[i - 2])      # the layer of step i-2 has read xs[bb]
+                xs[bb].copy_(xh, non_blocking=True)
+                ev_in[i].record(s_in)
+            stream.wait_event(ev_in[i])
+            if i >= 2:
+                stream.wait_event(ev_out[i - 2])         # ys[bb] of step i-2 is on the host
+            flush()
+            vx.encoder_layer_fwd(cfg, L, xs[bb], out=ys[bb], ws=ws)
+            ev_comp[i].record(stream)
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(ev_comp[i])
+                yh.copy_(ys[bb], non_blocking=True)
+                ev_out[i].record(s_out)
+        stream.wait_stream(s_out)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / K
 
     ms_e2e = float("nan")
     if not args.no_e2e:
-        for _ in range(3):
-            e2e_step()
-        torch.cuda.synchronize()
+        e2e_run(3)
         barrier(device)
-        ms_e2e_local, _, _ = timed_steps(torch, e2e_step, max(20, min(args.steps, 200)), flush, stream)
-        ms_e2e = reduce_max(ms_e2e_local, device)
+        ms_e2e = reduce_max(e2e_run(max(20, min(args.steps, 200))), device)
     sampler.stop()
     clocks = sampler.summary(t0, t1)
 
@@ -603,7 +632,9 @@ def main(argv=None):
             "layer_tflops": layer_flops(B, T) / (ms / 1e3) / 1e12,
             "layer_frac_of_measured_peak": layer_flops(B, T) / (ms / 1e3) / 1e12 / tf_burst,
             "e2e": {"value": frames_all / (ms_e2e / 1e3), "unit": UNIT,
-                    "h2d_bytes_per_step": B * T * d * 4, "d2h_bytes_per_step": B * T * d * 4},
+                    "h2d_bytes_per_step": B * T * d * 4, "d2h_bytes_per_step": B * T * d * 4,
+                    "method": "pinned host buffers; H2D, layer (after a 256 MiB L2 flush) and D2H of consecutive "
+                              "steps on three streams with two device buffers each way; timed over the whole run"},
             "gpu_launches": int(launches),
             "roofline": roof,
             "kernels": per_kernel,

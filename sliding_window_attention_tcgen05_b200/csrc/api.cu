@@ -52,6 +52,14 @@ bool pair_gemm_disabled() {
   return off;
 }
 
+bool ring_tma_disabled() {
+  static const bool off = [] {
+    const char* e = std::getenv("VX_RING_TMA");
+    return e && e[0] == '0';
+  }();
+  return off;
+}
+
 bool tma_store_disabled() {
   static const bool off = [] {
     const char* e = std::getenv("VX_TMA_STORE");

@@ -29,6 +29,7 @@ uint64_t wait_limit_ns();
 bool pdl_enabled();   // programmatic dependent launch (default on; VX_PDL=0 disables)
 bool pair_gemm_disabled();   // two-CTA GEMM tiles (default on; VX_PAIR_GEMM=0 disables)
 bool tma_store_disabled();   // TMA stores of GEMM outputs (default on; VX_TMA_STORE=0 disables)
+bool ring_tma_disabled();    // TMA-fed ring attention (default on; VX_RING_TMA=0 uses cp.async)
 
 // Launches `k` on `stream`, with programmatic dependent launch when enabled.
 template <class... KArgs, class... Args>
