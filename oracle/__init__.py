@@ -31,7 +31,15 @@ Readings where the page is silent (each pinned by a test in tests/):
     the previous chunk: the last 2 mel frames (conv1 taps) and the last 2
     conv1 outputs (conv2 taps) are carried; the first chunk starts from zeros;
   * projector: frames 4j .. 4j+3 are concatenated in time order into token j
-    (frame-major reshape of [B, T, d] to [B, T/4, 4d]), exact (erf) GELU.
+    (frame-major reshape of [B, T, d] to [B, T/4, 4d]), exact (erf) GELU;
+  * log-mel frontend (section "Frontend"): power spectrum |STFT|^2 of
+    400-sample frames (periodic Hann, hop 160, n_fft 400) at 16 kHz, a slaney
+    filterbank of 128 bands over 0-8000 Hz (slaney mel scale, area
+    normalisation), log10 of max(mel, 1e-10), the fixed global maximum of the
+    Realtime model: max(log, 1.5 - 8), then (x + 4) / 4; with centring
+    (the first chunk / a whole clip) the signal is reflect-padded by 200
+    samples on both sides and the last STFT frame is dropped; without it the
+    frames are those lying wholly inside the given samples.
 
 Parity against the real checkpoint is unpinned: the pages print no
 activations and no trained weights are available.
@@ -47,7 +55,7 @@ __all__ = [
     "rms_norm", "rope_inv_freq", "rope", "swa_attention", "swa_attention_rows",
     "silu", "gelu", "encoder_layer", "ring_from_sequence", "stream_step_layer",
     "stream_step", "conv_stem", "conv_out_len", "encoder", "as64", "conv_stem_step",
-    "projector",
+    "projector", "slaney_mel_filterbank", "log_mel", "log_mel_frames",
 ]
 
 
@@ -331,3 +339,68 @@ def projector(x, w1, w2, factor=4):
     T4 = T // factor
     tok = x[:, :T4 * factor, :].reshape(B, T4, factor * d)
     return gelu(tok @ as64(w1).T) @ as64(w2).T
+
+
+# ------------------------------------------------------------------ frontend
+
+SAMPLE_RATE, N_FFT, HOP, N_MELS, F_MAX, LOG_MEL_MAX = 16000, 400, 160, 128, 8000.0, 1.5
+
+
+def _hz_to_mel(f):
+    """Slaney mel scale: linear (3 f / 200) below 1000 Hz, logarithmic above
+    (27 mels per factor 6.4 in frequency), 15 mels at 1000 Hz."""
+    f = np.asarray(f, dtype=np.float64)
+    lin = f / (200.0 / 3.0)
+    log = 15.0 + np.log(np.maximum(f, 1e-300) / 1000.0) / (math.log(6.4) / 27.0)
+    return np.where(f >= 1000.0, log, lin)
+
+
+def _mel_to_hz(m):
+    m = np.asarray(m, dtype=np.float64)
+    lin = m * (200.0 / 3.0)
+    log = 1000.0 * np.exp((m - 15.0) * (math.log(6.4) / 27.0))
+    return np.where(m >= 15.0, log, lin)
+
+
+def slaney_mel_filterbank(n_mels=N_MELS, n_fft=N_FFT, sr=SAMPLE_RATE, f_min=0.0, f_max=F_MAX):
+    """[n_mels, n_fft // 2 + 1] triangles between n_mels + 2 points evenly spaced
+    on the slaney mel scale from f_min to f_max, each scaled by 2 / (its width
+    in Hz) (area normalisation)."""
+    hz = _mel_to_hz(np.linspace(_hz_to_mel(f_min), _hz_to_mel(f_max), n_mels + 2))
+    freqs = np.arange(n_fft // 2 + 1) * (sr / n_fft)
+    fb = np.zeros((n_mels, freqs.size))
+    for m in range(n_mels):
+        lo, mid, hi = hz[m], hz[m + 1], hz[m + 2]
+        up = (freqs - lo) / (mid - lo)
+        down = (hi - freqs) / (hi - mid)
+        fb[m] = np.maximum(0.0, np.minimum(up, down)) * (2.0 / (hi - lo))
+    return fb
+
+
+def _hann_periodic(n=N_FFT):
+    return 0.5 - 0.5 * np.cos(2.0 * math.pi * np.arange(n) / n)
+
+
+def log_mel_frames(frames):
+    """Normalised log-mel of already cut frames [..., 400] (float64)."""
+    spec = np.abs(np.fft.rfft(as64(frames) * _hann_periodic(), n=N_FFT, axis=-1)) ** 2    # [..., 201]
+    mel = spec @ slaney_mel_filterbank().T                                               # [..., 128]
+    log = np.log10(np.maximum(mel, 1e-10))
+    log = np.maximum(log, LOG_MEL_MAX - 8.0)
+    return (log + 4.0) / 4.0
+
+
+def log_mel(audio, center=True):
+    """Streaming log-mel frontend of the Realtime model: audio [B, N] at 16 kHz
+    -> [B, 128, F].  center: reflect-pad 200 samples on both sides, frames at
+    hop 160, last frame dropped (F = N // 160); else frames wholly inside the
+    samples (F = 1 + (N - 400) // 160 for N >= 400)."""
+    x = as64(audio)
+    if center:
+        x = np.pad(x, ((0, 0), (N_FFT // 2, N_FFT // 2)), mode="reflect")
+    n_frames = 1 + (x.shape[1] - N_FFT) // HOP if x.shape[1] >= N_FFT else 0
+    if center:
+        n_frames -= 1
+    idx = np.arange(n_frames)[:, None] * HOP + np.arange(N_FFT)[None, :]
+    return np.transpose(log_mel_frames(x[:, idx]), (0, 2, 1))
+
