@@ -379,8 +379,9 @@ def component_c4(vx, torch, flush, hbm, tf):
 
 def component_next(vx, torch, flush, hbm, tf):
     """The widened rows: the streaming conv-stem step (64 streams x 8 mel frames
-    -> 4 frames, warm padding cache) and the audio projector on the encoder
-    output of the 4 x 6000-mel workload ([4, 3000, 1280] -> [4, 750, 3072])."""
+    -> 4 frames, warm padding cache), the audio projector on the encoder
+    output of the 4 x 6000-mel workload ([4, 3000, 1280] -> [4, 750, 3072])
+    and the log-mel frontend producing that workload's input (4 x 60 s)."""
     g = torch.Generator(device="cuda").manual_seed(501)
 
     def nrm(shape, std):
@@ -410,8 +411,17 @@ def component_next(vx, torch, flush, hbm, tf):
         proj()
     ms_p, _, _ = timed_steps(torch, proj, 20, flush, torch.cuda.current_stream())
     proj_flop = 2 * 3000 * 5120 * 3072 + 2 * 3000 * 3072 * 3072
+    audio = torch.randn(4, 960000, generator=g, device="cuda") * 0.1
+    melo = torch.empty(4, 128, 6000, device="cuda")
+    wsm = vx.Workspace(vx.lib.vx_log_mel_workspace(4, 960000))
+    lm = lambda: vx.log_mel_fwd(audio, True, out=melo, ws=wsm)
+    for _ in range(3):
+        lm()
+    ms_m, _, _ = timed_steps(torch, lm, 20, flush, torch.cuda.current_stream())
     return {"conv_step_64x8": {"ms_per_step": ms_c, "frames_per_s": S * 4 / ms_c * 1e3,
                                "gbs": conv_bytes / ms_c / 1e6, "tflops": conv_flop / ms_c / 1e9},
+            "log_mel_4x60s": {"ms_per_call": ms_m, "mel_frames_per_s": 24000 / ms_m * 1e3,
+                              "gbs": (4 * 960000 * 4 + 4 * 128 * 6000 * 4) / ms_m / 1e6},
             "projector_4x3000": {"ms_per_call": ms_p, "tokens_per_s": 3000 / ms_p * 1e3,
                                  "tflops": proj_flop / ms_p / 1e9, "frac_of_measured_peak": proj_flop / ms_p / 1e9 / tf}}
 

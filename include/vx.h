@@ -245,6 +245,26 @@ VX_API vx_status vx_conv_stem_step(const float *mel_new, const void *w1p, const 
                             void *ws, size_t ws_bytes, cudaStream_t stream);
 VX_API size_t vx_conv_stem_step_workspace(int S, int n_mels, int n_new, int d);
 
+/* Streaming log-mel frontend of the Realtime model (transcribe.cpp notes
+ * "Voxtral", section "Frontend"): 16 kHz audio, 400-sample frames with a
+ * periodic Hann window at hop 160 (n_fft 400), power spectrum, slaney mel
+ * filterbank of 128 bands over 0-8000 Hz (area normalised), log10 of
+ * max(mel, 1e-10), the fixed global maximum of the Realtime model
+ * (max(log, 1.5 - 8)), then (x + 4) / 4.  Every frame depends on its own 400
+ * samples only, so a stream is processed chunk by chunk.
+ *   audio: [B, N] fp32;  mel: [B, 128, F] fp32 (the layout vx_conv_stem_fwd reads)
+ *   center = 1 (a whole clip, or a stream's first chunk): reflect-padded by 200
+ *     samples on both sides, the last frame dropped: F = N / 160 (N > 200, else
+ *     VX_ERR_UNSUPPORTED);
+ *   center = 0 (later chunks): the frames lying wholly inside the samples,
+ *     F = 1 + (N - 400) / 160 (0 when N < 400); pass the samples from
+ *     160 t0 - 200 on to continue the centred frame grid at frame t0.
+ * With F = 0 nothing is read or written.  Arithmetic in fp32.  Workspace:
+ * vx_log_mel_workspace(). */
+VX_API vx_status vx_log_mel_fwd(const float *audio, float *mel, int B, int N, int center,
+                         void *ws, size_t ws_bytes, cudaStream_t stream);
+VX_API size_t vx_log_mel_workspace(int B, int N);
+
 /* Audio projector (transcribe.cpp notes "Voxtral", section "Architecture ->
  * Voxtral Realtime 2602", Projector): the encoder output x [B, T, d] fp32 is
  * reshaped to [B, T/4, 4d] (frames 4j .. 4j+3 concatenated in time order, the

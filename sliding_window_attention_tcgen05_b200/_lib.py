@@ -64,6 +64,8 @@ SIGNATURES = {
     "vx_conv_stem_step_workspace": (_S, [_I, _I, _I, _I]),
     "vx_projector_fwd": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _P, _S, _P]),
     "vx_projector_workspace": (_S, [_I, _I, _I, _I]),
+    "vx_log_mel_fwd": (_I, [_P, _P, _I, _I, _I, _P, _S, _P]),
+    "vx_log_mel_workspace": (_S, [_I, _I]),
     "vx_encoder_fwd": (_I, [_CFG, _P, _I, _I, _I, _P, _P, _P, _P, _W, _I, _P, _P, _P, _S, _P]),
     "vx_encoder_workspace": (_S, [_CFG, _I, _I, _I]),
     "vx_stream_prefill": (_I, [_CFG, _W, _R, _P, _P, _I, _P, _P, _S, _P]),

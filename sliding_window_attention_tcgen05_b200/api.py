@@ -235,6 +235,19 @@ def conv_stem_step(mel_new, w1p, b1, w2p, b2, cache: ConvCache, out=None, ws: Wo
     return out
 
 
+def log_mel_fwd(audio, center: bool = True, out=None, ws: Workspace | None = None):
+    """Streaming log-mel frontend: audio [B, N] fp32 at 16 kHz -> [B, 128, F] fp32."""
+    B, N = audio.shape
+    F = N // 160 if center else (1 + (N - 400) // 160 if N >= 400 else 0)
+    if out is None:
+        out = torch.empty(B, 128, F, dtype=torch.float32, device=audio.device)
+    need = lib.vx_log_mel_workspace(B, N)
+    ws = _ws(ws, need, audio.device)
+    p, n = ws.get(need)
+    check(lib.vx_log_mel_fwd(_p(audio), _p(out), B, N, int(center), p, n, _stream()), "vx_log_mel_fwd")
+    return out
+
+
 def projector_fwd(x, w1, w2, out=None, ws: Workspace | None = None):
     """Audio projector: x [B, T, d] fp32 -> [B, T // 4, hidden] fp32 (w1 [hidden, 4d], w2 [hidden, hidden] bf16)."""
     B, T, d = x.shape

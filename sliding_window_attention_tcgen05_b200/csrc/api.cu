@@ -842,6 +842,30 @@ vx_status vx_projector_fwd(const float* x, const void* w1, const void* w2, float
   return VX_OK;
 }
 
+size_t vx_log_mel_workspace(int B, int N) {
+  (void)B;
+  (void)N;
+  return align_up(kStatusBytes + align_up(log_mel_table_bytes(), kAlign), kAlign);
+}
+
+vx_status vx_log_mel_fwd(const float* audio, float* mel, int B, int N, int center, void* ws, size_t ws_bytes,
+                         cudaStream_t stream) {
+  VX_CHECK_ARG(B > 0 && N > 0, "bad log-mel shape B=%d N=%d", B, N);
+  if (center && N <= 200) {
+    set_error("vx_log_mel_fwd: centred frames need more than 200 samples (got %d) for the reflect padding", N);
+    return VX_ERR_UNSUPPORTED;
+  }
+  if (log_mel_frames(N, center) == 0) return VX_OK;   // no whole frame: nothing is read or written
+  VX_CHECK_ARG(audio && mel, "audio / mel must not be null");
+  Launch L;
+  vx_status st;
+  if ((st = make_launch(&L, ws, ws_bytes, vx_log_mel_workspace(B, N), stream)) != VX_OK) return st;
+  Carve cv{static_cast<uint8_t*>(ws), kStatusBytes};
+  void* tables = cv.take(log_mel_table_bytes());
+  VX_CUDA(traced(L, "log_mel", 2, [&] { return launch_log_mel(L, audio, mel, B, N, center, tables); }));
+  return VX_OK;
+}
+
 size_t vx_encoder_workspace(const vx_layer_cfg* cfg, int B, int n_mels, int Tm) {
   if (!cfg || B <= 0 || Tm <= 0) return kStatusBytes;
   const int To = (Tm - 1) / 2 + 1;

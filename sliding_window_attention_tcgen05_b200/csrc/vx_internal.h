@@ -178,6 +178,13 @@ cudaError_t launch_conv_cache_save(const Launch& L, const uint16_t* xpad, const 
 // x [B, T, d] fp32 -> tok [B * (T/4), 4 d] bf16 (frames 4j..4j+3 of a clip form token j).
 cudaError_t launch_frames_to_tokens(const Launch& L, const float* x, uint16_t* tok, int B, int T, int d);
 
+// Log-mel frontend (16 kHz, n_fft 400, hop 160, 128 slaney bands, fixed max 1.5):
+// audio [B, N] fp32 -> mel [B, 128, log_mel_frames(N, center)] fp32; tables:
+// log_mel_table_bytes() of scratch (filterbank, window, twiddles).
+int log_mel_frames(int N, int center);
+size_t log_mel_table_bytes();
+cudaError_t launch_log_mel(const Launch& L, const float* audio, float* mel, int B, int N, int center, void* tables);
+
 cudaError_t launch_selftest_wait(const Launch& L);
 
 }  // namespace vx
