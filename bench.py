@@ -377,6 +377,14 @@ def component_c4(vx, torch, flush, hbm, tf):
             "kernel_ms_per_forward": {k: v["ms_per_step"] for k, v in tr.items()}}
 
 
+# Log-mel frontend arithmetic per 10 ms frame: window (400 mul), the 201-bin
+# DFT as 2 x 400 FMAs per bin, power (3 flop per bin) and the dense
+# 128 x 201 filterbank product; its bound is the fp32 CUDA-core rate:
+# 148 SMs x 128 fp32 lanes x 2 flop x 1.965 GHz.
+LOG_MEL_FLOP_PER_FRAME = 400 + 201 * 400 * 4 + 201 * 3 + 128 * 201 * 2
+FP32_ALU_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
+
+
 def component_next(vx, torch, flush, hbm, tf):
     """The widened rows: the streaming conv-stem step (64 streams x 8 mel frames
     -> 4 frames, warm padding cache), the audio projector on the encoder
@@ -421,7 +429,9 @@ def component_next(vx, torch, flush, hbm, tf):
     return {"conv_step_64x8": {"ms_per_step": ms_c, "frames_per_s": S * 4 / ms_c * 1e3,
                                "gbs": conv_bytes / ms_c / 1e6, "tflops": conv_flop / ms_c / 1e9},
             "log_mel_4x60s": {"ms_per_call": ms_m, "mel_frames_per_s": 24000 / ms_m * 1e3,
-                              "gbs": (4 * 960000 * 4 + 4 * 128 * 6000 * 4) / ms_m / 1e6},
+                              "gbs": (4 * 960000 * 4 + 4 * 128 * 6000 * 4) / ms_m / 1e6,
+                              "tflops_fp32": 24000 * LOG_MEL_FLOP_PER_FRAME / ms_m / 1e9,
+                              "frac_of_fp32_alu_peak": 24000 * LOG_MEL_FLOP_PER_FRAME / ms_m / 1e9 / FP32_ALU_TFLOPS},
             "projector_4x3000": {"ms_per_call": ms_p, "tokens_per_s": 3000 / ms_p * 1e3,
                                  "tflops": proj_flop / ms_p / 1e9, "frac_of_measured_peak": proj_flop / ms_p / 1e9 / tf}}
 
