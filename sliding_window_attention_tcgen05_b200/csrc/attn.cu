@@ -36,6 +36,29 @@ __device__ __forceinline__ void store_bf16x32(uint16_t* dst, const float (&v)[32
                  pack_bf16x2(v[8 * j + 4], v[8 * j + 5]), pack_bf16x2(v[8 * j + 6], v[8 * j + 7]));
 }
 
+// The softmax of a 128-key tile is bound by the softmax warps' instruction
+// issue, so the exponent arguments and the row sums use sm_100's packed
+// fp32x2 FMA / add (each lane of a packed op rounds like the scalar op, so
+// the results are those of the scalar code).
+__device__ __forceinline__ uint64_t f2_pack(float a, float b) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+  return r;
+}
+__device__ __forceinline__ void f2_unpack(uint64_t r, float& a, float& b) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(r));
+}
+__device__ __forceinline__ uint64_t ffma2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t fadd2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+
 // Max of 32 values as a balanced tree (short dependency chains).
 __device__ __forceinline__ float tree_max32(const float* v) {
   float t[16];
@@ -46,6 +69,33 @@ __device__ __forceinline__ float tree_max32(const float* v) {
 #pragma unroll
     for (int i = 0; i < w; ++i) t[i] = fmaxf(t[i], t[i + w]);
   return t[0];
+}
+
+// pv[e] = 2^(s[e] * sl2 - mu) for 32 scores, the argument two at a time.
+__device__ __forceinline__ void exp2_scaled32(const float* s, float sl2, float mu, float (&pv)[32]) {
+  const uint64_t sc = f2_pack(sl2, sl2), nm = f2_pack(-mu, -mu);
+#pragma unroll
+  for (int e = 0; e < 32; e += 2) {
+    float x0, x1;
+    f2_unpack(ffma2(f2_pack(s[e], s[e + 1]), sc, nm), x0, x1);
+    pv[e] = ex2_approx(x0);
+    pv[e + 1] = ex2_approx(x1);
+  }
+}
+
+// Sum of 32 values as the tree t[e] = v[e] + v[e + 16], then halving; two
+// neighbouring nodes of a level per packed add.
+__device__ __forceinline__ float sum32_tree(const float (&v)[32]) {
+  uint64_t t[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) t[i] = fadd2(f2_pack(v[2 * i], v[2 * i + 1]), f2_pack(v[2 * i + 16], v[2 * i + 17]));
+#pragma unroll
+  for (int w = 4; w >= 1; w >>= 1)
+#pragma unroll
+    for (int i = 0; i < w; ++i) t[i] = fadd2(t[i], t[i + w]);
+  float a, b;
+  f2_unpack(t[0], a, b);
+  return a + b;
 }
 
 // swa_attn_pair_kernel (many work items): one CTA per SM walks pairs of work
@@ -347,16 +397,8 @@ swa_attn_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
           float pv[32];
-#pragma unroll
-          for (int e = 0; e < 32; ++e) pv[e] = ex2_approx(fmaf(sv[c * 32 + e], sl2, -mu));
-          float t[16];
-#pragma unroll
-          for (int e = 0; e < 16; ++e) t[e] = pv[e] + pv[e + 16];
-#pragma unroll
-          for (int wdt = 8; wdt >= 1; wdt >>= 1)
-#pragma unroll
-            for (int e = 0; e < wdt; ++e) t[e] += t[e + wdt];
-          rs += t[0];
+          exp2_scaled32(sv + c * 32, sl2, mu, pv);
+          rs += sum32_tree(pv);
           uint32_t pk[16];
 #pragma unroll
           for (int e = 0; e < 16; ++e) pk[e] = pack_bf16x2(pv[2 * e], pv[2 * e + 1]);
@@ -657,16 +699,8 @@ swa_attn_split_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_cons
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
           float pv[32];
-#pragma unroll
-          for (int e = 0; e < 32; ++e) pv[e] = ex2_approx(fmaf(sv[c * 32 + e], sl2, -mu));
-          float t[16];
-#pragma unroll
-          for (int e = 0; e < 16; ++e) t[e] = pv[e] + pv[e + 16];
-#pragma unroll
-          for (int wdt = 8; wdt >= 1; wdt >>= 1)
-#pragma unroll
-            for (int e = 0; e < wdt; ++e) t[e] += t[e + wdt];
-          rs += t[0];
+          exp2_scaled32(sv + c * 32, sl2, mu, pv);
+          rs += sum32_tree(pv);
           uint32_t pk[16];
 #pragma unroll
           for (int e = 0; e < 16; ++e) pk[e] = pack_bf16x2(pv[2 * e], pv[2 * e + 1]);
