@@ -59,7 +59,7 @@ def parse_args(argv=None):
     ap.add_argument("--impl", choices=("vx", "reference"), default="vx")
     ap.add_argument("--no-components", action="store_true", help="skip the C2/C3/C4 component timings")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--components-only", default="", help="comma list of c2,c3,c4,next (profiling runs)")
+    ap.add_argument("--components-only", default="", help="comma list of c0,c2,c3,c4,next (profiling runs)")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-copy end-to-end pass (profiling runs)")
     ap.add_argument("--no-trace", action="store_true", help="skip the traced per-kernel pass (profiling runs)")
     ap.add_argument("--c3-layers", type=int, default=32, help="layers of the streaming-step component (profiling runs)")
@@ -288,6 +288,26 @@ def traced_kernels(vx, torch, step, K, flush):
 
 
 # ------------------------------------------------------------- components
+
+def component_c0(vx, torch, flush, hbm, tf):
+    """The tiny fp32 case: q, k, v [1, 64, 2, 64] (seed 0, drawn in that order),
+    window 16, RoPE theta 1e6 at pos0 0, through the public fp32 attention call
+    (RoPE kernel + CUDA-core attention kernel); latency per call, L2 flushed
+    between calls outside the events."""
+    import synth
+    q, k, v = (torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32)).cuda()
+               for a in synth.attention_qkv(1, 64, 2, 64, seed=0))
+    o = torch.empty_like(q)
+    ws = vx.Workspace(vx.lib.vx_swa_attn_workspace(0, 1, 64, 2, 64, 1))
+    step = lambda: vx.swa_attn_fwd(q, k, v, 16, apply_rope=True, rope_theta=1e6, pos0=0, out=o, ws=ws)
+    for _ in range(5):
+        step()
+    ms, _, _ = timed_steps(torch, step, 200, flush, torch.cuda.current_stream())
+    tr = traced_kernels(vx, torch, step, 20, flush)
+    fl = attn_flops(1, 64, 2, 64, 16)
+    return {"us_per_call": ms * 1e3, "kernels_us": {k2: v2["ms_per_launch"] * 1e3 for k2, v2 in tr.items()},
+            "mflop": fl / 1e6, "note": "launch-latency bound: 0.46 MFLOP"}
+
 
 def component_c2(vx, torch, flush, hbm, tf):
     out = {}
@@ -520,8 +540,8 @@ def main(argv=None):
             if c == "c3":
                 out[c] = component_c3(vx, torch, flush, hbm, tf_burst, L=args.c3_layers)
             else:
-                out[c] = {"c2": component_c2, "c4": component_c4, "next": component_next}[c](vx, torch, flush, hbm,
-                                                                                              tf_burst)
+                out[c] = {"c0": component_c0, "c2": component_c2, "c4": component_c4,
+                          "next": component_next}[c](vx, torch, flush, hbm, tf_burst)
         if rank == 0:
             print(json.dumps({"components": out}), flush=True)
         return 0
@@ -630,8 +650,8 @@ def main(argv=None):
     comps = None
     if world == 1 and not args.no_components:
         comps = {}
-        for name, fn in (("swa_c2", component_c2), ("stream_step_c3", component_c3), ("encoder_c4", component_c4),
-                         ("next_rows", component_next)):
+        for name, fn in (("swa_c0", component_c0), ("swa_c2", component_c2), ("stream_step_c3", component_c3),
+                         ("encoder_c4", component_c4), ("next_rows", component_next)):
             try:
                 comps[name] = fn(vx, torch, flush, hbm, tf_burst)
             except Exception as e:   # report, never hide

@@ -69,7 +69,7 @@ __global__ void mel_tables_kernel(float* __restrict__ fb, float* __restrict__ wi
   }
 }
 
-__global__ void __launch_bounds__(kMelThreads)
+__global__ void __launch_bounds__(kMelThreads, 3)   // 3 CTAs (24 warps) per SM
 log_mel_kernel(const float* __restrict__ audio, float* __restrict__ mel, const float* __restrict__ fbt,
                const float* __restrict__ win, const float2* __restrict__ tw, int N, int F, int center) {
   extern __shared__ __align__(16) float smem_f[];
