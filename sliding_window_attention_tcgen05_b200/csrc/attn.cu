@@ -124,17 +124,34 @@ constexpr int kOtherRegs = 56;
 struct AttnItem {
   int q0, h, b, kt0, n;   // first query, head, clip, first key tile, key tiles
 };
-__device__ __forceinline__ AttnItem attn_item(const AttnArgs& a, int item) {
-  const int nqt = (a.T + 127) / 128;
+__device__ __forceinline__ AttnItem item_at(const AttnArgs& a, int qt, int h, int b) {
   AttnItem it;
-  const int qt = item % nqt;
-  const int r = item / nqt;
-  it.h = r % a.H;
-  it.b = r / a.H;
+  it.h = h;
+  it.b = b;
   it.q0 = qt * 128;
   it.kt0 = max(0, it.q0 - a.window + 1) / 128;
   it.n = min(a.T - 1, it.q0 + 127) / 128 - it.kt0 + 1;
   return it;
+}
+// Item `item` in query-tile-fastest order.
+__device__ __forceinline__ AttnItem attn_item(const AttnArgs& a, int item) {
+  const int nqt = (a.T + 127) / 128;
+  const int r = item / nqt;
+  return item_at(a, item % nqt, r % a.H, r / a.H);
+}
+// Round r of this CTA in the split kernel's order: items sorted heaviest first
+// (query tiles in descending order; a tile's key-tile count never decreases
+// with its index), dealt to the CTAs round by round in alternating
+// directions, which evens out the CTAs' total key tiles.  False past this
+// CTA's last item (only the last round can be partial).
+__device__ __forceinline__ bool split_item(const AttnArgs& a, int n_items, int r, AttnItem& it) {
+  const int G = gridDim.x, x = blockIdx.x;
+  const int pos = r * G + ((r & 1) ? G - 1 - x : x);
+  if (pos >= n_items) return false;
+  const int hb = a.H * a.B;
+  const int rest = pos % hb;
+  it = item_at(a, (a.T + 127) / 128 - 1 - pos / hb, rest % a.H, rest / a.H);
+  return true;
 }
 // Ring position of tile t of item X in a pair whose items have nA, nB tiles,
 // loaded interleaved (A0, B0, A1, B1, ...), then the longer item's rest.
@@ -448,9 +465,8 @@ swa_attn_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
 }
 
 // swa_attn_split_kernel (few work items): one CTA per SM walks work items
-// (128-query tile, head, clip),
-// item = blockIdx.x + k * gridDim.x, query tiles fastest so that CTAs running
-// at the same time share K/V tiles through L2.  Within an item the key tiles
+// (128-query tile, head, clip) in the order of split_item (heaviest first,
+// alternating directions; with few items, all K/V tiles stay in L2).  Within an item the key tiles
 // of 128 that meet the tile's causal window alternate between two softmax
 // warpgroups (tile u -> warpgroup u % 2), each keeping its own running max /
 // sum / output for the same 128 rows; the two are merged at the end of the
@@ -521,8 +537,8 @@ swa_attn_split_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_cons
       int filled = 0;
       int U = 0;   // K/V tiles loaded so far (ring position)
       bool ok = true;
-      for (int item = blockIdx.x, k = 0; ok && item < n_items; item += gridDim.x, ++k) {
-        const AttnItem it = attn_item(a, item);
+      AttnItem it;
+      for (int k = 0; ok && split_item(a, n_items, k, it); ++k) {
         const int qb = k & 1;
         if (!mbar_wait(bar(QE + qb), ((k >> 1) & 1) ^ 1, wc, 10)) break;   // both issuers are done with it
         mbar_arrive_expect_tx(bar(QF + qb), kTile);
@@ -560,8 +576,8 @@ swa_attn_split_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_cons
       int jg = 0;      // this warpgroup's tiles so far (all items)
       int ubase = 0;   // ring position of the current item's tile 0
       bool ok = true;
-      for (int item = blockIdx.x, k = 0; ok && item < n_items; item += gridDim.x, ++k) {
-        const AttnItem it = attn_item(a, item);
+      AttnItem it;
+      for (int k = 0; ok && split_item(a, n_items, k, it); ++k) {
         const int nX = (it.n + 1 - X) / 2;
         const int qb = k & 1;
         ok = mbar_wait(bar(QF + qb), (k >> 1) & 1, wc, 13);
@@ -627,8 +643,8 @@ swa_attn_split_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_cons
     const int W = a.window;
     int jg = 0;   // this warpgroup's tiles so far (all items)
 
-    for (int item = blockIdx.x, k = 0; item < n_items; item += gridDim.x, ++k) {
-      const AttnItem it = attn_item(a, item);
+    AttnItem it;
+    for (int k = 0; split_item(a, n_items, k, it); ++k) {
       const int q0 = it.q0;
       const int i = q0 + r;
       const int nX = (it.n + 1 - X) / 2;   // tiles u = X, X + 2, ... < n
