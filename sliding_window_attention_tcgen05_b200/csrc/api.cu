@@ -19,8 +19,10 @@
 #include <cstring>
 #include <cmath>
 #include <atomic>
+#include <map>
 #include <mutex>
 #include <string>
+#include <utility>
 #include <vector>
 
 #include <cudaTypedefs.h>
@@ -58,6 +60,19 @@ bool ring_tma_disabled() {
     return e && e[0] == '0';
   }();
   return off;
+}
+
+cudaError_t ensure_dynamic_smem(const void* kernel, size_t smem) {
+  int dev = 0;
+  if (cudaError_t e = cudaGetDevice(&dev)) return e;
+  static std::mutex mu;
+  static std::map<std::pair<const void*, int>, size_t> done;   // (kernel, device) -> bytes set
+  std::lock_guard<std::mutex> lock(mu);
+  auto it = done.find({kernel, dev});
+  if (it != done.end() && it->second >= smem) return cudaSuccess;
+  cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  if (e == cudaSuccess) done[{kernel, dev}] = smem;
+  return e;
 }
 
 bool tma_store_disabled() {

@@ -31,10 +31,18 @@ bool pair_gemm_disabled();   // two-CTA GEMM tiles (default on; VX_PAIR_GEMM=0 d
 bool tma_store_disabled();   // TMA stores of GEMM outputs (default on; VX_TMA_STORE=0 disables)
 bool ring_tma_disabled();    // TMA-fed ring attention (default on; VX_RING_TMA=0 uses cp.async)
 
+// A kernel launched with more than 48 KB of dynamic shared memory needs
+// cudaFuncAttributeMaxDynamicSharedMemorySize on every device that runs it:
+// sets it once per (kernel, current device).  Thread-safe.
+cudaError_t ensure_dynamic_smem(const void* kernel, size_t smem);
+
 // Launches `k` on `stream`, with programmatic dependent launch when enabled.
 template <class... KArgs, class... Args>
 cudaError_t launch_kernel(void (*k)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
                           Args&&... args) {
+  if (smem > 48 * 1024) {
+    if (cudaError_t e = ensure_dynamic_smem(reinterpret_cast<const void*>(k), smem)) return e;
+  }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
   cfg.blockDim = block;
