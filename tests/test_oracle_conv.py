@@ -45,16 +45,36 @@ def test_conv_stem_is_causal():
     assert np.max(np.abs(oracle.conv_stem(m3, **w)[:, t] - base[:, t])) > 1e-4
 
 
-def test_encoder_composes_stem_layers_and_final_norm():
+def _zero_branch_layers(dims, n, seed):
+    """Layers whose O and down projections are zero: each layer then adds
+    exactly bo + bd to the residual stream (attention and MLP branches vanish)."""
+    layers = []
+    for l in range(n):
+        p = synth.layer_params(dims, seed=synth.layer_seed(seed, l))
+        p["wo"] = np.zeros_like(p["wo"])
+        p["wd"] = np.zeros_like(p["wd"])
+        layers.append(p)
+    return layers
+
+
+def test_encoder_is_stem_then_each_layer_once_then_final_norm():
+    # With zero-branch layers the encoder is, in closed form,
+    #   RMSNorm(stem(mel) + sum_l (bo_l + bd_l); g),
+    # the stem taken from torch's conv1d on the left-padded input.  A dropped,
+    # repeated or reordered-with-the-norm layer changes the bias sum or the
+    # normalisation, so it fails here.
     dims = synth.LayerDims(d_model=12, n_heads=2, head_dim=6, ffn_hidden=20, window=3)
     conv = _small_conv(5)
-    layers = [synth.layer_params(dims, seed=synth.layer_seed(6, l)) for l in range(2)]
+    layers = _zero_branch_layers(dims, 3, 6)
     g = synth.final_norm_gain(12, seed=7)
-    mel = synth.mel(1, 8, 14, seed=8)
+    mel = synth.mel(1, 8, 14, seed=8).astype(np.float64)
     out = oracle.encoder(mel, conv, layers, g, dims)
-    x = oracle.conv_stem(mel, **conv)
-    for p in layers:
-        x = oracle.encoder_layer(x, p, dims)
-    # final RMSNorm with gain g: out / g has RMS sqrt(ms / (ms + eps)) per frame
-    ms = np.mean(x * x, -1)
-    np.testing.assert_allclose(np.sqrt(np.mean((out / g) ** 2, -1)), np.sqrt(ms / (ms + dims.eps)), rtol=1e-12)
+    t = {k: torch.from_numpy(v.astype(np.float64)) for k, v in conv.items()}
+    h = F.gelu(F.conv1d(F.pad(torch.from_numpy(mel), (2, 0)), t["w1"], t["b1"]), approximate="none")
+    h = F.gelu(F.conv1d(F.pad(h, (2, 0)), t["w2"], t["b2"], stride=2), approximate="none")
+    x = h.permute(0, 2, 1).numpy() + sum(p["bo"].astype(np.float64) + p["bd"].astype(np.float64) for p in layers)
+    # out / g is x scaled per frame by 1 / sqrt(mean(x^2) + eps)
+    scale = 1.0 / np.sqrt(np.mean(x * x, axis=-1, keepdims=True) + dims.eps)
+    np.testing.assert_allclose(out / g.astype(np.float64), x * scale, rtol=1e-12, atol=1e-12)
+    # and with one layer fewer the result differs
+    assert np.max(np.abs(oracle.encoder(mel, conv, layers[:2], g, dims) - out)) > 1e-3

@@ -166,3 +166,28 @@ def test_query_bias_enters_scores():
     a = oracle.encoder_layer(x, p, SMALL)
     p2 = dict(p, bq=p["bq"] * 0)
     assert np.max(np.abs(oracle.encoder_layer(x, p2, SMALL) - a)) > 1e-5
+
+
+def test_stream_step_final_norm_closed_form():
+    # With zero-branch layers a streaming step through L layers adds
+    # sum_l (bo_l + bd_l) to the new frames (the ring only feeds the vanished
+    # attention branch); final_g then applies the encoder's final RMSNorm:
+    #   out = (x + sum b) / sqrt(mean((x + sum b)^2) + eps) * g.
+    dims = SMALL
+    layers = []
+    for l in range(3):
+        p = _params(seed=synth.layer_seed(12, l))
+        p["wo"] = np.zeros_like(p["wo"])
+        p["wd"] = np.zeros_like(p["wd"])
+        layers.append(p)
+    S, n, P = 2, 4, 7
+    x = synth.frames(S, n, dims.d_model, seed=13).astype(np.float64)
+    rings = [synth.ring_kv(S, dims.n_heads, dims.window, dims.head_dim, seed=14 + l) for l in range(3)]
+    g = synth.final_norm_gain(dims.d_model, seed=15).astype(np.float64)
+    raw, _, pos = oracle.stream_step(x, layers, dims, rings, np.full(S, P))
+    out, _, _ = oracle.stream_step(x, layers, dims, rings, np.full(S, P), final_g=g)
+    h = x + sum(p["bo"].astype(np.float64) + p["bd"].astype(np.float64) for p in layers)
+    np.testing.assert_allclose(raw, h, rtol=1e-13, atol=1e-13)
+    want = h / np.sqrt(np.mean(h * h, axis=-1, keepdims=True) + dims.eps) * g
+    np.testing.assert_allclose(out, want, rtol=1e-12, atol=1e-12)
+    assert np.all(pos == P + n)

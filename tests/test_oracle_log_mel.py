@@ -86,3 +86,42 @@ def test_streaming_continuation_equals_whole_clip_interior():
     n = cont.shape[2]
     np.testing.assert_allclose(cont[:, :, :min(n, whole.shape[2] - t0 - 2)],
                                whole[:, :, t0:t0 + min(n, whole.shape[2] - t0 - 2)], rtol=0, atol=1e-12)
+
+
+def _torchaudio_fb():
+    """The slaney filterbank as torchaudio builds it (float32), [128, 201] float64."""
+    return TAF.melscale_fbanks(201, 0.0, 8000.0, 128, 16000, norm="slaney", mel_scale="slaney").double().numpy().T
+
+
+@pytest.mark.parametrize("A", [1.0, 0.03, 1e-3])
+def test_impulse_at_frame_centre_band_values_closed_form(A):
+    # An impulse of amplitude A at sample 160 t sits at the centre of centred
+    # frame t, where the periodic Hann window is exactly 1, so that frame's
+    # power spectrum is A^2 at every bin and band m holds A^2 * sum_k fb[m, k].
+    # The normalisation then fixes every value: log10, the fixed floor
+    # 1.5 - 8 = -6.5, and (x + 4) / 4.  A = 1e-3 puts every band below the
+    # floor, A = 0.03 and 1.0 none (a natural log or a missing clamp fails).
+    x = np.zeros((1, 3200))
+    x[0, 160 * 5] = A
+    got = oracle.log_mel(x)[0, :, 5]
+    mel = A * A * _torchaudio_fb().sum(axis=1)
+    want = (np.maximum(np.log10(mel), -6.5) + 4.0) / 4.0
+    np.testing.assert_allclose(got, want, rtol=0, atol=2e-6)
+
+
+def test_bin_centred_tone_band_values_closed_form():
+    # A 1000 Hz cosine of amplitude A is 25 whole periods of a 400-sample
+    # frame.  With the periodic Hann window its DFT has |X[25]| = 100 A and
+    # |X[24]| = |X[26]| = 50 A and nothing else, whatever the phase; so band m
+    # of every interior frame is A^2 (2500 fb[m,24] + 1e4 fb[m,25] + 2500
+    # fb[m,26]), and bands without those bins sit at the -6.5 floor.
+    A = 0.25
+    n = np.arange(16000)
+    x = (A * np.cos(2 * math.pi * 1000.0 * n / 16000.0 + 0.7))[None, :]
+    out = oracle.log_mel(x)[0]
+    fb = _torchaudio_fb()
+    mel = A * A * (2500.0 * fb[:, 24] + 1e4 * fb[:, 25] + 2500.0 * fb[:, 26])
+    want = (np.maximum(np.log10(np.maximum(mel, 1e-30)), -6.5) + 4.0) / 4.0
+    assert np.sum(want > -0.625) >= 2 and np.sum(want == -0.625) >= 100
+    for t in (3, 50, 97):
+        np.testing.assert_allclose(out[:, t], want, rtol=0, atol=2e-6)

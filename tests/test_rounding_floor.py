@@ -1,13 +1,22 @@
 """Derivation of the 32-layer encoder tolerance (CPU only).
 
-The GPU path rounds every tensor-core operand to bf16: the RMSNorm outputs,
-q/k/v, the softmax probabilities P, the attention output, the SwiGLU
-activation, and the conv-stem hidden frames.  This test runs the oracle's
-float64 arithmetic with exactly those roundings added (nothing else changed)
-and measures its distance to the plain oracle on the frames that
-tests/test_gpu_layer.py::test_c4_full_encoder_prefix compares.  That distance
-is a floor for ANY implementation with bf16 activations: it exceeds the 3e-2
-max-abs bar after 32 layers while the relative L2 error stays under 1e-2.
+The GPU path rounds every tensor-core operand to bf16.  Two kinds of rounding
+are in that list:
+  * forced by the configs' "bf16 weights and activations": every activation
+    that is a GEMM operand or is stored between kernels -- the RMSNorm outputs
+    (QKV and gate/up operands), q/k/v, the attention output (O-projection
+    operand), the SwiGLU activation (down-projection operand) and the
+    conv-stem hidden frames (conv2 operand);
+  * a choice of this implementation: the softmax probabilities P, rounded to
+    bf16 so that P V runs on the tensor cores (an fp32 P V on CUDA cores would
+    not round them).
+This test runs the oracle's float64 arithmetic with those roundings added
+(nothing else changed), once with the forced ones only and once with bf16 P as
+well, and measures the distance to the plain oracle on the frames that
+tests/test_gpu_layer.py::test_c4_full_encoder_prefix compares.  The forced
+roundings alone give max-abs 3.8e-2 (bf16 P as well: 3.6e-2): after 32 layers
+any implementation with bf16 activations sits above the 3e-2 max-abs bar,
+while the relative L2 error stays under 1e-2 (7e-3).
 Hence the 32-layer encoder test keeps rel-L2 <= 1e-2 and bounds max-abs by
 C4_MAX_ABS below (the floor measured here, 3.6e-2, plus headroom).  The same
 holds for the 32-layer streaming step, whose output is the unnormalised
@@ -28,6 +37,15 @@ C4_MAX_ABS = 5e-2
 C4_FRAMES = 256
 C3_MAX_ABS = 1e-1
 C3_SAMPLE = (0, 37, 63)
+# The streaming config as stated (ring filled by a prefill of 1000 frames,
+# then a 4-frame step; tests/test_gpu_stream.py::test_c3_stated_config_prefill_then_step)
+# compares 32-layer outputs of streams 0 and 63.  Its floor, computed by
+# tests/derive_stream_floor.py (too slow for this suite: 32 whole-sequence
+# layers over 1004 frames twice), is max-abs 7.6e-2 / rel 6.4e-3 on the raw
+# residual stream (values up to +-11) and 3.0e-2 / 6.4e-3 after the final
+# RMSNorm; the bounds below add headroom, rel-L2 stays at 1e-2.
+C3_STATED_MAX_ABS = 1e-1
+C3_STATED_NORMED_MAX_ABS = 5e-2
 
 
 @functools.lru_cache(maxsize=1)
@@ -39,7 +57,7 @@ def _r(x):
     return synth.bf16_round(np.asarray(x, dtype=np.float32)).astype(np.float64)
 
 
-def _layer_bf16_operands(x, p, dims):
+def _layer_bf16_operands(x, p, dims, round_p=True):
     B, T, _ = x.shape
     H, D, W = dims.n_heads, dims.head_dim, dims.window
     pos = np.arange(T)
@@ -53,7 +71,7 @@ def _layer_bf16_operands(x, p, dims):
         lo = max(0, i - W + 1)
         s = np.einsum("bhd,bjhd->bhj", q[:, i], k[:, lo:i + 1]) / np.sqrt(D)
         e = np.exp(s - s.max(-1, keepdims=True))
-        a[:, i] = np.einsum("bhj,bjhd->bhd", _r(e), v[:, lo:i + 1]) / e.sum(-1, keepdims=True)
+        a[:, i] = np.einsum("bhj,bjhd->bhd", _r(e) if round_p else e, v[:, lo:i + 1]) / e.sum(-1, keepdims=True)
     h = x + _r(a.reshape(B, T, H * D)) @ f(p["wo"]).T + f(p["bo"])
     y1 = _r(oracle.rms_norm(h, p["ffn_norm_g"], dims.eps))
     act = _r(oracle.silu(y1 @ f(p["wg"]).T) * (y1 @ f(p["wu"]).T))
@@ -78,7 +96,8 @@ def _stem_bf16_operands(mel, conv):
 
 
 @pytest.mark.slow
-def test_bf16_operand_floor_of_the_32_layer_encoder():
+@pytest.mark.parametrize("round_p", [False, True])
+def test_bf16_operand_floor_of_the_32_layer_encoder(round_p):
     dims = synth.VOXTRAL_RT
     layers = _stack32()
     conv = synth.conv_params(seed=3)
@@ -87,7 +106,7 @@ def test_bf16_operand_floor_of_the_32_layer_encoder():
     ref = oracle.encoder(mel, conv, layers, g, dims)
     x = _stem_bf16_operands(mel, conv)
     for p in layers:
-        x = _layer_bf16_operands(x, p, dims)
+        x = _layer_bf16_operands(x, p, dims, round_p)
     out = oracle.rms_norm(x, g, dims.eps)
     err = out - ref
     max_abs = np.abs(err).max()
