@@ -159,3 +159,9 @@ def ring_kv(S, H, W, D, seed=6):
     k = bf16_round(_normal(rng, (S, H, W, D)))
     v = bf16_round(_normal(rng, (S, H, W, D)))
     return k, v
+
+
+def audio(B, N, seed=9, std=0.1):
+    """16 kHz audio samples ~ N(0, std^2) (white noise), float32 [B, N]."""
+    rng = np.random.default_rng(seed)
+    return _normal(rng, (B, N), std)

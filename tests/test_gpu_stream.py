@@ -11,7 +11,7 @@ import torch
 
 import oracle
 import synth
-from test_rounding_floor import C3_MAX_ABS, C3_SAMPLE
+from test_rounding_floor import C3_MAX_ABS, C3_SAMPLE, C3_STATED_MAX_ABS, C3_STATED_NORMED_MAX_ABS
 from gpu_util import cfg_of, compare_bf16, dev, host, layer_params_dev, layer_stack
 
 pytestmark = pytest.mark.gpu
@@ -181,3 +181,48 @@ def test_cuda_graph_replay_of_a_step():
     vx.stream_step(cfg_of(dims), Ls, ring_a, xin)   # second eager step on ring_a
     torch.cuda.synchronize()
     assert torch.all(ring_b.pos == 24) and torch.equal(ring_a.k, ring_b.k)
+
+
+def test_c3_stated_config_prefill_then_step():
+    # The streaming config as stated: 32 layers of the one-layer shape, 64
+    # streams, the ring filled by vx_stream_prefill from 1000 seeded frames
+    # per stream (so it has wrapped: frames 250..999 in slots f mod 750),
+    # then one 4-frame step at positions 1000..1003.  The step must equal
+    # (i) the GPU whole-sequence output of frames 1000..1003 (a prefill over
+    # all 1004 frames) and (ii) the oracle over those 1004 frames x 32 layers
+    # (streams 0 and 63).  Raw outputs are the unnormalised residual stream;
+    # with the final RMSNorm (final_g) they are the encoder's output.
+    vx = _vx()
+    dims = synth.VOXTRAL_RT
+    L, S, n, P = 32, 64, 4, 1000
+    layers = layer_stack(dims, L, 1)
+    Ls = [vx.pack_layer(cfg_of(dims), layer_params_dev(p)) for p in layers]
+    cfg = cfg_of(dims)
+    g = synth.final_norm_gain(dims.d_model, seed=5)
+    gd = dev(g, torch.bfloat16)
+    x = synth.frames(S, P + n, dims.d_model, seed=7)
+    xd = dev(x)
+    ring = vx.KVRing(cfg, L, S)
+    ws = vx.Workspace()
+    out = {}
+    for fg in (None, gd):
+        vx.stream_prefill(cfg, Ls, ring, xd[:, :P].contiguous(), ws=ws)
+        assert torch.all(ring.pos == P)
+        out[fg is None] = host(vx.stream_step(cfg, Ls, ring, xd[:, P:].contiguous(), final_g=fg, ws=ws))
+        assert torch.all(ring.pos == P + n)
+    whole = host(vx.stream_prefill(cfg, Ls, ring, xd, ws=ws)[:, P:])
+    whole_n = host(vx.stream_prefill(cfg, Ls, ring, xd, final_g=gd, ws=ws)[:, P:])
+    del ring, ws
+    torch.cuda.empty_cache()
+    raw, normed = out[True], out[False]
+    compare_bf16(raw, whole, "C3 stated: step vs GPU whole sequence (raw)", max_abs=C3_STATED_MAX_ABS)
+    compare_bf16(normed, whole_n, "C3 stated: step vs GPU whole sequence (final norm)", max_abs=C3_STATED_NORMED_MAX_ABS)
+    # the oracle over 1004 frames x 32 layers for two streams
+    sample = [0, 63]
+    h = np.asarray(x[sample], dtype=np.float64)
+    for p in layers:
+        h = oracle.encoder_layer(h, p, dims)
+    want = h[:, P:]
+    compare_bf16(raw[sample], want, "C3 stated: step vs oracle (raw)", max_abs=C3_STATED_MAX_ABS)
+    compare_bf16(normed[sample], oracle.rms_norm(want, g, dims.eps), "C3 stated: step vs oracle (final norm)",
+                 max_abs=C3_STATED_NORMED_MAX_ABS)
