@@ -151,8 +151,11 @@ VX_API vx_status vx_pack_conv_weight(const void *w, void *w_packed, int out_ch, 
 
 /* ------------------------------------------------------------- operations */
 
-/* Causal sliding-window multi-head attention with RoPE (the encoder's
- * attention: each frame attends to itself and the W-1 frames before it).
+/* Causal sliding-window multi-head attention with RoPE: the attention of
+ * the encoder layer in the transcribe.cpp notes "Voxtral", section
+ * "Architecture -> Voxtral Realtime 2602" (causal attention over a sliding
+ * window of 750 frames, RoPE theta 1e6, head_dim 64, 32 heads): each frame
+ * attends to itself and the W-1 frames before it.
  *   o_i = sum_{j: i-W < j <= i} softmax_j(<q'_i, k'_j> * scale) v_j per head,
  * with q', k' = RoPE(q, k) at positions pos0 + t when apply_rope != 0
  * (split-halves pairing, inv_freq_m = rope_theta^(-2m/D)).
@@ -174,13 +177,20 @@ VX_API size_t vx_swa_attn_workspace(vx_dtype dt, int B, int T, int H, int D, int
  * and the status word of the bounded waits) is one static device array of
  * 32 MiB + 256 bytes inside this library, held by every GPU that loads the
  * library until the process exits.  Inputs and outputs are still the caller's.
- * Limit: with apply_rope, the rotated q and k (2 * B*T*H*64 elements) plus
- * T * 256 bytes of table must fit in 32 MiB (about B*T*H <= 126000 for bf16,
- * half that for fp32); larger calls return VX_ERR_INVALID_ARG with a message
- * and enqueue nothing.
+ * Limit: with apply_rope, each rotated tensor takes B*T*H*64*es bytes
+ * (es = 2 for bf16, 4 for fp32) rounded up to a multiple of 256, and the
+ * cos/sin table T*256 bytes; 2 * that rounded size + T*256 must be at most
+ * 32 MiB (33554432 bytes).  For bf16 that is B*T*H + T <= 131072 when B*T*H
+ * is even (e.g. B=1, H=32: T <= 3971); for fp32, 2*B*T*H + T <= 131072.
+ * Without RoPE no scratch beyond the status word is used and any size runs.
+ * Larger calls return VX_ERR_INVALID_ARG with a message and enqueue nothing.
  * The first call on each device looks up the array's device address (with
- * that device current) and caches it; make that first call before any stream
- * capture.  Every call clears the status word and overwrites the rotated q/k,
+ * that device current) and caches it together with the current context; it
+ * is looked up again when the context changes (e.g. after cudaDeviceReset).
+ * Make that first call before any stream capture.  Its kernels are counted by
+ * vx_launch_count and timed by vx_trace_enable / vx_trace_read like those of
+ * vx_swa_attn_fwd.  Every call clears the status word and overwrites the
+ * rotated q/k,
  * and all calls share the one array: calls whose work overlaps on the GPU
  * (other streams, other threads) race on it.  A bounded wait that expires is
  * recorded only in that private status word; use vx_swa_attn_fwd with a
@@ -199,7 +209,11 @@ VX_API vx_status vx_rms_norm_fwd(const float *x, const float *r, const void *g, 
                           void *y, vx_dtype y_dt, int M, int d, float eps,
                           void *ws, size_t ws_bytes, cudaStream_t stream);
 
-/* One encoder layer over B clips of T frames (whole-sequence, causal):
+/* One encoder layer over B clips of T frames (whole-sequence, causal), as the
+ * transcribe.cpp notes "Voxtral", section "Architecture -> Voxtral Realtime
+ * 2602", state it: RMSNorm pre-norm, q/v/o projections with bias and k
+ * without, RoPE (theta 1e6, head_dim 64), causal sliding-window attention
+ * (750), and a SwiGLU MLP with bias on the down projection only:
  *   y0 = RMSNorm(x); q,k,v = y0 W^T + b; RoPE(q,k) at pos0 + t;
  *   h = x + SWA(q,k,v) Wo^T + bo; out = h + (silu(y1 Wg^T + bg) * (y1 Wu^T + bu)) Wd^T + bd,
  *   y1 = RMSNorm(h).
@@ -210,7 +224,10 @@ VX_API vx_status vx_encoder_layer_fwd(const vx_layer_cfg *cfg, const vx_layer_we
                                void *ws, size_t ws_bytes, cudaStream_t stream);
 VX_API size_t vx_encoder_layer_workspace(const vx_layer_cfg *cfg, int B, int T);
 
-/* Causal conv stem: left-pad-only Conv1d(n_mels -> d, k3, s1) + GELU, then
+/* Causal conv stem (transcribe.cpp notes "Voxtral", section "Architecture ->
+ * Voxtral Realtime 2602": causal convolutions with left padding only; shapes
+ * of the stem as in the 2507 section): left-pad-only
+ * Conv1d(n_mels -> d, k3, s1) + GELU, then
  * Conv1d(d -> d, k3, s2) + GELU (exact erf GELU, left zero padding of 2 frames
  * before each conv).  mel: [B, n_mels, Tm] fp32; w1p: [d, 3, n_mels] and
  * w2p: [d, 3, d] bf16 (vx_pack_conv_weight); b1, b2: [d] bf16;
@@ -301,8 +318,12 @@ VX_API vx_status vx_stream_prefill(const vx_layer_cfg *cfg, const vx_layer_weigh
                             const void *final_g, void *ws, size_t ws_bytes,
                             cudaStream_t stream);
 
-/* Streaming step: n_new (1..8) new frames per stream, for every stream of the
- * ring, through the ring's n_layers layers.  Per layer, new frame f = pos[s]+t
+/* Streaming step (transcribe.cpp notes "Voxtral", section "Architecture ->
+ * Voxtral Realtime 2602": 8 mel frames = 4 encoder frames per 80 ms step; the
+ * W-slot ring replaces the append-only frame buffer of the Core AI card's
+ * streaming encoder, section "Usage / Known limitations"): n_new (1..8) new
+ * frames per stream, for every stream of the ring, through the ring's
+ * n_layers layers.  Per layer, new frame f = pos[s]+t
  * attends frames f' with f - W < f' <= f: older frames from the ring, the rest
  * from this step; every in-window ring slot is read before the new K/V are
  * written to slots (pos[s] + t) mod W.  Advances pos[s] += n_new at the end.

@@ -46,22 +46,6 @@ const char* last_error() { return g_err; }
 static std::atomic<uint64_t> g_wait_limit_ns{1000000000ull};
 uint64_t wait_limit_ns() { return g_wait_limit_ns.load(); }
 
-bool pair_gemm_disabled() {
-  static const bool off = [] {
-    const char* e = std::getenv("VX_PAIR_GEMM");
-    return e && e[0] == '0';
-  }();
-  return off;
-}
-
-bool ring_tma_disabled() {
-  static const bool off = [] {
-    const char* e = std::getenv("VX_RING_TMA");
-    return e && e[0] == '0';
-  }();
-  return off;
-}
-
 cudaError_t ensure_dynamic_smem(const void* kernel, size_t smem) {
   int dev = 0;
   if (cudaError_t e = cudaGetDevice(&dev)) return e;
@@ -75,25 +59,7 @@ cudaError_t ensure_dynamic_smem(const void* kernel, size_t smem) {
   return e;
 }
 
-bool tma_store_disabled() {
-  static const bool off = [] {
-    const char* e = std::getenv("VX_TMA_STORE");
-    return e && e[0] == '0';
-  }();
-  return off;
-}
-
-bool pdl_enabled() {
-  static const bool on = [] {
-    const char* e = std::getenv("VX_PDL");
-    return !(e && e[0] == '0');
-  }();
-  return on;
-}
-
 // ------------------------------------------------------------- tracing --
-// Kernel launches go through traced(): it counts them and, when tracing is on
-// for the calling thread, brackets them with CUDA events on the launch stream.
 static std::atomic<uint64_t> g_launches{0};
 struct TraceRec {
   const char* name;
@@ -104,7 +70,10 @@ static thread_local std::vector<TraceRec> t_recs;
 static thread_local std::vector<cudaEvent_t> t_pool;
 static thread_local size_t t_pool_used = 0;
 
-static cudaEvent_t trace_event() {
+void count_launches(int n) { g_launches.fetch_add(static_cast<uint64_t>(n)); }
+bool trace_enabled() { return t_trace; }
+
+cudaEvent_t trace_event() {
   if (t_pool_used == t_pool.size()) {
     cudaEvent_t e;
     if (cudaEventCreate(&e) != cudaSuccess) return nullptr;
@@ -113,16 +82,21 @@ static cudaEvent_t trace_event() {
   return t_pool[t_pool_used++];
 }
 
-template <class F>
-cudaError_t traced(const Launch& L, const char* name, int kernels, F&& f) {
-  g_launches.fetch_add(static_cast<uint64_t>(kernels));
-  if (!t_trace) return f();
-  cudaEvent_t a = trace_event(), b = trace_event();
-  if (a) cudaEventRecord(a, L.stream);
-  const cudaError_t e = f();
-  if (b) cudaEventRecord(b, L.stream);
-  if (a && b) t_recs.push_back({name, a, b});
-  return e;
+void trace_record(const char* name, cudaEvent_t a, cudaEvent_t b) { t_recs.push_back({name, a, b}); }
+
+const char* rms_trace_name(int nparts, bool h_out, int y_kind) {
+  // "rmsnorm_p<n>[_h][_y16|_y32]": the partial sums it reduces, whether it
+  // writes h, and the normalised output's type (none when it only reduces).
+  static const std::vector<std::string> names = [] {
+    std::vector<std::string> v;
+    for (int n = 0; n <= kMaxSplitsTraced; ++n)
+      for (int h = 0; h < 2; ++h)
+        for (int y = 0; y < 3; ++y)
+          v.push_back("rmsnorm_p" + std::to_string(n) + (h ? "_h" : "") + (y == 1 ? "_y16" : y == 2 ? "_y32" : ""));
+    return v;
+  }();
+  if (nparts < 0 || nparts > kMaxSplitsTraced || y_kind < 0 || y_kind > 2) return "rmsnorm";
+  return names[(nparts * 2 + (h_out ? 1 : 0)) * 3 + y_kind].c_str();
 }
 
 int current_sm_count() {
@@ -232,6 +206,16 @@ vx_status make_launch(Launch* L, void* ws, size_t ws_bytes, size_t need, cudaStr
     return VX_ERR_CUDA;
   }
   return VX_OK;
+}
+
+// A traced RMSNorm / partial-sum reduction launch (see launch_rmsnorm).
+cudaError_t rmsnorm(const Launch& L, const float* x, const float* parts, int nparts, int64_t part_stride,
+                    const uint16_t* bias, const uint16_t* g, float* h_out, void* y, bool y_bf16, int M, int d,
+                    float eps) {
+  const int yk = (g && y) ? (y_bf16 ? 1 : 2) : 0;
+  return traced(L, rms_trace_name(nparts, h_out != nullptr, yk), 1, [&] {
+    return launch_rmsnorm(L, x, parts, nparts, part_stride, bias, g, h_out, y, y_bf16, M, d, eps);
+  });
 }
 
 vx_status check_cfg(const vx_layer_cfg* c) {
@@ -347,7 +331,7 @@ vx_status launch_planned(const Launch& L, const char* name, const CUtensorMap* t
   if (!tmap_bf16_2d(&tmB, Bw, a_in.K, a_in.N, ldb, p.pair ? p.bn / 2 : p.bn)) return VX_ERR_CUDA;
   GemmArgs a = a_in;
   std::memset(&tmD, 0, sizeof(tmD));
-  a.tma_store = (!tma_store_disabled() && tmap_gemm_out(&tmD, a, epi)) ? 1 : 0;
+  a.tma_store = tmap_gemm_out(&tmD, a, epi) ? 1 : 0;
   VX_CUDA(traced(L, name, 1, [&] { return launch_gemm(L, *tmA, tmB, tmD, a, epi, p); }));
   return VX_OK;
 }
@@ -431,11 +415,9 @@ vx_status run_layer(const Launch& L, const vx_layer_cfg& c, const vx_layer_weigh
   // 1. x_l = reduce(in); y0 = RMSNorm(x_l)
   const bool pending_in = in.parts != nullptr || in.bias != nullptr;
   const float* xl = pending_in ? bf.xmat : in.base;
-  VX_CUDA(traced(L, "rmsnorm", 1, [&] {
-    return launch_rmsnorm(L, in.base, in.parts, in.nparts, pstride, in.bias,
+  VX_CUDA(rmsnorm(L, in.base, in.parts, in.nparts, pstride, in.bias,
                           static_cast<const uint16_t*>(w.attn_norm_g), pending_in ? bf.xmat : nullptr, bf.y0, true, M,
-                          d, c.eps);
-  }));
+                          d, c.eps));
   // 2. QKV + bias + RoPE at (pos[s] or pos0) + t
   {
     GemmArgs a = base_args(L, M, 3 * HD, d);
@@ -455,16 +437,12 @@ vx_status run_layer(const Launch& L, const vx_layer_cfg& c, const vx_layer_weigh
                               sl2);
     }));
   } else {
-    CUtensorMap tq, tk, tv;
-    const int64_t rs = 3LL * HD, bs = static_cast<int64_t>(rows) * 3 * HD;
-    if (!tmap_attn_operand(&tq, bf.qkv, nseq, rows, H, rs, bs)) return VX_ERR_CUDA;
-    if (!tmap_attn_operand(&tk, bf.qkv + HD, nseq, rows, H, rs, bs)) return VX_ERR_CUDA;
-    if (!tmap_attn_operand(&tv, bf.qkv + 2 * HD, nseq, rows, H, rs, bs)) return VX_ERR_CUDA;
+    const AttnOperands op{bf.qkv, bf.qkv + HD, bf.qkv + 2 * HD, 3LL * HD, static_cast<int64_t>(rows) * 3 * HD};
     AttnArgs aa;
     aa.out = bf.att; aa.o_row = HD; aa.o_head = 64; aa.o_batch = static_cast<int64_t>(rows) * HD;
     aa.B = nseq; aa.T = rows; aa.H = H; aa.window = c.window; aa.scale_log2 = sl2;
     aa.status = L.status; aa.limit_ns = L.limit_ns;
-    VX_CUDA(traced(L, "swa_attn_tc", 1, [&] { return launch_attn_bf16(L, tq, tk, tv, aa); }));
+    VX_CUDA(traced(L, "swa_attn_tc", 1, [&] { return launch_attn_bf16(L, op, aa); }));
     if (ring && ring->fill)
       VX_CUDA(traced(L, "ring_fill", 1, [&] {
         return launch_ring_fill(L, bf.qkv, 3LL * HD, HD, ring->k, ring->v, nseq, rows, H, ring->W);
@@ -477,11 +455,9 @@ vx_status run_layer(const Launch& L, const vx_layer_cfg& c, const vx_layer_weigh
     return st;
   // 5. y1 = RMSNorm(h), materialising h when it is pending
   const bool pending_h = hp.parts != nullptr;
-  VX_CUDA(traced(L, "rmsnorm", 1, [&] {
-    return launch_rmsnorm(L, hp.base, hp.parts, hp.nparts, pstride, hp.bias,
+  VX_CUDA(rmsnorm(L, hp.base, hp.parts, hp.nparts, pstride, hp.bias,
                           static_cast<const uint16_t*>(w.ffn_norm_g), pending_h ? bf.h : nullptr, bf.y0, true, M, d,
-                          c.eps);
-  }));
+                          c.eps));
   // 6. gate/up + SwiGLU
   {
     GemmArgs a = base_args(L, M, 2 * F, d);
@@ -497,7 +473,7 @@ vx_status run_layer(const Launch& L, const vx_layer_cfg& c, const vx_layer_weigh
 // y = reduce(p) unless p already is y.
 cudaError_t reduce_into(const Launch& L, const Pending& p, float* y, int M, int d) {
   if (p.base == y && p.parts == nullptr && p.bias == nullptr) return cudaSuccess;
-  return launch_rmsnorm(L, p.base, p.parts, p.nparts, static_cast<int64_t>(M) * d, p.bias, nullptr, y, nullptr, false,
+  return rmsnorm(L, p.base, p.parts, p.nparts, static_cast<int64_t>(M) * d, p.bias, nullptr, y, nullptr, false,
                         M, d, 1.0f);
 }
 
@@ -701,17 +677,14 @@ vx_status vx_swa_attn_fwd(const void* q, const void* k, const void* v, void* o, 
     }));
     return VX_OK;
   }
-  CUtensorMap tq, tk, tv;
   const int64_t rs = int64_t(H) * 64, bs = int64_t(T) * H * 64;
-  if (!tmap_attn_operand(&tq, qq, B, T, H, rs, bs)) return VX_ERR_CUDA;
-  if (!tmap_attn_operand(&tk, kk, B, T, H, rs, bs)) return VX_ERR_CUDA;
-  if (!tmap_attn_operand(&tv, v, B, T, H, rs, bs)) return VX_ERR_CUDA;
+  const AttnOperands op{qq, kk, v, rs, bs};
   AttnArgs aa;
   aa.out = o; aa.o_row = rs; aa.o_head = 64; aa.o_batch = bs;
   aa.B = B; aa.T = T; aa.H = H; aa.window = window;
   aa.scale_log2 = scale * 1.4426950408889634f;
   aa.status = L.status; aa.limit_ns = L.limit_ns;
-  VX_CUDA(traced(L, "swa_attn_tc", 1, [&] { return launch_attn_bf16(L, tq, tk, tv, aa); }));
+  VX_CUDA(traced(L, "swa_attn_tc", 1, [&] { return launch_attn_bf16(L, op, aa); }));
   return VX_OK;
 }
 
@@ -729,10 +702,8 @@ vx_status vx_rms_norm_fwd(const float* x, const float* r, const void* g, float* 
   Launch L;
   vx_status st = make_launch(&L, ws, ws_bytes, kStatusBytes, stream);
   if (st != VX_OK) return st;
-  VX_CUDA(traced(L, "rmsnorm", 1, [&] {
-    return launch_rmsnorm(L, x, r, r ? 1 : 0, 0, nullptr, static_cast<const uint16_t*>(g), h_out, y, y_dt == VX_BF16,
-                          M, d, eps);
-  }));
+  VX_CUDA(rmsnorm(L, x, r, r ? 1 : 0, 0, nullptr, static_cast<const uint16_t*>(g), h_out, y, y_dt == VX_BF16,
+                          M, d, eps));
   return VX_OK;
 }
 
@@ -756,7 +727,7 @@ vx_status vx_encoder_layer_fwd(const vx_layer_cfg* cfg, const vx_layer_weights* 
   if ((st = run_layer(L, *cfg, *w, Pending{x, nullptr, 0, nullptr}, &out, y, B, T, pos0, bf, nullptr)) != VX_OK)
     return st;
   if (out.base != y || out.parts || out.bias)
-    VX_CUDA(traced(L, "reduce_out", 1, [&] { return reduce_into(L, out, y, B * T, cfg->d_model); }));
+    VX_CUDA(reduce_into(L, out, y, B * T, cfg->d_model));
   return VX_OK;
 }
 
@@ -917,10 +888,8 @@ vx_status vx_encoder_fwd(const vx_layer_cfg* cfg, const float* mel, int B, int n
     cur = next;
   }
   const int64_t pstride = static_cast<int64_t>(B) * To * cfg->d_model;
-  VX_CUDA(traced(L, "rmsnorm", 1, [&] {
-    return launch_rmsnorm(L, cur.base, cur.parts, cur.nparts, pstride, cur.bias,
-                          static_cast<const uint16_t*>(final_g), nullptr, out, false, B * To, cfg->d_model, cfg->eps);
-  }));
+  VX_CUDA(rmsnorm(L, cur.base, cur.parts, cur.nparts, pstride, cur.bias,
+                          static_cast<const uint16_t*>(final_g), nullptr, out, false, B * To, cfg->d_model, cfg->eps));
   return VX_OK;
 }
 
@@ -950,12 +919,10 @@ vx_status vx_stream_prefill(const vx_layer_cfg* cfg, const vx_layer_weights* lay
   }
   const int64_t pstride = static_cast<int64_t>(S) * T * cfg->d_model;
   if (final_g) {
-    VX_CUDA(traced(L, "rmsnorm", 1, [&] {
-      return launch_rmsnorm(L, cur.base, cur.parts, cur.nparts, pstride, cur.bias,
-                            static_cast<const uint16_t*>(final_g), nullptr, y, false, S * T, cfg->d_model, cfg->eps);
-    }));
+    VX_CUDA(rmsnorm(L, cur.base, cur.parts, cur.nparts, pstride, cur.bias,
+                            static_cast<const uint16_t*>(final_g), nullptr, y, false, S * T, cfg->d_model, cfg->eps));
   } else if (cur.base != y || cur.parts || cur.bias) {
-    VX_CUDA(traced(L, "reduce_out", 1, [&] { return reduce_into(L, cur, y, S * T, cfg->d_model); }));
+    VX_CUDA(reduce_into(L, cur, y, S * T, cfg->d_model));
   }
   VX_CUDA(traced(L, "pos_add", 1, [&] { return launch_pos_add(L, ring->pos, S, T, true); }));
   return VX_OK;
@@ -998,11 +965,9 @@ vx_status vx_stream_step(const vx_layer_cfg* cfg, const vx_layer_weights* layers
   }
   // y = reduce(last layer output), then the optional final RMSNorm.
   const int64_t pstride = static_cast<int64_t>(M) * cfg->d_model;
-  VX_CUDA(traced(L, "rmsnorm", 1, [&] {
-    return launch_rmsnorm(L, cur.base, cur.parts, cur.nparts, pstride, cur.bias,
+  VX_CUDA(rmsnorm(L, cur.base, cur.parts, cur.nparts, pstride, cur.bias,
                           static_cast<const uint16_t*>(final_g), final_g ? nullptr : y, final_g ? y : nullptr, false,
-                          M, cfg->d_model, cfg->eps);
-  }));
+                          M, cfg->d_model, cfg->eps));
   VX_CUDA(traced(L, "pos_add", 1, [&] { return launch_pos_add(L, ring->pos, S, n_new, false); }));
   return VX_OK;
 }

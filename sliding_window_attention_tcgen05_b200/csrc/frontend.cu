@@ -175,12 +175,6 @@ cudaError_t launch_log_mel(const Launch& L, const float* audio, float* mel, int 
   float* fb = static_cast<float*>(tables);   // [201][128]
   float* win = fb + kMels * kBins;
   float2* tw = reinterpret_cast<float2*>(win + kNfft);
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(log_mel_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kMelSmem);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
   cudaError_t e = launch_kernel(mel_tables_kernel, dim3(kMels + 1), dim3(256), 0, L.stream, fb, win, tw);
   if (e != cudaSuccess) return e;
   return launch_kernel(log_mel_kernel, dim3((F + kFpc - 1) / kFpc, B), dim3(kMelThreads), kMelSmem, L.stream, audio,

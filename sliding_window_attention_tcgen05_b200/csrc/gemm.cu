@@ -792,20 +792,10 @@ gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
 }
 
 // ------------------------------------------------------------- launchers --
-template <class K>
-cudaError_t set_smem(K kernel, int bytes, bool& done) {
-  if (done) return cudaSuccess;
-  cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
-  if (e == cudaSuccess) done = true;   // per instantiation; a racing second call is harmless
-  return e;
-}
-
 template <int BN, int EPI>
 cudaError_t launch_one(const Launch& L, const CUtensorMap& tmA, const CUtensorMap& tmB, const CUtensorMap& tmD,
                        const GemmArgs& a) {
   using C = OneCfg<BN>;
-  static bool attr_set = false;
-  if (cudaError_t e = set_smem(gemm_tc_kernel<BN, EPI>, C::S::kTotal, attr_set)) return e;
   const int tiles = ((a.M + kBM - 1) / kBM) * (a.N / BN) * a.k_splits;
   const int grid = tiles < L.sm_count ? tiles : L.sm_count;
   return launch_kernel(gemm_tc_kernel<BN, EPI>, dim3(grid), dim3(kThreads), C::S::kTotal, L.stream, tmA, tmB, tmD,
@@ -816,8 +806,6 @@ template <int BN, int EPI>
 cudaError_t launch_pair(const Launch& L, const CUtensorMap& tmA, const CUtensorMap& tmB, const CUtensorMap& tmD,
                         const GemmArgs& a) {
   using C = PairCfg<BN>;
-  static bool attr_set = false;
-  if (cudaError_t e = set_smem(gemm_tc2_kernel<BN, EPI>, C::S::kTotal, attr_set)) return e;
   const int tiles = ((a.M + 255) / 256) * (a.N / BN) * a.k_splits;
   const int pairs = L.sm_count / 2;
   const int grid = 2 * (tiles < pairs ? tiles : pairs);
@@ -870,7 +858,7 @@ GemmPlan plan_gemm(int M, int N, int K, int epi, int max_splits, int sm) {
   double best_t = 1e30;
   const int nkb = K / kBK;
   const bool can_split = epi == EPI_F32;
-  for (int pair = pair_gemm_disabled() ? 0 : 1; pair >= 0; --pair) {
+  for (int pair = 1; pair >= 0; --pair) {
     for (int bn = 256; bn >= 128; bn /= 2) {
       if (N % bn != 0) continue;
       for (int s = 1; s <= (can_split ? max_splits : 1); s *= 2) {

@@ -26,11 +26,33 @@ static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratch
 
 constexpr int kMaxDevices = 64;
 std::mutex g_noalloc_mu;
-void* g_noalloc_ptr[kMaxDevices] = {nullptr};
+struct ScratchAddr {
+  CUcontext ctx;   // the context the address was looked up in
+  void* ptr;
+};
+ScratchAddr g_noalloc_addr[kMaxDevices] = {};
+
+// The current context, through the runtime's driver entry point (no -lcuda).
+CUcontext current_context() {
+  using Fn = CUresult (*)(CUcontext*);
+  static Fn fn = [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return static_cast<Fn>(nullptr);
+    return reinterpret_cast<Fn>(p);
+  }();
+  CUcontext c = nullptr;
+  if (fn == nullptr || fn(&c) != CUDA_SUCCESS) return nullptr;
+  return c;
+}
 
 // Device address of g_noalloc_scratch on the current device.  In host code
-// the array's name is only a stand-in, so the address is looked up once per
-// device (with that device current) and cached.
+// the array's name is only a stand-in, so the address is looked up (with the
+// device current) on the first call on each device and cached.  The cache
+// also remembers the context it came from and looks the address up again
+// when that context has changed (after cudaDeviceReset, say).
 vx_status noalloc_scratch(void** out) {
   int dev = -1;
   cudaError_t e = cudaGetDevice(&dev);
@@ -38,8 +60,10 @@ vx_status noalloc_scratch(void** out) {
     vx::set_error("vx_swa_attn_fwd_noalloc: no usable current CUDA device (%s)", cudaGetErrorString(e));
     return VX_ERR_CUDA;
   }
+  const CUcontext ctx = current_context();
   std::lock_guard<std::mutex> lk(g_noalloc_mu);
-  if (g_noalloc_ptr[dev] == nullptr) {
+  ScratchAddr& c = g_noalloc_addr[dev];
+  if (c.ptr == nullptr || ctx == nullptr || c.ctx != ctx) {
     void* p = nullptr;
     e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
     if (e != cudaSuccess || p == nullptr) {
@@ -47,9 +71,10 @@ vx_status noalloc_scratch(void** out) {
                     cudaGetErrorString(e));
       return VX_ERR_CUDA;
     }
-    g_noalloc_ptr[dev] = p;
+    c.ctx = current_context();   // the lookup made the runtime's context current
+    c.ptr = p;
   }
-  *out = g_noalloc_ptr[dev];
+  *out = c.ptr;
   return VX_OK;
 }
 
@@ -113,7 +138,9 @@ vx_status vx_swa_attn_fwd_noalloc(const void* q, const void* k, const void* v, v
     void* qr = sc;
     void* kr = sc + (one + 255) / 256 * 256;
     void* tb = sc + 2 * ((one + 255) / 256 * 256);
-    if ((e = launch_rope(L, q, k, qr, kr, tb, dt == VX_BF16, B, T, H, pos0, rope_theta)) != cudaSuccess) {
+    if ((e = traced(L, "rope", 2, [&] {
+           return launch_rope(L, q, k, qr, kr, tb, dt == VX_BF16, B, T, H, pos0, rope_theta);
+         })) != cudaSuccess) {
       set_error("vx_swa_attn_fwd_noalloc: RoPE launch failed: %s", cudaGetErrorString(e));
       return VX_ERR_CUDA;
     }
@@ -121,20 +148,19 @@ vx_status vx_swa_attn_fwd_noalloc(const void* q, const void* k, const void* v, v
     kk = kr;
   }
   if (dt == VX_F32) {
-    e = launch_attn_f32(L, static_cast<const float*>(qq), static_cast<const float*>(kk),
-                        static_cast<const float*>(v), static_cast<float*>(o), B, T, H, window, scale);
+    e = traced(L, "swa_attn_f32", 1, [&] {
+      return launch_attn_f32(L, static_cast<const float*>(qq), static_cast<const float*>(kk),
+                             static_cast<const float*>(v), static_cast<float*>(o), B, T, H, window, scale);
+    });
   } else {
-    CUtensorMap tq, tk, tv;
     const int64_t rs = int64_t(H) * 64, bs = int64_t(T) * H * 64;
-    if (!tmap_attn_operand(&tq, qq, B, T, H, rs, bs) || !tmap_attn_operand(&tk, kk, B, T, H, rs, bs) ||
-        !tmap_attn_operand(&tv, v, B, T, H, rs, bs))
-      return VX_ERR_CUDA;
+    const AttnOperands op{qq, kk, v, rs, bs};
     AttnArgs aa;
     aa.out = o; aa.o_row = rs; aa.o_head = 64; aa.o_batch = bs;
     aa.B = B; aa.T = T; aa.H = H; aa.window = window;
     aa.scale_log2 = scale * 1.4426950408889634f;
     aa.status = L.status; aa.limit_ns = L.limit_ns;
-    e = launch_attn_bf16(L, tq, tk, tv, aa);
+    e = traced(L, "swa_attn_tc", 1, [&] { return launch_attn_bf16(L, op, aa); });
   }
   if (e != cudaSuccess) {
     set_error("vx_swa_attn_fwd_noalloc: attention launch failed: %s", cudaGetErrorString(e));

@@ -1,17 +1,17 @@
 // stream.cu -- the streaming-step kernels over the per-layer ring KV cache.
 //
-// ring_attn_kernel: one CTA per (head, stream).  The NQ new frames of the
+// ring_attn_tma_kernel: one CTA per (head, stream).  The NQ new frames of the
 //   stream (positions p .. p+NQ-1, p = pos[s]) attend their causal window:
-//   the n_old = min(p, W-1) newest cached frames (ring slots f mod W) plus the
-//   new frames themselves.  The kernel is bound by HBM (each (stream, head)
-//   reads 192 KB of K/V for 4 query rows); K/V chunks stream through a
-//   cp.async shared-memory ring and the dot products run on mma.sync
-//   fragments, which keeps the instruction count per key far below the load
-//   time (tcgen05's M >= 64 tiles would be almost all padding for 4 rows).
-//   Only after every ring read of the CTA has completed are the NQ new K/V
-//   rows written to slots (p + t) mod W (a slot about to be overwritten may
-//   still be inside an earlier query's window).  The (stream, head) ring
-//   segment is touched by this CTA only, so no other ordering is needed.
+//   the cached frames still inside it (ring slot f mod W) plus the new frames
+//   themselves.  The kernel is bound by HBM (each (stream, head) reads 192 KB
+//   of K/V for 4 query rows); K/V chunks arrive by TMA and the dot products
+//   run on mma.sync fragments, which keeps the instruction count per key far
+//   below the load time (tcgen05's M >= 64 tiles would be almost all padding
+//   for 4 rows).  Only after every ring read of the CTA has completed are the
+//   NQ new K/V rows written to slots (p + t) mod W (a slot about to be
+//   overwritten may still be inside an earlier query's window).  The
+//   (stream, head) ring segment is touched by this CTA only, so no other
+//   ordering is needed.
 // ring_fill_kernel: writes the K/V of the last W frames of a whole-sequence
 //   forward into the ring (streaming prefill).
 // pos_add_kernel: pos[s] += n (or = n).
@@ -21,17 +21,8 @@ namespace vx {
 
 namespace {
 
-constexpr int kRingThreads = 128;          // 4 warps, 16 keys each per chunk
 constexpr int kChunk = 64;                 // keys per pipeline stage
-constexpr int kStages = 4;
 constexpr int kStageBytes = 2 * kChunk * 128;   // K and V rows of one chunk (8 KB each)
-
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint32_t src_bytes) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
 __device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
   asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
@@ -54,207 +45,6 @@ __device__ __forceinline__ void mma_bf16_16816(float (&d)[4], uint32_t a0, uint3
 // Byte offset of 16-byte column c of row r in a 128-byte-row tile, XOR-swizzled
 // so that eight rows at the same column hit eight different bank groups.
 __device__ __forceinline__ uint32_t swz(int r, int c) { return r * 128 + ((c ^ (r & 7)) << 4); }
-
-// One CTA per (head h, stream s).  Keys kk = 0 .. n_old-1 are the cached frames
-// f0 + kk (ring slot (f0 + kk) mod W), kk = n_old .. n_old+NQ-1 the new frames.
-// Chunks of 64 keys (K and V rows) stream through a 4-stage cp.async ring; each
-// of the 4 warps takes 16 keys of a chunk and runs S = Q K^T and O += P V on
-// mma.sync m16n8k16 fragments (query rows NQ..15 are zero padding), with an
-// online softmax per query row.  The warps are merged through shared memory,
-// and only then (every ring read done) are the NQ new K/V rows appended.
-template <int NQ>
-__global__ void __launch_bounds__(kRingThreads)
-ring_attn_kernel(const uint16_t* __restrict__ qkv, int64_t ld_qkv, int HD,
-                 uint16_t* __restrict__ ring_k, uint16_t* __restrict__ ring_v,
-                 const int64_t* __restrict__ pos, int H, int W, uint16_t* __restrict__ out,
-                 float scale_log2) {
-  static_assert(NQ >= 1 && NQ <= 8, "1..8 new frames");
-  extern __shared__ __align__(128) uint8_t smem_raw[];
-  uint8_t* stage_base = smem_raw;                                      // kStages x (K 8 KB | V 8 KB)
-  float* sm_m = reinterpret_cast<float*>(smem_raw + kStages * kStageBytes);   // [4 warps][8]
-  float* sm_l = sm_m + 4 * 8;                                          // [4][8]
-  float* sm_o = sm_l + 4 * 8;                                          // [4][8][64]
-
-  pdl_wait();
-  pdl_trigger();
-  const int h = blockIdx.x;
-  const int s = blockIdx.y;
-  const int tid = threadIdx.x;
-  const int warp = tid >> 5, lane = tid & 31;
-  const int64_t p = pos[s];
-  const int n_old = static_cast<int>(p < W - 1 ? p : W - 1);
-  const int total = n_old + NQ;
-  const int nchunks = (total + kChunk - 1) / kChunk;
-  const int64_t seg = (static_cast<int64_t>(s) * H + h) * W * 64;
-  const uint16_t* rk = ring_k + seg;
-  const uint16_t* rv = ring_v + seg;
-  const int f0_slot = static_cast<int>((p - n_old) % W);
-  const uint16_t* newk = qkv + static_cast<int64_t>(s) * NQ * ld_qkv + HD + h * 64;
-
-  // Issue the cp.async copies of chunk c into its stage (rows past `total` are zero-filled).
-  auto load_chunk = [&](int c) {
-    const uint32_t sbase = smem_addr(stage_base + (c % kStages) * kStageBytes);
-#pragma unroll
-    for (int i = 0; i < (2 * kChunk * 8) / kRingThreads; ++i) {
-      const int idx = tid + kRingThreads * i;
-      const int row = idx >> 3;            // 0..127: K rows 0..63, V rows 64..127
-      const int col = idx & 7;
-      const int part = row >> 6;           // 0 K, 1 V
-      const int r = row & 63;
-      const int kk = c * kChunk + r;
-      const uint16_t* src = part ? rv : rk;
-      uint32_t bytes = 16;
-      if (kk < n_old) {
-        int slot = f0_slot + kk;
-        if (slot >= W) slot -= W;
-        src += static_cast<int64_t>(slot) * 64 + col * 8;
-      } else if (kk < total) {
-        src = newk + static_cast<int64_t>(kk - n_old) * ld_qkv + part * HD + col * 8;
-      } else {
-        src = rk;                          // any valid address; nothing is read
-        bytes = 0;
-      }
-      cp_async16(sbase + part * (kChunk * 128) + swz(r, col), src, bytes);
-    }
-  };
-
-  // Q as the A operand (rows = queries, zero beyond NQ), 4 k-steps of 16 dims.
-  const int qrow = lane >> 2;             // this lane's query row (c0/c1); c2/c3 are rows + 8 (padding)
-  const int qcol = (lane & 3) * 2;
-  uint32_t qa[4][2];
-#pragma unroll
-  for (int ks = 0; ks < 4; ++ks) {
-    qa[ks][0] = 0; qa[ks][1] = 0;
-    if (qrow < NQ) {
-      const uint16_t* qr = qkv + (static_cast<int64_t>(s) * NQ + qrow) * ld_qkv + h * 64 + ks * 16 + qcol;
-      qa[ks][0] = *reinterpret_cast<const uint32_t*>(qr);
-      qa[ks][1] = *reinterpret_cast<const uint32_t*>(qr + 8);
-    }
-  }
-
-  float o[8][4];
-#pragma unroll
-  for (int nb = 0; nb < 8; ++nb) o[nb][0] = o[nb][1] = o[nb][2] = o[nb][3] = 0.f;
-  float m_run = -INFINITY, l_part = 0.f;   // row qrow: running max; this lane's share of the row sum
-
-#pragma unroll
-  for (int c = 0; c < kStages - 1; ++c) {
-    if (c < nchunks) load_chunk(c);
-    cp_async_commit();
-  }
-  for (int c = 0; c < nchunks; ++c) {
-    cp_async_wait<kStages - 2>();
-    __syncthreads();
-    const uint32_t kb = smem_addr(stage_base + (c % kStages) * kStageBytes);
-    const uint32_t vb = kb + kChunk * 128;
-    const int r0 = warp * 16;               // this warp's 16 keys within the chunk
-    // S = Q K^T for two n-blocks of 8 keys.
-    float sacc[2][4];
-#pragma unroll
-    for (int nb = 0; nb < 2; ++nb) {
-      sacc[nb][0] = sacc[nb][1] = sacc[nb][2] = sacc[nb][3] = 0.f;
-      const int krow = r0 + nb * 8 + (lane & 7);
-#pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        uint32_t b0, b1, b2, b3;
-        ldsm_x4(kb + swz(krow, half * 4 + (lane >> 3)), b0, b1, b2, b3);
-        mma_bf16_16816(sacc[nb], qa[2 * half][0], 0u, qa[2 * half][1], 0u, b0, b1);
-        mma_bf16_16816(sacc[nb], qa[2 * half + 1][0], 0u, qa[2 * half + 1][1], 0u, b2, b3);
-      }
-    }
-    // Mask and scale: key kk is in query r's window iff n_old + r - W < kk <= n_old + r.
-    const int kk0 = c * kChunk + r0 + qcol;
-    float x[2][2];
-    float cmax = -INFINITY;
-#pragma unroll
-    for (int nb = 0; nb < 2; ++nb) {
-#pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        const int kk = kk0 + nb * 8 + e;
-        const bool ok = qrow < NQ && kk <= n_old + qrow && kk > n_old + qrow - W;
-        x[nb][e] = ok ? sacc[nb][e] * scale_log2 : -INFINITY;
-        cmax = fmaxf(cmax, x[nb][e]);
-      }
-    }
-    cmax = fmaxf(cmax, __shfl_xor_sync(0xffffffffu, cmax, 1));
-    cmax = fmaxf(cmax, __shfl_xor_sync(0xffffffffu, cmax, 2));
-    const float m_new = fmaxf(m_run, cmax);
-    const float mu = (m_new == -INFINITY) ? 0.f : m_new;
-    const float alpha = ex2_approx(m_run - mu);
-    float pr[2][2];
-#pragma unroll
-    for (int nb = 0; nb < 2; ++nb)
-#pragma unroll
-      for (int e = 0; e < 2; ++e) pr[nb][e] = ex2_approx(x[nb][e] - mu);
-    l_part = l_part * alpha + (pr[0][0] + pr[0][1]) + (pr[1][0] + pr[1][1]);
-    m_run = m_new;
-    // O = alpha * O + P V  (P as the A operand: rows 8..15 zero)
-    const uint32_t pa0 = pack_bf16x2(pr[0][0], pr[0][1]);
-    const uint32_t pa2 = pack_bf16x2(pr[1][0], pr[1][1]);
-#pragma unroll
-    for (int nb = 0; nb < 8; ++nb) { o[nb][0] *= alpha; o[nb][1] *= alpha; }
-#pragma unroll
-    for (int dc = 0; dc < 8; dc += 2) {
-      uint32_t b0, b1, b2, b3;
-      // matrices: (keys 0-7, d-chunk dc), (keys 8-15, dc), (keys 0-7, dc+1), (keys 8-15, dc+1)
-      const int vrow = r0 + (lane & 7) + ((lane >> 3) & 1) * 8;
-      const int vcol = dc + (lane >> 4);
-      ldsm_x4_t(vb + swz(vrow, vcol), b0, b1, b2, b3);
-      mma_bf16_16816(o[dc], pa0, 0u, pa2, 0u, b0, b1);
-      mma_bf16_16816(o[dc + 1], pa0, 0u, pa2, 0u, b2, b3);
-    }
-    // Refill the stage consumed in the previous iteration (every warp passed
-    // this iteration's barrier after finishing it).
-    if (c + kStages - 1 < nchunks) load_chunk(c + kStages - 1);
-    cp_async_commit();
-  }
-  cp_async_wait<0>();
-
-  // Per warp: full row sums, then merge the four warps through shared memory.
-  float l_row = l_part + __shfl_xor_sync(0xffffffffu, l_part, 1);
-  l_row += __shfl_xor_sync(0xffffffffu, l_row, 2);
-  if (qrow < NQ) {
-    if ((lane & 3) == 0) {
-      sm_m[warp * 8 + qrow] = m_run;
-      sm_l[warp * 8 + qrow] = l_row;
-    }
-#pragma unroll
-    for (int nb = 0; nb < 8; ++nb) {
-      sm_o[(warp * 8 + qrow) * 64 + nb * 8 + qcol] = o[nb][0];
-      sm_o[(warp * 8 + qrow) * 64 + nb * 8 + qcol + 1] = o[nb][1];
-    }
-  }
-  __syncthreads();   // also orders every ring read of this CTA before the writes below
-  for (int idx = tid; idx < NQ * 64; idx += kRingThreads) {
-    const int qi = idx >> 6, d = idx & 63;
-    float M = -INFINITY;
-#pragma unroll
-    for (int g = 0; g < 4; ++g) M = fmaxf(M, sm_m[g * 8 + qi]);
-    float Lsum = 0.f, acc = 0.f;
-#pragma unroll
-    for (int g = 0; g < 4; ++g) {
-      const float mg = sm_m[g * 8 + qi];
-      if (mg == -INFINITY) continue;
-      const float w = ex2_approx(mg - M);
-      Lsum = fmaf(sm_l[g * 8 + qi], w, Lsum);
-      acc = fmaf(sm_o[(g * 8 + qi) * 64 + d], w, acc);
-    }
-    const __nv_bfloat16 r = __float2bfloat16_rn(acc / Lsum);
-    out[(static_cast<int64_t>(s) * NQ + qi) * HD + h * 64 + d] = *reinterpret_cast<const uint16_t*>(&r);
-  }
-  // Append the new frames: slot (p + t) mod W.
-  for (int idx = tid; idx < NQ * 16; idx += kRingThreads) {
-    const int t = idx >> 4;
-    const int part = (idx >> 3) & 1;   // 0: K, 1: V
-    const int c = idx & 7;
-    const uint16_t* src = newk + static_cast<int64_t>(t) * ld_qkv + part * HD + c * 8;
-    const int dslot = static_cast<int>((p + t) % W);
-    uint16_t* dst = (part ? ring_v : ring_k) + seg + static_cast<int64_t>(dslot) * 64 + c * 8;
-    *reinterpret_cast<uint4*>(dst) = *reinterpret_cast<const uint4*>(src);
-  }
-}
-
-constexpr int kRingSmem = kStages * kStageBytes + (4 * 8 * 2 + 4 * 8 * 64) * 4;
 
 // Grid (frames, S); 256 threads cover H heads x 8 chunks of 16 bytes x {K, V}.
 __global__ void ring_fill_kernel(const uint16_t* __restrict__ qkv, int64_t ld_qkv, int HD,
@@ -531,28 +321,8 @@ template <int NQ>
 cudaError_t launch_ring_tma_nq(const Launch& L, const CUtensorMap& tk, const CUtensorMap& tv, const uint16_t* qkv,
                                int64_t ld_qkv, int HD, uint16_t* rk, uint16_t* rv, const int64_t* pos, int S, int H,
                                int W, uint16_t* out, float sl2) {
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e =
-        cudaFuncSetAttribute(ring_attn_tma_kernel<NQ>, cudaFuncAttributeMaxDynamicSharedMemorySize, kRingTmaSmem);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
   return launch_kernel(ring_attn_tma_kernel<NQ>, dim3(H, S), dim3(kRingTmaThreads), kRingTmaSmem, L.stream, tk, tv,
                        qkv, ld_qkv, HD, rk, rv, pos, H, W, out, sl2, L.status, L.limit_ns);
-}
-
-template <int NQ>
-cudaError_t launch_ring_nq(const Launch& L, const uint16_t* qkv, int64_t ld_qkv, int HD, uint16_t* rk,
-                           uint16_t* rv, const int64_t* pos, int S, int H, int W, uint16_t* out, float sl2) {
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(ring_attn_kernel<NQ>, cudaFuncAttributeMaxDynamicSharedMemorySize, kRingSmem);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
-  return launch_kernel(ring_attn_kernel<NQ>, dim3(H, S), dim3(kRingThreads), kRingSmem, L.stream, qkv, ld_qkv, HD, rk,
-                       rv, pos, H, W, out, sl2);
 }
 
 }  // namespace
@@ -560,30 +330,17 @@ cudaError_t launch_ring_nq(const Launch& L, const uint16_t* qkv, int64_t ld_qkv,
 cudaError_t launch_ring_attn(const Launch& L, const uint16_t* qkv, int64_t ld_qkv, int HD,
                              uint16_t* ring_k, uint16_t* ring_v, const int64_t* pos, int S, int H,
                              int W, int n_new, uint16_t* out, float scale_log2) {
-  if (!ring_tma_disabled()) {
-    // One layer's ring as [S * H * W rows, 64] bf16 tiles of 64 rows.
-    CUtensorMap tk, tv;
-    const uint64_t rows = static_cast<uint64_t>(S) * H * W;
-    if (!tmap_bf16_2d(&tk, ring_k, 64, rows, 64, kChunk) || !tmap_bf16_2d(&tv, ring_v, 64, rows, 64, kChunk))
-      return cudaErrorInvalidValue;
-    switch (n_new) {
+  // One layer's ring as [S * H * W rows, 64] bf16 tiles of 64 rows.
+  CUtensorMap tk, tv;
+  const uint64_t rows = static_cast<uint64_t>(S) * H * W;
+  if (!tmap_bf16_2d(&tk, ring_k, 64, rows, 64, kChunk) || !tmap_bf16_2d(&tv, ring_v, 64, rows, 64, kChunk))
+    return cudaErrorInvalidValue;
+  switch (n_new) {
 #define VX_RING_TMA(n) \
   case n: return launch_ring_tma_nq<n>(L, tk, tv, qkv, ld_qkv, HD, ring_k, ring_v, pos, S, H, W, out, scale_log2);
-      VX_RING_TMA(1) VX_RING_TMA(2) VX_RING_TMA(3) VX_RING_TMA(4)
-      VX_RING_TMA(5) VX_RING_TMA(6) VX_RING_TMA(7) VX_RING_TMA(8)
+    VX_RING_TMA(1) VX_RING_TMA(2) VX_RING_TMA(3) VX_RING_TMA(4)
+    VX_RING_TMA(5) VX_RING_TMA(6) VX_RING_TMA(7) VX_RING_TMA(8)
 #undef VX_RING_TMA
-      default: return cudaErrorInvalidValue;
-    }
-  }
-  switch (n_new) {
-    case 1: return launch_ring_nq<1>(L, qkv, ld_qkv, HD, ring_k, ring_v, pos, S, H, W, out, scale_log2);
-    case 2: return launch_ring_nq<2>(L, qkv, ld_qkv, HD, ring_k, ring_v, pos, S, H, W, out, scale_log2);
-    case 3: return launch_ring_nq<3>(L, qkv, ld_qkv, HD, ring_k, ring_v, pos, S, H, W, out, scale_log2);
-    case 4: return launch_ring_nq<4>(L, qkv, ld_qkv, HD, ring_k, ring_v, pos, S, H, W, out, scale_log2);
-    case 5: return launch_ring_nq<5>(L, qkv, ld_qkv, HD, ring_k, ring_v, pos, S, H, W, out, scale_log2);
-    case 6: return launch_ring_nq<6>(L, qkv, ld_qkv, HD, ring_k, ring_v, pos, S, H, W, out, scale_log2);
-    case 7: return launch_ring_nq<7>(L, qkv, ld_qkv, HD, ring_k, ring_v, pos, S, H, W, out, scale_log2);
-    case 8: return launch_ring_nq<8>(L, qkv, ld_qkv, HD, ring_k, ring_v, pos, S, H, W, out, scale_log2);
     default: return cudaErrorInvalidValue;
   }
 }

@@ -26,17 +26,14 @@ struct Launch {
 
 int current_sm_count();
 uint64_t wait_limit_ns();
-bool pdl_enabled();   // programmatic dependent launch (default on; VX_PDL=0 disables)
-bool pair_gemm_disabled();   // two-CTA GEMM tiles (default on; VX_PAIR_GEMM=0 disables)
-bool tma_store_disabled();   // TMA stores of GEMM outputs (default on; VX_TMA_STORE=0 disables)
-bool ring_tma_disabled();    // TMA-fed ring attention (default on; VX_RING_TMA=0 uses cp.async)
 
 // A kernel launched with more than 48 KB of dynamic shared memory needs
 // cudaFuncAttributeMaxDynamicSharedMemorySize on every device that runs it:
 // sets it once per (kernel, current device).  Thread-safe.
 cudaError_t ensure_dynamic_smem(const void* kernel, size_t smem);
 
-// Launches `k` on `stream`, with programmatic dependent launch when enabled.
+// Launches `k` on `stream` with programmatic dependent launch (the kernel may
+// start while the previous kernel of the stream runs; see pdl_wait()).
 template <class... KArgs, class... Args>
 cudaError_t launch_kernel(void (*k)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
                           Args&&... args) {
@@ -52,9 +49,34 @@ cudaError_t launch_kernel(void (*k)(KArgs...), dim3 grid, dim3 block, size_t sme
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = pdl_enabled() ? 1 : 0;
+  cfg.numAttrs = 1;
   return cudaLaunchKernelEx(&cfg, k, std::forward<Args>(args)...);
 }
+
+// ------------------------------------------------------------- tracing --
+// Every kernel launch goes through traced(): it counts the launches and,
+// while tracing is enabled for the calling thread (vx_trace_enable), brackets
+// them with CUDA events recorded on the launch stream (read by vx_trace_read).
+void count_launches(int n);
+bool trace_enabled();
+cudaEvent_t trace_event();   // from a per-thread pool; null if none could be made
+void trace_record(const char* name, cudaEvent_t a, cudaEvent_t b);
+
+template <class F>
+cudaError_t traced(const Launch& L, const char* name, int kernels, F&& f) {
+  count_launches(kernels);
+  if (!trace_enabled()) return f();
+  cudaEvent_t a = trace_event(), b = trace_event();
+  if (a) cudaEventRecord(a, L.stream);
+  const cudaError_t e = f();
+  if (b) cudaEventRecord(b, L.stream);
+  if (a && b) trace_record(name, a, b);
+  return e;
+}
+
+// Trace name of an RMSNorm / partial-sum reduction launch (static string).
+constexpr int kMaxSplitsTraced = 8;
+const char* rms_trace_name(int nparts, bool h_out, int y_kind /* 0 none, 1 bf16, 2 fp32 */);
 
 // cuTensorMapEncodeTiled through the runtime's driver entry point (no -lcuda).
 bool encode_tmap(CUtensorMap* map, CUtensorMapDataType dt, int rank, const void* base,
@@ -137,11 +159,17 @@ struct AttnArgs {
   DevStatus* status;
   uint64_t limit_ns;
 };
-// tmQ/tmK/tmV: 4-D bf16 maps {64 (d), H, T, B} with box {64, 1, 128, 1}.
-cudaError_t launch_attn_bf16(const Launch& L, const CUtensorMap& tmQ, const CUtensorMap& tmK,
-                             const CUtensorMap& tmV, const AttnArgs& a);
-bool tmap_attn_operand(CUtensorMap* map, const void* base, int B, int T, int H,
-                       int64_t row_stride, int64_t batch_stride);
+// Keys per tile of the bf16 attention kernel.
+constexpr int kAttnKeyTile = 64;
+// q, k, v: bf16 [B, T, H, 64] with element strides row_stride (t) and
+// batch_stride (b) (heads contiguous in 64s); read through 4-D TMA maps.
+struct AttnOperands {
+  const void* q;
+  const void* k;
+  const void* v;
+  int64_t row_stride, batch_stride;
+};
+cudaError_t launch_attn_bf16(const Launch& L, const AttnOperands& op, const AttnArgs& a);
 
 // fp32 CUDA-core sliding-window attention on pre-rotated q, k: [B, T, H, 64].
 cudaError_t launch_attn_f32(const Launch& L, const float* q, const float* k, const float* v,

@@ -3,7 +3,8 @@ allocate device memory (real-time audio callbacks, plug-in hosts that own
 every allocation, fixed memory budgets).  Its scratch is a static device
 array inside libvx; these tests call it through the C ABI and compare it with
 vx_swa_attn_fwd (which uses a caller-supplied workspace) on two calls in a
-row, within the tolerances the other GPU tests use.
+row, and with the float64 oracle, within the tolerances the other GPU tests
+use; they also check both sides of its size limit.
 
 This file is named to be collected last, so a run that stops at the first
 failure has already run every other test."""
@@ -13,6 +14,7 @@ import numpy as np
 import pytest
 import torch
 
+import oracle
 import synth
 from gpu_util import BF16_MAX_ABS, BF16_REL_L2, F32_MAX_ABS, dev, host
 
@@ -33,7 +35,8 @@ def _noalloc(vx, q, k, v, o, window, apply_rope=1, theta=1e6, pos0=0):
 
 
 def _check(got, want, bf16):
-    g, w = host(got), host(want)
+    g = host(got)
+    w = want if isinstance(want, np.ndarray) else host(want)
     err = np.abs(g - w).max()
     if bf16:
         rel = np.linalg.norm(g - w) / np.linalg.norm(w)
@@ -55,6 +58,12 @@ def test_noalloc_matches_workspace_entry_point_on_two_calls(dtype):
         ref = vx.swa_attn_fwd(q, k, v, W, pos0=pos0)
         torch.cuda.synchronize()
         _check(o, ref, bf16)
+        # and against the oracle on sampled rows (the window's edges, the end)
+        rows = sorted({0, 1, W - 1, W, T // 2, T - 1})
+        pos = pos0 + np.arange(T)
+        qh, kh, vh = (host(x) for x in (q, k, v))
+        want = oracle.swa_attention_rows(oracle.rope(qh, pos, 1e6), oracle.rope(kh, pos, 1e6), vh, W, rows)
+        _check(o[:, rows], want, bf16)
 
 
 def test_noalloc_without_rope_and_repeat_is_deterministic():
@@ -70,13 +79,31 @@ def test_noalloc_without_rope_and_repeat_is_deterministic():
     _check(a, ref, True)
 
 
-def test_noalloc_rejects_sizes_beyond_its_static_scratch():
+def test_noalloc_size_limit_both_sides():
+    # bf16 with RoPE: 2 * roundup256(B*T*H*128) + T*256 <= 32 MiB, i.e.
+    # B*T*H + T <= 131072 for even B*T*H.  B=1, H=32: T = 3971 fits
+    # (33 * 3971 = 131043), T = 3972 does not (131076).
     vx = _lib()
-    # bf16: B*T*H must stay <= 131072; 2 x 4096 x 32 = 262144 is too large
-    q = torch.zeros(2, 4096, 32, 64, dtype=torch.bfloat16, device="cuda")
+    H, W = 32, 750
+    q, k, v = synth.attention_qkv(1, 3972, H, 64, seed=9, bf16=True)
+    q, k, v = (dev(x, torch.bfloat16) for x in (q, k, v))
     o = torch.empty_like(q)
-    assert _noalloc(vx, q, q, q, o, 750) == 1
+    assert _noalloc(vx, q, k, v, o, W) == 1
     assert b"static limit" in vx.lib.vx_last_error()
-    # without RoPE it needs no scratch and runs
-    assert _noalloc(vx, q, q, q, o, 750, apply_rope=0) == 0
+    qs, ks, vs = (x[:, :3971].contiguous() for x in (q, k, v))
+    os_ = torch.empty_like(qs)
+    assert _noalloc(vx, qs, ks, vs, os_, W) == 0, vx.lib.vx_last_error()
+    ref = vx.swa_attn_fwd(qs, ks, vs, W)
+    torch.cuda.synchronize()
+    _check(os_, ref, True)
+    # without RoPE it needs no scratch beyond the status word and runs at any size
+    q2 = torch.zeros(2, 4096, 32, 64, dtype=torch.bfloat16, device="cuda")
+    o2 = torch.empty_like(q2)
+    assert _noalloc(vx, q2, q2, q2, o2, 750, apply_rope=0) == 0
+    # fp32 with RoPE: 2 * B*T*H + T <= 131072; B=1, H=16: T = 3971 fits, 3972 does not
+    qf = torch.zeros(1, 3972, 16, 64, dtype=torch.float32, device="cuda")
+    of = torch.empty_like(qf)
+    assert _noalloc(vx, qf, qf, qf, of, 750) == 1
+    qf2 = qf[:, :3971].contiguous()
+    assert _noalloc(vx, qf2, qf2, qf2, torch.empty_like(qf2), 750) == 0, vx.lib.vx_last_error()
     torch.cuda.synchronize()
