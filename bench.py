@@ -3,27 +3,39 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl vx|reference]
 
-Workload (one "step"): one full encoder layer over one clip of 1500 frames
-(d 1280, 32 heads x 64, SwiGLU 5120, causal window 750, RoPE theta 1e6), bf16
-operands with fp32 accumulation and an fp32 residual stream: RMSNorm -> QKV
-GEMM + RoPE -> sliding-window attention -> O-proj + residual -> RMSNorm ->
-gate/up GEMM + SwiGLU -> down GEMM + residual, all in libvx's sm_100a kernels.
-Inputs are synthetic and seeded, resident in HBM before the timed region; L2
-is flushed (a 256 MiB write) between timed steps, outside the step's events.
+Workload (one "step"): the full streaming encoder forward of 4 clips of 6000
+log-mel frames (128 bins, values ~ N(0,1)): the causal conv stem (Conv1d
+128->1280 k3 s1 + GELU, Conv1d 1280->1280 k3 s2 + GELU, left padding only,
+6000 -> 3000 frames), 32 encoder layers (d_model 1280, 32 heads x 64, SwiGLU
+5120, causal window 750, RoPE theta 1e6; RMSNorm -> QKV GEMM + RoPE ->
+sliding-window attention -> O-proj + residual -> RMSNorm -> gate/up GEMM +
+SwiGLU -> down GEMM + residual) and the final RMSNorm, through the public call
+vx_encoder_fwd: bf16 operands, fp32 accumulation and residual stream, every
+step in libvx's sm_100a kernels.  Weights are random with the distributions
+of the synthetic workload (projection/conv weights N(0, 0.02), biases
+N(0, 0.01), gains 1 + N(0, 0.02)); inputs are resident in HBM before the
+timed region; L2 is flushed (a 256 MiB write) between timed steps, outside
+the step's events (the 1.93 GB of layer weights exceed L2 anyway).
 
-`value` is encoder frames/s over all ranks (each rank runs an independent
-replica: the path shards by clip with no collective).  `e2e` repeats the
-measurement through the same public call with the input copied from pinned
-host memory and the output copied back inside the timed region.
-`roofline` reports the dominant kernel, timed live with CUDA events on its
-launch stream (libvx's trace mode).  On one GPU the line also carries
-`components`: the attention-only sweep (TFLOP/s), the 32-layer streaming step
-(GB/s) and the full 32-layer encoder (frames/s).  `cpu_baseline` times the
-float64 oracle on this host's cores on a bounded sample of the same workload.
+`value` is encoder frames/s (3000 output frames per clip) over all ranks: each
+rank runs an independent replica (the path shards by clip with no
+collective).  `e2e` repeats the measurement through the same public call with
+the mel input copied from pinned host memory and the encoder output copied
+back inside the timed region.  `roofline` reports the dominant kernel of the
+step, timed live with CUDA events on its launch stream (libvx's trace mode).
+`cpu_baseline` times the float64 oracle on this host's cores on a bounded
+sample of the same workload (the stem and two of the 32 layers of one clip,
+the forward extrapolated).  On one GPU the line also carries `components`:
+one encoder layer (1 x 1500 frames), the tiny fp32 attention case, the
+attention-only sweep (8 x {1500, 3000, 6000} frames, with the tile-skip
+ratio), the 32-layer 64-stream streaming step, and the widened rows (conv-stem
+step, projector, log-mel frontend, the 312-mel first chunk and the steady
+8-mel chunk of the streaming mode); each carries the oracle timed on a
+bounded sample beside it.
 
-`--impl reference` times that oracle alone (the reference arm of this build:
-the pages ship no runnable reference), printing the same line with
-"impl": "reference".
+`--impl reference` times the oracle alone on the same workload (the reference
+arm of this build: the pages ship no runnable reference), printing the same
+line with "impl": "reference".
 """
 from __future__ import annotations
 
@@ -32,10 +44,10 @@ import datetime
 import hashlib
 import json
 import os
+import re
 import subprocess
 import sys
 import tempfile
-import threading
 import time
 
 import numpy as np
@@ -45,21 +57,25 @@ sys.path.insert(0, ROOT)
 
 METRIC = "encoder frames/sec (1 B200); SWA TFLOP/s & % bf16 peak; stream-step GB/s"
 UNIT = "frames/s"
+C4 = dict(B=4, n_mels=128, Tm=6000, To=3000, d=1280, H=32, D=64, F=5120, W=750, L=32)
 C1 = dict(B=1, T=1500, d=1280, H=32, D=64, F=5120, W=750)
-WORKLOAD = ("one encoder layer (C1): B=1 clip x T=1500 frames, d_model 1280, 32 heads x 64, SwiGLU 5120, "
-            "causal window 750, RoPE theta 1e6; bf16 operands, fp32 accumulate and residual")
+WORKLOAD = ("streaming encoder forward: B=4 clips x 6000 log-mel frames (128 bins) -> causal conv stem -> "
+            "3000 frames -> 32 encoder layers (d_model 1280, 32 heads x 64, SwiGLU 5120, causal window 750, "
+            "RoPE theta 1e6) -> final RMSNorm; bf16 operands, fp32 accumulate and residual")
 L2_FLUSH_BYTES = 256 << 20
+PEAK_KIND = "fallback"   # "measured" once MEASURED_PEAKS.json has been read
 
 
 def parse_args(argv=None):
     ap = argparse.ArgumentParser(description="Voxtral Realtime encoder hot-path benchmark")
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=2000)
-    ap.add_argument("--warmup", type=int, default=50)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=("vx", "reference"), default="vx")
-    ap.add_argument("--no-components", action="store_true", help="skip the C2/C3/C4 component timings")
+    ap.add_argument("--no-components", action="store_true", help="skip the component timings")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--components-only", default="", help="comma list of c0,c2,c3,c4,next (profiling runs)")
+    ap.add_argument("--no-oracle", action="store_true", help="skip the components' oracle timings")
+    ap.add_argument("--components-only", default="", help="comma list of c0,c1,c2,c3,next (profiling runs)")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-copy end-to-end pass (profiling runs)")
     ap.add_argument("--no-trace", action="store_true", help="skip the traced per-kernel pass (profiling runs)")
     ap.add_argument("--c3-layers", type=int, default=32, help="layers of the streaming-step component (profiling runs)")
@@ -151,36 +167,7 @@ class ClockSampler:
                 "reasons": reasons, "samples": len(inside)}
 
 
-# ---------------------------------------------------------------- workload
-
-def make_layer(vx, torch, seed=1, device="cuda"):
-    """Random-init bf16 layer weights of the C1 shape (synth distributions), packed."""
-    import synth
-    cfg = vx.VOXTRAL_RT
-    p = synth.layer_params(synth.VOXTRAL_RT, seed=seed)
-    t = {k: (None if v is None else torch.from_numpy(v).to(device).to(torch.bfloat16)) for k, v in p.items()}
-    return cfg, vx.pack_layer(cfg, t)
-
-
-def device_layers(vx, torch, n, seed, device):
-    """n layers drawn on the device (torch RNG; distributions of synth.layer_params)."""
-    cfg = vx.VOXTRAL_RT
-    g = torch.Generator(device=device).manual_seed(seed)
-    d, hd, f = cfg.d_model, cfg.hd, cfg.ffn_hidden
-
-    def nrm(shape, std, mean=0.0):
-        return (torch.randn(shape, generator=g, device=device) * std + mean).to(torch.bfloat16)
-
-    layers = []
-    for _ in range(n):
-        p = {"attn_norm_g": nrm((d,), 0.02, 1.0), "wq": nrm((hd, d), 0.02), "wk": nrm((hd, d), 0.02),
-             "wv": nrm((hd, d), 0.02), "bq": nrm((hd,), 0.01), "bv": nrm((hd,), 0.01),
-             "wo": nrm((d, hd), 0.02), "bo": nrm((d,), 0.01), "ffn_norm_g": nrm((d,), 0.02, 1.0),
-             "wg": nrm((f, d), 0.02), "wu": nrm((f, d), 0.02), "wd": nrm((d, f), 0.02), "bd": nrm((d,), 0.01),
-             "bg": None, "bu": None}
-        layers.append(vx.pack_layer(cfg, p))
-    return cfg, layers
-
+# ------------------------------------------------------- algorithmic work
 
 def gemm_flops(M, d=1280, hd=2048, F=5120):
     return {"gemm_qkv_rope": 2 * M * d * 3 * hd, "gemm_o_residual": 2 * M * hd * d,
@@ -200,15 +187,51 @@ def layer_flops(B, T, W=750):
     return sum(gemm_flops(M).values()) + attn_flops(B, T, 32, 64, W)
 
 
-def kernel_work(name, B, T):
-    """(amount, unit, bound) of algorithmic work of one launch in the C1 layer."""
-    M = B * T
-    if name in gemm_flops(M):
+def stem_flops(B, Tm, n_mels=128, d=1280):
+    To = (Tm - 1) // 2 + 1
+    return {"gemm_conv1_gelu": 2 * B * Tm * d * 3 * n_mels, "gemm_conv2_gelu": 2 * B * To * d * 3 * d}
+
+
+def encoder_flops(B=4, Tm=6000, L=32):
+    To = (Tm - 1) // 2 + 1
+    return sum(stem_flops(B, Tm).values()) + L * layer_flops(B, To)
+
+
+def attn_tiles(T, W, tile=128):
+    """Key tiles of 128 the attention kernel visits for one (clip, head), the
+    tiles of the full causal square (query tile x key tile, key <= query), and
+    the fraction of the visited tiles' 128 x 128 scores that are attended
+    pairs: the kernel visits, for query tile q0 .. q0+127, key tiles
+    floor(max(0, q0 - W + 1) / 128) .. floor(min(T - 1, q0 + 127) / 128)."""
+    nqt = (T + tile - 1) // tile
+    visited = 0
+    for qt in range(nqt):
+        q0 = qt * tile
+        visited += min(T - 1, q0 + tile - 1) // tile - max(0, q0 - W + 1) // tile + 1
+    causal = nqt * (nqt + 1) // 2
+    return {"visited": visited, "causal_tiles": causal, "all_tiles": nqt * nqt,
+            "useful_frac": attended_pairs(T, W) / (visited * tile * tile)}
+
+
+_RMS = re.compile(r"rmsnorm_p(\d+)(_h)?(_y16|_y32)?$")
+
+
+def kernel_work(name, wl):
+    """(amount, unit, bound) of algorithmic work of one launch named `name` in
+    the workload wl = {"M": layer rows, "attn": (B, T, H, W), "stem": (B, Tm)}."""
+    M = wl.get("M")
+    if M and name in gemm_flops(M):
         return gemm_flops(M)[name], "flop", "tensor"
-    if name == "swa_attn_tc":
-        return attn_flops(B, T, 32, 64, 750), "flop", "tensor"
-    if name == "rmsnorm":
-        return M * 1280 * (4 + 2) + 1280 * 2, "byte", "hbm"
+    if wl.get("stem") and name in stem_flops(*wl["stem"]):
+        return stem_flops(*wl["stem"])[name], "flop", "tensor"
+    if name == "swa_attn_tc" and wl.get("attn"):
+        B, T, H, W = wl["attn"]
+        return attn_flops(B, T, H, 64, W), "flop", "tensor"
+    m = _RMS.match(name)
+    if m and M:
+        # x read, the partial sums read, h written (_h), the normalised output written
+        per = 4 + 4 * int(m.group(1)) + (4 if m.group(2) else 0) + {"_y16": 2, "_y32": 4, None: 0}[m.group(3)]
+        return M * 1280 * per + 1280 * 2, "byte", "hbm"
     return None, None, None
 
 
@@ -220,9 +243,16 @@ def src_digest(*names):
     return h.hexdigest()[:16]
 
 
-KERNEL_SRC = {"gemm_qkv_rope": ("gemm.cu", "vx_common.cuh"), "gemm_o_residual": ("gemm.cu", "vx_common.cuh"),
-              "gemm_gate_up_swiglu": ("gemm.cu", "vx_common.cuh"), "gemm_down_residual": ("gemm.cu", "vx_common.cuh"),
-              "swa_attn_tc": ("attn.cu", "vx_common.cuh"), "rmsnorm": ("misc.cu",), "ring_attn": ("stream.cu",)}
+def _kernel_src(name):
+    if name.startswith("gemm_"):
+        return ("gemm.cu", "vx_common.cuh")
+    if name == "swa_attn_tc":
+        return ("attn.cu", "vx_common.cuh")
+    if name.startswith("rmsnorm"):
+        return ("misc.cu",)
+    if name == "ring_attn":
+        return ("stream.cu",)
+    return ()
 
 
 def ncu_traffic(kernel, workload):
@@ -235,7 +265,8 @@ def ncu_traffic(kernel, workload):
     except (OSError, ValueError):
         return None
     e = db.get(f"{kernel}@{workload}")
-    if not e or e.get("src") != src_digest(*KERNEL_SRC.get(kernel, ())):
+    src = _kernel_src(kernel)
+    if not e or not src or e.get("src") != src_digest(*src):
         return None
     return e.get("dram_bytes_per_launch")
 
@@ -247,6 +278,39 @@ def peaks():
         return p["hbm_gbs"], p["bf16_tflops"], p.get("bf16_tflops_sustained", p["bf16_tflops"]), "measured"
     except (OSError, ValueError, KeyError):
         return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+def roofline(tr, wl, tf, hbm, peak_kind, workload_key, peak_note):
+    """Roofline entry of the kernel with the largest time per step in trace tr."""
+    dom = max(tr, key=lambda k: tr[k]["ms_per_step"])
+    work, wunit, bound = kernel_work(dom, wl)
+    if work is None:
+        roof = {"bound": None, "achieved": None, "peak": None, "unit": None, "frac": None}
+    elif bound == "tensor":
+        achieved = work / (tr[dom]["ms_per_launch"] / 1e3) / 1e12
+        roof = {"bound": "tensor", "achieved": achieved, "peak": tf, "unit": "TFLOP/s", "frac": achieved / tf,
+                "peak_kind": f"{peak_kind} bf16 dense ({peak_note})"}
+    else:
+        achieved = work / (tr[dom]["ms_per_launch"] / 1e3) / 1e9
+        roof = {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
+                "peak_kind": f"{peak_kind} HBM copy"}
+    roof.update({"kernel": dom, "work_per_launch": work, "work_unit": wunit,
+                 "ms_per_launch": tr[dom]["ms_per_launch"], "launches_per_step": tr[dom]["launches_per_step"],
+                 "share_of_step": tr[dom]["ms_per_step"] / sum(v["ms_per_step"] for v in tr.values()),
+                 "traffic": ncu_traffic(dom, workload_key)})
+    return roof
+
+
+def per_kernel_table(tr, wl):
+    out = {}
+    for k, v in tr.items():
+        e = {"ms_per_launch": v["ms_per_launch"], "launches_per_step": v["launches_per_step"],
+             "ms_per_step": v["ms_per_step"]}
+        w, u, b = kernel_work(k, wl)
+        if w is not None:
+            e["tflops" if u == "flop" else "gbs"] = w / (v["ms_per_launch"] / 1e3) / (1e12 if u == "flop" else 1e9)
+        out[k] = e
+    return out
 
 
 # -------------------------------------------------------------- timed loops
@@ -275,28 +339,104 @@ def traced_kernels(vx, torch, step, K, flush):
         for _ in range(K):
             flush()
             step()
-            buf = ctypes.create_string_buffer(1 << 16)
+            buf = ctypes.create_string_buffer(1 << 18)
             vx.lib.vx_trace_read(buf, len(buf))
             for line in buf.value.decode().splitlines():
                 name, ms = line.rsplit(" ", 1)
                 acc.setdefault(name, []).append(float(ms))
     finally:
         vx.lib.vx_trace_enable(0)
-    # launches per step of each name -> mean per launch and per step
     return {k: {"ms_per_launch": float(np.mean(v)), "launches_per_step": len(v) / K,
                 "ms_per_step": float(np.sum(v)) / K} for k, v in acc.items()}
 
 
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        return max(i.get("num_threads", 1) for i in threadpool_info()) or os.cpu_count()
+    except Exception:
+        return os.cpu_count()
+
+
+def _clock(fn):
+    t = time.perf_counter()
+    fn()
+    return time.perf_counter() - t
+
+
+# ----------------------------------------------------------------- weights
+
+def device_layers(vx, torch, n, seed, device):
+    """n layers drawn on the device (torch RNG; distributions of synth.layer_params), packed."""
+    cfg = vx.VOXTRAL_RT
+    g = torch.Generator(device=device).manual_seed(seed)
+    d, hd, f = cfg.d_model, cfg.hd, cfg.ffn_hidden
+
+    def nrm(shape, std, mean=0.0):
+        return (torch.randn(shape, generator=g, device=device) * std + mean).to(torch.bfloat16)
+
+    layers = []
+    for _ in range(n):
+        p = {"attn_norm_g": nrm((d,), 0.02, 1.0), "wq": nrm((hd, d), 0.02), "wk": nrm((hd, d), 0.02),
+             "wv": nrm((hd, d), 0.02), "bq": nrm((hd,), 0.01), "bv": nrm((hd,), 0.01),
+             "wo": nrm((d, hd), 0.02), "bo": nrm((d,), 0.01), "ffn_norm_g": nrm((d,), 0.02, 1.0),
+             "wg": nrm((f, d), 0.02), "wu": nrm((f, d), 0.02), "wd": nrm((d, f), 0.02), "bd": nrm((d,), 0.01),
+             "bg": None, "bu": None}
+        layers.append(vx.pack_layer(cfg, p))
+    return cfg, layers
+
+
+def device_stem(vx, torch, seed, device):
+    """Packed conv-stem weights and the final norm gain, drawn on the device."""
+    g = torch.Generator(device=device).manual_seed(seed)
+
+    def nrm(shape, std, mean=0.0):
+        return (torch.randn(shape, generator=g, device=device) * std + mean).to(torch.bfloat16)
+
+    w1p = vx.pack_conv_weight(nrm((1280, 128, 3), 0.02))
+    w2p = vx.pack_conv_weight(nrm((1280, 1280, 3), 0.02))
+    return w1p, nrm((1280,), 0.01), w2p, nrm((1280,), 0.01), nrm((1280,), 0.02, 1.0)
+
+
 # ------------------------------------------------------------- components
 
-def component_c0(vx, torch, flush, hbm, tf):
+def component_c1(vx, torch, flush, hbm, tf, oracle_on):
+    """One encoder layer over 1 clip x 1500 frames (vx_encoder_layer_fwd)."""
+    cfg, (L,) = device_layers(vx, torch, 1, 100, "cuda")
+    g = torch.Generator(device="cuda").manual_seed(101)
+    x = torch.randn(1, 1500, 1280, generator=g, device="cuda")
+    y = torch.empty_like(x)
+    ws = vx.Workspace(vx.lib.vx_encoder_layer_workspace(__import__("ctypes").byref(cfg.c()), 1, 1500))
+    step = lambda: vx.encoder_layer_fwd(cfg, L, x, out=y, ws=ws)
+    for _ in range(20):
+        step()
+    ms, _, _ = timed_steps(torch, step, 200, flush, torch.cuda.current_stream())
+    tr = traced_kernels(vx, torch, step, 50, flush)
+    wl = {"M": 1500, "attn": (1, 1500, 32, 750)}
+    fl = layer_flops(1, 1500)
+    out = {"ms_per_step": ms, "frames_per_s": 1500 / ms * 1e3, "tflops": fl / ms / 1e9,
+           "frac_of_measured_peak": fl / ms / 1e9 / tf,
+           "roofline": roofline(tr, wl, tf, hbm, PEAK_KIND, "C1", "burst"),
+           "kernels": per_kernel_table(tr, wl)}
+    if oracle_on:
+        import oracle
+        import synth
+        p = synth.layer_params(synth.VOXTRAL_RT, seed=1)
+        xs = synth.frames(1, 1500, 1280, seed=2)
+        t = _clock(lambda: oracle.encoder_layer(xs, p, synth.VOXTRAL_RT))
+        out["oracle"] = {"frames_per_s": 1500 / t, "s": t, "cores": blas_threads(),
+                         "sample": "one full layer over 1 x 1500 frames, float64 numpy oracle"}
+    return out
+
+
+def component_c0(vx, torch, flush, hbm, tf, oracle_on):
     """The tiny fp32 case: q, k, v [1, 64, 2, 64] (seed 0, drawn in that order),
     window 16, RoPE theta 1e6 at pos0 0, through the public fp32 attention call
     (RoPE kernel + CUDA-core attention kernel); latency per call, L2 flushed
     between calls outside the events."""
     import synth
-    q, k, v = (torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32)).cuda()
-               for a in synth.attention_qkv(1, 64, 2, 64, seed=0))
+    qkv = synth.attention_qkv(1, 64, 2, 64, seed=0)
+    q, k, v = (torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32)).cuda() for a in qkv)
     o = torch.empty_like(q)
     ws = vx.Workspace(vx.lib.vx_swa_attn_workspace(0, 1, 64, 2, 64, 1))
     step = lambda: vx.swa_attn_fwd(q, k, v, 16, apply_rope=True, rope_theta=1e6, pos0=0, out=o, ws=ws)
@@ -305,11 +445,19 @@ def component_c0(vx, torch, flush, hbm, tf):
     ms, _, _ = timed_steps(torch, step, 200, flush, torch.cuda.current_stream())
     tr = traced_kernels(vx, torch, step, 20, flush)
     fl = attn_flops(1, 64, 2, 64, 16)
-    return {"us_per_call": ms * 1e3, "kernels_us": {k2: v2["ms_per_launch"] * 1e3 for k2, v2 in tr.items()},
-            "mflop": fl / 1e6, "note": "launch-latency bound: 0.46 MFLOP"}
+    out = {"us_per_call": ms * 1e3, "kernels_us": {k2: v2["ms_per_launch"] * 1e3 for k2, v2 in tr.items()},
+           "mflop": fl / 1e6, "note": "launch-latency bound: 0.46 MFLOP"}
+    if oracle_on:
+        import oracle
+        pos = np.arange(64)
+        t = min(_clock(lambda: oracle.swa_attention(oracle.rope(qkv[0], pos, 1e6), oracle.rope(qkv[1], pos, 1e6),
+                                                    qkv[2], 16)) for _ in range(5))
+        out["oracle"] = {"us_per_call": t * 1e6, "cores": blas_threads(),
+                         "sample": "the whole case (RoPE + attention), float64 numpy oracle, best of 5"}
+    return out
 
 
-def component_c2(vx, torch, flush, hbm, tf):
+def component_c2(vx, torch, flush, hbm, tf, oracle_on):
     out = {}
     g = torch.Generator(device="cuda").manual_seed(20)
     for T in (1500, 3000, 6000):
@@ -323,24 +471,44 @@ def component_c2(vx, torch, flush, hbm, tf):
         ms, _, _ = timed_steps(torch, step, 10, flush, torch.cuda.current_stream())
         fl = attn_flops(8, T, 32, 64, 750)
         ka = tr["swa_attn_tc"]["ms_per_launch"]
-        out[f"T{T}"] = {"ms_per_call": ms, "attn_kernel_ms": ka, "rope_ms": tr.get("rope", {}).get("ms_per_step"),
-                        "gflop": fl / 1e9, "kernel_tflops": fl / ka / 1e9, "kernel_frac_of_measured_peak": fl / ka / 1e9 / tf,
-                        "call_tflops": fl / ms / 1e9}
+        e = {"ms_per_call": ms, "attn_kernel_ms": ka, "rope_ms": tr.get("rope", {}).get("ms_per_step"),
+             "gflop": fl / 1e9, "kernel_tflops": fl / ka / 1e9, "kernel_frac_of_measured_peak": fl / ka / 1e9 / tf,
+             "call_tflops": fl / ms / 1e9, "tiles_per_clip_head": attn_tiles(T, 750)}
+        if oracle_on:
+            import oracle
+            qh, kh, vh = (x[:1].float().cpu().numpy() for x in (q, k, v))
+            rows = list(range(T - 16, T))   # rows with full 750-key windows: the per-row cost of most rows
+            pos = np.arange(T)
+            t = _clock(lambda: oracle.swa_attention_rows(oracle.rope(qh, pos, 1e6), oracle.rope(kh, pos, 1e6),
+                                                         vh, 750, rows))
+            rows_all = 8 * T
+            e["oracle"] = {"s_per_call_extrapolated": t / 16 * rows_all, "tflops": fl / (t / 16 * rows_all) / 1e12,
+                           "cores": blas_threads(),
+                           "sample": f"16 query rows of clip 0 (all 32 heads, full 750-key windows, RoPE of the "
+                                     f"clip included) timed, extrapolated to the {rows_all} rows of the call"}
+        out[f"T{T}"] = e
         del q, k, v, o, ws
     return out
 
 
-def component_c3(vx, torch, flush, hbm, tf, L=32):
+def component_c3(vx, torch, flush, hbm, tf, oracle_on, L=32):
+    """The 32-layer streaming step of 64 streams x 4 new frames over a ring
+    filled by vx_stream_prefill from 1000 frames per stream (wrapped)."""
     cfg, layers = device_layers(vx, torch, L, 300, "cuda")
     S, n, P = 64, 4, 1000
     ring = vx.KVRing(cfg, L, S)
     g = torch.Generator(device="cuda").manual_seed(301)
-    ring.k.normal_(generator=g)
-    ring.v.normal_(generator=g)
-    ring.pos.fill_(P)
+    xp = torch.randn(S, P, cfg.d_model, generator=g, device="cuda")
+    wsp = vx.Workspace()
+    vx.stream_prefill(cfg, layers, ring, xp, ws=wsp)
+    torch.cuda.synchronize()
+    del xp, wsp
+    torch.cuda.empty_cache()
     x = torch.randn(S, n, cfg.d_model, generator=g, device="cuda")
     y = torch.empty_like(x)
     ws = vx.Workspace(vx.lib.vx_stream_step_workspace(__import__("ctypes").byref(cfg.c()), S, n))
+    # Every step appends 4 frames per stream (pos 1000, 1004, ...): the ring
+    # stays full, so every step moves the same bytes.
     step = lambda: vx.stream_step(cfg, layers, ring, x, out=y, ws=ws)
     for _ in range(3):
         step()
@@ -365,36 +533,28 @@ def component_c3(vx, torch, flush, hbm, tf, L=32):
     ring_ms = tr["ring_attn"]["ms_per_launch"]
     ring_bytes = (749 + 4) * 64 * 2 * 2 * 32 * S + 4 * 64 * 2 * 2 * 32 * S
     del gr
-    return {"ms_per_step_eager": ms, "ms_per_step_graph": ms_g, "bytes_per_step": total,
-            "gbs_graph": total / ms_g / 1e6, "frac_of_measured_hbm": total / ms_g / 1e6 / hbm,
-            "frames_per_s_graph": S * n / ms_g * 1e3,
-            "ring_attn_ms_per_launch": ring_ms, "ring_attn_gbs": ring_bytes / ring_ms / 1e6,
-            "kernel_ms_per_step": {k: v["ms_per_step"] for k, v in tr.items()}}
-
-
-def component_c4(vx, torch, flush, hbm, tf):
-    cfg, layers = device_layers(vx, torch, 32, 400, "cuda")
-    g = torch.Generator(device="cuda").manual_seed(401)
-
-    def nrm(shape, std):
-        return (torch.randn(shape, generator=g, device="cuda") * std).to(torch.bfloat16)
-
-    w1p = vx.pack_conv_weight(nrm((1280, 128, 3), 0.02))
-    w2p = vx.pack_conv_weight(nrm((1280, 1280, 3), 0.02))
-    b1, b2, fg = nrm((1280,), 0.01), nrm((1280,), 0.01), (1 + nrm((1280,), 0.02).float()).to(torch.bfloat16)
-    mel = torch.randn(4, 128, 6000, generator=g, device="cuda")
-    out = torch.empty(4, 3000, 1280, device="cuda")
-    ws = vx.Workspace(vx.lib.vx_encoder_workspace(__import__("ctypes").byref(cfg.c()), 4, 128, 6000))
-    step = lambda: vx.encoder_fwd(cfg, mel, w1p, b1, w2p, b2, layers, fg, out=out, ws=ws)
-    for _ in range(2):
-        step()
-    tr = traced_kernels(vx, torch, step, 2, lambda: None)
-    ms, _, _ = timed_steps(torch, step, 5, lambda: None, torch.cuda.current_stream())
-    stem = 2 * 4 * 6000 * 1280 * 128 * 3 + 2 * 4 * 3000 * 1280 * 1280 * 3
-    fl = stem + 32 * layer_flops(4, 3000)
-    return {"ms_per_forward": ms, "frames_per_s": 12000 / ms * 1e3, "tflop_per_forward": fl / 1e12,
-            "tflops": fl / ms / 1e9, "frac_of_measured_peak": fl / ms / 1e9 / tf,
-            "kernel_ms_per_forward": {k: v["ms_per_step"] for k, v in tr.items()}}
+    wl = {"M": S * n}
+    out = {"ms_per_step_eager": ms, "ms_per_step_graph": ms_g, "bytes_per_step": total,
+           "gbs_graph": total / ms_g / 1e6, "frac_of_measured_hbm": total / ms_g / 1e6 / hbm,
+           "frames_per_s_graph": S * n / ms_g * 1e3,
+           "ring_attn_ms_per_launch": ring_ms, "ring_attn_gbs": ring_bytes / ring_ms / 1e6,
+           "ring_fill": "vx_stream_prefill over 1000 frames per stream (ring wrapped), then steps at pos 1000, 1004, ...",
+           "kernels": per_kernel_table(tr, wl)}
+    if oracle_on:
+        import oracle
+        import synth
+        dims = synth.VOXTRAL_RT
+        lp = [synth.layer_params(dims, seed=synth.layer_seed(1, l)) for l in range(L)]
+        ns = 2
+        rings = [synth.ring_kv(ns, dims.n_heads, dims.window, dims.head_dim, seed=1000 + l) for l in range(L)]
+        xs = synth.frames(ns, n, 1280, seed=3)
+        t = _clock(lambda: oracle.stream_step(xs, lp, dims, rings, np.full(ns, P)))
+        out["oracle"] = {"ms_per_step_extrapolated": t / ns * S * 1e3, "frames_per_s": ns * n / t,
+                         "cores": blas_threads(),
+                         "sample": f"the oracle streaming step (32 layers, ring at pos 1000) for {ns} of the 64 "
+                                   f"streams, extrapolated to 64 (streams are independent)"}
+    del ring
+    return out
 
 
 # Log-mel frontend arithmetic per 10 ms frame: window (400 mul), the 201-bin
@@ -405,19 +565,22 @@ LOG_MEL_FLOP_PER_FRAME = 400 + 201 * 400 * 4 + 201 * 3 + 128 * 201 * 2
 FP32_ALU_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
 
 
-def component_next(vx, torch, flush, hbm, tf):
+def component_next(vx, torch, flush, hbm, tf, oracle_on):
     """The widened rows: the streaming conv-stem step (64 streams x 8 mel frames
     -> 4 frames, warm padding cache), the audio projector on the encoder
-    output of the 4 x 6000-mel workload ([4, 3000, 1280] -> [4, 750, 3072])
-    and the log-mel frontend producing that workload's input (4 x 60 s)."""
+    output of the 4 x 6000-mel workload ([4, 3000, 1280] -> [4, 750, 3072]),
+    the log-mel frontend producing that workload's input (4 x 60 s), and the
+    streaming mode of the Core AI card (section "Streaming"): the batched
+    first chunk of 312 mel frames (log-mel -> conv stem -> 32-layer prefill
+    that fills the ring: the time to first token's encoder part) and the
+    steady 8-mel chunk (log-mel -> conv-stem step -> 32-layer streaming step
+    -> projector of the 4 new frames into one audio token), for 64 streams."""
     g = torch.Generator(device="cuda").manual_seed(501)
 
     def nrm(shape, std):
         return (torch.randn(shape, generator=g, device="cuda") * std).to(torch.bfloat16)
 
-    w1p = vx.pack_conv_weight(nrm((1280, 128, 3), 0.02))
-    w2p = vx.pack_conv_weight(nrm((1280, 1280, 3), 0.02))
-    b1, b2 = nrm((1280,), 0.01), nrm((1280,), 0.01)
+    w1p, b1, w2p, b2, fg = device_stem(vx, torch, 502, "cuda")
     S = 64
     cache = vx.ConvCache(S, 128, 1280)
     mel = torch.randn(S, 128, 8, generator=g, device="cuda")
@@ -429,12 +592,12 @@ def component_next(vx, torch, flush, hbm, tf):
     ms_c, _, _ = timed_steps(torch, step, 50, lambda: None, torch.cuda.current_stream())
     conv_flop = 2 * S * 8 * 1280 * 128 * 3 + 2 * S * 4 * 1280 * 1280 * 3
     conv_bytes = (1280 * 128 * 3 + 1280 * 1280 * 3) * 2 + S * 128 * 8 * 4 + S * 4 * 1280 * 4
-    w1 = nrm((3072, 5120), 0.02)
-    w2 = nrm((3072, 3072), 0.02)
+    pw1 = nrm((3072, 5120), 0.02)
+    pw2 = nrm((3072, 3072), 0.02)
     x = torch.randn(4, 3000, 1280, generator=g, device="cuda")
     out = torch.empty(4, 750, 3072, device="cuda")
     wsp = vx.Workspace(vx.lib.vx_projector_workspace(4, 3000, 1280, 3072))
-    proj = lambda: vx.projector_fwd(x, w1, w2, out=out, ws=wsp)
+    proj = lambda: vx.projector_fwd(x, pw1, pw2, out=out, ws=wsp)
     for _ in range(3):
         proj()
     ms_p, _, _ = timed_steps(torch, proj, 20, flush, torch.cuda.current_stream())
@@ -446,72 +609,127 @@ def component_next(vx, torch, flush, hbm, tf):
     for _ in range(3):
         lm()
     ms_m, _, _ = timed_steps(torch, lm, 20, flush, torch.cuda.current_stream())
-    return {"conv_step_64x8": {"ms_per_step": ms_c, "frames_per_s": S * 4 / ms_c * 1e3,
-                               "gbs": conv_bytes / ms_c / 1e6, "tflops": conv_flop / ms_c / 1e9},
-            "log_mel_4x60s": {"ms_per_call": ms_m, "mel_frames_per_s": 24000 / ms_m * 1e3,
-                              "gbs": (4 * 960000 * 4 + 4 * 128 * 6000 * 4) / ms_m / 1e6,
-                              "tflops_fp32": 24000 * LOG_MEL_FLOP_PER_FRAME / ms_m / 1e9,
-                              "frac_of_fp32_alu_peak": 24000 * LOG_MEL_FLOP_PER_FRAME / ms_m / 1e9 / FP32_ALU_TFLOPS},
-            "projector_4x3000": {"ms_per_call": ms_p, "tokens_per_s": 3000 / ms_p * 1e3,
-                                 "tflops": proj_flop / ms_p / 1e9, "frac_of_measured_peak": proj_flop / ms_p / 1e9 / tf}}
+    res = {"conv_step_64x8": {"ms_per_step": ms_c, "frames_per_s": S * 4 / ms_c * 1e3,
+                              "gbs": conv_bytes / ms_c / 1e6, "tflops": conv_flop / ms_c / 1e9},
+           "log_mel_4x60s": {"ms_per_call": ms_m, "mel_frames_per_s": 24000 / ms_m * 1e3,
+                             "gbs": (4 * 960000 * 4 + 4 * 128 * 6000 * 4) / ms_m / 1e6,
+                             "tflops_fp32": 24000 * LOG_MEL_FLOP_PER_FRAME / ms_m / 1e9,
+                             "frac_of_fp32_alu_peak": 24000 * LOG_MEL_FLOP_PER_FRAME / ms_m / 1e9 / FP32_ALU_TFLOPS},
+           "projector_4x3000": {"ms_per_call": ms_p, "tokens_per_s": 3000 / ms_p * 1e3,
+                                "tflops": proj_flop / ms_p / 1e9, "frac_of_measured_peak": proj_flop / ms_p / 1e9 / tf}}
+    del x, out, audio, melo, wsm, wsp
+    torch.cuda.empty_cache()
+
+    # Streaming mode: 312-mel first chunk, then 8-mel chunks, 64 streams.
+    cfg, layers = device_layers(vx, torch, 32, 503, "cuda")
+    first_samples = 160 * 312 + 200
+    aud0 = torch.randn(S, first_samples, generator=g, device="cuda") * 0.1
+    audc = torch.randn(S, 160 * 7 + 400, generator=g, device="cuda") * 0.1
+    ring = vx.KVRing(cfg, 32, S)
+    wf = vx.Workspace()
+    wsm0 = vx.Workspace()
+
+    def first_chunk():
+        cache.reset()
+        m0 = vx.log_mel_fwd(aud0, True, ws=wsm0)[:, :, :312].contiguous()
+        h0 = vx.conv_stem_step(m0, w1p, b1, w2p, b2, cache, ws=wf)
+        return vx.stream_prefill(cfg, layers, ring, h0, final_g=fg, ws=wf)
+
+    def chunk():
+        mc = vx.log_mel_fwd(audc, False, ws=wsm0)
+        hc = vx.conv_stem_step(mc, w1p, b1, w2p, b2, cache, ws=wf)
+        yc = vx.stream_step(cfg, layers, ring, hc, final_g=fg, ws=wf)
+        return vx.projector_fwd(yc, pw1, pw2, ws=wf)
+
+    for _ in range(3):
+        first_chunk()
+        chunk()
+    ms_first, _, _ = timed_steps(torch, first_chunk, 10, flush, torch.cuda.current_stream())
+    first_chunk()
+    ms_chunk, _, _ = timed_steps(torch, chunk, 20, lambda: None, torch.cuda.current_stream())
+    res["stream_first_chunk_64x312"] = {
+        "ms_per_call": ms_first, "encoder_frames": S * 156, "frames_per_s": S * 156 / ms_first * 1e3,
+        "note": "log-mel (centred) + conv stem + 32-layer prefill filling the ring, final norm; 64 streams at "
+                "once.  Context only: the Core AI card's 0.148 s TTFT is one stream on Apple hardware with the "
+                "decoder included"}
+    res["stream_chunk_64x8"] = {
+        "ms_per_chunk": ms_chunk, "encoder_frames_per_s": S * 4 / ms_chunk * 1e3,
+        "tokens_per_s": S / ms_chunk * 1e3,
+        "note": "log-mel (8 frames) + conv-stem step + 32-layer streaming step + projector (one token per "
+                "stream); ring at pos >= 156.  Context only: the card's 59.6 ms chunk includes the decoder"}
+    del ring
+    return res
 
 
 # ------------------------------------------------------------- cpu legs
 
-def oracle_sample(frames: int):
-    """One oracle encoder layer over the first `frames` frames of the C1 input
-    (causal, so those outputs are exact); returns seconds."""
+def oracle_encoder_sample(n_layers=2):
+    """The oracle on one clip of the workload: the conv stem over 6000 mel
+    frames and n_layers of the 32 encoder layers over the 3000 frames it
+    gives.  Returns (stem seconds, mean seconds per layer)."""
     import oracle
     import synth
-    p = synth.layer_params(synth.VOXTRAL_RT, seed=1)
-    x = synth.frames(1, C1["T"], C1["d"], seed=2)[:, :frames]
-    t = time.perf_counter()
-    oracle.encoder_layer(x, p, synth.VOXTRAL_RT)
-    return time.perf_counter() - t
+    dims = synth.VOXTRAL_RT
+    conv = synth.conv_params(seed=3)
+    mel = synth.mel(1, 128, C4["Tm"], seed=4)
+    x = None
+
+    def stem():
+        nonlocal x
+        x = oracle.conv_stem(mel, **conv)
+
+    ts = _clock(stem)
+    tl = []
+    for l in range(n_layers):
+        p = synth.layer_params(dims, seed=synth.layer_seed(1, l))
+        tl.append(_clock(lambda: oracle.encoder_layer(x, p, dims)))
+    return ts, float(np.mean(tl))
 
 
-def blas_threads():
-    try:
-        from threadpoolctl import threadpool_info
-        return max(i.get("num_threads", 1) for i in threadpool_info()) or os.cpu_count()
-    except Exception:
-        return os.cpu_count()
+def oracle_forward_s(ts, tl):
+    """Seconds of one clip's forward: the stem and 32 layers of equal cost (the
+    final norm is negligible)."""
+    return ts + C4["L"] * tl
 
 
-def cpu_baseline(budget_s=12.0):
-    """The oracle as it stands on this host: full C1 layers repeated until ~budget_s."""
-    n, total = 0, 0.0
-    while total < budget_s and n < 20:
-        total += oracle_sample(C1["T"])
-        n += 1
-    return {"value": n * C1["T"] / total, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
-            "sample": f"{n} full C1 layer(s) ({n} x {C1['T']} frames) of the float64 numpy oracle, "
-                      f"{total:.1f} s of CPU time on {os.cpu_count()} host cores"}
+def cpu_baseline():
+    ts, tl = oracle_encoder_sample(2)
+    t = oracle_forward_s(ts, tl)
+    return {"value": C4["To"] / t, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+            "sample": f"one of the 4 clips: the float64 numpy oracle's conv stem over 6000 mel frames ({ts:.1f} s) "
+                      f"and 2 of the 32 layers over its 3000 frames ({tl:.1f} s each) timed on {os.cpu_count()} host "
+                      f"cores; the forward extrapolated as stem + 32 x layer = {t:.0f} s per 3000 frames"}
 
 
 def run_reference(args):
     rank, world, _ = dist_env()
     if rank != 0:
         return 0
-    frames = 375   # a quarter of the C1 clip per step (causal: exact outputs for those frames)
     for _ in range(args.warmup):
-        oracle_sample(frames)
-    t = [oracle_sample(frames) for _ in range(args.steps)]
-    ms = 1e3 * float(np.mean(t))
-    value = frames / (ms / 1e3)
+        oracle_encoder_sample(1)
+    per = [oracle_forward_s(*oracle_encoder_sample(1)) for _ in range(args.steps)]
+    s = float(np.mean(per))
+    value = C4["To"] / s
+    sample = ("per step, one of the 4 clips: the float64 numpy oracle's conv stem over 6000 mel frames and one "
+              "of the 32 layers over its 3000 frames timed; the clip's forward extrapolated as stem + 32 x layer")
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": s * 1e3, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": WORKLOAD, "B": C1["B"], "T": C1["T"], "parallelism": "replicas",
-                       "l2": "n/a (CPU)"},
+            "config": {"workload": WORKLOAD, "B": C4["B"], "n_mels": C4["n_mels"], "Tm": C4["Tm"],
+                       "frames_out": C4["To"], "layers": C4["L"], "parallelism": "replicas", "l2": "n/a (CPU)"},
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
-                             "sample": f"first {frames} frames of the C1 clip per step, float64 numpy oracle"},
+                             "sample": sample},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
     return 0
 
 
 # ------------------------------------------------------------------ main
+
+COMPONENTS = {"c1": ("encoder_layer_c1", component_c1), "c0": ("swa_c0", component_c0),
+              "c2": ("swa_c2", component_c2), "c3": ("stream_step_c3", component_c3),
+              "next": ("next_rows", component_next)}
+
 
 def main(argv=None):
     args = parse_args(argv)
@@ -527,32 +745,38 @@ def main(argv=None):
     torch.cuda.set_device(device)
     if world > 1:
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=180), device_id=device)
+    global PEAK_KIND
     hbm, tf_burst, tf_sust, peak_kind = peaks()
+    PEAK_KIND = peak_kind
 
     flush_buf = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
     flush = lambda: flush_buf.zero_()
     stream = torch.cuda.current_stream()
+    oracle_on = rank == 0 and world == 1 and not args.no_oracle
 
     comps_only = [c for c in args.components_only.split(",") if c]
     if comps_only:
         out = {}
         for c in comps_only:
+            name, fn = COMPONENTS[c]
             if c == "c3":
-                out[c] = component_c3(vx, torch, flush, hbm, tf_burst, L=args.c3_layers)
+                out[name] = component_c3(vx, torch, flush, hbm, tf_burst, oracle_on, L=args.c3_layers)
             else:
-                out[c] = {"c0": component_c0, "c2": component_c2, "c4": component_c4,
-                          "next": component_next}[c](vx, torch, flush, hbm, tf_burst)
+                out[name] = fn(vx, torch, flush, hbm, tf_burst, oracle_on)
         if rank == 0:
             print(json.dumps({"components": out}), flush=True)
         return 0
 
-    B, T, d = C1["B"], C1["T"], C1["d"]
-    cfg, L = make_layer(vx, torch, device=device)
-    g = torch.Generator(device=device).manual_seed(2 + rank)
-    x = torch.randn(B, T, d, generator=g, device=device)
-    y = torch.empty_like(x)
-    ws = vx.Workspace(vx.lib.vx_encoder_layer_workspace(__import__("ctypes").byref(cfg.c()), B, T), device=device)
-    step = lambda: vx.encoder_layer_fwd(cfg, L, x, out=y, ws=ws)
+    # ---- the timed workload: the 4 x 6000-mel encoder forward
+    B, Tm, To = C4["B"], C4["Tm"], C4["To"]
+    cfg, layers = device_layers(vx, torch, C4["L"], 400, device)
+    w1p, b1, w2p, b2, fg = device_stem(vx, torch, 401, device)
+    g = torch.Generator(device=device).manual_seed(402 + rank)
+    mel = torch.randn(B, C4["n_mels"], Tm, generator=g, device=device)
+    out = torch.empty(B, To, C4["d"], device=device)
+    ws = vx.Workspace(vx.lib.vx_encoder_workspace(__import__("ctypes").byref(cfg.c()), B, C4["n_mels"], Tm),
+                      device=device)
+    step = lambda: vx.encoder_fwd(cfg, mel, w1p, b1, w2p, b2, layers, fg, out=out, ws=ws)
 
     for _ in range(args.warmup):
         step()
@@ -569,19 +793,20 @@ def main(argv=None):
     torch.cuda.synchronize()
     barrier(device)
     ms = reduce_max(ms_local, device)
-    frames_all = reduce_sum(B * T, device)
+    frames_all = reduce_sum(B * To, device)
     value = frames_all / (ms / 1e3)
 
     # End to end through the public call from pinned host buffers: every step
-    # copies its input in (H2D), runs the layer and reads its output back (D2H).
-    # Like a server fed a stream of clips, the copies of neighbouring steps run
-    # on their own streams (two device buffers each way), overlapping the
-    # layer; the L2 flush before each step's layer is inside the timed region.
-    xh = torch.empty(B, T, d, dtype=torch.float32, pin_memory=True)
-    xh.copy_(x.cpu())
-    yh = torch.empty_like(xh, pin_memory=True)
-    xs = [x, torch.empty_like(x)]
-    ys = [y, torch.empty_like(y)]
+    # copies its mel input in (H2D), runs the encoder and reads its output
+    # back (D2H).  Like a server fed a stream of clips, the copies of
+    # neighbouring steps run on their own streams (two device buffers each
+    # way), overlapping the encoder; the L2 flush before each step is inside
+    # the timed region.
+    mh = torch.empty(mel.shape, dtype=torch.float32, pin_memory=True)
+    mh.copy_(mel.cpu())
+    oh = torch.empty(out.shape, dtype=torch.float32, pin_memory=True)
+    ms_dev = [mel, torch.empty_like(mel)]
+    os_dev = [out, torch.empty_like(out)]
     s_in, s_out = torch.cuda.Stream(device=device), torch.cuda.Stream(device=device)
 
     def e2e_run(K):
@@ -596,18 +821,18 @@ def main(argv=None):
             bb = i % 2
             with torch.cuda.stream(s_in):
                 if i >= 2:
-                    s_in.wait_event(ev_comp[i - 2])      # the layer of step i-2 has read xs[bb]
-                xs[bb].copy_(xh, non_blocking=True)
+                    s_in.wait_event(ev_comp[i - 2])      # the encoder of step i-2 has read ms_dev[bb]
+                ms_dev[bb].copy_(mh, non_blocking=True)
                 ev_in[i].record(s_in)
             stream.wait_event(ev_in[i])
             if i >= 2:
-                stream.wait_event(ev_out[i - 2])         # ys[bb] of step i-2 is on the host
+                stream.wait_event(ev_out[i - 2])         # os_dev[bb] of step i-2 is on the host
             flush()
-            vx.encoder_layer_fwd(cfg, L, xs[bb], out=ys[bb], ws=ws)
+            vx.encoder_fwd(cfg, ms_dev[bb], w1p, b1, w2p, b2, layers, fg, out=os_dev[bb], ws=ws)
             ev_comp[i].record(stream)
             with torch.cuda.stream(s_out):
                 s_out.wait_event(ev_comp[i])
-                yh.copy_(ys[bb], non_blocking=True)
+                oh.copy_(os_dev[bb], non_blocking=True)
                 ev_out[i].record(s_out)
         stream.wait_stream(s_out)
         e1.record(stream)
@@ -616,44 +841,28 @@ def main(argv=None):
 
     ms_e2e = float("nan")
     if not args.no_e2e:
-        e2e_run(3)
+        e2e_run(2)
         barrier(device)
-        ms_e2e = reduce_max(e2e_run(max(20, min(args.steps, 200))), device)
+        ms_e2e = reduce_max(e2e_run(max(5, args.steps)), device)
     sampler.stop()
     clocks = sampler.summary(t0, t1)
 
-    # dominant kernel, timed live per launch (trace mode), and its roofline
-    tr = traced_kernels(vx, torch, step, 0 if args.no_trace else 50, flush)
-    if not tr:
-        tr = {"none": {"ms_per_launch": float("nan"), "launches_per_step": 0, "ms_per_step": 0.0}}
-    dom = max(tr, key=lambda k: tr[k]["ms_per_step"])
-    work, wunit, bound = kernel_work(dom, B, T)
-    if work is None:
-        roof = {"bound": None, "achieved": None, "peak": None, "unit": None, "frac": None}
-    elif bound == "tensor":
-        achieved = work / (tr[dom]["ms_per_launch"] / 1e3) / 1e12
-        roof = {"bound": "tensor", "achieved": achieved, "peak": tf_burst, "unit": "TFLOP/s",
-                "frac": achieved / tf_burst, "peak_kind": f"{peak_kind} bf16 dense (burst)"}
+    # per-kernel times of the step, traced live; the dominant kernel's roofline
+    tr = traced_kernels(vx, torch, step, 0 if args.no_trace else 3, flush)
+    wl = {"M": B * To, "attn": (B, To, 32, C4["W"]), "stem": (B, Tm)}
+    if tr:
+        roof = roofline(tr, wl, tf_burst, hbm, peak_kind, "C4", "burst")
+        kernels = per_kernel_table(tr, wl)
     else:
-        achieved = work / (tr[dom]["ms_per_launch"] / 1e3) / 1e9
-        roof = {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
-                "peak_kind": f"{peak_kind} HBM copy"}
-    roof.update({"kernel": dom, "work_per_launch": work, "work_unit": wunit,
-                 "ms_per_launch": tr[dom]["ms_per_launch"], "traffic": ncu_traffic(dom, "C1")})
-    per_kernel = {k: {"ms_per_launch": v["ms_per_launch"], "launches_per_step": v["launches_per_step"]}
-                  for k, v in tr.items()}
-    for k, v in per_kernel.items():
-        w, u, b = kernel_work(k, B, T)
-        if w is not None:
-            v["tflops" if u == "flop" else "gbs"] = w / (v["ms_per_launch"] / 1e3) / (1e12 if u == "flop" else 1e9)
+        roof, kernels = {"bound": None, "achieved": None, "peak": None, "unit": None, "frac": None,
+                         "traffic": None}, {}
 
     comps = None
     if world == 1 and not args.no_components:
         comps = {}
-        for name, fn in (("swa_c0", component_c0), ("swa_c2", component_c2), ("stream_step_c3", component_c3),
-                         ("encoder_c4", component_c4), ("next_rows", component_next)):
+        for key, (name, fn) in COMPONENTS.items():
             try:
-                comps[name] = fn(vx, torch, flush, hbm, tf_burst)
+                comps[name] = fn(vx, torch, flush, hbm, tf_burst, oracle_on)
             except Exception as e:   # report, never hide
                 comps[name] = {"error": repr(e)}
             torch.cuda.empty_cache()
@@ -663,21 +872,25 @@ def main(argv=None):
         cpu = cpu_baseline()
 
     if rank == 0:
+        fl = encoder_flops(B, Tm)
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": WORKLOAD, "B": B, "T": T, "parallelism": f"replicas x{world}",
-                       "l2": "flushed between timed steps (256 MiB write outside the step events)"},
-            "layer_tflops": layer_flops(B, T) / (ms / 1e3) / 1e12,
-            "layer_frac_of_measured_peak": layer_flops(B, T) / (ms / 1e3) / 1e12 / tf_burst,
+            "config": {"workload": WORKLOAD, "B": B, "n_mels": C4["n_mels"], "Tm": Tm, "frames_out": To,
+                       "layers": C4["L"], "parallelism": f"replicas x{world}",
+                       "l2": "flushed between timed steps (256 MiB write outside the step events); the 1.93 GB "
+                             "of layer weights exceed L2"},
+            "encoder_tflops": fl / (ms / 1e3) / 1e12,
+            "encoder_frac_of_measured_peak": fl / (ms / 1e3) / 1e12 / tf_burst,
             "e2e": {"value": frames_all / (ms_e2e / 1e3), "unit": UNIT,
-                    "h2d_bytes_per_step": B * T * d * 4, "d2h_bytes_per_step": B * T * d * 4,
-                    "method": "pinned host buffers; H2D, layer (after a 256 MiB L2 flush) and D2H of consecutive "
-                              "steps on three streams with two device buffers each way; timed over the whole run"},
+                    "h2d_bytes_per_step": int(mel.numel() * 4), "d2h_bytes_per_step": int(out.numel() * 4),
+                    "method": "vx_encoder_fwd from pinned host mel to pinned host output; H2D, encoder (after a "
+                              "256 MiB L2 flush) and D2H of consecutive steps on three streams with two device "
+                              "buffers each way; timed over the whole run"},
             "gpu_launches": int(launches),
             "roofline": roof,
-            "kernels": per_kernel,
+            "kernels": kernels,
             "clocks": clocks,
             "cpu_baseline": cpu,
             "components": comps,

@@ -63,6 +63,30 @@ def test_algorithmic_work_counts():
     assert sum(bench.gemm_flops(1500).values()) == 2 * 1500 * 30146560
     assert bench.layer_flops(1, 1500) == pytest.approx(97.35e9, rel=1e-3)
     assert bench.attn_flops(8, 6000, 32, 64, 750) == pytest.approx(276.50e9, rel=1e-3)
+    # the encoder workload: stem 141.6 GFLOP + 32 layers of 4 x 3000 frames = 25.36 TFLOP
+    assert sum(bench.stem_flops(4, 6000).values()) == pytest.approx(141.6e9, rel=1e-3)
+    assert bench.encoder_flops(4, 6000) == pytest.approx(25.36e12, rel=1e-3)
+
+
+def test_attention_tile_counts():
+    # key tiles of 128 visited per (clip, head): 63 / 147 / 308 of 144 / 576 / 2209
+    for T, visited, total in ((1500, 63, 144), (3000, 147, 576), (6000, 308, 2209)):
+        t = bench.attn_tiles(T, 750)
+        assert (t["visited"], t["all_tiles"]) == (visited, total)
+        assert 0.8 < t["useful_frac"] < 0.85
+    # a window covering the clip visits the whole causal triangle
+    t = bench.attn_tiles(1000, 2000)
+    assert t["visited"] == t["causal_tiles"] == 8 * 9 // 2
+
+
+def test_rmsnorm_trace_names_count_their_bytes():
+    M = 1500
+    w = lambda name: bench.kernel_work(name, {"M": M})[0] - 1280 * 2
+    assert w("rmsnorm_p0_y16") == M * 1280 * (4 + 2)            # x in, bf16 y out
+    assert w("rmsnorm_p2_h_y16") == M * 1280 * (4 + 8 + 4 + 2)  # + two partial sums in, h out
+    assert w("rmsnorm_p1_h") == M * 1280 * (4 + 4 + 4)          # a reduction only
+    assert w("rmsnorm_p0_y32") == M * 1280 * (4 + 4)            # the final norm
+    assert bench.kernel_work("gemm_conv2_gelu", {"stem": (4, 6000)})[0] == 2 * 4 * 3000 * 1280 * 3 * 1280
 
 
 def test_reference_arm_prints_one_json_line():
