@@ -50,28 +50,55 @@ __device__ __forceinline__ uint64_t fadd2(uint64_t a, uint64_t b) {
   return d;
 }
 
-// Max of 32 values as a balanced tree (short dependency chains).
-__device__ __forceinline__ float tree_max32(const float* v) {
-  float t[16];
-#pragma unroll
-  for (int i = 0; i < 16; ++i) t[i] = fmaxf(v[i], v[i + 16]);
-#pragma unroll
-  for (int w = 8; w >= 1; w >>= 1)
-#pragma unroll
-    for (int i = 0; i < w; ++i) t[i] = fmaxf(t[i], t[i + w]);
-  return t[0];
+// Three-input maximum (sm_100's max.f32 with three sources).
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
 }
 
-// pv[e] = 2^(s[e] * sl2 - mu) for 32 scores, the argument two at a time.
-__device__ __forceinline__ void exp2_scaled32(const float* s, float sl2, float mu, float (&pv)[32]) {
+// Max of 64 values: a three-input tree (64 -> 22 -> 8 -> 3 -> 1), short
+// dependency chains, 32 instructions.
+__device__ __forceinline__ float tree_max64(const float* v) {
+  float t[22];
+#pragma unroll
+  for (int i = 0; i < 21; ++i) t[i] = fmax3(v[3 * i], v[3 * i + 1], v[3 * i + 2]);
+  t[21] = v[63];
+  float u[8];
+#pragma unroll
+  for (int i = 0; i < 7; ++i) u[i] = fmax3(t[3 * i], t[3 * i + 1], t[3 * i + 2]);
+  u[7] = t[21];
+  return fmax3(fmax3(u[0], u[1], u[2]), fmax3(u[3], u[4], u[5]), fmaxf(u[6], u[7]));
+}
+
+// v[e] = v[e] * sl2 - mu for 64 scores, two at a time.
+__device__ __forceinline__ void exp2_args64(float (&v)[64], float sl2, float mu) {
   const uint64_t sc = f2_pack(sl2, sl2), nm = f2_pack(-mu, -mu);
 #pragma unroll
-  for (int e = 0; e < 32; e += 2) {
-    float x0, x1;
-    f2_unpack(ffma2(f2_pack(s[e], s[e + 1]), sc, nm), x0, x1);
-    pv[e] = ex2_approx(x0);
-    pv[e + 1] = ex2_approx(x1);
-  }
+  for (int e = 0; e < 64; e += 2) f2_unpack(ffma2(f2_pack(v[e], v[e + 1]), sc, nm), v[e], v[e + 1]);
+}
+
+// 2^x on the MUFU unit as a volatile asm: the compiler keeps these in
+// program order with the token hand-off around them.
+__device__ __forceinline__ float ex2_ordered(float x) {
+  float y;
+  asm volatile("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// Sum of 32 values as the tree t[e] = v[e] + v[e + 16], then halving; two
+// neighbouring nodes of a level per packed add.
+__device__ __forceinline__ float sum32_tree(const float (&v)[32]) {
+  uint64_t t[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) t[i] = fadd2(f2_pack(v[2 * i], v[2 * i + 1]), f2_pack(v[2 * i + 16], v[2 * i + 17]));
+#pragma unroll
+  for (int w = 4; w >= 1; w >>= 1)
+#pragma unroll
+    for (int i = 0; i < w; ++i) t[i] = fadd2(t[i], t[i + w]);
+  float a, b;
+  f2_unpack(t[0], a, b);
+  return a + b;
 }
 
 // The softmax warpgroups take most of the register file (setmaxnreg): 8
@@ -86,21 +113,26 @@ constexpr int kOtherRegs = 56;
 // and one K/V ring that carries the union of their key ranges once (the two
 // windows overlap in all but two 64-key tiles, so each K/V tile crosses L2
 // once for both).  Key tiles are 64 keys wide so that each warpgroup's TMEM
-// holds two S buffers (64 columns each), its output O (64 columns) and a row
-// sum L (16 columns): S(j+1) is computed while the softmax of tile j runs, and
-// the softmax of tile j+1 never waits for the P V product of tile j, because
-// P(j) is written back (bf16 pairs) into S(j)'s own columns and the next use of
-// that buffer is tile j+2.  The row sum is accumulated on the tensor cores as
-// P times a constant tile of ones (L += P 1), from exactly the bf16 P that
-// enters O += P V; O and L are rescaled in place only when a row's running
-// maximum grows by more than kRescaleSlack.  Only the key tiles that meet the
-// causal window are visited, and masks are applied only on edge tiles.
+// holds three S buffers (64 columns each) and its output O (64 columns): S of
+// the next two tiles is computed while the softmax of a tile runs, and P(j)
+// is written back (bf16 pairs) into S(j)'s own columns, whose next use is
+// tile j+3.  O is rescaled in place only when a row's running maximum grows by
+// more than kRescaleSlack.  Only the key tiles that meet the causal window are
+// visited, and masks are applied only on edge tiles, per warp.
+// Measured on B200 (per-phase clock stamps of one CTA): a 64-key tile costs a
+// softmax warp ~470 cycles outside its exponentials and ~550 cycles of MUFU
+// issue (64 warp-wide ex2 at 8 cycles each); the tensor core is ~20% busy and
+// the MMA issue rate (~50 cycles per instruction per issuing thread) is not
+// the limit.  Warp q of each warpgroup shares a scheduler's MUFU with warp q
+// of the other, so the two take turns at their exponentials (a token passed
+// through an mbarrier, see the softmax loop); computing part of the
+// exponentials on the FMA pipe instead measured slower.
 // Warps 0-3 / 4-7: softmax warpgroups 0 / 1 (TMEM lane = query row); warp 8:
 // TMA producer; warps 9 / 10: the tensor-core products of warpgroup 0 / 1.
 constexpr int kWsStages = 6;                     // K/V ring stages (64-key tiles)
 constexpr int kKvTile = kAttnKeyTile * 64 * 2;   // 8 KB: 64 keys x 64 dims bf16
-constexpr int kOnesBytes = 16 * 128;             // 16 rows (N) x 64 keys (K) of bf16 ones
-constexpr int kAttnSmemWs = 4 * kTile + 2 * kWsStages * kKvTile + kOnesBytes + 1024 + 512;
+constexpr int kSBuf = 3;                         // S buffers per warpgroup
+constexpr int kAttnSmemWs = 4 * kTile + 2 * kWsStages * kKvTile + 1024 + 512;
 
 struct PairItem {
   int b, h, p;        // clip, head, pair index (query tiles 2p, 2p+1)
@@ -151,11 +183,12 @@ swa_attn_ws_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
   uint8_t* sQ = smem;                                  // Q[X][buffer]: 4 tiles of 16 KB
   uint8_t* sK = sQ + 4 * kTile;                        // K ring: kWsStages x 8 KB
   uint8_t* sV = sK + kWsStages * kKvTile;              // V ring
-  uint8_t* sOnes = sV + kWsStages * kKvTile;           // 2 KB of bf16 ones (the L product's B operand)
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sOnes + kOnesBytes);
-  // per warpgroup X: QF/QE [X*2 + buf], SF/PF/BF [X*2 + b], OD/OFREE/DR [X]
-  constexpr int QF = 0, QE = 4, KF = 8, VF = KF + kWsStages, KVE = VF + kWsStages, SF = KVE + kWsStages,
-                PF = SF + 4, BF = PF + 4, OD = BF + 4, OFREE = OD + 2, DR = OFREE + 2, NBAR = DR + 2;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sV + kWsStages * kKvTile);
+  // per warpgroup X: QF/QE [X*2 + buf], SF/PF/BF [X*3 + b], OD/OFREE/DR [X]
+  // KF[stage]: the stage's K and V tiles have landed (one barrier, both copies' bytes)
+  constexpr int QF = 0, QE = 4, KF = 8, KVE = KF + kWsStages, SF = KVE + kWsStages,
+                PF = SF + 2 * kSBuf, BF = PF + 2 * kSBuf, OD = BF + 2 * kSBuf, OFREE = OD + 2, DR = OFREE + 2,
+                TOK = DR + 2, NBAR = TOK + 8;   // TOK[X * 4 + q]: warp q of warpgroup X may exponentiate
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + NBAR);
   int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
   auto bar = [&](int i) { return smem_addr(bars + i); };
@@ -166,17 +199,13 @@ swa_attn_ws_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < 4; ++i) { mbar_init(bar(QF + i), 1); mbar_init(bar(QE + i), 1); }
-    for (int s = 0; s < kWsStages; ++s) { mbar_init(bar(KF + s), 1); mbar_init(bar(VF + s), 1); mbar_init(bar(KVE + s), 2); }
-    for (int i = 0; i < 4; ++i) { mbar_init(bar(SF + i), 1); mbar_init(bar(PF + i), 128); mbar_init(bar(BF + i), 1); }
+    for (int s = 0; s < kWsStages; ++s) { mbar_init(bar(KF + s), 1); mbar_init(bar(KVE + s), 2); }
+    for (int i = 0; i < 2 * kSBuf; ++i) { mbar_init(bar(SF + i), 1); mbar_init(bar(PF + i), 128); mbar_init(bar(BF + i), 1); }
     for (int X = 0; X < 2; ++X) { mbar_init(bar(OD + X), 1); mbar_init(bar(OFREE + X), 4); mbar_init(bar(DR + X), 1); }
+    for (int i = 0; i < 8; ++i) mbar_init(bar(TOK + i), 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
-  // The ones tile (every element 1.0 in bf16, so the swizzle is irrelevant),
-  // written through the generic proxy and fenced for the tensor cores.
-  for (int i = threadIdx.x; i < kOnesBytes / 16; i += blockDim.x)
-    reinterpret_cast<uint4*>(sOnes)[i] = make_uint4(0x3F803F80u, 0x3F803F80u, 0x3F803F80u, 0x3F803F80u);
-  fence_proxy_async_smem();
   if (warp == 9) {
     tmem_alloc(smem_addr(tmem_slot), kTmemCols);
     tmem_relinquish();
@@ -218,10 +247,9 @@ swa_attn_ws_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
           const uint32_t ph = (U / kWsStages) & 1;
           if (!mbar_wait(bar(KVE + st), ph ^ 1, wc, 51)) { ok = false; break; }
           const int kt = it.u0 + u;
-          mbar_arrive_expect_tx(bar(KF + st), kKvTile);
+          mbar_arrive_expect_tx(bar(KF + st), 2 * kKvTile);
           tma_load_4d(smem_addr(sK + st * kKvTile), &tmK, bar(KF + st), 0, it.h, kt * kAttnKeyTile, it.b);
-          mbar_arrive_expect_tx(bar(VF + st), kKvTile);
-          tma_load_4d(smem_addr(sV + st * kKvTile), &tmV, bar(VF + st), 0, it.h, kt * kAttnKeyTile, it.b);
+          tma_load_4d(smem_addr(sV + st * kKvTile), &tmV, bar(KF + st), 0, it.h, kt * kAttnKeyTile, it.b);
           // The stage is released by each warpgroup that uses the tile (its
           // last product's commit); for a tile only one uses, the producer
           // arrives in the other's place (after the previous phase completed).
@@ -240,7 +268,6 @@ swa_attn_ws_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
         if (q_issued & (1u << qi)) mbar_wait(bar(QF + qi), (q_par >> qi) & 1u, dw, 52);
       for (int s = 0; s < kWsStages && s < filled; ++s) {
         mbar_wait(bar(KF + s), (last_par >> s) & 1u, dw, 52);
-        mbar_wait(bar(VF + s), (last_par >> s) & 1u, dw, 52);
       }
     } else if ((warp == 9 || warp == 10) && lane == 0) {
       // ------------- tensor-core products of warpgroup X
@@ -248,8 +275,6 @@ swa_attn_ws_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
       const uint32_t tX = tmem + X * 256;
       const uint32_t idesc_s = idesc_bf16_f32(128, kAttnKeyTile, 0);
       const uint32_t idesc_o = idesc_bf16_f32(128, 64, 1);
-      const uint32_t idesc_l = idesc_bf16_f32(128, 16, 0);
-      const uint32_t ones = smem_addr(sOnes);
       int jg = 0;      // this warpgroup's key tiles so far (all items)
       int kc = 0;      // this warpgroup's items so far
       int ubase = 0;   // ring position of the current pair item's first union tile
@@ -262,9 +287,9 @@ swa_attn_ws_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
           ok = mbar_wait(bar(QF + qi), (kc >> 1) & 1, wc, 53);
           const uint32_t qa = smem_addr(sQ + qi * kTile);
           const int uoff = it.kt0[X] - it.u0;
-          auto issue_s = [&](int t) -> bool {   // S(t) into buffer (jg + t) & 1
-            const int g = jg + t, bsel = g & 1, U = ubase + uoff + t, st = U % kWsStages;
-            if (!mbar_wait(bar(BF + X * 2 + bsel), ((g >> 1) & 1) ^ 1, wc, 54)) return false;   // P(t-2) consumed
+          auto issue_s = [&](int t) -> bool {   // S(t) into buffer (jg + t) % 3
+            const int g = jg + t, bsel = g % kSBuf, U = ubase + uoff + t, st = U % kWsStages;
+            if (!mbar_wait(bar(BF + X * kSBuf + bsel), ((g / kSBuf) & 1) ^ 1, wc, 54)) return false;   // P(t-3) consumed
             if (!mbar_wait(bar(KF + st), (U / kWsStages) & 1, wc, 55)) return false;
             tc_fence_after();
             const uint32_t ka = smem_addr(sK + st * kKvTile);
@@ -272,35 +297,33 @@ swa_attn_ws_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
             for (int kk = 0; kk < 4; ++kk)
               umma_bf16(tX + 64 * bsel, smem_desc_sw128(qa + 32 * kk, 16, 1024),
                         smem_desc_sw128(ka + 32 * kk, 16, 1024), idesc_s, kk > 0);
-            umma_commit(bar(SF + X * 2 + bsel));
+            umma_commit(bar(SF + X * kSBuf + bsel));
             return true;
           };
-          auto issue_pv = [&](int t) -> bool {   // O += P V, L += P 1 (P in S(t)'s columns)
-            const int g = jg + t, bsel = g & 1, U = ubase + uoff + t, st = U % kWsStages;
-            if (!mbar_wait(bar(PF + X * 2 + bsel), (g >> 1) & 1, wc, 56)) return false;
-            if (!mbar_wait(bar(VF + st), (U / kWsStages) & 1, wc, 57)) return false;
-            // O and L are overwritten by the item's first product: the
-            // warpgroup's previous item must have been read out.
+          auto issue_pv = [&](int t) -> bool {   // O += P V (P in S(t)'s columns)
+            const int g = jg + t, bsel = g % kSBuf, U = ubase + uoff + t, st = U % kWsStages;
+            if (!mbar_wait(bar(PF + X * kSBuf + bsel), (g / kSBuf) & 1, wc, 56)) return false;
+            // O is overwritten by the item's first product: the warpgroup's
+            // previous item must have been read out.
             if (t == 0 && !mbar_wait(bar(OFREE + X), (kc & 1) ^ 1, wc, 58)) return false;
             tc_fence_after();
             const uint32_t va = smem_addr(sV + st * kKvTile);
             const uint32_t pa = tX + 64 * bsel;
 #pragma unroll
-            for (int kk = 0; kk < 4; ++kk) {   // 16 keys per step: 8 TMEM columns of P, 16 rows of V
-              const uint32_t acc = (t > 0 || kk > 0) ? 1u : 0u;
-              umma_bf16_ts(tX + 128, pa + 8 * kk, smem_desc_sw128(va + kk * 2048, kKvTile, 1024), idesc_o, acc);
-              umma_bf16_ts(tX + 192, pa + 8 * kk, smem_desc_sw128(ones + 32 * kk, 16, 1024), idesc_l, acc);
-            }
-            umma_commit(bar(BF + X * 2 + bsel));   // S buffer free; O, L hold tile t
+            for (int kk = 0; kk < 4; ++kk)   // 16 keys per step: 8 TMEM columns of P, 16 rows of V
+              umma_bf16_ts(tX + 192, pa + 8 * kk, smem_desc_sw128(va + kk * 2048, kKvTile, 1024), idesc_o,
+                           (t > 0 || kk > 0) ? 1u : 0u);
+            umma_commit(bar(BF + X * kSBuf + bsel));   // S buffer free; O holds tile t
             umma_commit(bar(KVE + st));            // K/V tile: S(t) and P V (t) were this group's uses
             return true;
           };
           if (ok) ok = issue_s(0);
+          if (ok && n > 1) ok = issue_s(1);
           for (int t = 0; ok && t < n; ++t) {
-            if (t + 1 < n) ok = issue_s(t + 1);
+            if (t + 2 < n) ok = issue_s(t + 2);
             if (ok) ok = issue_pv(t);
           }
-          umma_commit(bar(OD + X));   // O and L of this item are final once its products are done
+          umma_commit(bar(OD + X));   // O of this item is final once its products are done
           umma_commit(bar(QE + qi));  // and so is the use of its Q buffer
           jg += n;
           ++kc;
@@ -320,23 +343,35 @@ swa_attn_ws_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
     const int r = threadIdx.x & 127;
     const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const uint32_t tX = tmem + X * 256 + lane_off;
-    const uint32_t tO = tX + 128, tL = tX + 192;
+    const uint32_t tO = tX + 192;
     const float sl2 = a.scale_log2;
     const int W = a.window;
     int jg = 0;   // this warpgroup's key tiles so far (all items)
     int kc = 0;   // this warpgroup's items so far
+    // Warp q of each warpgroup shares a scheduler (and its MUFU) with warp q
+    // of the other.  Their exponentials would otherwise run at the same time
+    // and their other phases too, leaving the MUFU idle in between; so over
+    // the first min(nA, nB) tiles of each pair item the two take turns,
+    // passing a token (an mbarrier, waited with the bounded wait) after each
+    // tile's exponentials.  Warpgroup 0 holds the token first.  Both count
+    // the same turns per item, so the phases always match.
+    const int q = warp & 3;
+    const uint32_t tok_mine = bar(TOK + X * 4 + q), tok_other = bar(TOK + (X ^ 1) * 4 + q);
+    int turns = 0;   // token-protected tiles so far
+    if (X == 1 && lane == 0) mbar_arrive(tok_other);
     bool ok = true;
     PairItem it;
     for (int rr = 0; ok && ws_item(a, n_items, rr, it); ++rr) {
       const int n = it.n[X];
       if (n == 0) continue;
+      const int m_turns = min(it.n[0], it.n[1]);
       const int q0 = it.q0[X];
       const int i = q0 + r;
-      float m_used = -INFINITY;
+      float m_used = -INFINITY, l_run = 0.f;
       for (int t = 0; t < n; ++t) {
-        const int g = jg + t, bsel = g & 1;
+        const int g = jg + t, bsel = g % kSBuf;
         const int key0 = (it.kt0[X] + t) * kAttnKeyTile;
-        bool w = mbar_wait(bar(SF + X * 2 + bsel), (g >> 1) & 1, wc, 60);
+        bool w = mbar_wait(bar(SF + X * kSBuf + bsel), (g / kSBuf) & 1, wc, 60);
         if (!__all_sync(0xffffffffu, w)) { ok = false; break; }
         tc_fence_after();
         const uint32_t tS = tX + 64 * bsel;
@@ -353,76 +388,104 @@ swa_attn_ws_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
           }
         }
         // Edge tile: keys outside (i - W, i] of this row, i.e. outside
-        // columns [lo, hi] of the tile, are masked.
-        if (key0 + kAttnKeyTile - 1 > q0 || key0 <= q0 + 127 - W) {
+        // columns [lo, hi] of the tile, are masked.  A tile meets the causal
+        // edge (keys after some row: e > hi) or the window's start (keys too
+        // old for some row: e < lo), both only when W < 192; each test is
+        // skipped when no row of this warp (rows wq0 .. wq0 + 31) needs it.
+        {
+          const int wq0 = q0 + (warp & 3) * 32;
           const int lo = i - W + 1 - key0, hi = i - key0;
+          const bool causal = key0 + kAttnKeyTile - 1 > wq0;        // some row of the warp has hi < 63
+          const bool window = key0 < wq0 + 31 - W + 1;              // some row of the warp has lo > 0
+          if (causal && window) {
 #pragma unroll
-          for (int e = 0; e < 64; ++e) sv[e] = (e >= lo && e <= hi) ? sv[e] : -INFINITY;
+            for (int e = 0; e < 64; ++e) sv[e] = (e >= lo && e <= hi) ? sv[e] : -INFINITY;
+          } else if (causal) {
+#pragma unroll
+            for (int e = 0; e < 64; ++e) sv[e] = e <= hi ? sv[e] : -INFINITY;
+          } else if (window) {
+#pragma unroll
+            for (int e = 0; e < 64; ++e) sv[e] = e >= lo ? sv[e] : -INFINITY;
+          }
         }
-        const float m_tile = fmaxf(tree_max32(sv), tree_max32(sv + 32)) * sl2;
+        const float m_tile = tree_max64(sv) * sl2;
         // Rescale decision (per row): a first finite max just sets m_used (O
-        // and L are still zero); a max more than the slack above m_used
-        // rescales O and L (all of this warpgroup's earlier products must be
+        // and l are still zero); a max more than the slack above m_used
+        // rescales O and l (all of this warpgroup's earlier products must be
         // done: the one of tile t-1 completes BF of its buffer).
         float corr = 1.f;
         if (m_tile > m_used + kRescaleSlack) {
           if (m_used != -INFINITY) corr = ex2_approx(m_used - m_tile);
           m_used = m_tile;
         }
+        l_run *= corr;
         if (t > 0 && __any_sync(0xffffffffu, corr != 1.f)) {
           const int gp = g - 1;
-          w = mbar_wait(bar(BF + X * 2 + (gp & 1)), (gp >> 1) & 1, wc, 61);
+          w = mbar_wait(bar(BF + X * kSBuf + gp % kSBuf), (gp / kSBuf) & 1, wc, 61);
           if (!__all_sync(0xffffffffu, w)) { ok = false; break; }
           tc_fence_after();
-          uint32_t o0[32], o1[32], l1[1];
+          uint32_t o0[32], o1[32];
           tmem_ld32(tO, o0);
           tmem_ld32(tO + 32, o1);
-          tmem_ld1(tL, l1);
           tmem_ld_wait();
 #pragma unroll
           for (int e = 0; e < 32; ++e) {
             o0[e] = __float_as_uint(__uint_as_float(o0[e]) * corr);
             o1[e] = __float_as_uint(__uint_as_float(o1[e]) * corr);
           }
-          l1[0] = __float_as_uint(__uint_as_float(l1[0]) * corr);
           tmem_st32(tO, o0);
           tmem_st32(tO + 32, o1);
-          tmem_st1(tL, l1);
         }
         const float mu = (m_used == -INFINITY) ? 0.f : m_used;
-        // p = 2^(s * scale_log2 - mu), written as bf16 pairs over S's first 32 columns
+        // p = 2^(s * scale_log2 - mu): the arguments first, then (holding the
+        // token) only the 64 exponentials back to back, then the row sum and
+        // P as bf16 pairs over S's first 32 columns while the partner warp
+        // exponentiates.
+        exp2_args64(sv, sl2, mu);
+        const bool turn = t < m_turns;
+        if (turn) {
+          w = mbar_wait(tok_mine, turns & 1, wc, 63);
+          if (!__all_sync(0xffffffffu, w)) { ok = false; break; }
+        }
+#pragma unroll
+        for (int e = 0; e < 64; ++e) sv[e] = ex2_ordered(sv[e]);
+        if (turn) {   // every exponential above is issued before this point (ordered asm): pass the token
+          __syncwarp();
+          if (lane == 0) mbar_arrive(tok_other);
+          ++turns;
+        }
+        float rs = 0.f;
 #pragma unroll
         for (int c = 0; c < 2; ++c) {
-          float pv[32];
-          exp2_scaled32(sv + c * 32, sl2, mu, pv);
+          rs += sum32_tree(*reinterpret_cast<const float(*)[32]>(sv + c * 32));
           uint32_t pk[16];
 #pragma unroll
-          for (int e = 0; e < 16; ++e) pk[e] = pack_bf16x2(pv[2 * e], pv[2 * e + 1]);
+          for (int e = 0; e < 16; ++e) pk[e] = pack_bf16x2(sv[c * 32 + 2 * e], sv[c * 32 + 2 * e + 1]);
           tmem_st16(tS + c * 16, pk);
         }
         tmem_st_wait();
         tc_fence_before();
-        mbar_arrive(bar(PF + X * 2 + bsel));
+        mbar_arrive(bar(PF + X * kSBuf + bsel));
+        l_run += rs;
       }
       if (!ok) break;
       jg += n;
 
-      // Output: O / L once the item's last product is done; O and L are then
+      // Output: O / l once the item's last product is done; O is then
       // released for the warpgroup's next item.
       bool w = mbar_wait(bar(OD + X), kc & 1, wc, 62);
       if (!__all_sync(0xffffffffu, w)) { ok = false; break; }
       tc_fence_after();
-      uint32_t x0[32], x1[32], l1[1];
+      uint32_t x0[32], x1[32];
       tmem_ld32(tO, x0);
       tmem_ld32(tO + 32, x1);
-      tmem_ld1(tL, l1);
       tmem_ld_wait();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(OFREE + X));
       ++kc;
       if (i < a.T) {
-        const float inv_l = 1.0f / __uint_as_float(l1[0]);
+        const float inv_l = 1.0f / l_run;
         uint16_t* dst = static_cast<uint16_t*>(a.out) + static_cast<int64_t>(it.b) * a.o_batch +
                         static_cast<int64_t>(i) * a.o_row + static_cast<int64_t>(it.h) * a.o_head;
         float v0[32], v1[32];
