@@ -52,7 +52,7 @@ rmsnorm_kernel(const float* __restrict__ x, const float* __restrict__ parts, int
   if (row >= M) return;
   const int64_t roff = static_cast<int64_t>(row) * d;
   float4 v[NV];
-  float4 pp[MAXP][NV];
+  float4 pp[MAXP > 0 ? MAXP : 1][NV];
   uint2 bw[NV], gw[NV];
 #pragma unroll
   for (int i = 0; i < NV; ++i) v[i] = reinterpret_cast<const float4*>(x + roff)[lane + 32 * i];
@@ -278,10 +278,16 @@ __global__ void selftest_wait_kernel(DevStatus* st, uint64_t limit_ns) {
 
 }  // namespace
 
+// Without partial sums the row needs no registers for them: a separate
+// instantiation keeps the register count (and so the rows in flight per SM)
+// of the common case at its lowest.
 template <bool BF16, int NV>
 static cudaError_t launch_rms_warp(const Launch& L, const float* x, const float* parts, int nparts, int64_t ps,
                                    const uint16_t* bias, const uint16_t* g, float* h_out, void* y, int M, int d,
                                    float eps) {
+  if (nparts == 0)
+    return launch_kernel(rmsnorm_kernel<BF16, NV, 0>, dim3((M + 3) / 4), dim3(128), 0, L.stream, x, parts, nparts,
+                         ps, bias, g, h_out, y, M, d, eps);
   return launch_kernel(rmsnorm_kernel<BF16, NV, 2>, dim3((M + 3) / 4), dim3(128), 0, L.stream, x, parts, nparts, ps,
                        bias, g, h_out, y, M, d, eps);
 }
