@@ -124,6 +124,10 @@ struct GemmArgs {
   // tmD is then a 3-D map {columns, M, splits} with a 64-byte swizzled box of
   // 64 bytes x 32 rows.
   int tma_store;
+  // Work-unit order: M-fastest (consecutive units share a weight panel of B
+  // through L2) or, when A is the larger operand, N-fastest (the units of one
+  // row panel of A run together, so A crosses DRAM once); set by launch_gemm.
+  int n_fastest;
   DevStatus* status;
   uint64_t limit_ns;
 };
