@@ -85,9 +85,9 @@ def test_bf16_deterministic():
 
 
 def test_bf16_many_items_per_cta_with_single_tile_query_tiles():
-    # More (query tile, head, clip) items than SMs, with many one-key-tile
-    # items (first query tile of each head): every CTA of the persistent kernel
-    # walks several items, including ones where a softmax warpgroup has no tile.
+    # More pair items (two neighbouring query tiles of one clip and head) than
+    # SMs, with short items (the first query tiles of each head see one or two
+    # 64-key tiles): every CTA of the persistent kernel walks several items.
     B, T, H, W = 4, 256, 48, 100
     q, k, v = synth.attention_qkv(B, T, H, 64, seed=11, bf16=True)
     args = [dev(x, torch.bfloat16) for x in (q, k, v)]
@@ -100,9 +100,9 @@ def test_bf16_many_items_per_cta_with_single_tile_query_tiles():
 
 
 def test_bf16_item_pairs_with_odd_item_count():
-    # 5 query tiles x 255 heads = 1275 items: the many-items kernel (two items
-    # per CTA at a time) with pairs that straddle heads and a last pair that
-    # has a single item.
+    # 5 query tiles per head: every third pair item has a single query tile,
+    # so its second softmax warpgroup idles for that item while the K/V ring
+    # and the MUFU turn-taking continue across items.
     B, T, H, W = 1, 640, 255, 300
     q, k, v = synth.attention_qkv(B, T, H, 64, seed=12, bf16=True)
     args = [dev(x, torch.bfloat16) for x in (q, k, v)]
@@ -112,3 +112,20 @@ def test_bf16_item_pairs_with_odd_item_count():
     assert vx.status_check(ws) == 0
     rows = [0, 127, 128, 383, 384, 639]
     compare_bf16(o[:, rows], _oracle_rows(q, k, v, W, rows), "bf16 odd item pairs")
+
+
+def test_bf16_running_max_grows_across_tiles():
+    # Scores that grow along the keys (k_j = 0.05 j e_0, q = 8 e_0, no RoPE:
+    # s_j = 0.05 j, +3.2 per 64-key tile) make the running maximum rise by
+    # more than the rescale slack (2^8) every few tiles, so O and the row sum
+    # are rescaled in place many times; W >= T keeps every key in the window.
+    B, T, H, W = 1, 700, 2, 700
+    q = np.zeros((B, T, H, 64), np.float32)
+    k = np.zeros((B, T, H, 64), np.float32)
+    q[..., 0] = 8.0
+    k[..., 0] = (0.05 * np.arange(T, dtype=np.float32))[None, :, None]
+    v = synth.attention_qkv(B, T, H, 64, seed=13, bf16=True)[2]
+    q, k = synth.bf16_round(q), synth.bf16_round(k)
+    o = _vx().swa_attn_fwd(dev(q, torch.bfloat16), dev(k, torch.bfloat16), dev(v, torch.bfloat16), window=W,
+                           apply_rope=False)
+    compare_bf16(host(o), oracle.swa_attention(q, k, v, W), "bf16 growing max")
