@@ -7,21 +7,25 @@
 //   gemm_tc_kernel<BN>   one CTA per 128 x BN tile (BN 128 / 256);
 //   gemm_tc2_kernel<BN>  a cluster of two CTAs per 256 x BN tile, issued as
 //                        tcgen05.mma.cta_group::2 (M = 256) by the leader CTA.
-// CTA = 10 warps: warps 0-7 epilogue (warp w reads TMEM lanes 32 (w % 4) ..,
-// i.e. 32 tile rows, and half of the tile's columns), warp 8 TMA producer,
-// warp 9 MMA issuer (owns the TMEM allocation).  A 192 KB TMA ->
+// CTA = 11 warps: warps 0-7 epilogue (warp w reads TMEM lanes 32 (w % 4) ..,
+// i.e. 32 tile rows, and half of the tile's columns), warps 8 and 10 TMA
+// producers (alternate K blocks), warp 9 MMA issuer (owns the TMEM
+// allocation).  A 192 KB TMA ->
 // shared memory ring guarded by mbarriers feeds the MMAs; two TMEM
 // accumulators let the epilogue of one tile overlap the main loop of the next.
 // Work units (m tile, K split, n tile) are visited M-fastest, so the CTAs
-// resident at one time share a weight (B) panel through L2, or N-fastest when
-// A is the larger operand (it then crosses DRAM once: measured on the 4 x 3000
-// frame encoder, the down projection read its 123 MB activation ~2.5 times
-// over in M-fastest order).
+// resident at one time share a weight (B) panel through L2, N-fastest when A
+// is the larger operand and too large for L2 (it then crosses DRAM once), or
+// in groups of four row panels (launch_gemm chooses).
 //
 // The main loop is bound by how fast TMA can fill one SM's shared memory, so
 // the tile shape is chosen to move the fewest bytes per MMA: a CTA pair
 // stages 16 KB of A and BN/2 rows of B per 64-wide K block for 128 x BN of
-// MMA work (plan_gemm picks the shape, see below).
+// MMA work (plan_gemm picks the shape, see below).  Issuing a 16 KB tile load
+// keeps the issuing thread ~160-250 cycles (measured), and with its barrier
+// wait and bookkeeping one thread needs about as long per K block as the
+// MMAs of a 256-wide block take, so it could never run ahead of them; two
+// producer threads in separate warps take alternate K blocks.
 //
 // Epilogue: each warp reads 32 rows x 32 columns at a time from TMEM (one row
 // per lane), applies the row-wise part of the epilogue (bias, RoPE pairs,
@@ -39,9 +43,15 @@ namespace vx {
 
 namespace {
 
-constexpr int kThreads = 320;   // warps 0-7 epilogue, 8 TMA producer, 9 MMA issuer
+constexpr int kThreads = 352;   // warps 0-7 epilogue, 8 and 10 TMA producers, 9 MMA issuer
 constexpr int kProducerWarp = 8;
 constexpr int kMmaWarp = 9;
+constexpr int kProducer2Warp = 10;
+
+// Producer index of a warp (0, 1), or -1.
+__device__ __forceinline__ int producer_of(int warp) {
+  return warp == kProducerWarp ? 0 : (warp == kProducer2Warp ? 1 : -1);
+}
 constexpr int kBM = 128;
 constexpr int kBK = 64;
 constexpr int kABytes = kBM * kBK * 2;
@@ -403,6 +413,56 @@ __device__ __forceinline__ void epilogue_tile(const GemmArgs& a, EpiPre<BN, EPI>
   }
 }
 
+// Work unit u -> (m tile, n tile, K split) in the launch's order (GemmArgs::order;
+// the grouped order is only set without K splits).
+__device__ __forceinline__ void unit_coords(const GemmArgs& a, int u, int m_tiles, int n_tiles, int& mt, int& nt,
+                                            int& ks) {
+  const int splits = a.k_splits;
+  if (a.order == kOrderGrouped) {
+    const int per = kOrderGroupRows * n_tiles;   // units of one group of row panels
+    const int g = u / per, r = u - g * per;
+    const int rem = m_tiles - g * kOrderGroupRows;
+    const int gm = rem < kOrderGroupRows ? rem : kOrderGroupRows;
+    mt = g * kOrderGroupRows + r % gm;
+    nt = r / gm;
+    ks = 0;
+  } else if (a.order == kOrderNFastest) {
+    nt = u % n_tiles;
+    const int r = u / n_tiles;
+    ks = r % splits;
+    mt = r / splits;
+  } else {
+    mt = u % m_tiles;
+    const int r = u / m_tiles;
+    ks = r % splits;
+    nt = r / splits;
+  }
+}
+
+// A-operand coordinates of consecutive K blocks (GemmArgs: tap = kb /
+// kb_per_tap, c = kb % kb_per_tap, x = (tap % a_stride) a_tap_ch + 64 c,
+// y = m0 + tap / a_stride), advanced one block at a time.
+struct ACoord {
+  int tap, c, x0, y;
+  __device__ __forceinline__ void set(const GemmArgs& a, int m0) {
+    x0 = (tap % a.a_stride) * a.a_tap_ch;
+    y = m0 + tap / a.a_stride;
+  }
+  __device__ __forceinline__ void start(const GemmArgs& a, int kb, int m0) {
+    tap = kb / a.kb_per_tap;
+    c = kb - tap * a.kb_per_tap;
+    set(a, m0);
+  }
+  __device__ __forceinline__ int x() const { return x0 + c * kBK; }
+  __device__ __forceinline__ void next(const GemmArgs& a, int m0) {
+    if (++c == a.kb_per_tap) {
+      c = 0;
+      ++tap;
+      set(a, m0);
+    }
+  }
+};
+
 // ---------------------------------------------------------------- 1 CTA --
 template <int BN>
 struct OneCfg {
@@ -465,67 +525,58 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
   const int n_tiles = a.N / BN;
   auto decode = [&](int u, int& m0, int& n0, int& ks) {
     int mt, nt;
-    if (a.n_fastest) {
-      nt = u % n_tiles;
-      const int r = u / n_tiles;
-      ks = r % splits;
-      mt = r / splits;
-    } else {
-      mt = u % m_tiles;
-      const int r = u / m_tiles;
-      ks = r % splits;
-      nt = r / splits;
-    }
+    unit_coords(a, u, m_tiles, n_tiles, mt, nt, ks);
     m0 = mt * kBM;
     n0 = nt * BN;
   };
 
   // The weights (B) do not depend on the previous kernel of the stream: the
-  // producer starts streaming the first stages' B tiles before waiting for it.
+  // producers start streaming the first stages' B tiles before waiting for
+  // it.  Their completions may reach a full barrier before it is armed (a
+  // barrier's transaction count may run negative within a phase).
+  const int prod = producer_of(warp);
   int npre = 0;
-  if (warp == kProducerWarp && lane == 0 && blockIdx.x < num_tiles) {
+  if (prod >= 0 && lane == 0 && blockIdx.x < num_tiles) {
     int m0, n0, ks;
     decode(blockIdx.x, m0, n0, ks);
     npre = nkb < S ? nkb : S;
-    for (int i = 0; i < npre; ++i) {
-      mbar_arrive_expect_tx(full(i), kABytes + C::kBBytes);
+    for (int i = prod; i < npre; i += 2)
       tma_load_2d(smem_addr(sB + i * C::kBBytes), &tmB, full(i), (ks * nkb + i) * kBK, n0);
-    }
   }
   // Inputs written by the previous kernel of the stream are read below.
   pdl_wait();
   pdl_trigger();
 
-  if (warp == kProducerWarp) {
+  if (prod >= 0) {
+    // Producer `prod` fills the stages of the K blocks it with it % 2 == prod.
     if (lane == 0) {
       int stage = 0;
       uint32_t phase = 0;
-      uint32_t issued = 0;    // bit s: stage s was filled at least once
-      uint32_t last_par = 0;  // bit s: parity of the last fill of stage s
-      int it = 0;             // k-block iterations issued so far
+      uint32_t issued = 0;    // bit s: this thread filled stage s at least once
+      uint32_t last_par = 0;  // bit s: parity of its last fill of stage s
+      int it = 0;             // k-block iterations so far
       for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
         int m0, n0, ks;
         decode(tile, m0, n0, ks);
+        ACoord ac;
+        ac.start(a, ks * nkb, m0);
         bool ok = true;
-        for (int kb = ks * nkb; kb < (ks + 1) * nkb; ++kb, ++it) {
-          const bool pre = it < npre;   // B already in flight, barrier already armed
-          if (!pre) {
+        for (int i = 0; i < nkb; ++i, ++it) {
+          if ((it & 1) == prod) {
             if (!mbar_wait(empty(stage), phase ^ 1, wc, 1)) { ok = false; break; }
             mbar_arrive_expect_tx(full(stage), kABytes + C::kBBytes);
+            tma_load_2d(smem_addr(sA + stage * kABytes), &tmA, full(stage), ac.x(), ac.y);
+            if (it >= npre)   // the first npre B tiles are in flight already
+              tma_load_2d(smem_addr(sB + stage * C::kBBytes), &tmB, full(stage), (ks * nkb + i) * kBK, n0);
+            issued |= 1u << stage;
+            last_par = (last_par & ~(1u << stage)) | (phase << stage);
           }
-          const int tap = kb / a.kb_per_tap;
-          const int c = (kb - tap * a.kb_per_tap) * kBK;
-          const int ax = (tap % a.a_stride) * a.a_tap_ch + c;
-          const int ay = m0 + tap / a.a_stride;
-          tma_load_2d(smem_addr(sA + stage * kABytes), &tmA, full(stage), ax, ay);
-          if (!pre) tma_load_2d(smem_addr(sB + stage * C::kBBytes), &tmB, full(stage), kb * kBK, n0);
-          issued |= 1u << stage;
-          last_par = (last_par & ~(1u << stage)) | (phase << stage);
+          ac.next(a, m0);
           if (++stage == S) { stage = 0; phase ^= 1; }
         }
         if (!ok) break;
       }
-      // Wait (bounded, even after an abort) for the copies this thread issued.
+      // Wait (bounded, even after an abort) for the stages this thread armed.
       int zero = 0;
       WaitCtx dw = wc;
       dw.abort_flag = &zero;
@@ -673,65 +724,57 @@ gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
   const int n_tiles = a.N / BN;
   auto decode = [&](int u, int& m0, int& n0, int& ks) {
     int mt, nt;
-    if (a.n_fastest) {
-      nt = u % n_tiles;
-      const int r = u / n_tiles;
-      ks = r % splits;
-      mt = r / splits;
-    } else {
-      mt = u % m_tiles;
-      const int r = u / m_tiles;
-      ks = r % splits;
-      nt = r / splits;
-    }
+    unit_coords(a, u, m_tiles, n_tiles, mt, nt, ks);
     m0 = mt * 256 + 128 * rank;
     n0 = nt * BN;
   };
 
-  // The weights (B) do not depend on the previous kernel of the stream: both
-  // CTAs start streaming their halves of the first stages' B tiles before
-  // waiting for it; the leader arms the full barriers for whole stages.
+  // The weights (B) do not depend on the previous kernel of the stream: the
+  // producers of each CTA start streaming their halves of the first stages'
+  // B tiles before waiting for it.  Their completions may reach the leader's
+  // full barriers before they are armed (a barrier's transaction count may
+  // run negative within a phase).
+  const int prod = producer_of(warp);
   int npre = 0;
-  if (warp == kProducerWarp && lane == 0 && cluster < num_tiles) {
+  if (prod >= 0 && lane == 0 && cluster < num_tiles) {
     int m0, n0, ks;
     decode(cluster, m0, n0, ks);
     npre = nkb < S ? nkb : S;
-    for (int i = 0; i < npre; ++i) {
-      if (rank == 0) mbar_arrive_expect_tx(full(i), 2 * C::kStageBytes);
+    for (int i = prod; i < npre; i += 2)
       tma_load_2d_pair(smem_addr(sB + i * C::kBHalfBytes), &tmB, map_to_cta(full(i), 0), (ks * nkb + i) * kBK,
                        n0 + (BN / 2) * rank);
-    }
   }
   // Inputs written by the previous kernel of the stream are read below.
   pdl_wait();
   pdl_trigger();
 
-  if (warp == kProducerWarp) {
+  if (prod >= 0) {
+    // Producer `prod` fills the stages of the K blocks it with it % 2 == prod;
+    // the leader's arms their full barriers for the pair's four copies.
     if (lane == 0) {
       int stage = 0;
       uint32_t phase = 0;
       uint32_t issued = 0, last_par = 0;
-      int it = 0;   // k-block iterations issued so far
+      int it = 0;   // k-block iterations so far
       for (int tile = cluster; tile < num_tiles; tile += nclusters) {
         int m0, n0, ks;
         decode(tile, m0, n0, ks);
+        ACoord ac;
+        ac.start(a, ks * nkb, m0);
         bool ok = true;
-        for (int kb = ks * nkb; kb < (ks + 1) * nkb; ++kb, ++it) {
-          const bool pre = it < npre;   // B already in flight, barrier already armed
-          if (!pre) {
+        for (int i = 0; i < nkb; ++i, ++it) {
+          if ((it & 1) == prod) {
             if (!mbar_wait(empty(stage), phase ^ 1, wc, 31)) { ok = false; break; }
+            const uint32_t fb = map_to_cta(full(stage), 0);   // the leader's full barrier
             if (rank == 0) mbar_arrive_expect_tx(full(stage), 2 * C::kStageBytes);
+            tma_load_2d_pair(smem_addr(sA + stage * kABytes), &tmA, fb, ac.x(), ac.y);
+            if (it >= npre)   // the first npre B tiles are in flight already
+              tma_load_2d_pair(smem_addr(sB + stage * C::kBHalfBytes), &tmB, fb, (ks * nkb + i) * kBK,
+                               n0 + (BN / 2) * rank);
+            issued |= 1u << stage;
+            last_par = (last_par & ~(1u << stage)) | (phase << stage);
           }
-          const uint32_t fb = map_to_cta(full(stage), 0);   // the leader's full barrier
-          const int tap = kb / a.kb_per_tap;
-          const int c = (kb - tap * a.kb_per_tap) * kBK;
-          const int ax = (tap % a.a_stride) * a.a_tap_ch + c;
-          const int ay = m0 + tap / a.a_stride;
-          tma_load_2d_pair(smem_addr(sA + stage * kABytes), &tmA, fb, ax, ay);
-          if (!pre)
-            tma_load_2d_pair(smem_addr(sB + stage * C::kBHalfBytes), &tmB, fb, kb * kBK, n0 + (BN / 2) * rank);
-          issued |= 1u << stage;
-          last_par = (last_par & ~(1u << stage)) | (phase << stage);
+          ac.next(a, m0);
           if (++stage == S) { stage = 0; phase ^= 1; }
         }
         if (!ok) break;
@@ -898,17 +941,26 @@ GemmPlan plan_gemm(int M, int N, int K, int epi, int max_splits, int sm) {
 cudaError_t launch_gemm(const Launch& L, const CUtensorMap& tmA, const CUtensorMap& tmB, const CUtensorMap& tmD,
                         const GemmArgs& args, int epi, const GemmPlan& p) {
   if (args.M <= 0) return cudaSuccess;
-  if (args.k_splits != p.splits || p.splits < 1 || (args.K / kBK) % p.splits != 0 || args.K % kBK != 0 ||
+  if (args.out == nullptr || args.k_splits != p.splits || p.splits < 1 || (args.K / kBK) % p.splits != 0 || args.K % kBK != 0 ||
       p.bn <= 0 || args.N % p.bn != 0 || (p.splits > 1 && epi != EPI_F32) ||
       (args.tma_store && epi != EPI_F32 && epi != EPI_QKV_ROPE && epi != EPI_SWIGLU))
     return cudaErrorInvalidValue;
   // Walk the work units so that the larger operand crosses DRAM once: A
   // goes first when it is the larger one and too large to stay in L2 while
-  // it is walked once per column tile (measured: the encoder's 31-123 MB
-  // activations gain from it, a one-layer batch's 6-15 MB ones lose a little).
+  // it is walked once per column tile (the encoder's 123 MB down-projection
+  // input read it ~2.5 times over in M-fastest order).  Activations of
+  // 16-64 MB (the encoder's QKV, gate/up and O inputs) are walked in groups
+  // of four row panels: measured on the 4 x 3000 frame encoder, the QKV
+  // projection 148 -> 142 us against either plain order, the others
+  // unchanged; a one-layer batch's 6-15 MB inputs keep the M-fastest order.
   GemmArgs a2 = args;
   const int64_t a_bytes = static_cast<int64_t>(args.M) * args.K * 2, b_bytes = static_cast<int64_t>(args.N) * args.K * 2;
-  a2.n_fastest = (a_bytes > b_bytes && a_bytes >= (int64_t(16) << 20)) ? 1 : 0;
+  if (a_bytes > b_bytes && a_bytes >= (int64_t(64) << 20))
+    a2.order = kOrderNFastest;
+  else if (a_bytes >= (int64_t(16) << 20) && args.k_splits == 1)
+    a2.order = kOrderGrouped;
+  else
+    a2.order = kOrderMFastest;
   const GemmArgs& a = a2;
   switch (epi) {
     case EPI_F32: return launch_epi<EPI_F32>(L, tmA, tmB, tmD, a, p);

@@ -97,6 +97,9 @@ enum EpiKind : int {
   EPI_GELU_F32 = 4,   // out fp32 = GELU(acc + bias)
 };
 
+constexpr int kOrderMFastest = 0, kOrderNFastest = 1, kOrderGrouped = 2;
+constexpr int kOrderGroupRows = 4;
+
 struct GemmArgs {
   int M, N, K;
   // Split-K: the K loop is cut into k_splits equal parts; part ks writes its
@@ -124,10 +127,11 @@ struct GemmArgs {
   // tmD is then a 3-D map {columns, M, splits} with a 64-byte swizzled box of
   // 64 bytes x 32 rows.
   int tma_store;
-  // Work-unit order: M-fastest (consecutive units share a weight panel of B
-  // through L2) or, when A is the larger operand, N-fastest (the units of one
-  // row panel of A run together, so A crosses DRAM once); set by launch_gemm.
-  int n_fastest;
+  // Work-unit order (kOrder*), set by launch_gemm: M-fastest (consecutive
+  // units share a weight panel of B through L2), N-fastest (the units of one
+  // row panel of A run together, so A crosses DRAM once) or groups of
+  // kOrderGroupRows row panels, M-fastest inside a group.
+  int order;
   DevStatus* status;
   uint64_t limit_ns;
 };
