@@ -9,7 +9,7 @@
 //                        tcgen05.mma.cta_group::2 (M = 256) by the leader CTA.
 // CTA = 11 warps: warps 0-7 epilogue (warp w reads TMEM lanes 32 (w % 4) ..,
 // i.e. 32 tile rows, and half of the tile's columns), warps 8 and 10 TMA
-// producers (alternate K blocks), warp 9 MMA issuer (owns the TMEM
+// producers (even / odd ring stages), warp 9 MMA issuer (owns the TMEM
 // allocation).  A 192 KB TMA ->
 // shared memory ring guarded by mbarriers feeds the MMAs; two TMEM
 // accumulators let the epilogue of one tile overlap the main loop of the next.
@@ -25,7 +25,7 @@
 // keeps the issuing thread ~160-250 cycles (measured), and with its barrier
 // wait and bookkeeping one thread needs about as long per K block as the
 // MMAs of a 256-wide block take, so it could never run ahead of them; two
-// producer threads in separate warps take alternate K blocks.
+// producer threads in separate warps split the ring's stages (even / odd).
 //
 // Epilogue: each warp reads 32 rows x 32 columns at a time from TMEM (one row
 // per lane), applies the row-wise part of the epilogue (bias, RoPE pairs,
@@ -55,20 +55,27 @@ __device__ __forceinline__ int producer_of(int warp) {
 constexpr int kBM = 128;
 constexpr int kBK = 64;
 constexpr int kABytes = kBM * kBK * 2;
-constexpr int kRingBytes = 192 * 1024;        // TMA ring per CTA
-constexpr int kStgBytes = 8 * 2048;           // per epilogue warp: 32 rows x 64 bytes
+constexpr int kSmemBytes = 227 * 1024;        // per CTA
+constexpr int kStgBufBytes = 2048;            // 32 rows x 64 bytes
 constexpr int kBiasBytes = 8 * 256 * 2;       // per epilogue warp: the tile's bias, BN <= 256
 constexpr int kBarBytes = 256;
 
-// Shared memory: [ring][staging][bias][barriers], 1024-aligned base.
-template <int STAGE_BYTES>
+// Staging buffers per epilogue warp: two for the QKV epilogue, whose stores
+// would otherwise wait for one another (measured: 4 x 3000 frame encoder, QKV
+// 144 -> 138 us), one elsewhere (a second one would cost a ring stage).
+constexpr int stg_bufs(int epi) { return epi == EPI_QKV_ROPE ? 2 : 1; }
+
+// Shared memory: [ring][staging][bias][barriers], 1024-aligned base; the TMA
+// ring takes as many stages as fit.
+template <int STAGE_BYTES, int NBUF>
 struct SmemCfg {
-  static constexpr int kStages = kRingBytes / STAGE_BYTES;
+  static constexpr int kStgBytes = 8 * NBUF * kStgBufBytes;
+  static constexpr int kStages = (kSmemBytes - kStgBytes - kBiasBytes - kBarBytes - 1024) / STAGE_BYTES;
   static constexpr int kStg = kStages * STAGE_BYTES;
   static constexpr int kBias = kStg + kStgBytes;
   static constexpr int kBars = kBias + kBiasBytes;
   static constexpr int kTotal = kBars + kBarBytes + 1024;
-  static_assert(kStages >= 4, "ring too shallow");
+  static_assert(kStages >= 3 && kStages <= 12, "ring depth");
   static_assert(kTotal <= 227 * 1024, "shared memory");
 };
 
@@ -187,26 +194,42 @@ __device__ __forceinline__ void store_bf16_chunk(uint16_t* out, int64_t ld_out, 
 
 // Output path of one staged chunk.  With TMA stores the chunk leaves shared
 // memory as one 64-byte x 32-row box (the staging swizzle is the tensor map's
-// 64-byte swizzle), written by lane 0; before the staging buffer is refilled,
-// lane 0 waits for the copy engine to have read it.
+// 64-byte swizzle), written by lane 0.  With two staging buffers they take
+// turns, so a chunk is staged while the copy engine still reads the previous
+// one: before a buffer is refilled, lane 0 waits until at most one store (the
+// other buffer's) is still reading; with one, until none is.  Without TMA
+// stores one buffer serves.
 struct ChunkOut {
   const CUtensorMap* tmD;   // null: stores from registers
   int row0;                 // first tile row of this warp
   int z;                    // K-split index (third map coordinate)
+  uint4* stg;               // the warp's staging buffers (128 x 16 bytes each)
+  int nbuf;                 // 1 or 2
+  int n;                    // chunks stored by this warp so far (across tiles)
 };
-__device__ __forceinline__ void stage_reuse(const ChunkOut& co, int lane) {
-  if (co.tmD) {
-    if (lane == 0) bulk_wait_read_all();
-    __syncwarp();
-  }
+__device__ __forceinline__ void bulk_wait_read_but_one() {
+  asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
 }
-__device__ __forceinline__ void tma_flush(const ChunkOut& co, const uint4* stg, int lane, int col0) {
+// The buffer for the next chunk, free to be written.
+__device__ __forceinline__ uint4* stage_buf(const ChunkOut& co, int lane) {
+  if (!co.tmD) return co.stg;
+  if (lane == 0) {
+    if (co.nbuf == 2)
+      bulk_wait_read_but_one();
+    else
+      bulk_wait_read_all();
+  }
+  __syncwarp();
+  return co.nbuf == 2 ? co.stg + 128 * (co.n & 1) : co.stg;
+}
+__device__ __forceinline__ void tma_flush(ChunkOut& co, const uint4* buf, int lane, int col0) {
   fence_proxy_async_smem();   // this lane's staging writes, visible to the copy engine
   __syncwarp();
   if (lane == 0) {
-    tma_store_3d(co.tmD, smem_addr(stg), col0, co.row0, co.z);
+    tma_store_3d(co.tmD, smem_addr(buf), col0, co.row0, co.z);
     bulk_commit_group();
   }
+  ++co.n;
 }
 
 // Per warp: TMEM lane quarter q = warp & 3 (tile rows 32 q ..), and one half
@@ -266,8 +289,7 @@ __device__ __forceinline__ void epilogue_prepare(const GemmArgs& a, EpiPre<BN, E
 // The accumulator part: tacc = this warp's TMEM lanes at the tile's column 0.
 template <int BN, int EPI>
 __device__ __forceinline__ void epilogue_tile(const GemmArgs& a, EpiPre<BN, EPI>& p, const uint16_t* sbias,
-                                              uint4* stg, uint32_t tacc, int n0, int ks, int warp, int lane,
-                                              const ChunkOut& co) {
+                                              uint32_t tacc, int n0, int ks, int warp, int lane, ChunkOut& co) {
   const bool use_bias = a.bias != nullptr && ks == 0;
   const int hf = warp >> 2;
   if constexpr (EPI == EPI_QKV_ROPE) {
@@ -294,7 +316,7 @@ __device__ __forceinline__ void epilogue_tile(const GemmArgs& a, EpiPre<BN, EPI>
       }
 #pragma unroll
       for (int part = 0; part < 2; ++part) {
-        stage_reuse(co, lane);
+        uint4* stg = stage_buf(co, lane);
         stage_bf16x32(stg, lane, part ? x1 : x0);
         if (co.tmD) {
           tma_flush(co, stg, lane, n0 + c + 32 * part);
@@ -322,7 +344,7 @@ __device__ __forceinline__ void epilogue_tile(const GemmArgs& a, EpiPre<BN, EPI>
       if (use_bias) { add_bias32_smem(gv, sbias + g + hh); add_bias32_smem(uv, sbias + g + 64 + hh); }
 #pragma unroll
       for (int i = 0; i < 32; ++i) gv[i] = silu_f(gv[i]) * uv[i];
-      stage_reuse(co, lane);
+      uint4* stg = stage_buf(co, lane);
       stage_bf16x32(stg, lane, gv);
       if (co.tmD) {
         tma_flush(co, stg, lane, (n0 + g) / 2 + hh);
@@ -348,6 +370,7 @@ __device__ __forceinline__ void epilogue_tile(const GemmArgs& a, EpiPre<BN, EPI>
       if constexpr (EPI == EPI_GELU_BF16) {
 #pragma unroll
         for (int i = 0; i < 32; ++i) v[i] = gelu_erf(v[i]);
+        uint4* stg = co.stg;   // no TMA stores for GELU outputs
         stage_bf16x32(stg, lane, v);
         __syncwarp();
         store_bf16_chunk(static_cast<uint16_t*>(a.out), a.ld_out, p.sr, stg, lane, n0 + c);
@@ -361,7 +384,7 @@ __device__ __forceinline__ void epilogue_tile(const GemmArgs& a, EpiPre<BN, EPI>
         }
 #pragma unroll
         for (int h16 = 0; h16 < 32; h16 += 16) {
-          stage_reuse(co, lane);
+          uint4* stg = stage_buf(co, lane);
           stage_f32x16(stg, lane, v + h16);
           __syncwarp();
           float4 o[4];
@@ -464,10 +487,10 @@ struct ACoord {
 };
 
 // ---------------------------------------------------------------- 1 CTA --
-template <int BN>
+template <int BN, int EPI>
 struct OneCfg {
   static constexpr int kBBytes = BN * kBK * 2;
-  using S = SmemCfg<kABytes + kBBytes>;
+  using S = SmemCfg<kABytes + kBBytes, stg_bufs(EPI)>;
   static constexpr int kTmemCols = 2 * BN;   // two accumulators
 };
 
@@ -475,7 +498,7 @@ template <int BN, int EPI>
 __global__ void __launch_bounds__(kThreads, 1)
 gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                const __grid_constant__ CUtensorMap tmD, const __grid_constant__ GemmArgs a) {
-  using C = OneCfg<BN>;
+  using C = OneCfg<BN, EPI>;
   constexpr int S = C::S::kStages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -548,7 +571,8 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
   pdl_trigger();
 
   if (prod >= 0) {
-    // Producer `prod` fills the stages of the K blocks it with it % 2 == prod.
+    // Producer `prod` fills the ring stages s with s % 2 == prod (so every
+    // fill of a stage, and its drain below, belongs to one thread).
     if (lane == 0) {
       int stage = 0;
       uint32_t phase = 0;
@@ -562,7 +586,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
         ac.start(a, ks * nkb, m0);
         bool ok = true;
         for (int i = 0; i < nkb; ++i, ++it) {
-          if ((it & 1) == prod) {
+          if ((stage & 1) == prod) {
             if (!mbar_wait(empty(stage), phase ^ 1, wc, 1)) { ok = false; break; }
             mbar_arrive_expect_tx(full(stage), kABytes + C::kBBytes);
             tma_load_2d(smem_addr(sA + stage * kABytes), &tmA, full(stage), ac.x(), ac.y);
@@ -586,6 +610,11 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
   } else if (warp == kMmaWarp) {
     if (lane == 0) {
       const uint32_t idesc = idesc_bf16_f32(kBM, BN, 0);
+      // Descriptors of stage 0's A and B; a stage, and a 16-deep K step (32
+      // bytes) inside the 128-byte swizzled rows, add to the address field
+      // (address / 16, 14 bits: shared memory stays below 256 KB).
+      const uint64_t desc_a0 = smem_desc_sw128(smem_addr(sA), 16, 1024);
+      const uint64_t desc_b0 = smem_desc_sw128(smem_addr(sB), 16, 1024);
       int stage = 0;
       uint32_t phase = 0;
       int local = 0;
@@ -599,13 +628,10 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
         for (int kb = 0; kb < nkb; ++kb) {
           if (!mbar_wait(full(stage), phase, wc, 3)) { ok = false; break; }
           tc_fence_after();
-          const uint32_t a0 = smem_addr(sA + stage * kABytes);
-          const uint32_t b0 = smem_addr(sB + stage * C::kBBytes);
+          const uint64_t da = desc_a0 + static_cast<uint32_t>(stage * (kABytes >> 4));
+          const uint64_t db = desc_b0 + static_cast<uint32_t>(stage * (C::kBBytes >> 4));
 #pragma unroll
-          for (int k = 0; k < kBK / 16; ++k) {
-            umma_bf16(d_tmem, smem_desc_sw128(a0 + 32 * k, 16, 1024),
-                      smem_desc_sw128(b0 + 32 * k, 16, 1024), idesc, (kb | k) != 0);
-          }
+          for (int k = 0; k < kBK / 16; ++k) umma_bf16(d_tmem, da + 2 * k, db + 2 * k, idesc, (kb | k) != 0);
           umma_commit(empty(stage));
           if (++stage == S) { stage = 0; phase ^= 1; }
         }
@@ -620,7 +646,8 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
       mbar_wait(drain, 0, dw, 6);
     }
   } else {
-    uint4* stg = reinterpret_cast<uint4*>(stg_all) + warp * 128;
+    uint4* stg = reinterpret_cast<uint4*>(stg_all) + warp * (stg_bufs(EPI) * 128);
+    int stg_n = 0;   // chunks this warp has stored (the staging buffers alternate across tiles)
     int local = 0;
     for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++local) {
       int m0, n0, ks;
@@ -635,8 +662,9 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
       if (!ok) break;
       tc_fence_after();
       const uint32_t tacc = tmem_base + ab * BN + (static_cast<uint32_t>((warp & 3) * 32) << 16);
-      const ChunkOut co{a.tma_store ? &tmD : nullptr, m0 + (warp & 3) * 32, ks};
-      epilogue_tile<BN, EPI>(a, pre, sbias, stg, tacc, n0, ks, warp, lane, co);
+      ChunkOut co{a.tma_store ? &tmD : nullptr, m0 + (warp & 3) * 32, ks, stg, stg_bufs(EPI), stg_n};
+      epilogue_tile<BN, EPI>(a, pre, sbias, tacc, n0, ks, warp, lane, co);
+      stg_n = co.n;
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(acc_empty(ab));
@@ -659,11 +687,11 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
 // to the empty / accumulator barriers of both CTAs; both CTAs' epilogue warps
 // release an accumulator on the leader's barrier.  Each CTA's epilogue handles
 // its 128 rows x BN columns from its own TMEM.
-template <int BN>
+template <int BN, int EPI>
 struct PairCfg {
   static constexpr int kBHalfBytes = (BN / 2) * kBK * 2;
   static constexpr int kStageBytes = kABytes + kBHalfBytes;
-  using S = SmemCfg<kStageBytes>;
+  using S = SmemCfg<kStageBytes, stg_bufs(EPI)>;
   static constexpr int kTmemCols = 2 * BN;
 };
 
@@ -671,7 +699,7 @@ template <int BN, int EPI>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                 const __grid_constant__ CUtensorMap tmD, const __grid_constant__ GemmArgs a) {
-  using C = PairCfg<BN>;
+  using C = PairCfg<BN, EPI>;
   constexpr int S = C::S::kStages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -749,8 +777,9 @@ gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
   pdl_trigger();
 
   if (prod >= 0) {
-    // Producer `prod` fills the stages of the K blocks it with it % 2 == prod;
-    // the leader's arms their full barriers for the pair's four copies.
+    // Producer `prod` fills the ring stages s with s % 2 == prod (so every
+    // fill of a stage, and its drain below, belongs to one thread); the
+    // leader's arms their full barriers for the pair's four copies.
     if (lane == 0) {
       int stage = 0;
       uint32_t phase = 0;
@@ -763,7 +792,7 @@ gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
         ac.start(a, ks * nkb, m0);
         bool ok = true;
         for (int i = 0; i < nkb; ++i, ++it) {
-          if ((it & 1) == prod) {
+          if ((stage & 1) == prod) {
             if (!mbar_wait(empty(stage), phase ^ 1, wc, 31)) { ok = false; break; }
             const uint32_t fb = map_to_cta(full(stage), 0);   // the leader's full barrier
             if (rank == 0) mbar_arrive_expect_tx(full(stage), 2 * C::kStageBytes);
@@ -790,6 +819,11 @@ gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
   } else if (warp == kMmaWarp) {
     if (lane == 0 && rank == 0) {
       const uint32_t idesc = idesc_bf16_f32(256, BN, 0);
+      // Descriptors of stage 0's A and B; a stage, and a 16-deep K step (32
+      // bytes) inside the 128-byte swizzled rows, add to the address field
+      // (address / 16, 14 bits: shared memory stays below 256 KB).
+      const uint64_t desc_a0 = smem_desc_sw128(smem_addr(sA), 16, 1024);
+      const uint64_t desc_b0 = smem_desc_sw128(smem_addr(sB), 16, 1024);
       int stage = 0;
       uint32_t phase = 0;
       int local = 0;
@@ -803,12 +837,10 @@ gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
         for (int kb = 0; kb < nkb; ++kb) {
           if (!mbar_wait(full(stage), phase, wc, 33)) { ok = false; break; }
           tc_fence_after();
-          const uint32_t a0 = smem_addr(sA + stage * kABytes);
-          const uint32_t b0 = smem_addr(sB + stage * C::kBHalfBytes);
+          const uint64_t da = desc_a0 + static_cast<uint32_t>(stage * (kABytes >> 4));
+          const uint64_t db = desc_b0 + static_cast<uint32_t>(stage * (C::kBHalfBytes >> 4));
 #pragma unroll
-          for (int k = 0; k < kBK / 16; ++k)
-            umma_bf16_pair(d_tmem, smem_desc_sw128(a0 + 32 * k, 16, 1024), smem_desc_sw128(b0 + 32 * k, 16, 1024),
-                           idesc, (kb | k) != 0);
+          for (int k = 0; k < kBK / 16; ++k) umma_bf16_pair(d_tmem, da + 2 * k, db + 2 * k, idesc, (kb | k) != 0);
           umma_commit_pair(empty(stage), 0x3);
           if (++stage == S) { stage = 0; phase ^= 1; }
         }
@@ -822,7 +854,8 @@ gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
       mbar_wait(drain, 0, dw, 36);
     }
   } else {
-    uint4* stg = reinterpret_cast<uint4*>(stg_all) + warp * 128;
+    uint4* stg = reinterpret_cast<uint4*>(stg_all) + warp * (stg_bufs(EPI) * 128);
+    int stg_n = 0;   // chunks this warp has stored (the staging buffers alternate across tiles)
     int local = 0;
     const uint32_t acc_empty_leader0 = map_to_cta(acc_empty(0), 0);
     const uint32_t acc_empty_leader1 = map_to_cta(acc_empty(1), 0);
@@ -839,8 +872,9 @@ gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
       if (!ok) break;
       tc_fence_after();
       const uint32_t tacc = tmem_base + ab * BN + (static_cast<uint32_t>((warp & 3) * 32) << 16);
-      const ChunkOut co{a.tma_store ? &tmD : nullptr, m0 + (warp & 3) * 32, ks};
-      epilogue_tile<BN, EPI>(a, pre, sbias, stg, tacc, n0, ks, warp, lane, co);
+      ChunkOut co{a.tma_store ? &tmD : nullptr, m0 + (warp & 3) * 32, ks, stg, stg_bufs(EPI), stg_n};
+      epilogue_tile<BN, EPI>(a, pre, sbias, tacc, n0, ks, warp, lane, co);
+      stg_n = co.n;
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(ab ? acc_empty_leader1 : acc_empty_leader0);
@@ -861,7 +895,7 @@ gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
 template <int BN, int EPI>
 cudaError_t launch_one(const Launch& L, const CUtensorMap& tmA, const CUtensorMap& tmB, const CUtensorMap& tmD,
                        const GemmArgs& a) {
-  using C = OneCfg<BN>;
+  using C = OneCfg<BN, EPI>;
   const int tiles = ((a.M + kBM - 1) / kBM) * (a.N / BN) * a.k_splits;
   const int grid = tiles < L.sm_count ? tiles : L.sm_count;
   return launch_kernel(gemm_tc_kernel<BN, EPI>, dim3(grid), dim3(kThreads), C::S::kTotal, L.stream, tmA, tmB, tmD,
@@ -871,7 +905,7 @@ cudaError_t launch_one(const Launch& L, const CUtensorMap& tmA, const CUtensorMa
 template <int BN, int EPI>
 cudaError_t launch_pair(const Launch& L, const CUtensorMap& tmA, const CUtensorMap& tmB, const CUtensorMap& tmD,
                         const GemmArgs& a) {
-  using C = PairCfg<BN>;
+  using C = PairCfg<BN, EPI>;
   const int tiles = ((a.M + 255) / 256) * (a.N / BN) * a.k_splits;
   const int pairs = L.sm_count / 2;
   const int grid = 2 * (tiles < pairs ? tiles : pairs);
