@@ -62,6 +62,21 @@ def test_c1_full_layer():
     assert torch.equal(y2, y)
 
 
+def test_c4_size_layer_last_clip():
+    # One encoder layer over the encoder workload's 4 x 3000 frames (M = 12000
+    # rows per GEMM), in the walk orders of this size (grouped row panels for
+    # the QKV, gate/up and O inputs, N-fastest for the down projection's): the
+    # last clip is checked whole against the oracle, the first on a prefix.
+    vx = _vx()
+    dims = synth.VOXTRAL_RT
+    p = synth.layer_params(dims, seed=21)
+    x = synth.frames(4, 3000, dims.d_model, seed=22)
+    L = vx.pack_layer(cfg_of(dims), layer_params_dev(p))
+    y = host(vx.encoder_layer_fwd(cfg_of(dims), L, dev(x)))
+    compare_bf16(y[3:], oracle.encoder_layer(x[3:], p, dims), "C4-size layer, clip 3")
+    compare_bf16(y[:1, :200], oracle.encoder_layer(x[:1, :200], p, dims), "C4-size layer, clip 0 prefix")
+
+
 def test_layer_pack_matches_parameters():
     vx = _vx()
     p = synth.layer_params(SMALL, seed=5, gate_up_bias=True)
