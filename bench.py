@@ -417,7 +417,7 @@ def component_c1(vx, torch, flush, hbm, tf, oracle_on):
     wl = {"M": 1500, "attn": (1, 1500, 32, 750)}
     fl = layer_flops(1, 1500)
     out = {"ms_per_step": ms, "frames_per_s": 1500 / ms * 1e3, "tflops": fl / ms / 1e9,
-           "frac_of_measured_peak": fl / ms / 1e9 / tf,
+           "frac_of_peak": fl / ms / 1e9 / tf,
            "roofline": roofline(tr, wl, tf, hbm, PEAK_KIND, "C1", "burst"),
            "kernels": per_kernel_table(tr, wl)}
     if oracle_on:
@@ -474,7 +474,7 @@ def component_c2(vx, torch, flush, hbm, tf, oracle_on):
         fl = attn_flops(8, T, 32, 64, 750)
         ka = tr["swa_attn_tc"]["ms_per_launch"]
         e = {"ms_per_call": ms, "attn_kernel_ms": ka, "rope_ms": tr.get("rope", {}).get("ms_per_step"),
-             "gflop": fl / 1e9, "kernel_tflops": fl / ka / 1e9, "kernel_frac_of_measured_peak": fl / ka / 1e9 / tf,
+             "gflop": fl / 1e9, "kernel_tflops": fl / ka / 1e9, "kernel_frac_of_peak": fl / ka / 1e9 / tf,
              "call_tflops": fl / ms / 1e9, "tiles_per_clip_head": attn_tiles(T, 750)}
         if oracle_on:
             import oracle
@@ -537,7 +537,7 @@ def component_c3(vx, torch, flush, hbm, tf, oracle_on, L=32):
     del gr
     wl = {"M": S * n}
     out = {"ms_per_step_eager": ms, "ms_per_step_graph": ms_g, "bytes_per_step": total,
-           "gbs_graph": total / ms_g / 1e6, "frac_of_measured_hbm": total / ms_g / 1e6 / hbm,
+           "gbs_graph": total / ms_g / 1e6, "frac_of_hbm": total / ms_g / 1e6 / hbm,
            "frames_per_s_graph": S * n / ms_g * 1e3,
            "ring_attn_ms_per_launch": ring_ms, "ring_attn_gbs": ring_bytes / ring_ms / 1e6,
            "ring_fill": "vx_stream_prefill over 1000 frames per stream (ring wrapped), then steps at pos 1000, 1004, ...",
@@ -618,7 +618,7 @@ def component_next(vx, torch, flush, hbm, tf, oracle_on):
                              "tflops_fp32": 24000 * LOG_MEL_FLOP_PER_FRAME / ms_m / 1e9,
                              "frac_of_fp32_alu_peak": 24000 * LOG_MEL_FLOP_PER_FRAME / ms_m / 1e9 / FP32_ALU_TFLOPS},
            "projector_4x3000": {"ms_per_call": ms_p, "tokens_per_s": 3000 / ms_p * 1e3,
-                                "tflops": proj_flop / ms_p / 1e9, "frac_of_measured_peak": proj_flop / ms_p / 1e9 / tf}}
+                                "tflops": proj_flop / ms_p / 1e9, "frac_of_peak": proj_flop / ms_p / 1e9 / tf}}
     del x, out, audio, melo, wsm, wsp
     torch.cuda.empty_cache()
 
@@ -854,7 +854,11 @@ def main(argv=None):
     tr = traced_kernels(vx, torch, step, 0 if args.no_trace else 3, flush)
     wl = {"M": B * To, "attn": (B, To, 32, C4["W"]), "stem": (B, Tm)}
     if tr:
-        roof = roofline(tr, wl, tf_burst, hbm, peak_kind, "C4", "burst")
+        # the dominant kernel is timed inside the whole ~26 ms forward: the
+        # sustained (power-capped) GEMM figure is its denominator
+        roof = roofline(tr, wl, tf_sust, hbm, peak_kind, "C4", "sustained")
+        if roof.get("bound") == "tensor":
+            roof["frac_of_burst"] = roof["achieved"] / tf_burst
         kernels = per_kernel_table(tr, wl)
     else:
         roof, kernels = {"bound": None, "achieved": None, "peak": None, "unit": None, "frac": None,
@@ -885,7 +889,11 @@ def main(argv=None):
                        "l2": "flushed between timed steps (256 MiB write outside the step events); the 1.93 GB "
                              "of layer weights exceed L2"},
             "encoder_tflops": fl / (ms / 1e3) / 1e12,
-            "encoder_frac_of_measured_peak": fl / (ms / 1e3) / 1e12 / tf_burst,
+            "encoder_frac_of_peak": fl / (ms / 1e3) / 1e12 / tf_sust,
+            "peaks": {"kind": peak_kind, "bf16_tflops_burst": tf_burst, "bf16_tflops_sustained": tf_sust,
+                      "hbm_gbs": hbm,
+                      "use": "encoder and its dominant kernel: sustained (timed inside the forward); "
+                             "components timed alone: burst; HBM-bound rows: the copy figure"},
             "e2e": {"value": frames_all / (ms_e2e / 1e3), "unit": UNIT,
                     "h2d_bytes_per_step": int(mel.numel() * 4), "d2h_bytes_per_step": int(out.numel() * 4),
                     "method": "vx_encoder_fwd from pinned host mel to pinned host output; H2D, encoder (after a "
