@@ -272,7 +272,7 @@ __device__ __forceinline__ void epilogue_prepare(const GemmArgs& a, EpiPre<BN, E
       const int64_t pos = (a.pos_arr ? (ok ? a.pos_arr[b] : 0) : a.pos0) + t;
       const float posf = static_cast<float>(pos);
 #pragma unroll
-      for (int j = 0; j < 32; ++j) rope_sincos(posf, a.inv_freq_hi[j], a.inv_freq_lo[j], &p.sn[j], &p.cs[j]);
+      for (int j = 0; j < 32; ++j) rope_sincos_fast(posf, a.inv_freq_hi[j], a.inv_freq_lo[j], &p.sn[j], &p.cs[j]);
     }
   }
   if constexpr (EPI == EPI_F32) {

@@ -408,7 +408,8 @@ __device__ __forceinline__ uint4 ld_global_cs_v4(const void* p) {
 // sin/cos of pos * inv_freq with the product's rounding error carried
 // separately and the argument reduced by 2*pi in two parts (Cody-Waite),
 // so the angle stays accurate for large positions.
-__device__ __forceinline__ void rope_sincos(float posf, float inv_hi, float inv_lo, float* s, float* c) {
+// The angle reduced to [-pi, pi] (see rope_sincos).
+__device__ __forceinline__ float rope_angle(float posf, float inv_hi, float inv_lo) {
   constexpr double kTwoPi = 6.283185307179586476925286766559;
   constexpr float kTwoPiHi = static_cast<float>(kTwoPi);
   constexpr float kTwoPiLo = static_cast<float>(kTwoPi - static_cast<double>(kTwoPiHi));
@@ -418,8 +419,17 @@ __device__ __forceinline__ void rope_sincos(float posf, float inv_hi, float inv_
   const float k = rintf(a_hi * kInvTwoPi);
   float r = fmaf(-k, kTwoPiHi, a_hi);
   r = fmaf(-k, kTwoPiLo, r);
-  r += a_lo;
-  sincosf(r, s, c);
+  return r + a_lo;
+}
+__device__ __forceinline__ void rope_sincos(float posf, float inv_hi, float inv_lo, float* s, float* c) {
+  sincosf(rope_angle(posf, inv_hi, inv_lo), s, c);
+}
+// The same with the hardware sine / cosine on the reduced angle (absolute
+// error ~2^-21 on [-pi, pi], far below the bf16 rounding of the rotated
+// values); for the QKV GEMM's epilogue, where 32 angles per row and tile
+// would otherwise cost more issue slots than the rest of the epilogue.
+__device__ __forceinline__ void rope_sincos_fast(float posf, float inv_hi, float inv_lo, float* s, float* c) {
+  __sincosf(rope_angle(posf, inv_hi, inv_lo), s, c);
 }
 
 }  // namespace vx
