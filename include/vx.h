@@ -173,15 +173,14 @@ VX_API size_t vx_swa_attn_workspace(vx_dtype dt, int B, int T, int H, int D, int
  * run attention (real-time audio callbacks that must not wait on the
  * driver's allocator, plug-in hosts that own every device allocation, code
  * under a fixed memory budget).  It takes no workspace and allocates nothing:
- * its scratch (the RoPE-rotated q and k, their per-position cos/sin table,
- * and the status word of the bounded waits) is one static device array of
- * 32 MiB + 256 bytes inside this library, held by every GPU that loads the
- * library until the process exits.  Inputs and outputs are still the caller's.
+ * its scratch (the RoPE-rotated q and k, and the status word of the bounded
+ * waits) is one static device array of 32 MiB + 256 bytes inside this
+ * library, held by every GPU that loads the library until the process exits.
+ * Inputs and outputs are still the caller's.
  * Limit: with apply_rope, each rotated tensor takes B*T*H*64*es bytes
- * (es = 2 for bf16, 4 for fp32) rounded up to a multiple of 256, and the
- * cos/sin table T*256 bytes; 2 * that rounded size + T*256 must be at most
- * 32 MiB (33554432 bytes).  For bf16 that is B*T*H + T <= 131072 when B*T*H
- * is even (e.g. B=1, H=32: T <= 3971); for fp32, 2*B*T*H + T <= 131072.
+ * (es = 2 for bf16, 4 for fp32) rounded up to a multiple of 256; 2 * that
+ * rounded size must be at most 32 MiB (33554432 bytes).  For bf16 that is
+ * B*T*H <= 131072 (e.g. B=1, H=32: T <= 4096); for fp32, B*T*H <= 65536.
  * Without RoPE no scratch beyond the status word is used and any size runs.
  * Larger calls return VX_ERR_INVALID_ARG with a message and enqueue nothing.
  * The first call on each device looks up the array's device address (with

@@ -634,7 +634,6 @@ size_t vx_swa_attn_workspace(vx_dtype dt, int B, int T, int H, int D, int apply_
     const size_t es = dt == VX_F32 ? 4 : 2;
     cv.take(size_t(B) * T * H * D * es);
     cv.take(size_t(B) * T * H * D * es);
-    cv.take(size_t(T) * 32 * 8);
   }
   return align_up(cv.off, kAlign);
 }
@@ -663,10 +662,7 @@ vx_status vx_swa_attn_fwd(const void* q, const void* k, const void* v, void* o, 
     const size_t es = dt == VX_F32 ? 4 : 2;
     void* qr = cv.take(size_t(B) * T * H * D * es);
     void* kr = cv.take(size_t(B) * T * H * D * es);
-    void* tb = cv.take(size_t(T) * 32 * 8);
-    VX_CUDA(traced(L, "rope", 2, [&] {
-      return launch_rope(L, q, k, qr, kr, tb, dt == VX_BF16, B, T, H, pos0, rope_theta);
-    }));
+    VX_CUDA(traced(L, "rope", 1, [&] { return launch_rope(L, q, k, qr, kr, dt == VX_BF16, B, T, H, pos0, rope_theta); }));
     qq = qr;
     kk = kr;
   }

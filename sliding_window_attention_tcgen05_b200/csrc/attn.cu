@@ -571,66 +571,69 @@ struct RopeArgs {
   float lo[32];
 };
 
-// table[t][m] = (cos, sin) of (pos0 + t) * inv_freq_m, t < T, m < 32.
-__global__ void rope_table_kernel(float2* __restrict__ table, int T, int64_t pos0, const __grid_constant__ RopeArgs f) {
-  pdl_wait();
-  pdl_trigger();
-  const int idx = blockIdx.x * blockDim.x + threadIdx.x;
-  if (idx >= T * 32) return;
-  const int t = idx >> 5, m = idx & 31;
-  float sn, cs;
-  rope_sincos(static_cast<float>(pos0 + t), f.hi[m], f.lo[m], &sn, &cs);
-  table[idx] = make_float2(cs, sn);
-}
-
-// Rotates q and k ([B, T, H, 64]) into qr and kr with the table: thread
-// handles pairs (m, m + 32) for 8 consecutive m of one (tensor, row, head).
+// Rotates q and k ([B, T, H, 64]) into qr and kr in one pass: warp per
+// (row, tensor).  Lane m computes the angle (pos0 + t) * inv_freq_m once;
+// each lane then takes the 8-pair groups g = lane % 4 (pairs m = 8g .. 8g+7
+// with m + 32) of heads lane / 4, lane / 4 + 8, ..., with its group's eight
+// cos / sin from the other lanes by shuffles, so every access is 16 bytes
+// and each angle is computed once per row and tensor.
 template <bool BF16>
-__global__ void rope_apply_kernel(const void* __restrict__ q, const void* __restrict__ k, void* __restrict__ qr,
-                                  void* __restrict__ kr, const float2* __restrict__ table, int64_t rows, int T, int H) {
+__global__ void __launch_bounds__(256) rope_rows_kernel(const void* __restrict__ q, const void* __restrict__ k,
+                                                        void* __restrict__ qr, void* __restrict__ kr, int64_t rows,
+                                                        int T, int H, int64_t pos0, const __grid_constant__ RopeArgs f) {
   pdl_wait();
   pdl_trigger();
-  const int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  const int64_t per = rows * H * 4;          // per tensor: (row, head, 8-pair group)
-  if (idx >= 2 * per) return;
-  const int which = idx >= per;
-  const int64_t j = which ? idx - per : idx;
-  const int g = static_cast<int>(j & 3);      // m = 8 g .. 8 g + 7
-  const int64_t rh = j >> 2;
-  const int t = static_cast<int>((rh / H) % T);
-  const int64_t e = rh * 64 + g * 8;
-  const float2* tb = table + t * 32 + g * 8;
-  float u[8], w[8];
-  if constexpr (BF16) {
-    const uint16_t* src = static_cast<const uint16_t*>(which ? k : q);
-    const uint4 a = *reinterpret_cast<const uint4*>(src + e);
-    const uint4 c = *reinterpret_cast<const uint4*>(src + e + 32);
-    u[0] = bf16lo(a.x); u[1] = bf16hi(a.x); u[2] = bf16lo(a.y); u[3] = bf16hi(a.y);
-    u[4] = bf16lo(a.z); u[5] = bf16hi(a.z); u[6] = bf16lo(a.w); u[7] = bf16hi(a.w);
-    w[0] = bf16lo(c.x); w[1] = bf16hi(c.x); w[2] = bf16lo(c.y); w[3] = bf16hi(c.y);
-    w[4] = bf16lo(c.z); w[5] = bf16hi(c.z); w[6] = bf16lo(c.w); w[7] = bf16hi(c.w);
-  } else {
-    const float* src = static_cast<const float*>(which ? k : q);
-#pragma unroll
-    for (int i = 0; i < 8; ++i) { u[i] = src[e + i]; w[i] = src[e + 32 + i]; }
-  }
-  float y1[8], y2[8];
+  const int64_t wid = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (wid >= 2 * rows) return;   // whole warps leave together
+  const int64_t row = wid >> 1;
+  const int which = static_cast<int>(wid & 1);
+  const int t = static_cast<int>(row % T);
+  float sn_m, cs_m;
+  rope_sincos(static_cast<float>(pos0 + t), f.hi[lane], f.lo[lane], &sn_m, &cs_m);
+  const int g = lane & 3;
+  float cs[8], sn[8];
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
-    const float2 cs = tb[i];
-    y1[i] = u[i] * cs.x - w[i] * cs.y;
-    y2[i] = w[i] * cs.x + u[i] * cs.y;
+    cs[i] = __shfl_sync(0xffffffffu, cs_m, 8 * g + i);
+    sn[i] = __shfl_sync(0xffffffffu, sn_m, 8 * g + i);
   }
-  if constexpr (BF16) {
-    uint16_t* dst = static_cast<uint16_t*>(which ? kr : qr);
-    *reinterpret_cast<uint4*>(dst + e) = make_uint4(pack_bf16x2(y1[0], y1[1]), pack_bf16x2(y1[2], y1[3]),
-                                                    pack_bf16x2(y1[4], y1[5]), pack_bf16x2(y1[6], y1[7]));
-    *reinterpret_cast<uint4*>(dst + e + 32) = make_uint4(pack_bf16x2(y2[0], y2[1]), pack_bf16x2(y2[2], y2[3]),
-                                                         pack_bf16x2(y2[4], y2[5]), pack_bf16x2(y2[6], y2[7]));
-  } else {
-    float* dst = static_cast<float*>(which ? kr : qr);
+  for (int h = lane >> 2; h < H; h += 8) {
+    const int64_t e = (row * H + h) * 64 + 8 * g;
+    float u[8], w[8];
+    if constexpr (BF16) {
+      const uint16_t* src = static_cast<const uint16_t*>(which ? k : q);
+      const uint4 a = *reinterpret_cast<const uint4*>(src + e);
+      const uint4 c = *reinterpret_cast<const uint4*>(src + e + 32);
+      u[0] = bf16lo(a.x); u[1] = bf16hi(a.x); u[2] = bf16lo(a.y); u[3] = bf16hi(a.y);
+      u[4] = bf16lo(a.z); u[5] = bf16hi(a.z); u[6] = bf16lo(a.w); u[7] = bf16hi(a.w);
+      w[0] = bf16lo(c.x); w[1] = bf16hi(c.x); w[2] = bf16lo(c.y); w[3] = bf16hi(c.y);
+      w[4] = bf16lo(c.z); w[5] = bf16hi(c.z); w[6] = bf16lo(c.w); w[7] = bf16hi(c.w);
+    } else {
+      const float4* src = reinterpret_cast<const float4*>(static_cast<const float*>(which ? k : q) + e);
+      const float4 a0 = src[0], a1 = src[1], c0 = src[8], c1 = src[9];
+      u[0] = a0.x; u[1] = a0.y; u[2] = a0.z; u[3] = a0.w; u[4] = a1.x; u[5] = a1.y; u[6] = a1.z; u[7] = a1.w;
+      w[0] = c0.x; w[1] = c0.y; w[2] = c0.z; w[3] = c0.w; w[4] = c1.x; w[5] = c1.y; w[6] = c1.z; w[7] = c1.w;
+    }
+    float y1[8], y2[8];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) { dst[e + i] = y1[i]; dst[e + 32 + i] = y2[i]; }
+    for (int i = 0; i < 8; ++i) {
+      y1[i] = u[i] * cs[i] - w[i] * sn[i];
+      y2[i] = w[i] * cs[i] + u[i] * sn[i];
+    }
+    if constexpr (BF16) {
+      uint16_t* dst = static_cast<uint16_t*>(which ? kr : qr);
+      *reinterpret_cast<uint4*>(dst + e) = make_uint4(pack_bf16x2(y1[0], y1[1]), pack_bf16x2(y1[2], y1[3]),
+                                                      pack_bf16x2(y1[4], y1[5]), pack_bf16x2(y1[6], y1[7]));
+      *reinterpret_cast<uint4*>(dst + e + 32) = make_uint4(pack_bf16x2(y2[0], y2[1]), pack_bf16x2(y2[2], y2[3]),
+                                                           pack_bf16x2(y2[4], y2[5]), pack_bf16x2(y2[6], y2[7]));
+    } else {
+      float4* dst = reinterpret_cast<float4*>(static_cast<float*>(which ? kr : qr) + e);
+      dst[0] = make_float4(y1[0], y1[1], y1[2], y1[3]);
+      dst[1] = make_float4(y1[4], y1[5], y1[6], y1[7]);
+      dst[8] = make_float4(y2[0], y2[1], y2[2], y2[3]);
+      dst[9] = make_float4(y2[4], y2[5], y2[6], y2[7]);
+    }
   }
 }
 
@@ -665,25 +668,19 @@ cudaError_t launch_attn_f32(const Launch& L, const float* q, const float* k, con
   return launch_kernel(swa_attn_f32_kernel, grid, dim3(128), 0, L.stream, q, k, v, o, T, H, window, scale);
 }
 
-cudaError_t launch_rope(const Launch& L, const void* q, const void* k, void* qr, void* kr, void* table, bool bf16,
-                        int B, int T, int H, int64_t pos0, float theta) {
+cudaError_t launch_rope(const Launch& L, const void* q, const void* k, void* qr, void* kr, bool bf16, int B, int T,
+                        int H, int64_t pos0, float theta) {
   RopeArgs f;
   for (int m = 0; m < 32; ++m) {
     const double inv = std::pow(static_cast<double>(theta), -2.0 * m / 64.0);
     f.hi[m] = static_cast<float>(inv);
     f.lo[m] = static_cast<float>(inv - static_cast<double>(f.hi[m]));
   }
-  float2* tb = static_cast<float2*>(table);
-  cudaError_t e = launch_kernel(rope_table_kernel, dim3((T * 32 + 255) / 256), dim3(256), 0, L.stream, tb, T, pos0, f);
-  if (e != cudaSuccess) return e;
   const int64_t rows = static_cast<int64_t>(B) * T;
-  const int64_t total = 2 * rows * H * 4;
-  const dim3 grid(static_cast<unsigned>((total + 255) / 256));
+  const dim3 grid(static_cast<unsigned>((2 * rows + 7) / 8));   // 8 warps per block
   if (bf16)
-    return launch_kernel(rope_apply_kernel<true>, grid, dim3(256), 0, L.stream, q, k, qr, kr,
-                         static_cast<const float2*>(tb), rows, T, H);
-  return launch_kernel(rope_apply_kernel<false>, grid, dim3(256), 0, L.stream, q, k, qr, kr,
-                       static_cast<const float2*>(tb), rows, T, H);
+    return launch_kernel(rope_rows_kernel<true>, grid, dim3(256), 0, L.stream, q, k, qr, kr, rows, T, H, pos0, f);
+  return launch_kernel(rope_rows_kernel<false>, grid, dim3(256), 0, L.stream, q, k, qr, kr, rows, T, H, pos0, f);
 }
 
 }  // namespace vx

@@ -5,9 +5,8 @@
 // they run attention: real-time audio callbacks that must not block on the
 // driver's allocator, plug-in hosts that own every device allocation, and
 // code running under a fixed memory budget that may not grow.  This entry
-// point takes no workspace.  Its scratch -- the RoPE-rotated q and k, their
-// cos/sin table, and the status word of the bounded waits -- lives in one
-// file-scope device array of
+// point takes no workspace.  Its scratch -- the RoPE-rotated q and k and the
+// status word of the bounded waits -- lives in one file-scope device array of
 // kNoAllocScratchBytes that every GPU loading this library holds until the
 // process exits.  Inputs and outputs are still the caller's.
 #include <cstring>
@@ -18,7 +17,7 @@
 
 namespace {
 
-// 256 bytes of status word, then room for the rotated q and k and the table.
+// 256 bytes of status word, then room for the rotated q and k.
 constexpr size_t kNoAllocStatusBytes = 256;
 constexpr size_t kNoAllocScratchBytes = (32u << 20) + kNoAllocStatusBytes;   // 32 MiB + status
 
@@ -107,8 +106,7 @@ vx_status vx_swa_attn_fwd_noalloc(const void* q, const void* k, const void* v, v
   }
   const size_t es = dt == VX_F32 ? 4 : 2;
   const size_t one = static_cast<size_t>(B) * T * H * D * es;   // one rotated tensor
-  const size_t table = static_cast<size_t>(T) * 32 * 8;       // cos / sin per position
-  const size_t need = apply_rope ? 2 * ((one + 255) / 256 * 256) + table : 0;
+  const size_t need = apply_rope ? 2 * ((one + 255) / 256 * 256) : 0;
   if (need > kNoAllocScratchBytes - kNoAllocStatusBytes) {
     set_error("vx_swa_attn_fwd_noalloc: B*T*H = %lld needs %zu bytes of scratch for the rotated q/k, more than "
               "the %zu-byte static limit (use vx_swa_attn_fwd with a workspace)",
@@ -137,9 +135,8 @@ vx_status vx_swa_attn_fwd_noalloc(const void* q, const void* k, const void* v, v
     unsigned char* sc = static_cast<unsigned char*>(base) + kNoAllocStatusBytes;
     void* qr = sc;
     void* kr = sc + (one + 255) / 256 * 256;
-    void* tb = sc + 2 * ((one + 255) / 256 * 256);
-    if ((e = traced(L, "rope", 2, [&] {
-           return launch_rope(L, q, k, qr, kr, tb, dt == VX_BF16, B, T, H, pos0, rope_theta);
+    if ((e = traced(L, "rope", 1, [&] {
+           return launch_rope(L, q, k, qr, kr, dt == VX_BF16, B, T, H, pos0, rope_theta);
          })) != cudaSuccess) {
       set_error("vx_swa_attn_fwd_noalloc: RoPE launch failed: %s", cudaGetErrorString(e));
       return VX_ERR_CUDA;

@@ -184,9 +184,9 @@ cudaError_t launch_attn_f32(const Launch& L, const float* q, const float* k, con
                             float* o, int B, int T, int H, int window, float scale);
 
 // RoPE of q and k ([B, T, H, 64], fp32 or bf16) into qr and kr (same layout
-// and dtype); table: T * 32 float2 of scratch for the per-position cos / sin.
-cudaError_t launch_rope(const Launch& L, const void* q, const void* k, void* qr, void* kr, void* table, bool bf16,
-                        int B, int T, int H, int64_t pos0, float theta);
+// and dtype), one kernel.
+cudaError_t launch_rope(const Launch& L, const void* q, const void* k, void* qr, void* kr, bool bf16, int B, int T,
+                        int H, int64_t pos0, float theta);
 
 // ---------------------------------------------------------------- others --
 // h = x + bias + sum_{k < nparts} parts[k * part_stride + .]  (parts/bias optional);

@@ -80,17 +80,16 @@ def test_noalloc_without_rope_and_repeat_is_deterministic():
 
 
 def test_noalloc_size_limit_both_sides():
-    # bf16 with RoPE: 2 * roundup256(B*T*H*128) + T*256 <= 32 MiB, i.e.
-    # B*T*H + T <= 131072 for even B*T*H.  B=1, H=32: T = 3971 fits
-    # (33 * 3971 = 131043), T = 3972 does not (131076).
+    # bf16 with RoPE: 2 * roundup256(B*T*H*128) <= 32 MiB, i.e.
+    # B*T*H <= 131072.  B=1, H=32: T = 4096 fits, T = 4097 does not.
     vx = _lib()
     H, W = 32, 750
-    q, k, v = synth.attention_qkv(1, 3972, H, 64, seed=9, bf16=True)
+    q, k, v = synth.attention_qkv(1, 4097, H, 64, seed=9, bf16=True)
     q, k, v = (dev(x, torch.bfloat16) for x in (q, k, v))
     o = torch.empty_like(q)
     assert _noalloc(vx, q, k, v, o, W) == 1
     assert b"static limit" in vx.lib.vx_last_error()
-    qs, ks, vs = (x[:, :3971].contiguous() for x in (q, k, v))
+    qs, ks, vs = (x[:, :4096].contiguous() for x in (q, k, v))
     os_ = torch.empty_like(qs)
     assert _noalloc(vx, qs, ks, vs, os_, W) == 0, vx.lib.vx_last_error()
     ref = vx.swa_attn_fwd(qs, ks, vs, W)
@@ -100,10 +99,11 @@ def test_noalloc_size_limit_both_sides():
     q2 = torch.zeros(2, 4096, 32, 64, dtype=torch.bfloat16, device="cuda")
     o2 = torch.empty_like(q2)
     assert _noalloc(vx, q2, q2, q2, o2, 750, apply_rope=0) == 0
-    # fp32 with RoPE: 2 * B*T*H + T <= 131072; B=1, H=16: T = 3971 fits, 3972 does not
-    qf = torch.zeros(1, 3972, 16, 64, dtype=torch.float32, device="cuda")
+    # fp32 with RoPE: 2 * B*T*H*256 <= 32 MiB, i.e. B*T*H <= 65536; B=1, H=16:
+    # T = 4096 fits, 4097 does not
+    qf = torch.zeros(1, 4097, 16, 64, dtype=torch.float32, device="cuda")
     of = torch.empty_like(qf)
     assert _noalloc(vx, qf, qf, qf, of, 750) == 1
-    qf2 = qf[:, :3971].contiguous()
+    qf2 = qf[:, :4096].contiguous()
     assert _noalloc(vx, qf2, qf2, qf2, torch.empty_like(qf2), 750) == 0, vx.lib.vx_last_error()
     torch.cuda.synchronize()
