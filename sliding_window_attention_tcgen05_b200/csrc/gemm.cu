@@ -32,8 +32,8 @@
 // SwiGLU gate x up, GELU), transposes the chunk through a swizzled 2 KB
 // shared-memory buffer and stores it with four lanes per row, so every store
 // writes whole 32-byte sectors.  The tile's bias is staged in shared memory,
-// and the RoPE angles and the residual of the first chunk are prepared before
-// the accumulator is ready.
+// and the rows' positions and the residual of the first chunk are prepared
+// before the accumulator is ready.
 #include <cmath>
 #include <cstdio>
 
@@ -235,14 +235,14 @@ __device__ __forceinline__ void tma_flush(ChunkOut& co, const uint4* buf, int la
 // Per warp: TMEM lane quarter q = warp & 3 (tile rows 32 q ..), and one half
 // of the tile's column work (warp >> 2).  Everything of a tile's epilogue
 // that does not need the accumulator is done before waiting for it: the bias
-// into this warp's shared-memory copy, the RoPE angles of this lane's row, the
-// residual of the first chunk.  Warps never wait for one another, so a warp
+// into this warp's shared-memory copy, the position of this lane's row, the
+// residual of the first chunk.  The RoPE angles are computed per head where
+// they are used (hardware sine / cosine): holding all 32 would spill.  Warps never wait for one another, so a warp
 // that leaves the tile loop on a timeout cannot stall the others.
 template <int BN, int EPI>
 struct EpiPre {
   StoreRows sr;
-  float cs[EPI == EPI_QKV_ROPE ? 32 : 1];
-  float sn[EPI == EPI_QKV_ROPE ? 32 : 1];
+  float posf;
   float4 res[EPI == EPI_F32 ? 4 : 1];
 };
 
@@ -270,9 +270,7 @@ __device__ __forceinline__ void epilogue_prepare(const GemmArgs& a, EpiPre<BN, E
       int b, t;
       out_row(a, mw + lane, ok, b, t);
       const int64_t pos = (a.pos_arr ? (ok ? a.pos_arr[b] : 0) : a.pos0) + t;
-      const float posf = static_cast<float>(pos);
-#pragma unroll
-      for (int j = 0; j < 32; ++j) rope_sincos_fast(posf, a.inv_freq_hi[j], a.inv_freq_lo[j], &p.sn[j], &p.cs[j]);
+      p.posf = static_cast<float>(pos);
     }
   }
   if constexpr (EPI == EPI_F32) {
@@ -309,9 +307,11 @@ __device__ __forceinline__ void epilogue_tile(const GemmArgs& a, EpiPre<BN, EPI>
       if (rope) {
 #pragma unroll
         for (int j = 0; j < 32; ++j) {
+          float sn, cs;
+          rope_sincos_fast(p.posf, a.inv_freq_hi[j], a.inv_freq_lo[j], &sn, &cs);
           const float u = x0[j], w = x1[j];
-          x0[j] = u * p.cs[j] - w * p.sn[j];
-          x1[j] = w * p.cs[j] + u * p.sn[j];
+          x0[j] = u * cs - w * sn;
+          x1[j] = w * cs + u * sn;
         }
       }
 #pragma unroll
