@@ -254,6 +254,7 @@ struct LayerBufs {
   uint16_t* act;   // [M, F]     bf16 SwiGLU output
   float* xmat;     // [M, d]     fp32 materialised layer input (when it arrives as partial sums)
   float* parts;    // [split_cap(M), M, d] fp32 split-K partial sums (null when split_cap(M) == 1)
+  int* norm_ctr;   // [M/32 + 2] counters of an RMSNorm run in a residual GEMM's tail (or null)
 };
 
 // Most K-splits a GEMM with M rows may use: few-row GEMMs have too few output
@@ -272,7 +273,15 @@ LayerBufs carve_layer(Carve& cv, const vx_layer_cfg& c, int64_t M) {
   const int cap = split_cap(M);
   b.xmat = cap > 1 ? static_cast<float*>(cv.take(M * d * 4)) : nullptr;
   b.parts = cap > 1 ? static_cast<float*>(cv.take(cap * M * d * 4)) : nullptr;
+  b.norm_ctr = (cap == 1 && d == 1280) ? static_cast<int*>(cv.take(((M + 31) / 32 + 2) * 4)) : nullptr;
   return b;
+}
+
+// The tail-norm counters start at zero (each kernel that uses them leaves them
+// at zero again).
+vx_status init_norm_ctr(const Launch& L, const LayerBufs& b, int64_t M) {
+  if (b.norm_ctr) VX_CUDA(cudaMemsetAsync(b.norm_ctr, 0, ((M + 31) / 32 + 2) * 4, L.stream));
+  return VX_OK;
 }
 
 size_t layer_ws_bytes(const vx_layer_cfg& c, int64_t M) {
@@ -357,14 +366,25 @@ struct Pending {
   const float* parts;
   int nparts;
   const uint16_t* bias;
+  bool normed;   // its consumer's RMSNorm has been written already (by the producing GEMM)
+};
+
+// An RMSNorm of a residual GEMM's output, run in that GEMM's tail: gain g,
+// output y (bf16 or fp32; may be the GEMM's own output).
+struct NormFuse {
+  const uint16_t* g;
+  void* y;
+  bool y_bf16;
 };
 
 // A residual GEMM  out = A W^T + bias + res  in the planned shape: fused into
 // the epilogue when the plan has one K-split, else as fp32 partial sums whose
 // reduction (with bias and residual) is left pending for the next RMSNorm.
+// With one K-split, a CTA-pair plan, d = 1280 and tail counters, the RMSNorm
+// nf of the output runs in the GEMM's tail (result->normed).
 vx_status residual_gemm(const Launch& L, const char* name, const void* A, int64_t lda, const void* W, int M, int N,
                         int K, const uint16_t* bias, const float* res, float* out, float* parts, int max_splits,
-                        Pending* result) {
+                        Pending* result, const NormFuse* nf = nullptr, int* norm_ctr = nullptr, float eps = 0.f) {
   GemmArgs a = base_args(L, M, N, K);
   const GemmPlan p = plan_gemm(M, N, K, EPI_F32, parts ? max_splits : 1, L.sm_count);
   a.ld_out = N;
@@ -378,6 +398,14 @@ vx_status residual_gemm(const Launch& L, const char* name, const void* A, int64_
     a.bias = bias;
     a.res = res; a.ld_res = N;
     *result = Pending{out, nullptr, 0, nullptr};
+    if (nf && norm_ctr && p.pair && N == 1280) {
+      a.norm_g = nf->g;
+      a.norm_y = nf->y;
+      a.norm_y_bf16 = nf->y_bf16 ? 1 : 0;
+      a.norm_eps = eps;
+      a.norm_ctr = norm_ctr;
+      result->normed = true;
+    }
   }
   return gemm(L, name, A, lda, W, a, EPI_F32, &p);
 }
@@ -404,7 +432,7 @@ struct RingLayer {
 //   out = h + bd + act Wd^T           (fused into y, or pending)
 vx_status run_layer(const Launch& L, const vx_layer_cfg& c, const vx_layer_weights& w, const Pending& in,
                     Pending* out, float* y, int nseq, int rows, int64_t pos0, const LayerBufs& bf,
-                    const RingLayer* ring) {
+                    const RingLayer* ring, const NormFuse* next_norm = nullptr) {
   const int d = c.d_model, H = c.n_heads, HD = H * c.head_dim, F = c.ffn_hidden;
   const int M = nseq * rows;
   const int64_t pstride = static_cast<int64_t>(M) * d;
@@ -412,12 +440,12 @@ vx_status run_layer(const Launch& L, const vx_layer_cfg& c, const vx_layer_weigh
   const float sl2 = (1.0f / std::sqrt(static_cast<float>(c.head_dim))) * 1.4426950408889634f;
   const bool step = ring && ring->step;
   vx_status st;
-  // 1. x_l = reduce(in); y0 = RMSNorm(x_l)
+  // 1. x_l = reduce(in); y0 = RMSNorm(x_l) (unless the previous GEMM wrote it)
   const bool pending_in = in.parts != nullptr || in.bias != nullptr;
   const float* xl = pending_in ? bf.xmat : in.base;
-  VX_CUDA(rmsnorm(L, in.base, in.parts, in.nparts, pstride, in.bias,
-                          static_cast<const uint16_t*>(w.attn_norm_g), pending_in ? bf.xmat : nullptr, bf.y0, true, M,
-                          d, c.eps));
+  if (!in.normed)
+    VX_CUDA(rmsnorm(L, in.base, in.parts, in.nparts, pstride, in.bias, static_cast<const uint16_t*>(w.attn_norm_g),
+                    pending_in ? bf.xmat : nullptr, bf.y0, true, M, d, c.eps));
   // 2. QKV + bias + RoPE at (pos[s] or pos0) + t
   {
     GemmArgs a = base_args(L, M, 3 * HD, d);
@@ -448,16 +476,17 @@ vx_status run_layer(const Launch& L, const vx_layer_cfg& c, const vx_layer_weigh
         return launch_ring_fill(L, bf.qkv, 3LL * HD, HD, ring->k, ring->v, nseq, rows, H, ring->W);
       }));
   }
-  // 4. h = x_l + bo + att Wo^T
+  // 4. h = x_l + bo + att Wo^T (with 5. in its tail when it can)
   Pending hp;
+  const NormFuse norm2{static_cast<const uint16_t*>(w.ffn_norm_g), bf.y0, true};
   if ((st = residual_gemm(L, "gemm_o_residual", bf.att, HD, w.wo, M, d, HD, static_cast<const uint16_t*>(w.bo), xl,
-                          bf.h, bf.parts, cap, &hp)) != VX_OK)
+                          bf.h, bf.parts, cap, &hp, &norm2, bf.norm_ctr, c.eps)) != VX_OK)
     return st;
   // 5. y1 = RMSNorm(h), materialising h when it is pending
   const bool pending_h = hp.parts != nullptr;
-  VX_CUDA(rmsnorm(L, hp.base, hp.parts, hp.nparts, pstride, hp.bias,
-                          static_cast<const uint16_t*>(w.ffn_norm_g), pending_h ? bf.h : nullptr, bf.y0, true, M, d,
-                          c.eps));
+  if (!hp.normed)
+    VX_CUDA(rmsnorm(L, hp.base, hp.parts, hp.nparts, pstride, hp.bias, static_cast<const uint16_t*>(w.ffn_norm_g),
+                    pending_h ? bf.h : nullptr, bf.y0, true, M, d, c.eps));
   // 6. gate/up + SwiGLU
   {
     GemmArgs a = base_args(L, M, 2 * F, d);
@@ -465,9 +494,9 @@ vx_status run_layer(const Launch& L, const vx_layer_cfg& c, const vx_layer_weigh
     a.bias = static_cast<const uint16_t*>(w.bgu);
     if ((st = gemm(L, "gemm_gate_up_swiglu", bf.y0, d, w.wgu, a, EPI_SWIGLU)) != VX_OK) return st;
   }
-  // 7. out = h + bd + act Wd^T
+  // 7. out = h + bd + act Wd^T (with the next RMSNorm in its tail when the caller names one and it can)
   return residual_gemm(L, "gemm_down_residual", bf.act, F, w.wd, M, d, F, static_cast<const uint16_t*>(w.bd), bf.h, y,
-                       bf.parts, cap, out);
+                       bf.parts, cap, out, next_norm, bf.norm_ctr, c.eps);
 }
 
 // y = reduce(p) unless p already is y.
@@ -719,6 +748,7 @@ vx_status vx_encoder_layer_fwd(const vx_layer_cfg* cfg, const vx_layer_weights* 
   if ((st = make_launch(&L, ws, ws_bytes, vx_encoder_layer_workspace(cfg, B, T), stream)) != VX_OK) return st;
   Carve cv{static_cast<uint8_t*>(ws), kStatusBytes};
   const LayerBufs bf = carve_layer(cv, *cfg, int64_t(B) * T);
+  if ((st = init_norm_ctr(L, bf, int64_t(B) * T)) != VX_OK) return st;
   Pending out;
   if ((st = run_layer(L, *cfg, *w, Pending{x, nullptr, 0, nullptr}, &out, y, B, T, pos0, bf, nullptr)) != VX_OK)
     return st;
@@ -877,15 +907,22 @@ vx_status vx_encoder_fwd(const vx_layer_cfg* cfg, const float* mel, int B, int n
   }
   Carve cv{static_cast<uint8_t*>(ws), kStatusBytes};
   const LayerBufs bf = carve_layer(cv, *cfg, int64_t(B) * To);
+  if ((st = init_norm_ctr(L, bf, int64_t(B) * To)) != VX_OK) return st;
   Pending cur{out, nullptr, 0, nullptr};
   for (int l = 0; l < n_layers; ++l) {
     Pending next;
-    if ((st = run_layer(L, *cfg, layers[l], cur, &next, out, B, To, 0, bf, nullptr)) != VX_OK) return st;
+    // The layer's last GEMM may run the next RMSNorm: the next layer's (into
+    // its normalised input) or the final one (in place, fp32).
+    const NormFuse nn = l + 1 < n_layers ? NormFuse{static_cast<const uint16_t*>(layers[l + 1].attn_norm_g), bf.y0, true}
+                                         : NormFuse{static_cast<const uint16_t*>(final_g), out, false};
+    if ((st = run_layer(L, *cfg, layers[l], cur, &next, out, B, To, 0, bf, nullptr, &nn)) != VX_OK) return st;
     cur = next;
   }
-  const int64_t pstride = static_cast<int64_t>(B) * To * cfg->d_model;
-  VX_CUDA(rmsnorm(L, cur.base, cur.parts, cur.nparts, pstride, cur.bias,
-                          static_cast<const uint16_t*>(final_g), nullptr, out, false, B * To, cfg->d_model, cfg->eps));
+  if (!cur.normed) {
+    const int64_t pstride = static_cast<int64_t>(B) * To * cfg->d_model;
+    VX_CUDA(rmsnorm(L, cur.base, cur.parts, cur.nparts, pstride, cur.bias, static_cast<const uint16_t*>(final_g),
+                    nullptr, out, false, B * To, cfg->d_model, cfg->eps));
+  }
   return VX_OK;
 }
 
@@ -904,6 +941,7 @@ vx_status vx_stream_prefill(const vx_layer_cfg* cfg, const vx_layer_weights* lay
   if ((st = make_launch(&L, ws, ws_bytes, vx_encoder_layer_workspace(cfg, S, T), stream)) != VX_OK) return st;
   Carve cv{static_cast<uint8_t*>(ws), kStatusBytes};
   const LayerBufs bf = carve_layer(cv, *cfg, int64_t(S) * T);
+  if ((st = init_norm_ctr(L, bf, int64_t(S) * T)) != VX_OK) return st;
   const int64_t layer_elems = int64_t(S) * cfg->n_heads * ring->window * cfg->head_dim;
   Pending cur{x, nullptr, 0, nullptr};
   for (int l = 0; l < ring->n_layers; ++l) {
@@ -950,6 +988,7 @@ vx_status vx_stream_step(const vx_layer_cfg* cfg, const vx_layer_weights* layers
   if ((st = make_launch(&L, ws, ws_bytes, vx_stream_step_workspace(cfg, S, n_new), stream)) != VX_OK) return st;
   Carve cv{static_cast<uint8_t*>(ws), kStatusBytes};
   const LayerBufs bf = carve_layer(cv, *cfg, M);
+  if ((st = init_norm_ctr(L, bf, M)) != VX_OK) return st;
   const int64_t layer_elems = int64_t(S) * cfg->n_heads * ring->window * cfg->head_dim;
   Pending cur{x_new, nullptr, 0, nullptr};
   for (int l = 0; l < ring->n_layers; ++l) {

@@ -679,6 +679,102 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
   }
 }
 
+// ------------------------------------------------------- RMSNorm in the tail --
+// A residual GEMM whose output feeds an RMSNorm normalises it in the same
+// kernel: the O and down projections of the 4 x 3000 frame encoder have 235
+// tiles for 74 CTA pairs, so most pairs sit idle through the last round, and
+// their epilogue warps normalise the rows that are already complete instead.
+// Each epilogue warp publishes its 32 rows of a tile (release add on the row
+// group's counter once its stores are complete); a warp normalising two rows
+// first waits (bounded) for their group's count to reach 2 per column tile.
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+__device__ __forceinline__ void red_release_add(int* p, int v) {
+  asm volatile("red.release.gpu.global.add.s32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+__device__ __forceinline__ int ld_acquire(const int* p) {
+  int v;
+  asm volatile("ld.acquire.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+// The group counter *c reaches target (bounded: false after the wait limit or
+// once another wait of the CTA gave up).  Lane 0 polls.
+__device__ __forceinline__ bool norm_wait_group(const int* c, int target, const WaitCtx& w, int lane) {
+  int ok = 1;
+  if (lane == 0) {
+    const uint64_t t0 = globaltimer_ns();
+    while (ld_acquire(c) < target) {
+      if (*w.abort_flag) { ok = 0; break; }
+      if (globaltimer_ns() - t0 > w.limit_ns) {
+        *w.abort_flag = 1;
+        report_timeout(w.status, 39);
+        ok = 0;
+        break;
+      }
+      __nanosleep(64);
+    }
+  }
+  ok = __shfl_sync(0xffffffffu, ok, 0);
+  if (ok) (void)ld_acquire(c);   // every lane acquires the stores it is about to read
+  return ok != 0;
+}
+
+// Normalises rows two at a time (taken from the work counter) once their row
+// group is complete: d = 1280 = 10 float4 per lane.
+__device__ __forceinline__ void norm_tail_rows(const GemmArgs& a, int n_tiles, int lane, const WaitCtx& w) {
+  constexpr int NV = 10;
+  const int ngroups = (a.M + 31) >> 5;
+  int* work = a.norm_ctr + ngroups;
+  const int target = 2 * n_tiles;
+  uint2 gw[NV];
+#pragma unroll
+  for (int i = 0; i < NV; ++i) gw[i] = __ldg(reinterpret_cast<const uint2*>(a.norm_g) + lane + 32 * i);
+  const float* out = static_cast<const float*>(a.out);
+  while (true) {
+    int r0 = 0;
+    if (lane == 0) r0 = atomicAdd(work, 2);
+    r0 = __shfl_sync(0xffffffffu, r0, 0);
+    if (r0 >= a.M) break;
+    if (!norm_wait_group(a.norm_ctr + (r0 >> 5), target, w, lane)) break;
+    const int nr = a.M - r0 < 2 ? a.M - r0 : 2;
+    float4 v[2][NV];
+#pragma unroll
+    for (int rr = 0; rr < 2; ++rr)
+      if (rr < nr) {
+#pragma unroll
+        for (int i = 0; i < NV; ++i)
+          v[rr][i] = __ldcg(reinterpret_cast<const float4*>(out + static_cast<int64_t>(r0 + rr) * a.ld_out) + lane + 32 * i);
+      }
+#pragma unroll
+    for (int rr = 0; rr < 2; ++rr) {
+      if (rr >= nr) break;
+      float ss = 0.f;
+#pragma unroll
+      for (int i = 0; i < NV; ++i)
+        ss = fmaf(v[rr][i].x, v[rr][i].x, fmaf(v[rr][i].y, v[rr][i].y, fmaf(v[rr][i].z, v[rr][i].z, fmaf(v[rr][i].w, v[rr][i].w, ss))));
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+      const float inv = rsqrtf(ss / static_cast<float>(a.N) + a.norm_eps);
+      const int64_t row = static_cast<int64_t>(r0 + rr) * a.N;
+#pragma unroll
+      for (int i = 0; i < NV; ++i) {
+        const float4 x = v[rr][i];
+        const uint2 g = gw[i];
+        const float o0 = x.x * inv * bf16lo(g.x), o1 = x.y * inv * bf16hi(g.x);
+        const float o2 = x.z * inv * bf16lo(g.y), o3 = x.w * inv * bf16hi(g.y);
+        if (a.norm_y_bf16) {
+          reinterpret_cast<uint2*>(static_cast<uint16_t*>(a.norm_y) + row)[lane + 32 * i] =
+              make_uint2(pack_bf16x2(o0, o1), pack_bf16x2(o2, o3));
+        } else {
+          reinterpret_cast<float4*>(static_cast<float*>(a.norm_y) + row)[lane + 32 * i] = make_float4(o0, o1, o2, o3);
+        }
+      }
+    }
+  }
+}
+
 // ------------------------------------------------------------ CTA pairs --
 // A cluster of two CTAs computes a 256 x BN tile with tcgen05.mma.cta_group::2
 // (M = 256).  CTA r loads its own 128 rows of A and rows [r BN/2, (r+1) BN/2)
@@ -878,12 +974,35 @@ gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(ab ? acc_empty_leader1 : acc_empty_leader0);
+      if (EPI == EPI_F32 && a.norm_g) {   // publish this warp's 32 rows of the tile once stored
+        if (!a.tma_store) __threadfence();
+        __syncwarp();
+        const int grp = (m0 + (warp & 3) * 32) >> 5;
+        if (lane == 0) {
+          if (a.tma_store) {
+            bulk_wait_all();             // its TMA stores are complete ...
+            fence_proxy_async_global();  // ... and ordered before the generic release below
+          }
+          __threadfence();
+          if (grp < ((a.M + 31) >> 5)) red_release_add(a.norm_ctr + grp, 1);
+        }
+      }
     }
     if (a.tma_store && lane == 0) bulk_wait_all();   // this warp's output stores are complete
+    if (EPI == EPI_F32 && a.norm_g && !*abort_flag) norm_tail_rows(a, n_tiles, lane, wc);
   }
 
   tc_fence_before();
   __syncthreads();
+  if (EPI == EPI_F32 && a.norm_g && threadIdx.x == 0) {
+    // The last CTA to finish sets the counters back to zero for the next launch.
+    const int ngroups = (a.M + 31) >> 5;
+    __threadfence();
+    if (atomicAdd(a.norm_ctr + ngroups + 1, 1) == static_cast<int>(gridDim.x) - 1) {
+      for (int i = 0; i < ngroups + 2; ++i) a.norm_ctr[i] = 0;
+      __threadfence();
+    }
+  }
   cluster_sync_all();   // no CTA of the pair still uses TMEM or the peer's barriers
   if (warp == kMmaWarp) {
     tc_fence_after();
@@ -977,7 +1096,9 @@ cudaError_t launch_gemm(const Launch& L, const CUtensorMap& tmA, const CUtensorM
   if (args.M <= 0) return cudaSuccess;
   if (args.out == nullptr || args.k_splits != p.splits || p.splits < 1 || (args.K / kBK) % p.splits != 0 || args.K % kBK != 0 ||
       p.bn <= 0 || args.N % p.bn != 0 || (p.splits > 1 && epi != EPI_F32) ||
-      (args.tma_store && epi != EPI_F32 && epi != EPI_QKV_ROPE && epi != EPI_SWIGLU))
+      (args.tma_store && epi != EPI_F32 && epi != EPI_QKV_ROPE && epi != EPI_SWIGLU) ||
+      (args.norm_g && (epi != EPI_F32 || !p.pair || p.splits != 1 || args.N != 1280 || args.ld_out != args.N ||
+                       !args.norm_y || !args.norm_ctr)))
     return cudaErrorInvalidValue;
   // Walk the work units so that the larger operand crosses DRAM once: A
   // goes first when it is the larger one and too large to stay in L2 while

@@ -132,6 +132,18 @@ struct GemmArgs {
   // row panel of A run together, so A crosses DRAM once) or groups of
   // kOrderGroupRows row panels, M-fastest inside a group.
   int order;
+  // Pair kernel, EPI_F32 without K splits, N == 1280: when norm_g is set, the
+  // epilogue warps also normalise the output once it is stored: out row r ->
+  // norm_y row r = out_r / rms(out_r) * norm_g (RMSNorm, eps norm_eps; bf16
+  // when norm_y_bf16, else fp32; norm_y may be out itself).  norm_ctr: one int
+  // per 32 rows (stores of that row group done: 2 per column tile), a work
+  // counter and a finished-CTA counter, all zero at launch; the kernel's last
+  // CTA sets them back to zero.
+  const uint16_t* norm_g;
+  void* norm_y;
+  int norm_y_bf16;
+  float norm_eps;
+  int* norm_ctr;
   DevStatus* status;
   uint64_t limit_ns;
 };
