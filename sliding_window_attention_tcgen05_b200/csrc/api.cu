@@ -280,7 +280,9 @@ LayerBufs carve_layer(Carve& cv, const vx_layer_cfg& c, int64_t M) {
 // The tail-norm counters start at zero (each kernel that uses them leaves them
 // at zero again).
 vx_status init_norm_ctr(const Launch& L, const LayerBufs& b, int64_t M) {
-  if (b.norm_ctr) VX_CUDA(cudaMemsetAsync(b.norm_ctr, 0, ((M + 31) / 32 + 2) * 4, L.stream));
+  if (b.norm_ctr) VX_CUDA(traced(L, "zero_ctr", 1, [&] {
+    return launch_zero_ints(L, b.norm_ctr, static_cast<int>((M + 31) / 32 + 2));
+  }));
   return VX_OK;
 }
 

@@ -276,6 +276,16 @@ __global__ void selftest_wait_kernel(DevStatus* st, uint64_t limit_ns) {
   }
 }
 
+// Sets n ints to zero (counters in a caller's workspace), as a kernel of the
+// stream rather than a copy-engine memset, which could queue behind the
+// caller's copies.
+__global__ void zero_ints_kernel(int* __restrict__ p, int n) {
+  pdl_wait();
+  pdl_trigger();
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < n) p[i] = 0;
+}
+
 }  // namespace
 
 // Without partial sums the row needs no registers for them: a separate
@@ -363,6 +373,10 @@ cudaError_t launch_frames_to_tokens(const Launch& L, const float* x, uint16_t* t
   const int64_t blocks = (n8 + 255) / 256;
   return launch_kernel(frames_to_tokens_kernel, dim3(static_cast<unsigned>(blocks < 4096 ? blocks : 4096)), dim3(256),
                        0, L.stream, x, tok, T, T4, d, n8);
+}
+
+cudaError_t launch_zero_ints(const Launch& L, int* p, int n) {
+  return launch_kernel(zero_ints_kernel, dim3((n + 255) / 256), dim3(256), 0, L.stream, p, n);
 }
 
 cudaError_t launch_selftest_wait(const Launch& L) {

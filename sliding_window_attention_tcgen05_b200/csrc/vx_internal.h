@@ -215,6 +215,8 @@ cudaError_t launch_ring_attn(const Launch& L, const uint16_t* qkv, int64_t ld_qk
 cudaError_t launch_ring_fill(const Launch& L, const uint16_t* qkv, int64_t ld_qkv, int HD,
                              uint16_t* ring_k, uint16_t* ring_v, int S, int T, int H, int W);
 cudaError_t launch_pos_add(const Launch& L, int64_t* pos, int S, int64_t n, bool set);
+// p[0 .. n) = 0.
+cudaError_t launch_zero_ints(const Launch& L, int* p, int n);
 
 cudaError_t launch_pack_layer(const Launch& L, int d, int HD, int F, const uint16_t* wq,
                               const uint16_t* wk, const uint16_t* wv, const uint16_t* bq,
