@@ -6,8 +6,8 @@
 //   the key tiles that meet the causal window visited.
 // swa_attn_f32_kernel: fp32 CUDA-core reference-precision path (one warp per
 //   query row), used for fp32 inputs.
-// rope_table_kernel / rope_apply_kernel: RoPE pre-pass of vx_swa_attn_fwd on raw
-//   q, k (a per-position cos/sin table, then one vectorised rotation pass).
+// rope_rows_kernel: RoPE pre-pass of vx_swa_attn_fwd on raw q, k (one pass,
+//   each angle computed once per row).
 #include <cmath>
 
 #include "vx_internal.h"
