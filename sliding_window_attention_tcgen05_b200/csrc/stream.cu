@@ -84,10 +84,11 @@ __global__ void pos_add_kernel(int64_t* pos, int S, int64_t n, int set) {
 // of new frame p + r iff d >= r + 1 (i.e. f > p + r - W).  The NQ new frames
 // are attended by warp 0 in one extra 16-key block read from the qkv rows.
 constexpr int kRingTmaThreads = 160;   // 4 consumer warps + 1 TMA producer warp
-// Three 16 KB stages (54.5 KB of shared memory) let four CTAs share an SM.
-// Measured on the 64-stream, 32-layer step: the kernel is bound by how many
-// CTAs run at once, not by the stages in flight per CTA (2 / 3 / 4 / 6 / 8
-// stages = 5 / 4 / 3 / 2 / 1 CTAs per SM: 78.2 / 75.5 / 76.2 / 92.4 / 154 us).
+// Three 16 KB stages (54.5 KB of shared memory) let four CTAs share an SM
+// (86 registers also allow four).  Measured on the 64-stream, 32-layer step:
+// the kernel is bound by how many CTAs run at once more than by the stages in
+// flight per CTA (3 / 4 / 6 / 8 stages = 4 / 3 / 2 / 1 CTAs per SM: 75.5 /
+// 76.2 / 92.4 / 154 us; 2 stages, still 4 CTAs per SM: 78.2 us).
 constexpr int kRingTmaStages = 3;
 constexpr int kRingTmaSmem = 1024 + kRingTmaStages * kStageBytes + 2 * 16 * 128 + 256;
 
