@@ -59,6 +59,37 @@ def test_small_stream_matches_oracle_and_whole_sequence(prefill, n_new, steps):
     assert torch.all(ring.pos == T)
 
 
+@pytest.mark.parametrize("window,S,prefill,n_new", [(16, 600, 21, 1), (16, 600, 21, 8), (200, 300, 230, 4),
+                                                     (200, 160, 37, 3)])
+def test_many_items_per_ring_cta(window, S, prefill, n_new):
+    # More (stream, head) items than the ring kernel keeps resident (a few CTAs
+    # per SM), so each CTA walks several items through one stage ring, items of
+    # one chunk (W = 16) or of several with a ragged last one (W = 200, wrapped
+    # or not).  Every stream must equal the whole-sequence output, and sampled
+    # streams the oracle.
+    vx = _vx()
+    dims = synth.LayerDims(d_model=256, n_heads=4, head_dim=64, ffn_hidden=512, window=window)
+    layers = layer_stack(dims, 1, 71)
+    steps = 2
+    T = prefill + n_new * steps
+    x = synth.frames(S, T, dims.d_model, seed=72)
+    Ls = [vx.pack_layer(cfg_of(dims), layer_params_dev(p)) for p in layers]
+    ring = vx.KVRing(cfg_of(dims), 1, S)
+    vx.stream_prefill(cfg_of(dims), Ls, ring, dev(x[:, :prefill]))
+    whole_gpu = host(vx.stream_prefill(cfg_of(dims), Ls, vx.KVRing(cfg_of(dims), 1, S), dev(x)))
+    sample = [0, S // 2 + 1, S - 1]
+    xs = x[sample]
+    rings = _oracle_rings(xs, layers, dims, prefill)
+    pos = np.full(len(sample), prefill)
+    for st in range(steps):
+        rows = slice(prefill + st * n_new, prefill + (st + 1) * n_new)
+        got = host(vx.stream_step(cfg_of(dims), Ls, ring, dev(x[:, rows])))
+        compare_bf16(got, whole_gpu[:, rows], f"step {st} vs whole-sequence GPU")
+        want, rings, pos = oracle.stream_step(xs[:, rows], layers, dims, rings, pos)
+        compare_bf16(got[sample], want, f"step {st} vs oracle")
+    assert torch.all(ring.pos == T)
+
+
 def test_ring_slots_bit_exact_across_wrap():
     # Layer 0's K/V depend only on the layer input, so after [prefill T, step 4]
     # the layer-0 ring must equal, bit for bit, the ring after prefill T + 4;
