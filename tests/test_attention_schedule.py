@@ -8,7 +8,8 @@ Checked for many (T, W, B, H, grid): every (clip, head, query tile) is
 processed exactly once; the visited key tiles hold every key of every row's
 window (i - W < j <= i, causal) and each of them holds a key of some row's
 window; the union range covers both tiles' ranges with no gap; the rounds
-are dealt heaviest first."""
+are dealt heaviest first.  The streaming kernel's slot-order mask over the
+ring is checked against the window rule as well."""
 import pytest
 
 KEY_TILE = 64
@@ -91,3 +92,24 @@ def test_key_tiles_cover_exactly_the_windows(T, W):
             for t in range(kt0, kt0 + n):   # every visited tile is needed by some row
                 assert any(max(0, i - W + 1) < (t + 1) * KEY_TILE and i >= t * KEY_TILE for i in rows)
         assert covered == set(range(u0, u0 + nu)), "the union has a gap or extra tiles"
+
+
+@pytest.mark.parametrize("W", [1, 2, 5, 16, 64, 65, 750])
+def test_ring_slot_mask_is_the_window(W):
+    # The streaming kernel walks the ring in slot order and keeps slot j as a
+    # key of new frame p + r (r < n_new) iff j < min(p, W), d >= r + 1 and
+    # p - W + d >= 0, with d = (j - p) mod W.  By the ring rule (frame f in
+    # slot f mod W, frames max(0, p - W) .. p - 1 cached) that must be the set
+    # of cached frames in the window of p + r: p + r - W < f <= p + r, f < p.
+    for p in list(range(0, 3 * W + 3)) + [1000, 1003]:
+        nslots = min(p, W)
+        cached = {f % W: f for f in range(max(0, p - W), p)}
+        for r in range(8):
+            got = set()
+            for j in range(W):
+                d = (j - p) % W
+                if j < nslots and d >= r + 1 and p - W + d >= 0:
+                    got.add(p - W + d)
+                    assert cached.get(j) == p - W + d, "slot holds another frame"
+            want = {f for f in cached.values() if p + r - W < f <= p + r}
+            assert got == want, (p, r)
